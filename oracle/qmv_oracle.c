@@ -1,0 +1,511 @@
+/*
+ * qmv_oracle.c -- plain, slow, obviously-correct CPU oracle for weight-only
+ * block-quantized matvec.  TEST INFRASTRUCTURE ONLY: nothing in the product
+ * path (the CUDA library and its Python binding) may call, link or include
+ * this file.  It shares no header, helper, table or constant generator with
+ * the CUDA code.
+ *
+ * Sources (cited by page title and section):
+ *   [P1] "Stream D -- Quantization (FP4 + QAT-int4): feasibility, first
+ *        result, and plan", sec. 1 "Toolchain reality" (E2M1 / OCP MX dtype,
+ *        per-block 32 along in-features, e8m0 scale formula, 2 values per
+ *        byte packing) and sec. 2 "The de-risk experiment" (fp4 fake-quant
+ *        numerics; int4/int8 symmetric-with-clipping, MSE-optimal clip).
+ *   [P2] "Dense-path int4km coverage + flagship Qwen3.6-35B -- session
+ *        findings & methods", sec. 8 "FP4 (E2M1) dense matvec" (per-K-block
+ *        e8m0 scale times a fixed 16-value E2M1 grid; per-row 16-entry
+ *        k-means codebook for int4km; y = x W^T at q=1).
+ *   [P3] "coreai-optimization (coreai-opt) reference -- quantization &
+ *        palettization", sections "Quantization" (symmetric, per-block 32),
+ *        "Palettization" (scalar 1-D k-means, 2^n_bits LUT, per-channel
+ *        grouping) and "Theoretical size" (fp16 scales, LUT bytes).
+ *   [P5] "Compression (palettization & quantization)", section "Per-channel
+ *        int8 on a big-vocab LM head: use per-block-32".
+ *
+ * Where the pages leave a step open, the reading taken is stated at the
+ * function.  Every floating-point step is written so that its rounding is
+ * fixed by IEEE-754 (float ops in float, the MSE and the matvec in double,
+ * no contraction: build with -ffp-contract=off, never -ffast-math).
+ *
+ * Parity status: every function here is pinned by tests under
+ * tests/test_oracle_pins.py except oracle_kmeans_int4km's LUT *values*,
+ * which no page fixes (see its comment): "parity unpinned" for those values;
+ * its invariants (exact reconstruction of <=16 distinct values, monotone
+ * SSE, nearest-entry indices) are pinned.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_FLAG_NONFINITE 1u      /* a block/row held Inf or NaN */
+#define ORC_FLAG_SCALE_OVERFLOW 2u /* no clip gave a finite fp16 scale */
+#define ORC_FLAG_BAD_EXPERT 4u     /* gather: expert id outside [0, E) */
+
+#define ORC_FMT_FP4 0
+#define ORC_FMT_INT4 1
+#define ORC_FMT_INT4KM 2
+#define ORC_FMT_INT8 3
+
+/* ------------------------------------------------------------------ */
+/* IEEE binary16 <-> binary32, written from the format definition.     */
+/* ------------------------------------------------------------------ */
+
+/* binary16 bits -> exact float value. */
+static float orc_f16_to_f32(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int ex = (h >> 10) & 0x1F;
+  int man = h & 0x3FF;
+  double v;
+  if (ex == 0x1F) {
+    v = man ? NAN : INFINITY;
+  } else if (ex == 0) {
+    v = ldexp((double)man, -24); /* subnormal: man * 2^-24 */
+  } else {
+    v = ldexp((double)(1024 + man), ex - 25); /* (1 + man/1024) * 2^(ex-15) */
+  }
+  return (float)(sign ? -v : v);
+}
+
+/* float -> binary16 bits, round to nearest, ties to even; overflow -> Inf. */
+static uint16_t orc_f32_to_f16(float f) {
+  uint16_t sign = signbit(f) ? 0x8000 : 0;
+  double a = fabs((double)f);
+  if (isnan(f)) return (uint16_t)(sign | 0x7E00);
+  if (isinf(f)) return (uint16_t)(sign | 0x7C00);
+  if (a >= 65520.0) return (uint16_t)(sign | 0x7C00); /* halfway to 2^16 rounds up */
+  if (a < ldexp(1.0, -14)) {
+    /* subnormal range: value = m * 2^-24, m in [0, 1024] (1024 = min normal) */
+    double m = nearbyint(a * ldexp(1.0, 24)); /* exact scaling, RNE rounding */
+    return (uint16_t)(sign | (uint16_t)m);
+  }
+  int e2;
+  (void)frexp(a, &e2); /* a = fr * 2^e2, fr in [0.5, 1) */
+  int E = e2 - 1;      /* a in [2^E, 2^(E+1)) */
+  double m = nearbyint(ldexp(a, 10 - E)); /* in [1024, 2048] */
+  if (m == 2048.0) {
+    m = 1024.0;
+    E += 1;
+  }
+  if (E > 15) return (uint16_t)(sign | 0x7C00);
+  return (uint16_t)(sign | (uint16_t)((E + 15) << 10) | (uint16_t)(m - 1024.0));
+}
+
+/* Exported for the pin tests (compared against a library float16 cast). */
+uint16_t oracle_f32_to_f16(float f) { return orc_f32_to_f16(f); }
+float oracle_f16_to_f32(uint16_t h) { return orc_f16_to_f32(h); }
+
+/* ------------------------------------------------------------------ */
+/* FP4 E2M1 with an e8m0 scale per 32-block  [P1 sec.1, sec.2; P2 sec.8] */
+/* ------------------------------------------------------------------ */
+
+/* The E2M1 magnitudes, code 0..7: sign-magnitude 4-bit float with 2
+ * exponent bits and 1 mantissa bit (OCP MX E2M1). */
+static const double orc_e2m1_grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* Magnitude code of v >= 0: nearest grid point, ties to the even code
+ * (round-to-nearest-even on the 1-bit mantissa); values above 6 land on 6
+ * (saturation), which the argmin gives by itself. */
+static int orc_e2m1_mag(double v) {
+  int best = 0;
+  double bd = fabs(v - orc_e2m1_grid[0]);
+  for (int c = 1; c < 8; c++) {
+    double d = fabs(v - orc_e2m1_grid[c]);
+    if (d < bd || (d == bd && (c % 2 == 0) && (best % 2 == 1))) {
+      best = c;
+      bd = d;
+    }
+  }
+  return best;
+}
+
+int oracle_e2m1_code(float v) { /* exported for pins: full 4-bit code */
+  int mag = orc_e2m1_mag(fabs((double)v));
+  return (signbit(v) ? 8 : 0) | mag;
+}
+
+/* floor(log2(a)) for finite a > 0, exactly (frexp on the exact double). */
+static int orc_floor_log2(float a) {
+  int e2;
+  (void)frexp((double)a, &e2);
+  return e2 - 1;
+}
+
+/* e8m0 scale byte of a block: scale = 2^(floor(log2(amax)) - 2), the
+ * E2M1 target exponent being 2 [P1 sec.1].  Reading: amax == 0 gives the
+ * smallest scale (byte 0); the exponent is clamped to the e8m0 range
+ * [-127, 127] (byte 255 is NaN in e8m0 and is never produced). */
+int oracle_e8m0_byte(float amax) {
+  int e;
+  if (amax == 0.0f)
+    e = -127;
+  else
+    e = orc_floor_log2(amax) - 2;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e + 127;
+}
+
+/* codes: uint8 [N, K/2], element 2j in the low nibble, 2j+1 in the high
+ * nibble (reading of "2 values per byte", little-endian like 8 codes per
+ * uint32).  scales: uint8 [N, K/32] e8m0 bytes.  A block holding Inf/NaN
+ * is written as all-zero codes with scale byte 0 and raises a flag. */
+int oracle_encode_fp4(const float* W, int64_t N, int64_t K, uint8_t* codes,
+                      uint8_t* scales, uint32_t* flags_out) {
+  if (K % 32 != 0 || N < 0) return -2;
+  uint32_t flags = 0;
+  int64_t nb = K / 32;
+#pragma omp parallel for reduction(| : flags) schedule(static)
+  for (int64_t n = 0; n < N; n++) {
+    for (int64_t b = 0; b < nb; b++) {
+      const float* w = W + n * K + b * 32;
+      uint8_t* cb = codes + n * (K / 2) + b * 16;
+      float amax = 0.0f;
+      int finite = 1;
+      for (int i = 0; i < 32; i++) {
+        if (!isfinite(w[i])) finite = 0;
+        float a = fabsf(w[i]);
+        if (a > amax) amax = a;
+      }
+      if (!finite) {
+        flags |= ORC_FLAG_NONFINITE;
+        memset(cb, 0, 16);
+        scales[n * nb + b] = 0;
+        continue;
+      }
+      int byte = oracle_e8m0_byte(amax);
+      scales[n * nb + b] = (uint8_t)byte;
+      int e = byte - 127;
+      for (int i = 0; i < 32; i += 2) {
+        int c[2];
+        for (int u = 0; u < 2; u++) {
+          double v = ldexp(fabs((double)w[i + u]), -e); /* exact: w * 2^-e */
+          c[u] = (signbit(w[i + u]) ? 8 : 0) | orc_e2m1_mag(v);
+        }
+        cb[i / 2] = (uint8_t)(c[0] | (c[1] << 4));
+      }
+    }
+  }
+  if (flags_out) *flags_out = flags;
+  return 0;
+}
+
+static float orc_fp4_value(int code, int scale_byte) {
+  double v = ldexp(orc_e2m1_grid[code & 7], scale_byte - 127);
+  return (float)((code & 8) ? -v : v);
+}
+
+/* ------------------------------------------------------------------ */
+/* Symmetric int4 / int8, per-block 32, MSE-searched clip             */
+/* [P1 sec.2 "int4 / int8: symmetric-with-clipping, MSE-optimal clip"; */
+/*  P3 "Quantization"; P5 per-block-32 int8 head]                      */
+/* ------------------------------------------------------------------ */
+
+/* For each block and each clip alpha in list order:
+ *   s16  = fp16_RNE( float(alpha * amax) / float(qmax) )   (float ops)
+ *   q_i  = clamp(rint_even(w_i / float(s16)), -qmax, qmax)  (0 if s16 == 0)
+ *   err  = sum_i (double(w_i) - double(q_i) * double(s16))^2, i = 0..31 in order
+ * keep the first alpha with strictly smaller err.  Readings: range is
+ * [-qmax, qmax] with qmax = 7 (int4) or 127 (int8); the scale is fp16 (the
+ * size formula's 2-byte scales) and the codes are computed with the stored
+ * fp16 scale; a candidate whose fp16 scale overflows is skipped, and a block
+ * with no finite candidate is written as zeros with a flag.
+ * int4 storage: nibble = q + 8 (element 2j low nibble).  int8: two's
+ * complement byte.  scales: fp16 bits [N, K/32]. */
+int oracle_encode_int_sym(const float* W, int64_t N, int64_t K, int qmax,
+                          const float* clips, int n_clips, uint8_t* codes,
+                          uint16_t* scales, uint32_t* flags_out) {
+  if (K % 32 != 0 || N < 0 || (qmax != 7 && qmax != 127) || n_clips < 1) return -2;
+  uint32_t flags = 0;
+  int64_t nb = K / 32;
+  int bits = (qmax == 7) ? 4 : 8;
+#pragma omp parallel for reduction(| : flags) schedule(static)
+  for (int64_t n = 0; n < N; n++) {
+    for (int64_t b = 0; b < nb; b++) {
+      const float* w = W + n * K + b * 32;
+      float amax = 0.0f;
+      int finite = 1;
+      for (int i = 0; i < 32; i++) {
+        if (!isfinite(w[i])) finite = 0;
+        float a = fabsf(w[i]);
+        if (a > amax) amax = a;
+      }
+      int best_q[32];
+      uint16_t best_s = 0;
+      int have = 0;
+      double best_err = 0.0;
+      if (finite) {
+        for (int c = 0; c < n_clips; c++) {
+          float t = clips[c] * amax;
+          float sf = t / (float)qmax;
+          uint16_t sh = orc_f32_to_f16(sf);
+          if ((sh & 0x7C00) == 0x7C00) continue; /* fp16 overflow */
+          float s = orc_f16_to_f32(sh);
+          int q[32];
+          double err = 0.0;
+          for (int i = 0; i < 32; i++) {
+            if (s == 0.0f) {
+              q[i] = 0;
+            } else {
+              float r = rintf(w[i] / s);
+              if (r > (float)qmax) r = (float)qmax;
+              if (r < (float)-qmax) r = (float)-qmax;
+              q[i] = (int)r;
+            }
+            double d = (double)w[i] - (double)q[i] * (double)s;
+            err += d * d;
+          }
+          if (!have || err < best_err) {
+            have = 1;
+            best_err = err;
+            best_s = sh;
+            memcpy(best_q, q, sizeof(q));
+          }
+        }
+      }
+      if (!finite) flags |= ORC_FLAG_NONFINITE;
+      if (finite && !have) flags |= ORC_FLAG_SCALE_OVERFLOW;
+      if (!have) {
+        memset(best_q, 0, sizeof(best_q));
+        best_s = 0;
+      }
+      scales[n * nb + b] = best_s;
+      if (bits == 4) {
+        uint8_t* cb = codes + n * (K / 2) + b * 16;
+        for (int i = 0; i < 32; i += 2)
+          cb[i / 2] = (uint8_t)((best_q[i] + 8) | ((best_q[i + 1] + 8) << 4));
+      } else {
+        int8_t* cb = (int8_t*)codes + n * K + b * 32;
+        for (int i = 0; i < 32; i++) cb[i] = (int8_t)best_q[i];
+      }
+    }
+  }
+  if (flags_out) *flags_out = flags;
+  return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* int4km: per-row 16-entry LUT by scalar 1-D k-means                 */
+/* [P3 "Palettization": scalar k-means, 2^n_bits centroids, per-channel */
+/*  grouping; P2 sec.8: per-output-row 16-entry codebook]             */
+/* ------------------------------------------------------------------ */
+
+static int orc_cmp_float(const void* a, const void* b) {
+  float x = *(const float*)a, y = *(const float*)b;
+  return (x > y) - (x < y);
+}
+
+/* Nearest of the 16 centres to v, distance |v - c| in double, ties to the
+ * lower index. */
+static int orc_nearest16(const double* c, double v) {
+  int best = 0;
+  double bd = fabs(v - c[0]);
+  for (int k = 1; k < 16; k++) {
+    double d = fabs(v - c[k]);
+    if (d < bd) {
+      bd = d;
+      best = k;
+    }
+  }
+  return best;
+}
+
+/* Per row (n = K weights), readings where no page fixes the details:
+ *  1. sort the row ascending;
+ *  2. centre k starts at sorted[floor((2k+1) n / 32)], the (k+1/2)/16
+ *     quantile without interpolation;
+ *  3. `iters` Lloyd steps: assign each weight to the nearest centre (double
+ *     distance, ties to the lower index); each non-empty centre becomes
+ *     float(double sum of its members, added in ascending value order /
+ *     count); an empty centre keeps its value;
+ *  4. LUT = fp16_RNE(centres);
+ *  5. indices = nearest LUT entry (double distance, ties to lower index).
+ * idx: uint8 [N, K/2] (element 2j low nibble); lut: fp16 bits [N, 16].
+ * A row holding Inf/NaN is written as zeros and raises a flag.
+ * sse_trace (optional, [N, iters+1]): the SSE against the centres before
+ * each step and after the last, for the monotonicity pin. */
+int oracle_kmeans_int4km(const float* W, int64_t N, int64_t K, int iters,
+                         uint16_t* lut, uint8_t* idx, double* sse_trace,
+                         uint32_t* flags_out) {
+  if (K % 32 != 0 || N < 0 || iters < 0) return -2;
+  uint32_t flags = 0;
+#pragma omp parallel for reduction(| : flags) schedule(dynamic, 64)
+  for (int64_t n = 0; n < N; n++) {
+    const float* w = W + n * K;
+    int finite = 1;
+    for (int64_t i = 0; i < K; i++)
+      if (!isfinite(w[i])) finite = 0;
+    if (!finite) {
+      flags |= ORC_FLAG_NONFINITE;
+      memset(lut + n * 16, 0, 32);
+      memset(idx + n * (K / 2), 0, (size_t)(K / 2));
+      if (sse_trace)
+        for (int t = 0; t <= iters; t++) sse_trace[n * (iters + 1) + t] = NAN;
+      continue;
+    }
+    float* s = (float*)malloc((size_t)K * sizeof(float));
+    memcpy(s, w, (size_t)K * sizeof(float));
+    qsort(s, (size_t)K, sizeof(float), orc_cmp_float);
+    double c[16];
+    for (int k = 0; k < 16; k++) c[k] = (double)s[((2 * k + 1) * K) / 32];
+    for (int it = 0; it <= iters; it++) {
+      double sum[16] = {0}, sse = 0.0;
+      int64_t cnt[16] = {0};
+      for (int64_t i = 0; i < K; i++) {
+        double v = (double)s[i];
+        int j = orc_nearest16(c, v);
+        double d = v - c[j];
+        sse += d * d;
+        sum[j] += v;
+        cnt[j]++;
+      }
+      if (sse_trace) sse_trace[n * (iters + 1) + it] = sse;
+      if (it == iters) break;
+      for (int k = 0; k < 16; k++)
+        if (cnt[k] > 0) c[k] = (double)(float)(sum[k] / (double)cnt[k]);
+    }
+    free(s);
+    double cl[16];
+    for (int k = 0; k < 16; k++) {
+      uint16_t h = orc_f32_to_f16((float)c[k]);
+      lut[n * 16 + k] = h;
+      cl[k] = (double)orc_f16_to_f32(h);
+    }
+    uint8_t* ib = idx + n * (K / 2);
+    for (int64_t i = 0; i < K; i += 2) {
+      int a = orc_nearest16(cl, (double)w[i]);
+      int b = orc_nearest16(cl, (double)w[i + 1]);
+      ib[i / 2] = (uint8_t)(a | (b << 4));
+    }
+  }
+  if (flags_out) *flags_out = flags;
+  return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Dequantization (exact in float) and the fp64 matvec                */
+/* ------------------------------------------------------------------ */
+
+/* Dequantized weight (row n, column k) of one format.  aux is the scale
+ * plane (fp4: uint8 [N,K/32]; int4/int8: fp16 bits [N,K/32]) or the LUT
+ * (int4km: fp16 bits [N,16]). */
+static float orc_wdq(int fmt, const void* codes, const void* aux, int64_t K,
+                     int64_t n, int64_t k) {
+  int64_t nb = K / 32;
+  switch (fmt) {
+    case ORC_FMT_FP4: {
+      uint8_t byte = ((const uint8_t*)codes)[n * (K / 2) + k / 2];
+      int code = (k % 2) ? (byte >> 4) : (byte & 15);
+      return orc_fp4_value(code, ((const uint8_t*)aux)[n * nb + k / 32]);
+    }
+    case ORC_FMT_INT4: {
+      uint8_t byte = ((const uint8_t*)codes)[n * (K / 2) + k / 2];
+      int q = ((k % 2) ? (byte >> 4) : (byte & 15)) - 8;
+      float s = orc_f16_to_f32(((const uint16_t*)aux)[n * nb + k / 32]);
+      return (float)q * s;
+    }
+    case ORC_FMT_INT4KM: {
+      uint8_t byte = ((const uint8_t*)codes)[n * (K / 2) + k / 2];
+      int j = (k % 2) ? (byte >> 4) : (byte & 15);
+      return orc_f16_to_f32(((const uint16_t*)aux)[n * 16 + j]);
+    }
+    case ORC_FMT_INT8: {
+      int q = ((const int8_t*)codes)[n * K + k];
+      float s = orc_f16_to_f32(((const uint16_t*)aux)[n * nb + k / 32]);
+      return (float)q * s;
+    }
+  }
+  return NAN;
+}
+
+int oracle_dequant(int fmt, const void* codes, const void* aux, int64_t N,
+                   int64_t K, float* Wdq) {
+  if (K % 32 != 0 || N < 0 || fmt < 0 || fmt > 3) return -2;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; n++)
+    for (int64_t k = 0; k < K; k++) Wdq[n * K + k] = orc_wdq(fmt, codes, aux, K, n, k);
+  return 0;
+}
+
+/* r[b, i] = sum_k double(x[b,k]) * double(Wdq[rows[i], k]), k ascending,
+ * for the listed rows (all rows when rows == NULL, i = n).  x: fp16 bits
+ * [B, K]; r: double [B, nrows].  [P2 sec.8: y = x W^T at q=1; the batch
+ * rows are independent tokens.] */
+int oracle_matvec_rows(int fmt, const void* codes, const void* aux,
+                       const uint16_t* x, int B, int64_t N, int64_t K,
+                       const int64_t* rows, int64_t nrows, double* r) {
+  if (K % 32 != 0 || N < 0 || B < 1 || fmt < 0 || fmt > 3) return -2;
+  int64_t R = rows ? nrows : N;
+  double* xd = (double*)malloc((size_t)(B * K) * sizeof(double));
+  for (int64_t i = 0; i < (int64_t)B * K; i++) xd[i] = (double)orc_f16_to_f32(x[i]);
+  int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+  for (int64_t i = 0; i < R; i++) {
+    int64_t n = rows ? rows[i] : i;
+    if (n < 0 || n >= N) {
+      bad = 1;
+      continue;
+    }
+    for (int b = 0; b < B; b++) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; k++) acc += xd[b * K + k] * (double)orc_wdq(fmt, codes, aux, K, n, k);
+      r[(int64_t)b * R + i] = acc;
+    }
+  }
+  free(xd);
+  return bad ? -1 : 0;
+}
+
+/* Routed-expert gather matvec [P1 sec.1 gather_qmm over the selected
+ * experts only; P2 sec.3]: for token b and slot j, e = ids[b*topk + j];
+ * y[b, j, :] = W_e x_(b) (x_per_slot == 0, x [B, K]) or W_e x_(b,j)
+ * (x_per_slot == 1, x [B, topk, K]).  Stacks are the per-expert arrays laid
+ * out one after another ([E, N, ...]).  An id outside [0, E) gives a zero
+ * output row and a flag.  y: double [B, topk, N]. */
+int oracle_gather_matvec(int fmt, const void* codes, const void* aux, int E,
+                         int64_t N, int64_t K, const int32_t* ids, int B,
+                         int topk, const uint16_t* x, int x_per_slot,
+                         double* y, uint32_t* flags_out) {
+  if (K % 32 != 0 || N < 0 || B < 1 || topk < 1 || fmt < 0 || fmt > 3) return -2;
+  int64_t code_bytes = (fmt == ORC_FMT_INT8) ? N * K : N * (K / 2);
+  int64_t aux_bytes = (fmt == ORC_FMT_FP4) ? N * (K / 32)
+                      : (fmt == ORC_FMT_INT4KM) ? N * 16 * 2
+                                                : N * (K / 32) * 2;
+  uint32_t flags = 0;
+  for (int b = 0; b < B; b++) {
+    for (int j = 0; j < topk; j++) {
+      int e = ids[b * topk + j];
+      double* yo = y + ((int64_t)b * topk + j) * N;
+      if (e < 0 || e >= E) {
+        flags |= ORC_FLAG_BAD_EXPERT;
+        for (int64_t n = 0; n < N; n++) yo[n] = 0.0;
+        continue;
+      }
+      const uint8_t* ce = (const uint8_t*)codes + (int64_t)e * code_bytes;
+      const uint8_t* ae = (const uint8_t*)aux + (int64_t)e * aux_bytes;
+      const uint16_t* xb = x + (x_per_slot ? ((int64_t)b * topk + j) * K : (int64_t)b * K);
+      oracle_matvec_rows(fmt, ce, ae, xb, 1, N, K, NULL, N, yo);
+    }
+  }
+  if (flags_out) *flags_out = flags;
+  return 0;
+}
+
+/* Number of worker threads the OpenMP loops use (1 when built without). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  extern void omp_set_num_threads(int);
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}

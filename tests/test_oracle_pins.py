@@ -1,0 +1,444 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Nothing here re-types the oracle's formulas to compare them with themselves:
+each check is a library routine (numpy's float16 cast, ml_dtypes' E2M1 and
+e8m0 casts, numpy float64 matmul, scikit-learn's Lloyd k-means), a closed
+form written out by hand (tests/golden), an exhaustive/brute-force search,
+an invariant, or a figure printed by the pages (soft band).
+"""
+import math
+import os
+
+import ml_dtypes
+import numpy as np
+import pytest
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(12345)
+
+
+def _rows(name):
+    out = []
+    for line in open(os.path.join(GOLD, name)):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            out.append(line.split())
+    return out
+
+
+def _f(tok):
+    return float.fromhex(tok) if "0x" in tok else float(tok)
+
+
+# --------------------------------------------------------------------------
+# IEEE binary16 conversion (library: numpy's float16 cast is RNE)
+# --------------------------------------------------------------------------
+
+def test_f16_from_f32_matches_numpy(orc):
+    specials = [0.0, -0.0, 1.0, 65504.0, 65519.99, 65520.0, 65536.0, 1e9, 2.0 ** -14, 2.0 ** -24,
+                2.0 ** -25, 1.5 * 2.0 ** -25, 2.0 ** -26, 3.0 * 2.0 ** -26, 0.1, 1.0 / 3, -2.5e-7,
+                1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 2048.0 + 1.0, 2048.0 + 3.0, float("inf")]
+    vals = np.array(specials + list(RNG.standard_normal(4000) * 10.0 ** RNG.uniform(-9, 5, 4000)), np.float32)
+    # ties: values exactly halfway between fp16 neighbours
+    ties = (np.arange(1, 2000, dtype=np.float32) + np.float32(0.5)) * np.float32(2.0 ** -10)
+    vals = np.concatenate([vals, ties, -ties])
+    ref = vals.astype(np.float16).view(np.uint16)
+    got = np.array([orc.f32_to_f16_bits(float(v)) for v in vals], np.uint16)
+    bad = np.nonzero(ref != got)[0]
+    assert bad.size == 0, [(float(vals[i]), hex(ref[i]), hex(got[i])) for i in bad[:5]]
+
+
+def test_f16_to_f32_all_patterns(orc):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float32)
+    got = np.array([orc.f16_bits_to_f32(int(b)) for b in bits], np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(ref[~nan].view(np.uint32), got[~nan].view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# FP4 E2M1 + e8m0 (library: ml_dtypes float4_e2m1fn / float8_e8m0fnu)
+# --------------------------------------------------------------------------
+
+def test_e2m1_value_set_golden():
+    rows = _rows("e2m1_values.txt")
+    codes = np.array([int(r[0]) for r in rows], np.uint8)
+    vals = np.array([_f(r[1]) for r in rows], np.float32)
+    lib_vals = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    assert np.array_equal(lib_vals.view(np.uint32), vals.view(np.uint32))
+
+
+def test_e2m1_rounding_matches_library_near_every_threshold(orc):
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    cuts = [(a + b) / 2 for a, b in zip(grid, grid[1:])] + grid + [7.0, 8.0, 100.0]
+    vals = []
+    for c in cuts:
+        v = np.float32(c)
+        lo, hi = v, v
+        vals.append(v)
+        for _ in range(4):  # 4 ulps on each side of every tie and grid point
+            lo = np.nextafter(lo, np.float32(-1), dtype=np.float32)
+            hi = np.nextafter(hi, np.float32(100), dtype=np.float32)
+            vals += [lo, hi]
+    vals += list(RNG.uniform(0, 9, 3000).astype(np.float32))
+    vals = np.array(vals, np.float32)
+    vals = np.concatenate([vals, -vals, np.array([0.0, -0.0, 1e-30, -1e-30], np.float32)])
+    ref = vals.astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    got = np.array([orc.e2m1_code(float(v)) for v in vals], np.uint8)
+    bad = np.nonzero(ref != got)[0]
+    assert bad.size == 0, [(float(vals[i]), int(ref[i]), int(got[i])) for i in bad[:5]]
+
+
+def test_e8m0_closed_form_golden(orc):
+    for amax_s, byte_s, *_ in _rows("e8m0_scale_cases.txt"):
+        amax = float(np.float32(_f(amax_s)))
+        assert orc.e8m0_byte(amax) == int(byte_s), amax_s
+
+
+def test_e8m0_scale_is_library_e8m0_of_the_power_of_two(orc):
+    # the byte is the e8m0 encoding (per ml_dtypes) of 2^(floor(log2 amax) - 2)
+    amax = (np.abs(RNG.standard_normal(3000)) * 10.0 ** RNG.uniform(-30, 30, 3000)).astype(np.float32)
+    for a in amax:
+        b = orc.e8m0_byte(float(a))
+        ref = np.array([2.0 ** (b - 127)], np.float32).astype(ml_dtypes.float8_e8m0fnu).view(np.uint8)[0]
+        assert ref == b
+        # the block maximum lands in the top binade of E2M1: amax / scale in [4, 8)
+        r = float(a) / 2.0 ** (b - 127)
+        assert 4.0 <= r < 8.0, (a, b)
+
+
+def _fp4_lib_codes(W, scales):
+    """E2M1 codes of W / scale computed by the ml_dtypes cast (library)."""
+    s = np.repeat(np.ldexp(1.0, scales.astype(np.int32) - 127), 32, axis=1)
+    v = (W.astype(np.float64) / s).astype(np.float32)  # exact: power-of-two scaling
+    c = v.astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+
+
+def test_encode_fp4_matches_library_cast(orc):
+    W = (RNG.standard_normal((64, 256)) * 0.02).astype(np.float32)
+    W[:, [3, 100]] *= 20.0
+    W[5, :32] = 0.0
+    W[6, 32:64] = -1e-40  # subnormal block
+    codes, scales, flags = orc.encode_fp4(W)
+    assert flags == 0
+    assert np.array_equal(codes, _fp4_lib_codes(W, scales))
+    # element 2j in the low nibble: pin the packing with a one-element block
+    Z = np.zeros((1, 32), np.float32)
+    Z[0, 1] = 6.0
+    c, s, _ = orc.encode_fp4(Z)
+    assert s[0, 0] == 127 and c[0, 0] == 0x70 and not c[0, 1:].any()
+
+
+def test_fp4_round_trip_exact_on_grid(orc):
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], np.float32)
+    N, K = 200, 128
+    mags = grid[RNG.integers(0, 8, (N, K))]
+    mags.reshape(N, -1, 32)[:, :, 0] = RNG.choice([4.0, 6.0], (N, K // 32))  # block max in [4, 6]
+    sign = RNG.choice([-1.0, 1.0], (N, K)).astype(np.float32)
+    e = RNG.integers(-20, 20, (N, K // 32))
+    W = (sign * mags * np.repeat(np.ldexp(1.0, e), 32, axis=1)).astype(np.float32)
+    codes, scales, _ = orc.encode_fp4(W)
+    assert np.array_equal(scales.astype(np.int64) - 127, e)
+    D = orc.dequant(orc.FMT_FP4, codes, scales, N, K)
+    assert np.array_equal(D.view(np.uint32), W.view(np.uint32))  # bit-exact incl. signed zeros
+
+
+def test_fp4_dequant_matches_library_decode_and_error_bound(orc):
+    W = (RNG.standard_normal((128, 512)) * 0.02).astype(np.float32)
+    W[:, 7] *= 20
+    codes, scales, _ = orc.encode_fp4(W)
+    D = orc.dequant(orc.FMT_FP4, codes, scales, *W.shape)
+    c = np.empty(W.shape, np.uint8)
+    c[:, 0::2], c[:, 1::2] = codes & 15, codes >> 4
+    s = np.repeat(np.ldexp(1.0, scales.astype(np.int32) - 127), 32, axis=1)
+    ref = (c.view(ml_dtypes.float4_e2m1fn).astype(np.float64) * s).astype(np.float32)
+    assert np.array_equal(D.view(np.uint32), ref.view(np.uint32))
+    # |w - dq| <= half the local grid gap (x scale); above 6 saturation bounds it by 2 x scale
+    v = np.abs(W.astype(np.float64)) / s
+    gap = np.where(v <= 2, 0.5, np.where(v <= 4, 1.0, 2.0))
+    bound = np.where(v <= 6, gap / 2, 2.0) * s
+    assert np.all(np.abs(W.astype(np.float64) - D) <= bound)
+
+
+def test_fp4_negative_values_rounding_to_zero_keep_the_sign(orc):
+    W = np.zeros((1, 32), np.float32)
+    W[0, 0] = 4.0
+    W[0, 1] = -0.1  # |v| = 0.1 < 0.25 -> magnitude 0 with the sign bit set
+    codes, scales, _ = orc.encode_fp4(W)
+    assert (codes[0, 0] >> 4) == 8
+    D = orc.dequant(orc.FMT_FP4, codes, scales, 1, 32)
+    assert math.copysign(1.0, float(D[0, 1])) == -1.0 and D[0, 1] == 0.0
+
+
+def test_fp4_nonfinite_block_flags_and_zeroes(orc):
+    W = (RNG.standard_normal((2, 64)) * 0.02).astype(np.float32)
+    W[1, 40] = np.nan
+    codes, scales, flags = orc.encode_fp4(W)
+    assert flags & orc.FLAG_NONFINITE
+    assert not codes[1, 16:32].any() and scales[1, 1] == 0
+    assert np.array_equal(codes[:1], orc.encode_fp4(W[:1])[0])
+
+
+# --------------------------------------------------------------------------
+# symmetric int4 / int8 with MSE clip search
+# --------------------------------------------------------------------------
+
+def _unpack_int(codes, bits, K):
+    if bits == 4:
+        q = np.empty((codes.shape[0], K), np.int64)
+        q[:, 0::2], q[:, 1::2] = (codes & 15).astype(np.int64) - 8, (codes >> 4).astype(np.int64) - 8
+        return q
+    return codes.astype(np.int64)
+
+
+def _brute_q(w, s, qmax):
+    """Exhaustive search of the integer in [-qmax, qmax] nearest to the float32
+    quotient w / s, ties to the even integer."""
+    if s == 0:
+        return np.zeros_like(w, dtype=np.int64)
+    quot = (w.astype(np.float32) / np.float32(s)).astype(np.float64)
+    cand = np.arange(-qmax, qmax + 1)
+    d = np.abs(quot[:, None] - cand[None, :])
+    best = d.min(axis=1, keepdims=True)
+    ok = d == best
+    # among ties prefer the even integer
+    pick = np.where(ok & (cand[None, :] % 2 == 0), 1, 0) + ok.astype(int)
+    return cand[np.argmax(pick, axis=1)]
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_int_encode_brute_force(orc, bits):
+    qmax = 7 if bits == 4 else 127
+    clips = orc.INT4_CLIPS if bits == 4 else np.array([1.0, 0.9, 0.8, 0.7], np.float32)
+    W = (RNG.standard_normal((24, 128)) * 0.02).astype(np.float32)
+    W[:, 9] *= 20.0
+    W[3, :32] = 0.0
+    W[4, 32:64] = 1e-9  # tiny block: fp16 scale underflows toward subnormal / zero
+    enc = orc.encode_int4 if bits == 4 else orc.encode_int8
+    codes, scales, flags = enc(W, clips)
+    assert flags == 0
+    q = _unpack_int(codes, bits, W.shape[1])
+    for n in range(W.shape[0]):
+        for b in range(W.shape[1] // 32):
+            w = W[n, b * 32:(b + 1) * 32]
+            s = float(scales[n, b])
+            assert np.array_equal(q[n, b * 32:(b + 1) * 32], _brute_q(w, s, qmax)), (n, b)
+            amax = np.float32(np.max(np.abs(w)))
+            errs, svals = [], []
+            for a in clips:
+                sc = np.float16(np.float32(np.float32(a) * amax) / np.float32(qmax))  # library RNE cast
+                qq = _brute_q(w, float(sc), qmax)
+                errs.append(float(np.sum((w.astype(np.float64) - qq * float(sc)) ** 2)))
+                svals.append(sc)
+            chosen = float(np.sum((w.astype(np.float64) - q[n, b * 32:(b + 1) * 32] * s) ** 2))
+            assert chosen <= min(errs) * (1 + 1e-12) + 1e-300
+            assert any(np.float16(s) == sv for sv in svals)
+            # the first clip reaching the minimum is kept
+            first = int(np.argmin(errs))
+            if errs.count(errs[first]) == 1 or min(errs) == 0:
+                assert np.float16(s) == svals[first] or min(errs) == 0
+
+
+def test_int_special_blocks(orc):
+    W = np.zeros((3, 32), np.float32)
+    W[0, 5] = 0.7  # single non-zero element, alpha = 1: q = qmax, s = fp16(0.7/7)
+    W[2, :] = 65504.0 * 8  # scale 0.1*... overflow for int4 -> no finite clip
+    codes, scales, flags = orc.encode_int4(W, np.array([1.0], np.float32))
+    assert flags & orc.FLAG_SCALE_OVERFLOW
+    q = _unpack_int(codes, 4, 32)
+    assert q[0, 5] == 7 and np.count_nonzero(q[0]) == 1
+    assert scales[0, 0] == np.float16(np.float32(0.7) / np.float32(7))
+    assert not q[1].any() and scales[1, 0] == 0  # all-zero block
+    assert not q[2].any() and scales[2, 0] == 0
+    D = orc.dequant(orc.FMT_INT4, codes, scales, 3, 32)
+    assert D[0, 5] == np.float32(7) * np.float32(scales[0, 0])
+
+
+def test_int_dequant_matches_numpy(orc):
+    W = (RNG.standard_normal((16, 256)) * 0.02).astype(np.float32)
+    for bits, enc, fmt in ((4, orc.encode_int4, orc.FMT_INT4), (8, orc.encode_int8, orc.FMT_INT8)):
+        codes, scales, _ = enc(W)
+        D = orc.dequant(fmt, codes, scales, *W.shape)
+        ref = (_unpack_int(codes, bits, 256).astype(np.float32)
+               * np.repeat(scales.astype(np.float32), 32, axis=1))
+        assert np.array_equal(D, ref)
+
+
+def test_relerr_ordering_and_page_band(orc):
+    """fp4 error > int4-clip error > int8 error on outlier-bearing weights
+    (the pages' quality-gate ordering); the levels sit near the printed ones."""
+    gold = {r[0]: float(r[1]) for r in _rows("weight_relerr.txt")}
+    W = (RNG.standard_normal((512, 1024)) * 0.02).astype(np.float32)
+    W[:, RNG.permutation(1024)[:8]] *= 20.0
+    N, K = W.shape
+    err = {}
+    c, s, _ = orc.encode_fp4(W)
+    err["fp4"] = orc.dequant(orc.FMT_FP4, c, s, N, K)
+    c, s, _ = orc.encode_int4(W)
+    err["int4_clip"] = orc.dequant(orc.FMT_INT4, c, s, N, K)
+    c, s, _ = orc.encode_int8(W)
+    err["int8"] = orc.dequant(orc.FMT_INT8, c, s, N, K)
+    rel = {k: float(np.linalg.norm(W - v) / np.linalg.norm(W)) for k, v in err.items()}
+    assert rel["fp4"] > rel["int4_clip"] > rel["int8"]
+    W0 = (RNG.standard_normal((512, 1024)) * 0.02).astype(np.float32)  # no outliers
+    for name, fmt, enc in (("int8", orc.FMT_INT8, orc.encode_int8), ("int4_clip", orc.FMT_INT4, orc.encode_int4),
+                           ("fp4", orc.FMT_FP4, orc.encode_fp4)):
+        out = enc(W0)
+        r = float(np.linalg.norm(W0 - orc.dequant(fmt, out[0], out[1], 512, 1024)) / np.linalg.norm(W0))
+        assert 0.75 * gold[name] < r < 1.35 * gold[name], (name, r)
+
+
+# --------------------------------------------------------------------------
+# int4km k-means (LUT values: parity unpinned; invariants pinned)
+# --------------------------------------------------------------------------
+
+def test_kmeans_exact_on_few_distinct_values(orc):
+    """A row of <= 16 fp16-representable values, each occurring at least
+    n/16 times, is a fixed point of Lloyd from the quantile start (every
+    value is some starting centre: a run of >= n/16 equal sorted values holds
+    a quantile position), so it reconstructs exactly."""
+    N, K = 32, 256
+    W = np.zeros((N, K), np.float32)
+    for n in range(N):
+        nd = int(RNG.integers(1, 17))
+        vals = np.unique(np.float16(RNG.standard_normal(nd) * 0.05)).astype(np.float32)
+        nd = len(vals)
+        counts = np.full(nd, K // 16)
+        counts += np.bincount(RNG.integers(0, nd, K - counts.sum()), minlength=nd)
+        W[n] = RNG.permutation(np.repeat(vals, counts))
+    lut, idx, flags = orc.kmeans_int4km(W)
+    assert flags == 0
+    D = orc.dequant(orc.FMT_INT4KM, idx, lut, N, K)
+    assert np.array_equal(D, W)
+
+
+def test_kmeans_sse_monotone_and_nearest_indices(orc):
+    W = (RNG.standard_normal((64, 512)) * 0.02).astype(np.float32)
+    W[:, 3] *= 20
+    lut, idx, flags, sse = orc.kmeans_int4km(W, want_sse=True)
+    assert flags == 0
+    assert np.all(np.diff(sse, axis=1) <= 1e-18)
+    L = lut.astype(np.float64)
+    d = np.abs(W.astype(np.float64)[:, :, None] - L[:, None, :])
+    nearest = np.argmin(d, axis=2)  # argmin returns the lowest index on ties
+    got = np.empty_like(nearest)
+    got[:, 0::2], got[:, 1::2] = idx & 15, idx >> 4
+    assert np.array_equal(got, nearest)
+    assert np.all(np.diff(L, axis=1) >= 0)  # centres stay ordered on these rows
+
+
+def test_kmeans_matches_sklearn_lloyd(orc):
+    """Same quantile start, 20 Lloyd steps: scikit-learn's KMeans (float64
+    centres) lands within fp16 rounding of the oracle's LUT on almost every
+    row; the oracle rounds centres to float each step, so rare rows may take a
+    different tie path."""
+    from sklearn.cluster import KMeans
+    W = (RNG.standard_normal((40, 512)) * 0.02).astype(np.float32)
+    lut, _, _ = orc.kmeans_int4km(W)
+    agree = 0
+    for n in range(W.shape[0]):
+        s = np.sort(W[n])
+        init = s[[((2 * k + 1) * 512) // 32 for k in range(16)]].astype(np.float64)[:, None]
+        km = KMeans(16, init=init, n_init=1, max_iter=20, tol=0.0, algorithm="lloyd")
+        km.fit(W[n].astype(np.float64)[:, None])
+        ref = np.sort(km.cluster_centers_[:, 0]).astype(np.float16)
+        if np.array_equal(ref, lut[n]):
+            agree += 1
+    assert agree >= 0.9 * W.shape[0], agree
+
+
+def test_kmeans_quantile_start(orc):
+    W = (RNG.standard_normal((8, 256)) * 0.02).astype(np.float32)
+    lut, _, _ = orc.kmeans_int4km(W, iters=0)
+    for n in range(8):
+        s = np.sort(W[n])
+        assert np.array_equal(lut[n], s[[((2 * k + 1) * 256) // 32 for k in range(16)]].astype(np.float16))
+
+
+# --------------------------------------------------------------------------
+# matvec and gather
+# --------------------------------------------------------------------------
+
+def _encode_all(orc, W):
+    N, K = W.shape
+    out = {}
+    c, s, _ = orc.encode_fp4(W)
+    out[orc.FMT_FP4] = (c, s)
+    c, s, _ = orc.encode_int4(W)
+    out[orc.FMT_INT4] = (c, s)
+    lut, idx, _ = orc.kmeans_int4km(W)
+    out[orc.FMT_INT4KM] = (idx, lut)
+    c, s, _ = orc.encode_int8(W)
+    out[orc.FMT_INT8] = (c, s)
+    return out
+
+
+def test_matvec_one_hot_is_a_column_bit_exact(orc):
+    N, K = 48, 192
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    for fmt, (c, a) in _encode_all(orc, W).items():
+        D = orc.dequant(fmt, c, a, N, K)
+        ks = [0, 1, 31, 32, 33, 100, K - 1]
+        x = np.zeros((len(ks), K), np.float16)
+        x[np.arange(len(ks)), ks] = 1.0
+        r = orc.matvec(fmt, c, a, x, N, K)
+        for i, k in enumerate(ks):
+            assert np.array_equal(r[i], D[:, k].astype(np.float64)), (fmt, k)
+
+
+def test_matvec_matches_numpy_and_integer_sums(orc):
+    N, K = 64, 256
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    x = RNG.standard_normal((3, K)).astype(np.float16)
+    for fmt, (c, a) in _encode_all(orc, W).items():
+        D = orc.dequant(fmt, c, a, N, K).astype(np.float64)
+        r = orc.matvec(fmt, c, a, x, N, K)
+        ref = x.astype(np.float64) @ D.T
+        assert np.allclose(r, ref, rtol=1e-12, atol=1e-15)
+        rows = np.array([N - 1, 0, 17])
+        assert np.array_equal(orc.matvec(fmt, c, a, x, N, K, rows=rows), r[:, rows])
+    # integer-valued weights (fp4 grid x 2^1), all-ones x: exact integer sums
+    Wi = (RNG.integers(-3, 4, (N, K)) * 2).astype(np.float32)
+    Wi[:, ::32] = 12.0
+    c, s, _ = orc.encode_fp4(Wi)
+    r = orc.matvec(orc.FMT_FP4, c, s, np.ones((1, K), np.float16), N, K)
+    assert np.array_equal(r[0], Wi.sum(axis=1).astype(np.float64))
+
+
+def test_gather_is_dense_matvec_per_slot(orc):
+    E, N, K, B, topk = 6, 32, 128, 3, 2
+    Ws = (RNG.standard_normal((E, N, K)) * 0.02).astype(np.float32)
+    enc = [_encode_all(orc, Ws[e]) for e in range(E)]
+    ids = np.array([[0, 5], [2, 2], [7, -1]], np.int32)  # duplicate, then two bad ids
+    for x_per_slot in (0, 1):
+        x = RNG.standard_normal((B, topk, K) if x_per_slot else (B, K)).astype(np.float16)
+        for fmt in enc[0]:
+            cs = np.stack([enc[e][fmt][0] for e in range(E)])
+            aus = np.stack([enc[e][fmt][1] for e in range(E)])
+            y, flags = orc.gather_matvec(fmt, cs, aus, E, N, K, ids, x, x_per_slot)
+            assert flags & orc.FLAG_BAD_EXPERT
+            for b in range(B):
+                for j in range(topk):
+                    e = ids[b, j]
+                    if 0 <= e < E:
+                        xb = x[b, j] if x_per_slot else x[b]
+                        ref = orc.matvec(fmt, cs[e], aus[e], xb[None], N, K)[0]
+                        assert np.array_equal(y[b, j], ref)
+                    else:
+                        assert not y[b, j].any()
+
+
+def test_fp4_cos_vs_fp16_page_band(orc):
+    """cos(fp4 output, fp16-weight output) at the pages' three decode shapes."""
+    for name, K, N, cos_ref in _rows("fp4_cos_vs_fp16.txt"):
+        K, N, cos_ref = int(K), int(N), float(cos_ref)
+        n = min(N, 4096)  # a row sample of the big head: cos is a per-output statistic
+        W = (RNG.standard_normal((n, K)) * 0.02).astype(np.float32)
+        x = RNG.standard_normal((1, K)).astype(np.float16)
+        c, s, _ = orc.encode_fp4(W)
+        y4 = orc.matvec(orc.FMT_FP4, c, s, x, n, K)[0]
+        y16 = x.astype(np.float64) @ W.astype(np.float16).astype(np.float64).T
+        cos = float(y4 @ y16[0] / (np.linalg.norm(y4) * np.linalg.norm(y16)))
+        assert abs(cos - cos_ref) < 0.003, (name, cos)

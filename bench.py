@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-only block-quantized lm_head matvec on B200.
+
+Workload: the 248320 x 2048 lm_head at batch 1 (one decode token), one fused
+dequant-matvec per weight format per step: fp4 (E2M1 + e8m0), int4 (symmetric,
+MSE clip), int4km (per-row 16-entry palette), int8 (symmetric).  Weights are
+seeded synthetic N(0, 0.02) with two outlier input columns x20, encoded on the
+GPU by the library's own encoders (int4km: random per-row palettes of the same
+shape, as no GPU palette fit exists yet); activations N(0, 1) fp16.
+
+Metric: effective weight GB/s = algorithmic bytes (codes + scales/palette +
+x + y) / kernel time, and us per matvec.  Every input (~1.1 GB per step in
+total) is larger than L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) each rank runs an independent replica on its own GPU
+(the op has no cross-GPU exchange); `value` sums the ranks' bytes over the
+slowest rank's time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective weight GB/s (% of HBM peak) & us per 248320x2048 lm_head matvec"
+N_HEAD, K_HEAD = 248320, 2048
+FORMATS = ("fp4", "int4", "int4km", "int8")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def algorithmic_bytes(fmt: str, N: int, K: int, B: int) -> int:
+    """Bytes a matvec must move: packed codes + block scales (or palette) +
+    activations (fp16) + outputs (fp32)."""
+    codes = N * K // 2 if fmt != "int8" else N * K
+    aux = {"fp4": N * (K // 32), "int4": N * (K // 32) * 2, "int8": N * (K // 32) * 2, "int4km": N * 16 * 2}[fmt]
+    return codes + aux + B * K * 2 + B * N * 4
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_digest() -> str:
+    d = hashlib.sha256()
+    src = os.path.join(ROOT, "weight_only_quantized_qmv_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(src, name), "rb") as f:
+                d.update(name.encode() + f.read())
+    return d.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_fmt: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "qmv_matvec_lm_head_248320x2048_b1.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m = re.search(r"csrc_sha256_16:\s*([0-9a-f]+)", txt)
+    if not m or m.group(1) != csrc_digest():
+        return None
+    m = re.search(rf"dram_bytes_per_launch\[{kernel_fmt}\]:\s*([0-9]+)", txt)
+    return int(m.group(1)) if m else None
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons while the
+    timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="qmv_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_index)], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4], parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[4]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- workload
+
+def build_workload(device, formats=FORMATS):
+    import torch
+    import weight_only_quantized_qmv_b200 as q
+    from weight_only_quantized_qmv_b200 import synth
+    g = synth.generator(0, device)
+    W, _ = synth.weights(N_HEAD, K_HEAD, g, n_outlier_cols=2)
+    x = synth.activations(1, K_HEAD, g)
+    lut, idx = synth.palette_tables(N_HEAD, K_HEAD, g)
+    enc_ms = {}
+    ops = {}
+    for fmt, fn in (("fp4", q.encode_fp4), ("int4", q.encode_int4), ("int8", q.encode_int8)):
+        if fmt not in formats:
+            continue
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        codes, aux = fn(W)
+        b.record()
+        torch.cuda.synchronize()
+        enc_ms[fmt] = a.elapsed_time(b)
+        ops[fmt] = (codes, aux)
+    ops["int4km"] = (idx, lut)
+    del W
+    torch.cuda.empty_cache()
+    flags = q.status_fetch()
+    if flags:
+        raise RuntimeError(f"encoder status flags 0x{flags:x}")
+    return x, ops, enc_ms
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import weight_only_quantized_qmv_b200 as q
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    q.lib()
+    formats = tuple(args.formats)
+    x, ops, enc_ms = build_workload(dev, formats)
+    fmt_id = {"fp4": q.FMT_FP4, "int4": q.FMT_INT4, "int4km": q.FMT_INT4KM, "int8": q.FMT_INT8}
+    outs = {f: torch.empty((1, N_HEAD), dtype=torch.float32, device=dev) for f in formats}
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for f in formats:
+            c, a = ops[f]
+            q.matvec(fmt_id[f], c, a, x, out=outs[f], stream=stream)
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        tdist.barrier()
+    torch.cuda.synchronize()
+
+    # timed region: per-step events bracket each format's kernel
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(formats) + 1)] for _ in range(args.steps)]
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_index = cvd.split(",")[local_rank].strip() if cvd else str(local_rank)
+    with ClockSampler(gpu_index) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for s in range(args.steps):
+            e = evs[s]
+            e[0].record(stream)
+            for i, f in enumerate(formats):
+                c, a = ops[f]
+                q.matvec(fmt_id[f], c, a, x, out=outs[f], stream=stream)
+                e[i + 1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    clocks = clk.summary()
+    total_ms = t_start.elapsed_time(t_end)
+    per_fmt_ms = {f: [evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)]
+                  for i, f in enumerate(formats)}
+    flags = q.status_fetch()
+    if flags:
+        raise RuntimeError(f"kernel status flags 0x{flags:x}")
+
+    ms_step = total_ms / args.steps
+    if dist:
+        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    bytes_step = sum(algorithmic_bytes(f, N_HEAD, K_HEAD, 1) for f in formats)
+    value = bytes_step * world / (ms_step * 1e-3) / 1e9
+
+    peak, peak_src = hbm_peak()
+    per_fmt = {}
+    for f in formats:
+        us = statistics.mean(per_fmt_ms[f]) * 1e3
+        gbs = algorithmic_bytes(f, N_HEAD, K_HEAD, 1) / (us * 1e-6) / 1e9
+        per_fmt[f] = {"us": round(us, 3), "us_median": round(statistics.median(per_fmt_ms[f]) * 1e3, 3),
+                      "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
+                      "frac_of_8tbs": round(gbs / 8000.0, 4),
+                      "bytes": algorithmic_bytes(f, N_HEAD, K_HEAD, 1)}
+    dom = max(formats, key=lambda f: per_fmt[f]["us"])
+    roof = {"bound": "hbm", "kernel": f"mv_kernel<{dom}> lm_head 248320x2048 B=1",
+            "achieved": per_fmt[dom]["gbs"], "peak": peak, "unit": "GB/s",
+            "frac": round(per_fmt[dom]["gbs"] / peak, 4), "peak_source": f"{peak_src} (hbm copy)",
+            "traffic": profiled_traffic(dom), "algorithmic_bytes": per_fmt[dom]["bytes"]}
+
+    # extra measurements (outside the timed region): batch 4 / 16 verify
+    extra = measure_batches(q, ops, dev, stream) if not args.no_extras and "fp4" in formats else None
+
+    # end to end through the C ABI with host buffers: H2D x, the matvecs, D2H y
+    e2e = None if args.no_extras else measure_e2e(q, ops, fmt_id, x, dev, stream, formats,
+                                                    steps=min(200, max(20, args.steps // 10)))
+
+    return {
+        "ms_per_step": ms_step, "value": value, "per_fmt": per_fmt, "roofline": roof, "clocks": clocks,
+        "encode_ms": enc_ms, "batches": extra, "e2e": e2e, "bytes_step": bytes_step,
+        "gpu_launches": len(formats) * args.steps,
+    }
+
+
+def measure_batches(q, ops, dev, stream, reps=30):
+    import torch
+    from weight_only_quantized_qmv_b200 import synth
+    g = synth.generator(7, dev)
+    res = {}
+    for B in (4, 16):
+        x = synth.activations(B, K_HEAD, g)
+        out = torch.empty((B, N_HEAD), dtype=torch.float32, device=dev)
+        c, a = ops["fp4"]
+        for _ in range(3):
+            q.matvec_fp4(c, a, x, out=out, stream=stream)
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            q.matvec_fp4(c, a, x, out=out, stream=stream)
+            e1.record(stream)
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        us = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+        res[f"fp4_b{B}"] = {"us": round(us, 3),
+                            "gbs": round(algorithmic_bytes("fp4", N_HEAD, K_HEAD, B) / (us * 1e-6) / 1e9, 1)}
+    return res
+
+
+def measure_e2e(q, ops, fmt_id, x, dev, stream, formats, steps):
+    import torch
+    x_host = x.cpu().pin_memory()
+    y_host = {f: torch.empty((1, N_HEAD), dtype=torch.float32).pin_memory() for f in formats}
+    x_dev = torch.empty_like(x)
+    outs = {f: torch.empty((1, N_HEAD), dtype=torch.float32, device=dev) for f in formats}
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        for f in formats:
+            c, a = ops[f]
+            q.matvec(fmt_id[f], c, a, x_dev, out=outs[f], stream=stream)
+            y_host[f].copy_(outs[f], non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(5):
+        one()
+    times = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        one_start = time.perf_counter()
+        x_dev.copy_(x_host, non_blocking=True)
+        for f in formats:
+            c, a = ops[f]
+            q.matvec(fmt_id[f], c, a, x_dev, out=outs[f], stream=stream)
+            y_host[f].copy_(outs[f], non_blocking=True)
+        e1.record(stream)
+        stream.synchronize()
+        times.append((e0.elapsed_time(e1), (time.perf_counter() - one_start) * 1e3))
+    ms_dev = statistics.mean(t[0] for t in times)
+    ms_wall = statistics.mean(t[1] for t in times)
+    bytes_step = sum(algorithmic_bytes(f, N_HEAD, K_HEAD, 1) for f in formats)
+    return {"value": round(bytes_step / (ms_wall * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "ms_per_step_wall": round(ms_wall, 4), "ms_per_step_device": round(ms_dev, 4),
+            "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(len(formats) * N_HEAD * 4),
+            "steps": steps}
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(W_rows, x_np, seconds_target):
+    """Time the oracle's fp64 matvec on a row sample of the head for each
+    format; returns (GB/s on the algorithmic-bytes definition, rows, threads)."""
+    import numpy as np
+    import oracle
+    enc = {}
+    c, s, _ = oracle.encode_fp4(W_rows)
+    enc["fp4"] = (oracle.FMT_FP4, c, s)
+    c, s, _ = oracle.encode_int4(W_rows)
+    enc["int4"] = (oracle.FMT_INT4, c, s)
+    lut = np.sort(np.random.default_rng(0).standard_normal((W_rows.shape[0], 16)) * 0.02, axis=1).astype(np.float16)
+    idx = np.random.default_rng(1).integers(0, 256, (W_rows.shape[0], K_HEAD // 2), dtype=np.uint8)
+    enc["int4km"] = (oracle.FMT_INT4KM, idx, lut)
+    c, s, _ = oracle.encode_int8(W_rows)
+    enc["int8"] = (oracle.FMT_INT8, c, s)
+    R = W_rows.shape[0]
+    t0 = time.perf_counter()
+    done = 0
+    nbytes = 0
+    while True:
+        for f in FORMATS:
+            fid, c, a = enc[f]
+            oracle.matvec(fid, c, a, x_np, R, K_HEAD)
+            nbytes += algorithmic_bytes(f, R, K_HEAD, 1)
+        done += 1
+        if time.perf_counter() - t0 >= seconds_target:
+            break
+    dt = time.perf_counter() - t0
+    return nbytes / dt / 1e9, R, oracle.num_threads(), dt, done
+
+
+def cpu_baseline(W, x, seconds=12.0, rows=8192):
+    import numpy as np
+    Wn = W[:rows].cpu().numpy()
+    xn = x.cpu().numpy()
+    gbs, R, thr, dt, passes = oracle_sample(Wn, xn, seconds)
+    return {"value": round(gbs, 3), "unit": "GB/s", "cores": thr, "kind": "oracle",
+            "sample": f"fp64 oracle matvec, {R} of 248320 rows x 2048, all four formats, {passes} passes in "
+                      f"{dt:.1f} s (bytes scaled by the algorithmic-bytes definition)"}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on the host cores, each
+    step one bounded row-sample of the same workload."""
+    import numpy as np
+    import oracle
+    from weight_only_quantized_qmv_b200 import synth
+    import torch
+    g = synth.generator(0, "cpu")
+    budget_s = 150.0
+    per_step_s = budget_s / max(1, args.steps + args.warmup)
+    rows = 4096
+    W, _ = synth.weights(rows, K_HEAD, g, n_outlier_cols=2)
+    x = synth.activations(1, K_HEAD, g).numpy()
+    Wn = W.numpy()
+    # size the per-step row sample to the time budget
+    probe_gbs, _, thr, _, _ = oracle_sample(Wn[:256], x, 0.5)
+    bytes_per_row = sum(algorithmic_bytes(f, 1, K_HEAD, 1) for f in FORMATS)
+    R = int(max(16, min(rows, probe_gbs * 1e9 * per_step_s / bytes_per_row)))
+    enc = {}
+    c, s, _ = oracle.encode_fp4(Wn[:R])
+    enc["fp4"] = (oracle.FMT_FP4, c, s)
+    c, s, _ = oracle.encode_int4(Wn[:R])
+    enc["int4"] = (oracle.FMT_INT4, c, s)
+    enc["int4km"] = (oracle.FMT_INT4KM, np.random.default_rng(1).integers(0, 256, (R, K_HEAD // 2), dtype=np.uint8),
+                     np.sort(np.random.default_rng(0).standard_normal((R, 16)) * 0.02, axis=1).astype(np.float16))
+    c, s, _ = oracle.encode_int8(Wn[:R])
+    enc["int8"] = (oracle.FMT_INT8, c, s)
+
+    def step():
+        for f in FORMATS:
+            fid, cc, aa = enc[f]
+            oracle.matvec(fid, cc, aa, x, R, K_HEAD)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    bytes_step = sum(algorithmic_bytes(f, R, K_HEAD, 1) for f in FORMATS)
+    value = bytes_step * args.steps / dt / 1e9
+    sample = f"fp64 CPU oracle, {R} of 248320 rows x 2048 per format per step"
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"lm_head 248320x2048 batch 1, fp4+int4+int4km+int8 (row sample {R})",
+                   "l2": "n/a (host)"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": thr, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+# ----------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle leg")
+    ap.add_argument("--formats", nargs="+", choices=FORMATS, default=list(FORMATS),
+                    help="weight formats in the step (default: all four, the benchmark workload)")
+    ap.add_argument("--no-extras", action="store_true", help="skip the e2e and batch-4/16 measurements")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        r = run_ours(args, rank, world, local_rank)
+    finally:
+        pass
+    out = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            from weight_only_quantized_qmv_b200 import synth
+            g = synth.generator(0, "cuda")
+            W, _ = synth.weights(8192, K_HEAD, g, n_outlier_cols=2)
+            x = synth.activations(1, K_HEAD, g)
+            cpu = cpu_baseline(W, x)
+        out = {
+            "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16 operands, f32 accumulate", "data": "synthetic",
+            "config": {"workload": "lm_head 248320x2048 batch 1; one matvec per format per step "
+                                   f"({', '.join(args.formats)})",
+                       "l2": "inputs larger than L2 (~1.1 GB read per step), no flush",
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "per_format": r["per_fmt"], "roofline": r["roofline"], "cpu_baseline": cpu, "e2e": r["e2e"],
+            "gpu_launches": r["gpu_launches"] * world, "clocks": r["clocks"], "encode_ms": r["encode_ms"],
+            "batch_verify": r["batches"],
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+        tdist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

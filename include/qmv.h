@@ -1,0 +1,179 @@
+/*
+ * qmv.h -- C ABI of libqmv: weight-only block-quantized encoders and fused
+ * dequantize-and-matvec kernels for LLM decode on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the pages' statement of the problem:
+ *   [P1] "Stream D -- Quantization (FP4 + QAT-int4): feasibility, first
+ *        result, and plan": sec. 1 (E2M1 / OCP MX FP4 weights, per-block 32
+ *        along in-features, e8m0 scale 2^(floor(log2(max_abs)) - 2), two
+ *        values per byte; int4/int8/int4km gather formats for routed
+ *        experts) and sec. 2 (symmetric int4/int8 with an MSE-optimal clip).
+ *   [P2] "Dense-path int4km coverage + flagship Qwen3.6-35B -- session
+ *        findings & methods": sec. 1-3 (decode is weight-bandwidth bound; a
+ *        fused int4km matvec for lm_head and attention q/o; gather over the
+ *        selected experts only) and sec. 8 (FP4 dense matvec: fixed E2M1 grid
+ *        times a per-K-block e8m0 scale; per-row 16-entry k-means codebook).
+ *   [P3] "coreai-optimization (coreai-opt) reference -- quantization &
+ *        palettization": per-block symmetric quantization, 1-D k-means
+ *        palettes, fp16 scales, and the pitfall that layers whose dimension
+ *        does not divide the block are silently skipped (here: rejected).
+ *
+ * Conventions for every call below
+ *  - All array pointers are DEVICE pointers owned by the caller, 16-byte
+ *    aligned, row-major and densely packed.  Host pointers are marked
+ *    "host".  The library keeps no pointer after a call returns and
+ *    allocates no device memory in any call.
+ *  - `stream` is a cudaStream_t passed as void* (NULL: the legacy default
+ *    stream).  Calls only enqueue work on it; they never synchronize, except
+ *    qmv_status_fetch.
+ *  - Shapes: N output rows (out-features), K in-features with K % 32 == 0
+ *    (one quantization block = 32 consecutive in-features of one row).
+ *    B is the number of activation rows (decode tokens), 1 <= B <= 16.
+ *  - fp16 arrays are IEEE binary16 bit patterns (uint16_t).
+ *  - Packed 4-bit codes: element k of a row lives in byte k/2, low nibble
+ *    for even k, high nibble for odd k (the little-endian reading of eight
+ *    codes per 32-bit word).
+ *  - Errors: argument checks run on the host before anything is enqueued
+ *    and return QMV_ERR_ARG (null or misaligned pointer, bad format or clip
+ *    list), QMV_ERR_SHAPE (N < 1, K < 32, K % 32 != 0, E < 1) or
+ *    QMV_ERR_UNSUPPORTED (B or topk outside [1, 16], or a shape whose
+ *    activations do not fit the kernel's on-chip staging); a failed launch
+ *    returns QMV_ERR_CUDA.  Bad DATA is found on the device: the kernel sets
+ *    a bit of a library-owned device status word (QMV_FLAG_*) and carries
+ *    on; qmv_status_fetch reads and clears it.  No kernel traps.
+ *  - The library-owned status word is per device; calls that run on several
+ *    streams at once share it.
+ */
+#ifndef QMV_H
+#define QMV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QMV_OK = 0,
+  QMV_ERR_ARG = -1,
+  QMV_ERR_SHAPE = -2,
+  QMV_ERR_UNSUPPORTED = -3,
+  QMV_ERR_DATA = -4,
+  QMV_ERR_CUDA = -5
+} qmv_status;
+
+/* Weight formats. */
+enum {
+  QMV_FMT_FP4 = 0,    /* E2M1 codes + e8m0 scale byte per 32-block      */
+  QMV_FMT_INT4 = 1,   /* symmetric int4 (nibble = q + 8) + fp16 scale   */
+  QMV_FMT_INT4KM = 2, /* 4-bit index into a per-row 16-entry fp16 LUT   */
+  QMV_FMT_INT8 = 3    /* symmetric int8 (two's complement) + fp16 scale */
+};
+
+/* Device status bits (qmv_status_fetch). */
+#define QMV_FLAG_NONFINITE 0x1u      /* encode: a block held Inf/NaN (block written as zeros) */
+#define QMV_FLAG_SCALE_OVERFLOW 0x2u /* encode: no clip gave a finite fp16 scale (block zeroed) */
+#define QMV_FLAG_BAD_EXPERT 0x4u     /* gather: expert id outside [0, E) (that output row zeroed) */
+#define QMV_FLAG_TIMEOUT 0x8u        /* a pipeline wait gave up (internal fault; outputs invalid) */
+
+/* ---------------------------------------------------------------------
+ * Encoders (offline conversion; [P1] sec. 1-2).
+ * --------------------------------------------------------------------- */
+
+/* FP4 E2M1 encode.  Per row and 32-block: amax = max|w|; e = floor(log2(
+ * amax)) - 2 clamped to [-127, 127] (amax == 0 gives -127); scale byte =
+ * e + 127; code = sign bit | E2M1 magnitude of |w| * 2^-e rounded to nearest,
+ * ties to even, saturating at 6.  A negative weight that rounds to zero keeps
+ * its sign (code 8).
+ *   W       [N, K] float32 (in)
+ *   codes   [N, K/2] uint8 (out, packed as above)
+ *   scales  [N, K/32] uint8 e8m0 bytes (out)
+ * A block with Inf/NaN: codes 0, scale byte 0, QMV_FLAG_NONFINITE. */
+qmv_status qmv_encode_fp4(const float* W, int64_t N, int64_t K, uint8_t* codes,
+                          uint8_t* scales, void* stream);
+
+/* Symmetric int4 encode with MSE-searched clip.  Per block, for each clip
+ * alpha in list order: s = fp16_rne(float(alpha * amax) / 7); q_i =
+ * clamp(rint_even(w_i / s), -7, 7) (0 when s == 0); err = sum over i of
+ * (double(w_i) - q_i * double(s))^2 accumulated in order i = 0..31; the first
+ * alpha with the strictly smallest err wins.  A clip whose fp16 scale
+ * overflows is skipped; a block with none left is zeroed with
+ * QMV_FLAG_SCALE_OVERFLOW.
+ *   clips   host float32 [n_clips], 1 <= n_clips <= 16 (e.g. 1.00 .. 0.50)
+ *   codes   [N, K/2] uint8, nibble = q + 8 (out)
+ *   scales  [N, K/32] fp16 (out) */
+qmv_status qmv_encode_int4(const float* W, int64_t N, int64_t K, const float* clips,
+                           int n_clips, uint8_t* codes, uint16_t* scales, void* stream);
+
+/* Symmetric int8 encode: as qmv_encode_int4 with qmax = 127 and one
+ * two's-complement byte per weight.  clips = {1.0f} is plain absmax.
+ *   codes   [N, K] int8 (out);  scales [N, K/32] fp16 (out) */
+qmv_status qmv_encode_int8(const float* W, int64_t N, int64_t K, const float* clips,
+                           int n_clips, int8_t* codes, uint16_t* scales, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Fused dequantize + matvec, y = x Wdq^T with fp32 accumulation
+ * ([P2] sec. 1-3, 8).  x: [B, K] fp16; y: [B, N] float32 (overwritten).
+ * Block-scaled formats apply the scale to each 32-block's exact partial sum.
+ * --------------------------------------------------------------------- */
+
+/* codes [N, K/2] uint8 E2M1; scales [N, K/32] uint8 e8m0. */
+qmv_status qmv_matvec_fp4(const uint8_t* codes, const uint8_t* scales, const uint16_t* x,
+                          int B, int64_t N, int64_t K, float* y, void* stream);
+
+/* codes [N, K/2] uint8 (q + 8 nibbles); scales [N, K/32] fp16. */
+qmv_status qmv_matvec_int4(const uint8_t* codes, const uint16_t* scales, const uint16_t* x,
+                           int B, int64_t N, int64_t K, float* y, void* stream);
+
+/* idx [N, K/2] uint8 (4-bit LUT indices); lut [N, 16] fp16 per-row palette. */
+qmv_status qmv_matvec_int4km(const uint8_t* idx, const uint16_t* lut, const uint16_t* x,
+                             int B, int64_t N, int64_t K, float* y, void* stream);
+
+/* codes [N, K] int8; scales [N, K/32] fp16. */
+qmv_status qmv_matvec_int8(const int8_t* codes, const uint16_t* scales, const uint16_t* x,
+                           int B, int64_t N, int64_t K, float* y, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Routed-expert gather matvec ([P1] sec. 1 gather formats; [P2] sec. 3:
+ * only the selected experts' weights are read).  For token b and slot j,
+ * e = expert_ids[b*topk + j] and
+ *    y[b, j, :] = W_e x_b        (x_per_slot == 0, x [B, K])
+ *    y[b, j, :] = W_e x_{b,j}    (x_per_slot == 1, x [B, topk, K]).
+ * Each selected expert's weights are streamed once per call for all the
+ * (b, j) that chose it.
+ *   fmt          QMV_FMT_*; codes_stack / aux_stack are the per-format
+ *                arrays of qmv_matvec_* stacked over experts: [E, N, ...]
+ *   expert_ids   [B, topk] int32 (device)
+ *   y            [B, topk, N] float32 (out)
+ * An id outside [0, E) zeroes its output row and sets QMV_FLAG_BAD_EXPERT.
+ * The (b, j) pairs that chose one expert are served together, in column
+ * groups of up to 16 pairs per pass over that expert's weights. */
+qmv_status qmv_gather_matvec(int fmt, const void* codes_stack, const void* aux_stack, int E,
+                             int64_t N, int64_t K, const int32_t* expert_ids, int B, int topk,
+                             const uint16_t* x, int x_per_slot, float* y, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Test support and status
+ * --------------------------------------------------------------------- */
+
+/* Dequantize to float32 Wdq [N, K] with the same decode the matvec kernels
+ * use (exact: every format's dequantized value is a float32). */
+qmv_status qmv_dequant(int fmt, const void* codes, const void* aux, int64_t N, int64_t K,
+                       float* Wdq, void* stream);
+
+/* Synchronize `stream`, then read and clear the current device's status
+ * word into *flags (host).  Returns QMV_ERR_DATA when any QMV_FLAG_* bit was
+ * set, QMV_OK otherwise, QMV_ERR_CUDA if the stream reported an error. */
+qmv_status qmv_status_fetch(void* stream, uint32_t* flags);
+
+/* Text of the last error of this host thread ("" if none). */
+const char* qmv_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* qmv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMV_H */

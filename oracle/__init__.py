@@ -31,7 +31,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # QMV_ORACLE_LIB: load another build of the same source (the mutation
+        # tests point it at deliberately broken copies)
+        path = os.environ.get("QMV_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         P, I64, I32, U32P = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)
         L.oracle_f32_to_f16.argtypes = [ctypes.c_float]

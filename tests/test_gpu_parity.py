@@ -1,0 +1,443 @@
+"""GPU parity of libqmv (through its C ABI binding) against the CPU oracle.
+
+Bar: packed codes, scales and dequantized weights bit-exact; matvec outputs
+within max relative error 1e-3 of the fp64 oracle, read per activation row as
+||y_b - r_b||_inf / ||r_b||_inf (a per-element ratio is ill-conditioned where
+r is near zero).  The expected fp32-accumulation error is ~1e-6, so the
+tests also report the observed figure in their assertion messages.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from weight_only_quantized_qmv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+FMTS = ("fp4", "int4", "int4km", "int8")
+
+
+@pytest.fixture(scope="module")
+def q():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from weight_only_quantized_qmv_b200 import _build
+    _build.build()
+    import weight_only_quantized_qmv_b200 as q
+    q.lib()
+    assert q.status_fetch() == 0
+    return q
+
+
+def rel_err(y, r):
+    """max over activation rows of ||y_b - r_b||_inf / ||r_b||_inf."""
+    y = np.asarray(y, np.float64).reshape(r.shape)
+    num = np.abs(y - r).max(axis=-1)
+    den = np.abs(r).max(axis=-1)
+    den = np.where(den == 0, 1.0, den)
+    return float((num / den).max())
+
+
+def gen_w(N, K, seed=0, n_out=0, device="cuda"):
+    g = synth.generator(seed, device)
+    W, _ = synth.weights(N, K, g, n_outlier_cols=n_out)
+    return W, g
+
+
+def encode_gpu(q, fmt, W, W_np=None):
+    """GPU encode (fp4/int4/int8) or oracle fit (int4km: no GPU encoder)."""
+    if fmt == "fp4":
+        return q.encode_fp4(W)
+    if fmt == "int4":
+        return q.encode_int4(W)
+    if fmt == "int8":
+        return q.encode_int8(W)
+    lut, idx, _ = orc.kmeans_int4km(W.cpu().numpy() if W_np is None else W_np)
+    return torch.from_numpy(idx).cuda(), torch.from_numpy(lut).cuda()
+
+
+def encode_orc(fmt, Wn):
+    if fmt == "fp4":
+        c, s, f = orc.encode_fp4(Wn)
+    elif fmt == "int4":
+        c, s, f = orc.encode_int4(Wn)
+    elif fmt == "int8":
+        c, s, f = orc.encode_int8(Wn)
+    else:
+        s, c, f = orc.kmeans_int4km(Wn)
+    return c, s, f
+
+
+FID = {"fp4": orc.FMT_FP4, "int4": orc.FMT_INT4, "int4km": orc.FMT_INT4KM, "int8": orc.FMT_INT8}
+
+
+def np_bits(t):
+    a = t.cpu().numpy()
+    return a.view(np.uint8) if a.dtype in (np.int8, np.uint8) else a.view(np.uint16)
+
+
+# ---------------------------------------------------------------------------
+# encoders
+# ---------------------------------------------------------------------------
+
+def test_e2m1_hardware_conversion_matches_oracle_table(q):
+    """Blocks whose max is 4 or 7.99 have scale 2^0, so each code is the
+    hardware E2M1 conversion of the weight itself: it must equal the
+    oracle's nearest-even table at every tie and threshold."""
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    pts = [(a + b) / 2 for a, b in zip(grid, grid[1:])] + grid + [7.0]
+    vals = []
+    for c in pts:
+        v = np.float32(c)
+        vals.append(v)
+        lo = hi = v
+        for _ in range(3):
+            lo = np.nextafter(lo, np.float32(-1), dtype=np.float32)
+            hi = np.nextafter(hi, np.float32(9), dtype=np.float32)
+            vals += [lo, hi]
+    vals = np.array([v for v in vals if 0 <= v < 7.99], np.float32)
+    vals = np.concatenate([vals, -vals, np.array([-0.0, 1e-30, -1e-30], np.float32)])
+    n = (len(vals) + 30) // 31
+    W = np.zeros((n, 32), np.float32)
+    W[:, 0] = np.where(np.arange(n) % 2 == 0, 4.0, 7.99)
+    W[:, 1:].flat[:len(vals)] = vals
+    c_gpu, s_gpu = q.encode_fp4(torch.from_numpy(W).cuda())
+    c_orc, s_orc, _ = orc.encode_fp4(W)
+    assert np.array_equal(s_gpu.cpu().numpy(), s_orc)
+    assert (s_orc == 127).all()
+    assert np.array_equal(c_gpu.cpu().numpy(), c_orc)
+    assert q.status_fetch() == 0
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4", "int8"])
+@pytest.mark.parametrize("N,K", [(1, 32), (40, 96), (300, 544), (64, 2080), (33, 4096)])
+def test_encoder_bit_exact(q, fmt, N, K):
+    W, _ = gen_w(N, K, seed=N + K, n_out=max(1, K // 1000))
+    W[0, :32] = 0.0  # all-zero block
+    if N > 2:
+        W[1, 32 % K:32 % K + 32] = 1e-30  # tiny block: scale underflow paths
+        W[2, :] *= 1e4  # large row
+    Wn = W.cpu().numpy()
+    c_g, s_g = encode_gpu(q, fmt, W)
+    c_o, s_o, f = encode_orc(fmt, Wn)
+    assert f == 0
+    assert np.array_equal(np_bits(c_g), c_o.view(np.uint8))
+    assert np.array_equal(np_bits(s_g), s_o.view(np.uint8) if fmt == "fp4" else s_o.view(np.uint16))
+    assert q.status_fetch() == 0
+
+
+def test_c1_tiny_fp4_round_trip_and_matvec(q):
+    """512x1024 fp4, 8 outlier columns x20, x ~N(0,1) fp16, seed 0."""
+    g = synth.generator(0, "cpu")
+    W, _ = synth.weights(512, 1024, g, n_outlier_cols=8)
+    x = synth.activations(1, 1024, g)
+    Wn, xn = W.numpy(), x.numpy()
+    codes, scales = q.encode_fp4(W.cuda())
+    c_o, s_o, _ = orc.encode_fp4(Wn)
+    assert np.array_equal(codes.cpu().numpy(), c_o) and np.array_equal(scales.cpu().numpy(), s_o)
+    D = q.dequant(q.FMT_FP4, codes, scales).cpu().numpy()
+    D_o = orc.dequant(orc.FMT_FP4, c_o, s_o, 512, 1024)
+    assert np.array_equal(D.view(np.uint32), D_o.view(np.uint32))
+    y = q.matvec_fp4(codes, scales, x.cuda())
+    r = orc.matvec(orc.FMT_FP4, c_o, s_o, xn, 512, 1024)
+    assert rel_err(y.cpu().numpy(), r) < TOL
+    assert q.status_fetch() == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K", [(17, 96), (200, 544), (130, 2048), (64, 2080), (48, 4096)])
+def test_dequant_bit_exact(q, fmt, N, K):
+    W, _ = gen_w(N, K, seed=3 * N + K, n_out=2)
+    Wn = W.cpu().numpy()
+    c_o, s_o, _ = encode_orc(fmt, Wn)
+    c = torch.from_numpy(c_o).cuda()
+    s = torch.from_numpy(s_o).cuda()
+    D = q.dequant(q.__dict__["FMT_" + fmt.upper()], c, s).cpu().numpy()
+    D_o = orc.dequant(FID[fmt], c_o, s_o, N, K)
+    assert np.array_equal(D.view(np.uint32), D_o.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# fused dequant + matvec
+# ---------------------------------------------------------------------------
+
+def _inputs(fmt, N, K, B, seed):
+    g = synth.generator(seed, "cpu")
+    W, _ = synth.weights(N, K, g, n_outlier_cols=2)
+    x = synth.activations(B, K, g)
+    Wn = W.numpy()
+    c_o, s_o, _ = encode_orc(fmt, Wn) if fmt != "int4km" or N * K <= 2_000_000 else (None, None, 0)
+    if c_o is None:
+        lut, idx = synth.palette_tables(N, K, g)
+        c_o, s_o = idx.numpy(), lut.numpy()
+    return c_o, s_o, x.numpy()
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K", [(1, 32), (17, 96), (1000, 544), (600, 2048), (70, 2080), (130, 4096),
+                                 (40, 6144)])
+@pytest.mark.parametrize("B", [1, 3, 8, 9, 16])
+def test_matvec_parity(q, fmt, N, K, B):
+    c_o, s_o, xn = _inputs(fmt, N, K, B, seed=N * 7 + K + B)
+    c, s, x = torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(), torch.from_numpy(xn).cuda()
+    if B * K * 2 > 160 * 1024:
+        # activations beyond the on-chip staging are rejected on the host
+        with pytest.raises(q.QmvError) as ei:
+            q.matvec(q.__dict__["FMT_" + fmt.upper()], c, s, x)
+        assert ei.value.status == q.ERR_UNSUPPORTED
+        return
+    y = q.matvec(q.__dict__["FMT_" + fmt.upper()], c, s, x).cpu().numpy()
+    r = orc.matvec(FID[fmt], c_o, s_o, xn, N, K)
+    e = rel_err(y, r)
+    assert e < TOL, e
+    assert q.status_fetch() == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_matvec_one_hot_columns_bit_exact(q, fmt):
+    """x = e_k picks column k of Wdq: the kernel must return it exactly
+    (pins layout, nibble order, scale indexing and the k-permutation)."""
+    N, K = 100, 544
+    c_o, s_o, _ = _inputs(fmt, N, K, 1, seed=5)
+    ks = [0, 1, 7, 8, 31, 32, 100, 257, K - 1, K - 2, 300, 511, 64, 65, 200, 450]
+    x = np.zeros((len(ks), K), np.float16)
+    x[np.arange(len(ks)), ks] = 1.0
+    y = q.matvec(q.__dict__["FMT_" + fmt.upper()], torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(),
+                 torch.from_numpy(x).cuda()).cpu().numpy()
+    D = orc.dequant(FID[fmt], c_o, s_o, N, K)
+    for i, k in enumerate(ks):
+        assert np.array_equal(y[i], D[:, k]), (fmt, k)
+
+
+def test_matvec_output_guard_bands(q):
+    """Sentinels around the output rows stay untouched (no out-of-bounds
+    writes on a ragged last tile)."""
+    N, K, B = 37, 2048, 3
+    c_o, s_o, xn = _inputs("fp4", N, K, B, seed=11)
+    buf = torch.full((B * N + 64,), 12345.0, device="cuda")
+    out = buf[32:32 + B * N].view(B, N)
+    q.matvec_fp4(torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(), torch.from_numpy(xn).cuda(), out=out)
+    b = buf.cpu().numpy()
+    assert (b[:32] == 12345.0).all() and (b[32 + B * N:] == 12345.0).all()
+    assert rel_err(out.cpu().numpy(), orc.matvec(orc.FMT_FP4, c_o, s_o, xn, N, K)) < TOL
+
+
+def test_unaligned_fp4_scale_plane(q):
+    """A scale plane starting at an odd byte takes the staged-block path."""
+    N, K, B = 50, 2048, 2
+    c_o, s_o, xn = _inputs("fp4", N, K, B, seed=13)
+    sb = torch.zeros(s_o.size + 1, dtype=torch.uint8, device="cuda")
+    sb[1:] = torch.from_numpy(s_o.reshape(-1)).cuda()
+    s_view = sb[1:].view(N, K // 32)
+    y = q.matvec_fp4(torch.from_numpy(c_o).cuda(), s_view, torch.from_numpy(xn).cuda())
+    assert rel_err(y.cpu().numpy(), orc.matvec(orc.FMT_FP4, c_o, s_o, xn, N, K)) < TOL
+
+
+def test_matvec_is_deterministic(q):
+    N, K, B = 3000, 2048, 4
+    c_o, s_o, xn = _inputs("int4", N, K, B, seed=17)
+    args = (torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(), torch.from_numpy(xn).cuda())
+    y1 = q.matvec_int4(*args)
+    y2 = q.matvec_int4(*args)
+    assert torch.equal(y1, y2)
+
+
+# ---------------------------------------------------------------------------
+# gather over routed experts
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("B,topk,x_per_slot", [(1, 8, 0), (3, 2, 1), (8, 8, 0), (8, 8, 1), (16, 4, 0)])
+def test_gather_parity(q, fmt, B, topk, x_per_slot):
+    E, N, K = 12, 80, 544
+    g = synth.generator(B * 100 + topk, "cpu")
+    Ws = [synth.weights(N, K, g)[0].numpy() for _ in range(E)]
+    enc = [encode_orc(fmt, W) for W in Ws]
+    cs = np.stack([e[0] for e in enc])
+    aus = np.stack([e[1] for e in enc])
+    ids = synth.routing(B, topk, E, g).numpy()
+    if B >= 3:
+        ids[1, 0] = ids[0, 0]  # two tokens share an expert
+    x = synth.activations(B, K, g, extra_shape=(topk,) if x_per_slot else ()).numpy()
+    F = q.__dict__["FMT_" + fmt.upper()]
+    y = q.gather_matvec(F, torch.from_numpy(cs).cuda(), torch.from_numpy(aus).cuda(), torch.from_numpy(ids).cuda(),
+                        torch.from_numpy(x).cuda(), x_per_slot=bool(x_per_slot)).cpu().numpy()
+    r, fl = orc.gather_matvec(FID[fmt], cs, aus, E, N, K, ids, x, x_per_slot)
+    assert fl == 0
+    assert rel_err(y.reshape(-1, N), r.reshape(-1, N)) < TOL
+    # identical to the dense kernel on the chosen expert's weights, bit for bit
+    for b in range(B):
+        for j in range(topk):
+            e = ids[b, j]
+            xb = x[b, j] if x_per_slot else x[b]
+            yd = q.matvec(F, torch.from_numpy(cs[e]).cuda(), torch.from_numpy(aus[e]).cuda(),
+                          torch.from_numpy(xb[None].copy()).cuda()).cpu().numpy()[0]
+            assert np.array_equal(yd, y[b, j]), (b, j)
+    assert q.status_fetch() == 0
+
+
+def test_gather_bad_expert_id_flags_and_zeroes(q):
+    E, N, K, B, topk = 4, 64, 256, 2, 3
+    g = synth.generator(1, "cpu")
+    W = synth.weights(E * N, K, g)[0].numpy()
+    c, s, _ = orc.encode_fp4(W)
+    cs, ss = c.reshape(E, N, -1), s.reshape(E, N, -1)
+    ids = np.array([[0, 9, 2], [-1, 3, 3]], np.int32)
+    x = synth.activations(B, K, g).numpy()
+    y = torch.full((B, topk, N), 7.0, device="cuda")
+    q.gather_matvec(q.FMT_FP4, torch.from_numpy(cs).cuda(), torch.from_numpy(ss).cuda(), torch.from_numpy(ids).cuda(),
+                    torch.from_numpy(x).cuda(), out=y)
+    flags = q.status_fetch()
+    assert flags & q.FLAG_BAD_EXPERT
+    yn = y.cpu().numpy()
+    assert not yn[0, 1].any() and not yn[1, 0].any()
+    r, fl = orc.gather_matvec(orc.FMT_FP4, cs, ss, E, N, K, ids, x, 0)
+    assert fl & orc.FLAG_BAD_EXPERT
+    assert rel_err(yn.reshape(-1, N), r.reshape(-1, N)) < TOL
+
+
+# ---------------------------------------------------------------------------
+# data faults and argument errors
+# ---------------------------------------------------------------------------
+
+def test_nonfinite_weights_flag_and_zero_blocks(q):
+    W, _ = gen_w(8, 128, seed=2)
+    W[3, 40] = float("nan")
+    W[5, 100] = float("inf")
+    Wn = W.cpu().numpy()
+    for fmt in ("fp4", "int4", "int8"):
+        c, s = encode_gpu(q, fmt, W)
+        flags = q.status_fetch()
+        assert flags & q.FLAG_NONFINITE, fmt
+        c_o, s_o, f = encode_orc(fmt, Wn)
+        assert f & orc.FLAG_NONFINITE
+        assert np.array_equal(np_bits(c), c_o.view(np.uint8))
+
+
+def test_scale_overflow_flag(q):
+    W = torch.zeros(2, 32, device="cuda")
+    W[1, 0] = 1e6  # 1e6 / 7 > 65504: no finite fp16 scale for clip 1.0
+    c, s = q.encode_int4(W, clips=[1.0])
+    assert q.status_fetch() & q.FLAG_SCALE_OVERFLOW
+    c_o, s_o, f = orc.encode_int4(W.cpu().numpy(), np.array([1.0], np.float32))
+    assert f & orc.FLAG_SCALE_OVERFLOW
+    assert np.array_equal(c.cpu().numpy(), c_o) and np.array_equal(np_bits(s), s_o.view(np.uint16))
+
+
+def test_argument_errors_raise(q):
+    codes = torch.zeros(16, 64, dtype=torch.uint8, device="cuda")
+    scales = torch.zeros(16, 4, dtype=torch.uint8, device="cuda")
+    xb = torch.zeros(2 * 128 + 1, dtype=torch.float16, device="cuda")
+    with pytest.raises(q.QmvError) as ei:
+        q.matvec_fp4(codes, scales, xb[1:129])  # x misaligned by 2 bytes
+    assert ei.value.status == q.ERR_ARG
+    with pytest.raises(q.QmvError) as ei:
+        q.matvec_fp4(codes, scales, torch.zeros(17, 128, dtype=torch.float16, device="cuda"))
+    assert ei.value.status == q.ERR_UNSUPPORTED
+    assert q.status_fetch() == 0
+
+
+# ---------------------------------------------------------------------------
+# the workloads at full size (sampled rows against the oracle)
+# ---------------------------------------------------------------------------
+
+def sample_rows(N, n_rand=384, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = np.concatenate([np.arange(min(N, 48)), np.arange(max(0, N - 48), N), rng.integers(0, N, n_rand)])
+    return np.unique(rows)
+
+
+def _full_encode_check(q, fmt, W, rows):
+    c, s = encode_gpu(q, fmt, W)
+    c_o, s_o, f = encode_orc(fmt, W[torch.from_numpy(rows).cuda()].cpu().numpy())
+    assert f == 0
+    assert np.array_equal(np_bits(c)[rows], c_o.view(np.uint8))
+    assert np.array_equal(np_bits(s)[rows], s_o.view(np.uint8) if fmt == "fp4" else s_o.view(np.uint16))
+    return c, s, c_o, s_o
+
+
+def _sampled_matvec(q, fmt, c, s, c_o, s_o, xn, rows, K):
+    y = q.matvec(q.__dict__["FMT_" + fmt.upper()], c, s, torch.from_numpy(xn).cuda())
+    r = orc.matvec(FID[fmt], c_o, s_o, xn, len(rows), K)
+    e = rel_err(y.cpu().numpy()[:, rows], r)
+    assert e < TOL, (fmt, e)
+    return e
+
+
+@pytest.mark.slow
+def test_full_int8_head_130560x2048(q):
+    N, K = 130560, 2048
+    g = synth.generator(0, "cuda")
+    W, _ = synth.weights(N, K, g)
+    x = synth.activations(1, K, g).cpu().numpy()
+    rows = sample_rows(N)
+    c, s, c_o, s_o = _full_encode_check(q, "int8", W, rows)
+    _sampled_matvec(q, "int8", c, s, c_o, s_o, x, rows, K)
+    assert q.status_fetch() == 0
+
+
+@pytest.mark.slow
+def test_full_int4_and_fp4_head_248320x2048(q):
+    """int4 (11 clips) and fp4 on the same outlier-bearing head; fp4 at
+    batch 1, 4 and 16."""
+    N, K = 248320, 2048
+    g = synth.generator(0, "cuda")
+    W, _ = synth.weights(N, K, g, n_outlier_cols=2)
+    x16 = synth.activations(16, K, g).cpu().numpy()
+    rows = sample_rows(N)
+    c, s, c_o, s_o = _full_encode_check(q, "int4", W, rows)
+    _sampled_matvec(q, "int4", c, s, c_o, s_o, x16[:1], rows, K)
+    del c, s
+    c, s, c_o, s_o = _full_encode_check(q, "fp4", W, rows)
+    for B in (1, 4, 16):
+        _sampled_matvec(q, "fp4", c, s, c_o, s_o, x16[:B], rows, K)
+    assert q.status_fetch() == 0
+
+
+@pytest.mark.slow
+def test_full_int4km_head_248320x2048(q):
+    """int4km at full size with per-row palettes of the workload's shape
+    (random tables: the CPU fit of 248320 rows is covered at smaller sizes)."""
+    N, K = 248320, 2048
+    g = synth.generator(0, "cuda")
+    lut, idx = synth.palette_tables(N, K, g)
+    x = synth.activations(1, K, g).cpu().numpy()
+    rows = sample_rows(N)
+    y = q.matvec_int4km(idx, lut, torch.from_numpy(x).cuda())
+    r = orc.matvec(orc.FMT_INT4KM, idx.cpu().numpy()[rows], lut.cpu().numpy()[rows], x, len(rows), K)
+    assert rel_err(y.cpu().numpy()[:, rows], r) < TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("B", [1, 8])
+def test_full_decode_step_int4km(q, B):
+    """lm_head + 10 x (q_proj 2048->4096, o_proj 4096->2048) + routed experts
+    256 x (gate/up 2048->512, down 512->2048), top-8 routing."""
+    g = synth.generator(1000 + B, "cuda")
+    dense = [(248320, 2048)] + [(4096, 2048), (2048, 4096)] * 10
+    for i, (N, K) in enumerate(dense):
+        lut, idx = synth.palette_tables(N, K, g)
+        x = synth.activations(B, K, g).cpu().numpy()
+        rows = sample_rows(N, n_rand=64, seed=i)
+        y = q.matvec_int4km(idx, lut, torch.from_numpy(x).cuda())
+        r = orc.matvec(orc.FMT_INT4KM, idx.cpu().numpy()[rows], lut.cpu().numpy()[rows], x, len(rows), K)
+        assert rel_err(y.cpu().numpy()[:, rows], r) < TOL, (i, N, K)
+    E, topk = 256, 8
+    ids = synth.routing(B, topk, E, g)
+    for name, N, K, per_slot in (("gate", 512, 2048, 0), ("up", 512, 2048, 0), ("down", 2048, 512, 1)):
+        lut, idx = synth.palette_tables(E * N, K, g)
+        lut, idx = lut.view(E, N, 16), idx.view(E, N, K // 2)
+        x = synth.activations(B, K, g, extra_shape=(topk,) if per_slot else ())
+        y = q.gather_matvec(q.FMT_INT4KM, idx, lut, ids, x, x_per_slot=bool(per_slot)).cpu().numpy()
+        ids_n, xn = ids.cpu().numpy(), x.cpu().numpy()
+        for b in range(B):
+            for j in range(topk):
+                e = ids_n[b, j]
+                rows = sample_rows(N, n_rand=32, seed=b * topk + j)
+                xb = xn[b, j] if per_slot else xn[b]
+                r = orc.matvec(orc.FMT_INT4KM, idx[e].cpu().numpy()[rows], lut[e].cpu().numpy()[rows], xb[None],
+                               len(rows), K)
+                assert rel_err(y[b, j][rows][None], r) < TOL, (name, b, j)
+    assert q.status_fetch() == 0

@@ -241,6 +241,36 @@ def test_int_encode_brute_force(orc, bits):
                 assert np.float16(s) == svals[first] or min(errs) == 0
 
 
+def test_int_exact_ties_round_to_even(orc):
+    """Quotients exactly halfway between integers round to the even one: with
+    amax = 7 and clip 1, the int4 scale is exactly 1."""
+    w = np.array([7.0, 2.5, -2.5, 1.5, -1.5, 0.5, -0.5, 3.5, -3.5, 4.5, 5.5, 6.5] + [0.0] * 20, np.float32)
+    codes, scales, _ = orc.encode_int4(w[None], np.array([1.0], np.float32))
+    assert scales[0, 0] == 1.0
+    q = _unpack_int(codes, 4, 32)[0]
+    assert list(q[:12]) == [7, 2, -2, 2, -2, 0, 0, 4, -4, 4, 6, 6]
+    w8 = np.zeros((1, 32), np.float32)
+    w8[0, :6] = [127.0, 2.5, -2.5, 100.5, 101.5, -0.5]
+    codes8, scales8, _ = orc.encode_int8(w8)
+    assert scales8[0, 0] == 1.0
+    assert list(codes8[0, :6]) == [127, 2, -2, 100, 102, 0]
+
+
+def test_int_clip_tie_keeps_the_first(orc):
+    """Two clips whose fp16 scales sit one ulp either side of the optimum
+    c = amax / 7 give the same q and exactly the same SSE 49 u^2: the first
+    clip in list order is kept."""
+    c, u = 0.140625, 2.0 ** -13  # c on the fp16 grid, u its spacing there
+    w = np.zeros((1, 32), np.float32)
+    w[0, 0] = 7 * c
+    clips = np.array([1 - u / c, 1 + u / c], np.float32)
+    for order in (clips, clips[::-1].copy()):
+        codes, scales, _ = orc.encode_int4(w, order)
+        sc = np.float16(np.float32(np.float32(order[0]) * np.float32(7 * c)) / np.float32(7))
+        assert scales[0, 0] == sc, (order, scales[0, 0], sc)
+        assert _unpack_int(codes, 4, 32)[0, 0] == 7
+
+
 def test_int_special_blocks(orc):
     W = np.zeros((3, 32), np.float32)
     W[0, 5] = 0.7  # single non-zero element, alpha = 1: q = qmax, s = fp16(0.7/7)
@@ -312,6 +342,12 @@ def test_kmeans_exact_on_few_distinct_values(orc):
     assert flags == 0
     D = orc.dequant(orc.FMT_INT4KM, idx, lut, N, K)
     assert np.array_equal(D, W)
+    # rows with fewer than 16 values keep duplicate centres: an index must
+    # name the lowest of equal nearest entries
+    got = np.empty((N, K), np.int64)
+    got[:, 0::2], got[:, 1::2] = idx & 15, idx >> 4
+    d = np.abs(W.astype(np.float64)[:, :, None] - lut.astype(np.float64)[:, None, :])
+    assert np.array_equal(got, np.argmin(d, axis=2))
 
 
 def test_kmeans_sse_monotone_and_nearest_indices(orc):

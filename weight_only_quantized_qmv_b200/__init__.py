@@ -1,0 +1,226 @@
+"""weight_only_quantized_qmv_b200 -- Python binding of libqmv (B200, sm_100a).
+
+Argument marshalling only: every step of encode / matvec / gather runs in the
+library's CUDA kernels (libqmv.so, next to this file, built by _build.py).
+PyTorch supplies device memory and the current stream.  There is no CPU or
+library fallback: importing the binding without libqmv.so raises.
+
+The functions mirror the C ABI in include/qmv.h (same names without the
+``qmv_`` prefix).  Packed layouts: 4-bit codes uint8 [N, K/2] (element 2j in
+the low nibble), fp4 scales uint8 [N, K/32] (e8m0), int4/int8 scales float16
+[N, K/32], int4km palette float16 [N, 16]; activations float16 [B, K];
+outputs float32 [B, N].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqmv.so")
+
+FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8 = 0, 1, 2, 3
+FMT_NAMES = {FMT_FP4: "fp4", FMT_INT4: "int4", FMT_INT4KM: "int4km", FMT_INT8: "int8"}
+FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT, FLAG_TIMEOUT = 1, 2, 4, 8
+OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_DATA, ERR_CUDA = 0, -1, -2, -3, -4, -5
+
+# Clip lists of the workloads: int4 searches 1.00, 0.95, ..., 0.50 (float32
+# literals); int8 is plain symmetric absmax.
+INT4_CLIPS = [1.0 - 0.05 * i for i in range(11)]
+INT8_CLIPS = [1.0]
+
+
+class QmvError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"libqmv status {status}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+# (name, argtypes) of every exported entry point
+_P, _I64, _I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+SIGNATURES = {
+    "qmv_encode_fp4": [_P, _I64, _I64, _P, _P, _P],
+    "qmv_encode_int4": [_P, _I64, _I64, _P, _I32, _P, _P, _P],
+    "qmv_encode_int8": [_P, _I64, _I64, _P, _I32, _P, _P, _P],
+    "qmv_matvec_fp4": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
+    "qmv_matvec_int4": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
+    "qmv_matvec_int4km": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
+    "qmv_matvec_int8": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
+    "qmv_gather_matvec": [_I32, _P, _P, _I32, _I64, _I64, _P, _I32, _I32, _P, _I32, _P, _P],
+    "qmv_dequant": [_I32, _P, _P, _I64, _I64, _P, _P],
+    "qmv_status_fetch": [_P, ctypes.POINTER(ctypes.c_uint32)],
+    "qmv_last_error": [],
+    "qmv_version": [],
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libqmv.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libqmv.so not found at {LIB_PATH}: build it with "
+                              "`python -m weight_only_quantized_qmv_b200._build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in SIGNATURES.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_char_p if name in ("qmv_last_error", "qmv_version") else ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _call(name, *args):
+    rc = getattr(lib(), name)(*args)
+    if rc != OK:
+        raise QmvError(rc, lib().qmv_last_error().decode())
+    return rc
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def version() -> str:
+    return lib().qmv_version().decode()
+
+
+# ---------------------------------------------------------------- encoders
+
+def encode_fp4(W: torch.Tensor, stream=None):
+    """W float32 [N, K] -> (codes uint8 [N, K/2], scales uint8 [N, K/32])."""
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, K // 32), dtype=torch.uint8, device=W.device)
+    _call("qmv_encode_fp4", _ptr(W), N, K, _ptr(codes), _ptr(scales), _stream(stream))
+    return codes, scales
+
+
+def _encode_int(name, W, clips, bits, stream):
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    c = (ctypes.c_float * len(clips))(*[float(v) for v in clips])
+    codes = torch.empty((N, K * bits // 8), dtype=torch.uint8 if bits == 4 else torch.int8, device=W.device)
+    scales = torch.empty((N, K // 32), dtype=torch.float16, device=W.device)
+    _call(name, _ptr(W), N, K, c, len(clips), _ptr(codes), _ptr(scales), _stream(stream))
+    return codes, scales
+
+
+def encode_int4(W: torch.Tensor, clips=INT4_CLIPS, stream=None):
+    """-> (codes uint8 [N, K/2] (q + 8 nibbles), scales float16 [N, K/32])."""
+    return _encode_int("qmv_encode_int4", W, clips, 4, stream)
+
+
+def encode_int8(W: torch.Tensor, clips=INT8_CLIPS, stream=None):
+    """-> (codes int8 [N, K], scales float16 [N, K/32])."""
+    return _encode_int("qmv_encode_int8", W, clips, 8, stream)
+
+
+# ---------------------------------------------------------------- matvec
+
+_AUX = {FMT_FP4: torch.uint8, FMT_INT4: torch.float16, FMT_INT4KM: torch.float16, FMT_INT8: torch.float16}
+_CODES = {FMT_FP4: torch.uint8, FMT_INT4: torch.uint8, FMT_INT4KM: torch.uint8, FMT_INT8: torch.int8}
+_ENTRY = {FMT_FP4: "qmv_matvec_fp4", FMT_INT4: "qmv_matvec_int4", FMT_INT4KM: "qmv_matvec_int4km",
+          FMT_INT8: "qmv_matvec_int8"}
+
+
+def _nk(fmt, codes):
+    N = codes.shape[-2]
+    K = codes.shape[-1] * (1 if fmt == FMT_INT8 else 2)
+    return N, K
+
+
+def matvec(fmt: int, codes: torch.Tensor, aux: torch.Tensor, x: torch.Tensor, out=None, stream=None):
+    """y float32 [B, N] = x Wdq^T for x float16 [B, K] (or [K] -> [N])."""
+    _need(codes, "codes", _CODES[fmt])
+    _need(aux, "scales/lut", _AUX[fmt])
+    N, K = _nk(fmt, codes)
+    squeeze = x.dim() == 1
+    xx = x.unsqueeze(0) if squeeze else x
+    _need(xx, "x", torch.float16)
+    B = xx.shape[0]
+    if xx.shape[1] != K:
+        raise ValueError(f"x has {xx.shape[1]} features, weights have {K}")
+    if out is None:
+        out = torch.empty((B, N), dtype=torch.float32, device=codes.device)
+    _need(out, "out", torch.float32, (B, N))
+    _call(_ENTRY[fmt], _ptr(codes), _ptr(aux), _ptr(xx), B, N, K, _ptr(out), _stream(stream))
+    return out[0] if squeeze else out
+
+
+def matvec_fp4(codes, scales, x, out=None, stream=None):
+    return matvec(FMT_FP4, codes, scales, x, out, stream)
+
+
+def matvec_int4(codes, scales, x, out=None, stream=None):
+    return matvec(FMT_INT4, codes, scales, x, out, stream)
+
+
+def matvec_int4km(idx, lut, x, out=None, stream=None):
+    return matvec(FMT_INT4KM, idx, lut, x, out, stream)
+
+
+def matvec_int8(codes, scales, x, out=None, stream=None):
+    return matvec(FMT_INT8, codes, scales, x, out, stream)
+
+
+def gather_matvec(fmt: int, codes_stack: torch.Tensor, aux_stack: torch.Tensor, expert_ids: torch.Tensor,
+                  x: torch.Tensor, x_per_slot: bool = False, out=None, stream=None):
+    """y float32 [B, topk, N]; codes_stack [E, N, ...], aux_stack [E, N, ...],
+    expert_ids int32 [B, topk], x float16 [B, K] or [B, topk, K]."""
+    _need(codes_stack, "codes_stack", _CODES[fmt])
+    _need(aux_stack, "aux_stack", _AUX[fmt])
+    _need(expert_ids, "expert_ids", torch.int32)
+    _need(x, "x", torch.float16)
+    E = codes_stack.shape[0]
+    N, K = _nk(fmt, codes_stack)
+    B, topk = expert_ids.shape
+    want = (B, topk, K) if x_per_slot else (B, K)
+    if tuple(x.shape) != want:
+        raise ValueError(f"x must have shape {want}, got {tuple(x.shape)}")
+    if out is None:
+        out = torch.empty((B, topk, N), dtype=torch.float32, device=codes_stack.device)
+    _need(out, "out", torch.float32, (B, topk, N))
+    _call("qmv_gather_matvec", fmt, _ptr(codes_stack), _ptr(aux_stack), E, N, K, _ptr(expert_ids), B, topk,
+          _ptr(x), int(bool(x_per_slot)), _ptr(out), _stream(stream))
+    return out
+
+
+def dequant(fmt: int, codes: torch.Tensor, aux: torch.Tensor, stream=None) -> torch.Tensor:
+    """Exact float32 [N, K] dequantized weights (test support)."""
+    _need(codes, "codes", _CODES[fmt])
+    _need(aux, "aux", _AUX[fmt])
+    N, K = _nk(fmt, codes)
+    out = torch.empty((N, K), dtype=torch.float32, device=codes.device)
+    _call("qmv_dequant", fmt, _ptr(codes), _ptr(aux), N, K, _ptr(out), _stream(stream))
+    return out
+
+
+def status_fetch(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status flags."""
+    flags = ctypes.c_uint32(0)
+    rc = lib().qmv_status_fetch(_stream(stream), ctypes.byref(flags))
+    if rc not in (OK, ERR_DATA):
+        raise QmvError(rc, lib().qmv_last_error().decode())
+    return int(flags.value)

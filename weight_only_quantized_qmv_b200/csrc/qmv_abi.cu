@@ -1,0 +1,241 @@
+// qmv_abi.cu -- the extern "C" entry points of libqmv (declared in qmv.h):
+// host-side argument validation, the per-device status word, last-error text
+// and the kernel launches on the caller's stream.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "qmv_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+qmv_status fail(qmv_status code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+qmv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(QMV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Device status word: one per device (a __device__ variable exists once per
+// device that loads the module).  Kernels OR QMV_FLAG_* bits into it.
+__device__ uint32_t g_status_word;
+
+constexpr int kMaxDevices = 64;
+uint32_t* g_status_ptr[kMaxDevices] = {nullptr};
+int g_num_sms[kMaxDevices] = {0};
+
+// Per-device set-up (current device): the status word's device address and
+// the SM count.  Runs on a device's first call.
+qmv_status device_ctx(uint32_t** status, int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(QMV_ERR_UNSUPPORTED, "device %d out of range", dev);
+  if (!g_status_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    g_num_sms[dev] = sms;
+    g_status_ptr[dev] = static_cast<uint32_t*>(ptr);
+  }
+  *status = g_status_ptr[dev];
+  *num_sms = g_num_sms[dev];
+  return QMV_OK;
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qmv_status check_ptr(const void* p, const char* name) {
+  if (!p) return fail(QMV_ERR_ARG, "%s is null", name);
+  if (!aligned16(p)) return fail(QMV_ERR_ARG, "%s is not 16-byte aligned", name);
+  return QMV_OK;
+}
+
+qmv_status check_shape(int64_t N, int64_t K) {
+  if (N < 1) return fail(QMV_ERR_SHAPE, "N must be >= 1 (got %lld)", (long long)N);
+  if (K < 32 || K % 32 != 0)
+    return fail(QMV_ERR_SHAPE, "K must be a positive multiple of the 32-element block (got %lld)", (long long)K);
+  if (K > (int64_t)1 << 30 || N > (int64_t)1 << 40) return fail(QMV_ERR_SHAPE, "shape too large");
+  return QMV_OK;
+}
+
+#define QMV_TRY(x)                  \
+  do {                              \
+    const qmv_status _s = (x);      \
+    if (_s != QMV_OK) return _s;    \
+  } while (0)
+
+qmv_status encode_int(int qmax, const float* W, int64_t N, int64_t K, const float* clips, int n_clips,
+                      uint8_t* codes, uint16_t* scales, void* stream) {
+  QMV_TRY(check_ptr(W, "W"));
+  QMV_TRY(check_ptr(codes, "codes"));
+  if (!scales || (reinterpret_cast<uintptr_t>(scales) & 1u)) return fail(QMV_ERR_ARG, "scales null or misaligned");
+  QMV_TRY(check_shape(N, K));
+  if (!clips || n_clips < 1 || n_clips > 16) return fail(QMV_ERR_ARG, "clip list must hold 1..16 values");
+  qmv::ClipList cl{};
+  for (int i = 0; i < n_clips; ++i) {
+    if (!(clips[i] > 0.0f) || clips[i] != clips[i]) return fail(QMV_ERR_ARG, "clip %d is not a positive number", i);
+    cl.v[i] = clips[i];
+  }
+  cl.n = n_clips;
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  cudaError_t e = qmv::launch_encode_int(qmax, W, N, K, cl, codes, scales, st, sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "encode launch");
+  return QMV_OK;
+}
+
+qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
+                         int64_t K, float* y, void* stream, bool gather, int E, const int32_t* ids, int topk,
+                         int x_per_slot) {
+  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
+  QMV_TRY(check_ptr(codes, "codes"));
+  if (!aux) return fail(QMV_ERR_ARG, "scales/lut is null");
+  // the staged scale block copies handle any byte alignment; the palette and
+  // row-aligned scale copies need 16-byte alignment
+  if (fmt == QMV_FMT_INT4KM) QMV_TRY(check_ptr(aux, "lut"));
+  if (fmt != QMV_FMT_FP4 && (reinterpret_cast<uintptr_t>(aux) & 1u)) return fail(QMV_ERR_ARG, "fp16 scales misaligned");
+  QMV_TRY(check_ptr(x, "x"));
+  if (!y || (reinterpret_cast<uintptr_t>(y) & 3u)) return fail(QMV_ERR_ARG, "y null or misaligned");
+  QMV_TRY(check_shape(N, K));
+  if (B < 1 || B > 16) return fail(QMV_ERR_UNSUPPORTED, "B must be in [1, 16] (got %d)", B);
+  qmv::MvParams p{};
+  p.codes = static_cast<const uint8_t*>(codes);
+  p.aux = static_cast<const uint8_t*>(aux);
+  p.x = x;
+  p.y = y;
+  p.N = N;
+  p.K = K;
+  p.B = B;
+  p.gather = gather ? 1 : 0;
+  if (gather) {
+    if (E < 1) return fail(QMV_ERR_SHAPE, "E must be >= 1");
+    if (topk < 1 || topk > 16) return fail(QMV_ERR_UNSUPPORTED, "topk must be in [1, 16] (got %d)", topk);
+    if (!ids || (reinterpret_cast<uintptr_t>(ids) & 3u)) return fail(QMV_ERR_ARG, "expert_ids null or misaligned");
+    if (x_per_slot != 0 && x_per_slot != 1) return fail(QMV_ERR_ARG, "x_per_slot must be 0 or 1");
+    p.ids = ids;
+    p.E = E;
+    p.topk = topk;
+    p.x_per_slot = x_per_slot;
+  } else {
+    p.E = 1;
+    p.topk = 1;
+  }
+  if (!qmv::plan_matvec(fmt, p))
+    return fail(QMV_ERR_UNSUPPORTED, "activations (%d rows x %lld) do not fit the on-chip staging", p.n_xrows,
+                (long long)K);
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  p.status = st;
+  cudaError_t e = qmv::launch_matvec(fmt, p, sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "matvec launch");
+  return QMV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qmv_status qmv_encode_fp4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* scales, void* stream) {
+  QMV_TRY(check_ptr(W, "W"));
+  QMV_TRY(check_ptr(codes, "codes"));
+  if (!scales) return fail(QMV_ERR_ARG, "scales is null");
+  QMV_TRY(check_shape(N, K));
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  cudaError_t e = qmv::launch_encode_fp4(W, N, K, codes, scales, st, sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "encode_fp4 launch");
+  return QMV_OK;
+}
+
+qmv_status qmv_encode_int4(const float* W, int64_t N, int64_t K, const float* clips, int n_clips,
+                           uint8_t* codes, uint16_t* scales, void* stream) {
+  return encode_int(7, W, N, K, clips, n_clips, codes, scales, stream);
+}
+
+qmv_status qmv_encode_int8(const float* W, int64_t N, int64_t K, const float* clips, int n_clips,
+                           int8_t* codes, uint16_t* scales, void* stream) {
+  return encode_int(127, W, N, K, clips, n_clips, reinterpret_cast<uint8_t*>(codes), scales, stream);
+}
+
+qmv_status qmv_matvec_fp4(const uint8_t* codes, const uint8_t* scales, const uint16_t* x, int B, int64_t N,
+                          int64_t K, float* y, void* stream) {
+  return matvec_common(QMV_FMT_FP4, codes, scales, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
+}
+
+qmv_status qmv_matvec_int4(const uint8_t* codes, const uint16_t* scales, const uint16_t* x, int B, int64_t N,
+                           int64_t K, float* y, void* stream) {
+  return matvec_common(QMV_FMT_INT4, codes, scales, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
+}
+
+qmv_status qmv_matvec_int4km(const uint8_t* idx, const uint16_t* lut, const uint16_t* x, int B, int64_t N,
+                             int64_t K, float* y, void* stream) {
+  return matvec_common(QMV_FMT_INT4KM, idx, lut, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
+}
+
+qmv_status qmv_matvec_int8(const int8_t* codes, const uint16_t* scales, const uint16_t* x, int B, int64_t N,
+                           int64_t K, float* y, void* stream) {
+  return matvec_common(QMV_FMT_INT8, codes, scales, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
+}
+
+qmv_status qmv_gather_matvec(int fmt, const void* codes_stack, const void* aux_stack, int E, int64_t N, int64_t K,
+                             const int32_t* expert_ids, int B, int topk, const uint16_t* x, int x_per_slot,
+                             float* y, void* stream) {
+  if (B < 1 || B > 16) return fail(QMV_ERR_UNSUPPORTED, "B must be in [1, 16] (got %d)", B);
+  return matvec_common(fmt, codes_stack, aux_stack, x, B, N, K, y, stream, true, E, expert_ids, topk, x_per_slot);
+}
+
+qmv_status qmv_dequant(int fmt, const void* codes, const void* aux, int64_t N, int64_t K, float* Wdq, void* stream) {
+  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
+  QMV_TRY(check_ptr(codes, "codes"));
+  if (!aux) return fail(QMV_ERR_ARG, "aux is null");
+  if (fmt == QMV_FMT_INT4KM) QMV_TRY(check_ptr(aux, "lut"));
+  if (fmt != QMV_FMT_FP4 && (reinterpret_cast<uintptr_t>(aux) & 1u)) return fail(QMV_ERR_ARG, "fp16 scales misaligned");
+  QMV_TRY(check_ptr(Wdq, "Wdq"));
+  QMV_TRY(check_shape(N, K));
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  cudaError_t e = qmv::launch_dequant(fmt, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(aux), N, K,
+                                      Wdq, sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+  return QMV_OK;
+}
+
+qmv_status qmv_status_fetch(void* stream, uint32_t* flags) {
+  if (!flags) return fail(QMV_ERR_ARG, "flags is null");
+  *flags = 0;
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  const uint32_t zero = 0;
+  e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  *flags = v;
+  if (v) return fail(QMV_ERR_DATA, "device status flags 0x%x", v);
+  return QMV_OK;
+}
+
+const char* qmv_last_error(void) { return g_err; }
+
+const char* qmv_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,294 @@
+// qmv_device.cuh -- device helpers shared by the libqmv kernels (sm_100a):
+// mbarrier pipeline primitives with bounded waits, 1-D bulk async copies,
+// the m16n8k16 tensor-core step, and the per-format decoders that turn packed
+// weight codes into exact fp16 tensor-core operands.
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "qmv_internal.h"
+
+namespace qmv {
+
+// ---------------------------------------------------------------------------
+// Timers, status and pipeline waits
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of `bar` with parity `parity` to complete.  Bounded: after
+// kWaitLimitNs of wall time (or, when respect_abort, once another warp raised
+// `abort`) it records QMV_FLAG_TIMEOUT, raises `abort` and returns false
+// instead of spinning on.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s; a healthy wait is microseconds
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status, bool respect_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (respect_abort && *abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, QMV_FLAG_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// 1-D bulk async copy global -> shared (TMA engine, no tensor map), counted on
+// the mbarrier's transaction bytes.  dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (bulk copy) accesses of the same bytes.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Loads
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core step: D(16x8, f32) = A(16x16, f16, row) * B(16x8, f16, col) + C
+// Fragment of lane l (g = l/4, t = l%4):
+//   a0 = (row g,   k 2t,2t+1)   a1 = (row g+8, k 2t,2t+1)
+//   a2 = (row g,   k 2t+8,2t+9) a3 = (row g+8, k 2t+8,2t+9)
+//   b0 = (k 2t,2t+1; col g)     b1 = (k 2t+8,2t+9; col g)
+//   d0,d1 = (row g, cols 2t,2t+1)   d2,d3 = (row g+8, cols 2t,2t+1)
+// Products of fp16 operands are exact in fp32; the sum accumulates in fp32.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------------------
+// Byte/bit helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {  // (a & b) | c
+  uint32_t r;  // truth table: (0xF0 & 0xCC) | 0xAA = 0xEA
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t lop3_mux(uint32_t a, uint32_t b, uint32_t m) {  // m ? b : a, bitwise
+  uint32_t r;
+  // truth table over (a, b, m) = (0xF0, 0xCC, 0xAA): (m & b) | (~m & a) = 0xD8
+  asm("lop3.b32 %0, %1, %2, %3, 0xD8;" : "=r"(r) : "r"(a), "r"(b), "r"(m));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// byte `i` (0..3, compile-time) of w, two E2M1 codes -> f16x2 (low nibble in
+// the low half).  Exact: every E2M1 value is an fp16 value.
+template <int I>
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t w) {
+  uint32_t r;
+  if constexpr (I == 0)
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b0;\n}" : "=r"(r) : "r"(w));
+  else if constexpr (I == 1)
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b1;\n}" : "=r"(r) : "r"(w));
+  else if constexpr (I == 2)
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b2;\n}" : "=r"(r) : "r"(w));
+  else
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b3;\n}" : "=r"(r) : "r"(w));
+  return r;
+}
+
+// Eight non-negative floats -> four bytes of E2M1 code pairs (v[2j] in the low
+// nibble of byte j), round to nearest even, saturating at 6 (hardware
+// conversion; its first source operand fills the high nibble).
+__device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float (&v)[8]) {
+  uint32_t r;
+  asm("{\n .reg .b8 c0, c1, c2, c3;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n"
+      " mov.b32 %0, {c0, c1, c2, c3};\n}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+// e8m0 byte -> float 2^(byte - 127), exact (byte 0 is the subnormal 2^-127).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t byte) {
+  uint32_t bits = byte << 23;
+  return __uint_as_float(bits > 0x00400000u ? bits : 0x00400000u);
+}
+
+// ---------------------------------------------------------------------------
+// Per-format decoders: one 32-bit word of a row's codes (8 weights, k = 8t..8t+7
+// of one 32-block for the 4-bit formats; 4 weights for int8) -> fp16 operands
+// for the two m16n8k16 steps of that block.  The k order the decoder emits is
+// the order the activations are staged in shared memory (kXPerm below).
+// ---------------------------------------------------------------------------
+
+// FP4: pairs (k0,k1) (k2,k3) for step 0, (k4,k5) (k6,k7) for step 1.
+struct DecFp4 {
+  __device__ __forceinline__ static void run(uint32_t w, uint32_t& s0lo, uint32_t& s0hi, uint32_t& s1lo,
+                                             uint32_t& s1hi) {
+    s0lo = e2m1x2_to_f16x2<0>(w);
+    s0hi = e2m1x2_to_f16x2<1>(w);
+    s1lo = e2m1x2_to_f16x2<2>(w);
+    s1hi = e2m1x2_to_f16x2<3>(w);
+  }
+};
+
+// INT4 (nibble = q + 8): 0x6400 | n is the fp16 1024 + n; subtracting 1032
+// gives q exactly.  Nibbles at bits 4..7 of each half come out as 1024 + 16 n
+// and are mapped with an exact fma: (1024 + 16 n) / 16 - 72 = n - 8.
+// Emitted pairs: (k0,k4) (k1,k5) for step 0 and (k2,k6) (k3,k7) for step 1.
+struct DecInt4 {
+  __device__ __forceinline__ static void run(uint32_t w, uint32_t& s0lo, uint32_t& s0hi, uint32_t& s1lo,
+                                             uint32_t& s1hi) {
+    const uint32_t kMagic = 0x64006400u;  // fp16x2 (1024, 1024)
+    const uint32_t kSub = 0x64086408u;    // fp16x2 (1032, 1032)
+    const uint32_t kSixteenth = 0x2C002C00u;  // fp16x2 (1/16, 1/16)
+    const uint32_t kNeg72 = 0xD480D480u;  // fp16x2 (-72, -72)
+    const uint32_t w8 = w >> 8;
+    s0lo = hsub2_u32(lop3_and_or(w, 0x000F000Fu, kMagic), kSub);
+    s0hi = hfma2_u32(lop3_and_or(w, 0x00F000F0u, kMagic), kSixteenth, kNeg72);
+    s1lo = hsub2_u32(lop3_and_or(w8, 0x000F000Fu, kMagic), kSub);
+    s1hi = hfma2_u32(lop3_and_or(w8, 0x00F000F0u, kMagic), kSixteenth, kNeg72);
+  }
+};
+
+// INT8: one word holds 4 weights (k0..k3).  Bias each byte by 128, splice it
+// under 0x64 (fp16 1024 + u), subtract 1152: exact q.  Pairs (k0,k1) (k2,k3).
+__device__ __forceinline__ void dec_int8_word(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint32_t kSub = 0x64806480u;  // fp16x2 (1152, 1152)
+  lo = hsub2_u32(prmt(u, 0x64646464u, 0x5140u), kSub);
+  hi = hsub2_u32(prmt(u, 0x64646464u, 0x5342u), kSub);
+}
+
+// INT4KM: 16-entry fp16 palette of one row held as byte tables in registers:
+// lo[0..3] = low bytes of entries 0..15, hi[0..3] = high bytes.  Four indices
+// (one per byte lane of `sel`, bit 3 in `msk`) look up 4 bytes per table with
+// two byte-permutes over the 8-entry halves and a bitwise select on bit 3.
+struct Palette {
+  uint32_t lo0, lo1, lo2, lo3, hi0, hi1, hi2, hi3;
+};
+
+__device__ __forceinline__ Palette palette_from_words(const uint32_t (&e)[8]) {
+  // e[j] = entries 2j (low half) and 2j+1 (high half)
+  Palette p;
+  p.lo0 = prmt(e[0], e[1], 0x6420u);
+  p.lo1 = prmt(e[2], e[3], 0x6420u);
+  p.lo2 = prmt(e[4], e[5], 0x6420u);
+  p.lo3 = prmt(e[6], e[7], 0x6420u);
+  p.hi0 = prmt(e[0], e[1], 0x7531u);
+  p.hi1 = prmt(e[2], e[3], 0x7531u);
+  p.hi2 = prmt(e[4], e[5], 0x7531u);
+  p.hi3 = prmt(e[6], e[7], 0x7531u);
+  return p;
+}
+
+// w: 8 nibbles (k0..k7).  Emits (k0,k1) (k2,k3) (k4,k5) (k6,k7) as f16x2.
+__device__ __forceinline__ void dec_int4km(const Palette& p, uint32_t w, uint32_t& s0lo, uint32_t& s0hi,
+                                           uint32_t& s1lo, uint32_t& s1hi) {
+  const uint32_t w4 = w << 4;
+  const uint32_t wh = w >> 16;
+  const uint32_t sel0 = w & 0x7777u;   // nibbles 0..3, bit 3 cleared
+  const uint32_t sel1 = wh & 0x7777u;  // nibbles 4..7
+  const uint32_t m0 = prmt(w4, w, 0xD9C8u);  // byte i = 0xFF iff bit 3 of nibble i
+  const uint32_t m1 = prmt(w4, w, 0xFBEAu);  // nibbles 4..7
+  const uint32_t lo_a = lop3_mux(prmt(p.lo0, p.lo1, sel0), prmt(p.lo2, p.lo3, sel0), m0);
+  const uint32_t hi_a = lop3_mux(prmt(p.hi0, p.hi1, sel0), prmt(p.hi2, p.hi3, sel0), m0);
+  const uint32_t lo_b = lop3_mux(prmt(p.lo0, p.lo1, sel1), prmt(p.lo2, p.lo3, sel1), m1);
+  const uint32_t hi_b = lop3_mux(prmt(p.hi0, p.hi1, sel1), prmt(p.hi2, p.hi3, sel1), m1);
+  s0lo = prmt(lo_a, hi_a, 0x5140u);
+  s0hi = prmt(lo_a, hi_a, 0x7362u);
+  s1lo = prmt(lo_b, hi_b, 0x5140u);
+  s1hi = prmt(lo_b, hi_b, 0x7362u);
+}
+
+}  // namespace qmv

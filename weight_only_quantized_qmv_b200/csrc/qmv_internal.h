@@ -1,0 +1,87 @@
+// qmv_internal.h -- declarations shared by the libqmv translation units:
+// kernel parameter blocks, per-format geometry and the launchers the C ABI
+// (qmv_abi.cu) calls after validating its arguments.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "qmv.h"
+
+namespace qmv {
+
+// ---- fused dequant-matvec / gather kernel -----------------------------------
+constexpr int kConsumerWarps = 8;                    // warps that decode + multiply
+constexpr int kThreads = 32 * (1 + kConsumerWarps);  // + one producer warp
+constexpr int kTileRows = 16;                        // rows per tile: one m16 step
+constexpr int kMaxCols = 16;                         // activation columns per pass
+constexpr int kMaxStages = 8;
+constexpr int kMaxPairs = 256;                       // B * topk upper bound (16 * 16)
+constexpr int kSmemLimit = 227 * 1024;               // per-block opt-in maximum on sm_100
+
+// Aux (scale / palette) staging mode of a launch.
+enum AuxMode : int {
+  kAuxRows = 0,   // per-row bulk copies of the chunk's scale segment (aligned shapes)
+  kAuxBlock = 1,  // the tile's whole scale block, every stage (any K % 32 == 0)
+  kAuxLut = 2     // the tile's 16 x 16 fp16 palette, first chunk only
+};
+
+struct MvParams {
+  const uint8_t* codes;   // codes of expert 0 (dense: the matrix)
+  const uint8_t* aux;     // scales / palette of expert 0
+  const uint16_t* x;      // activations, fp16 bits
+  float* y;               // outputs
+  const int32_t* ids;     // gather: expert ids [B * topk]
+  uint32_t* status;       // library device status word
+  int64_t N, K;
+  int64_t code_row_bytes;  // bytes of codes per weight row
+  int64_t aux_row_bytes;   // bytes of scales per row (palette: 32)
+  int64_t expert_code_bytes, expert_aux_bytes;
+  int64_t tiles;           // ceil(N / 16)
+  int B;                   // dense: activation rows; gather: tokens
+  int topk, E, x_per_slot, gather;
+  int KC, nchunks;         // in-features per pipeline stage, stages per tile
+  int RS;                  // shared-memory bytes per staged code row
+  int AS;                  // shared-memory bytes per staged scale row (kAuxRows)
+  int aux_mode;
+  int stages, stage_bytes, aux_off;  // ring geometry; aux_off: scale region inside a stage
+  int XS;                  // shared-memory bytes per staged activation row
+  int n_xrows;             // activation rows staged
+  int off_red, off_x, off_stage;  // dynamic shared-memory offsets
+  int smem_bytes;
+};
+
+// Per-format constants (bits per weight, scale bytes per 32-block).
+struct FmtInfo {
+  int bits, scale_bytes, kc_max;
+  bool lut;
+};
+inline FmtInfo fmt_info(int fmt) {
+  switch (fmt) {
+    case QMV_FMT_FP4: return {4, 1, 2048, false};
+    case QMV_FMT_INT4: return {4, 2, 2048, false};
+    case QMV_FMT_INT4KM: return {4, 0, 2048, true};
+    default: return {8, 2, 1024, false};
+  }
+}
+
+// Fills the geometry of `p` (shapes and pointers already set).  Returns false
+// when the activations plus a two-stage ring do not fit in shared memory.
+bool plan_matvec(int fmt, MvParams& p);
+
+cudaError_t launch_matvec(int fmt, const MvParams& p, int num_sms, cudaStream_t stream);
+
+// ---- encoders / dequant ------------------------------------------------------
+struct ClipList {
+  float v[16];
+  int n;
+};
+
+cudaError_t launch_encode_fp4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* scales,
+                              uint32_t* status, int num_sms, cudaStream_t stream);
+cudaError_t launch_encode_int(int qmax, const float* W, int64_t N, int64_t K, const ClipList& clips,
+                              uint8_t* codes, uint16_t* scales, uint32_t* status, int num_sms,
+                              cudaStream_t stream);
+cudaError_t launch_dequant(int fmt, const uint8_t* codes, const uint8_t* aux, int64_t N, int64_t K, float* Wdq,
+                           int num_sms, cudaStream_t stream);
+
+}  // namespace qmv

@@ -74,7 +74,6 @@ enum {
 #define QMV_FLAG_NONFINITE 0x1u      /* encode: a block held Inf/NaN (block written as zeros) */
 #define QMV_FLAG_SCALE_OVERFLOW 0x2u /* encode: no clip gave a finite fp16 scale (block zeroed) */
 #define QMV_FLAG_BAD_EXPERT 0x4u     /* gather: expert id outside [0, E) (that output row zeroed) */
-#define QMV_FLAG_TIMEOUT 0x8u        /* a pipeline wait gave up (internal fault; outputs invalid) */
 
 /* ---------------------------------------------------------------------
  * Encoders (offline conversion; [P1] sec. 1-2).

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libqmv.so")
 
 FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8 = 0, 1, 2, 3
 FMT_NAMES = {FMT_FP4: "fp4", FMT_INT4: "int4", FMT_INT4KM: "int4km", FMT_INT8: "int8"}
-FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT, FLAG_TIMEOUT = 1, 2, 4, 8
+FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT = 1, 2, 4
 OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_DATA, ERR_CUDA = 0, -1, -2, -3, -4, -5
 
 # Clip lists of the workloads: int4 searches 1.00, 0.95, ..., 0.50 (float32

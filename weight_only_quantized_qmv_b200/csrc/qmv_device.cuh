@@ -1,7 +1,6 @@
 // qmv_device.cuh -- device helpers shared by the libqmv kernels (sm_100a):
-// mbarrier pipeline primitives with bounded waits, 1-D bulk async copies,
-// the m16n8k16 tensor-core step, and the per-format decoders that turn packed
-// weight codes into exact fp16 tensor-core operands.
+// shared-memory loads, the m16n8k16 tensor-core step, and the per-format
+// decoders that turn packed weight codes into exact fp16 tensor-core operands.
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -10,86 +9,8 @@
 
 namespace qmv {
 
-// ---------------------------------------------------------------------------
-// Timers, status and pipeline waits
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_fence_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase of `bar` with parity `parity` to complete.  Bounded: after
-// kWaitLimitNs of wall time (or, when respect_abort, once another warp raised
-// `abort`) it records QMV_FLAG_TIMEOUT, raises `abort` and returns false
-// instead of spinning on.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s; a healthy wait is microseconds
-
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status, bool respect_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0) {
-      if (respect_abort && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(status, QMV_FLAG_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
-// 1-D bulk async copy global -> shared (TMA engine, no tensor map), counted on
-// the mbarrier's transaction bytes.  dst, src and bytes must be multiples of 16.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
-// Orders this thread's generic-proxy shared-memory writes before later
-// async-proxy (bulk copy) accesses of the same bytes.
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -211,16 +132,59 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t byte) {
 // the order the activations are staged in shared memory (kXPerm below).
 // ---------------------------------------------------------------------------
 
-// FP4: pairs (k0,k1) (k2,k3) for step 0, (k4,k5) (k6,k7) for step 1.
-struct DecFp4 {
-  __device__ __forceinline__ static void run(uint32_t w, uint32_t& s0lo, uint32_t& s0hi, uint32_t& s1lo,
-                                             uint32_t& s1hi) {
-    s0lo = e2m1x2_to_f16x2<0>(w);
-    s0hi = e2m1x2_to_f16x2<1>(w);
-    s1lo = e2m1x2_to_f16x2<2>(w);
-    s1hi = e2m1x2_to_f16x2<3>(w);
+// A 32-bit constant the compiler cannot fold, so that multiplies by powers of
+// two stay integer multiply-adds (the FMA pipe) instead of turning into
+// shifts and masks on the half-rate integer ALU pipe.
+__device__ __forceinline__ uint32_t opaque(uint32_t c) {
+  uint32_t r;
+  asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(c));
+  return r;
+}
+
+// Multipliers the decoders use to move bytes with integer multiply-high.
+struct Mul {
+  uint32_t p8, p16, p24, p4, e23;  // 2^8, 2^16, 2^24, 2^4, 2^23
+  __device__ __forceinline__ static Mul make() {
+    Mul m;
+    m.p8 = opaque(1u << 8);
+    m.p16 = opaque(1u << 16);
+    m.p24 = opaque(1u << 24);
+    m.p4 = opaque(1u << 4);
+    m.e23 = opaque(1u << 23);
+    return m;
   }
 };
+
+// two E2M1 codes in the LOW byte of r -> f16x2 (low nibble in the low half)
+__device__ __forceinline__ uint32_t e2m1x2_lo_to_f16x2(uint32_t r) {
+  uint32_t o;
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b0;\n}" : "=r"(o) : "r"(r));
+  return o;
+}
+
+// FP4: pairs (k0,k1) (k2,k3) for step 0, (k4,k5) (k6,k7) for step 1.  The
+// upper bytes are brought down with multiply-high (w >> 8, w >> 16, w >> 24).
+struct DecFp4 {
+  __device__ __forceinline__ static void run(uint32_t w, uint32_t& s0lo, uint32_t& s0hi, uint32_t& s1lo,
+                                             uint32_t& s1hi, const Mul& m) {
+    s0lo = e2m1x2_lo_to_f16x2(w);
+    s0hi = e2m1x2_lo_to_f16x2(__umulhi(w, m.p24));
+    s1lo = e2m1x2_lo_to_f16x2(__umulhi(w, m.p16));
+    s1hi = e2m1x2_lo_to_f16x2(__umulhi(w, m.p8));
+  }
+};
+
+// Byte i (0..3) of u -> float 2^(byte - 126) (exact, always normal): the
+// e8m0 scale times 2.  Callers fold the factor 1/2 into their outputs.
+template <int I>
+__device__ __forceinline__ float e8m0_x2_to_f32(uint32_t u, const Mul& m) {
+  uint32_t t = u;
+  if constexpr (I == 0) t = u * m.p24;
+  if constexpr (I == 1) t = u * m.p16;
+  if constexpr (I == 2) t = u * m.p8;
+  const uint32_t byte = __umulhi(t, m.p8);  // t >> 24
+  return __uint_as_float(byte * m.e23 + m.e23);
+}
 
 // INT4 (nibble = q + 8): 0x6400 | n is the fp16 1024 + n; subtracting 1032
 // gives q exactly.  Nibbles at bits 4..7 of each half come out as 1024 + 16 n
@@ -228,12 +192,12 @@ struct DecFp4 {
 // Emitted pairs: (k0,k4) (k1,k5) for step 0 and (k2,k6) (k3,k7) for step 1.
 struct DecInt4 {
   __device__ __forceinline__ static void run(uint32_t w, uint32_t& s0lo, uint32_t& s0hi, uint32_t& s1lo,
-                                             uint32_t& s1hi) {
+                                             uint32_t& s1hi, const Mul& m) {
     const uint32_t kMagic = 0x64006400u;  // fp16x2 (1024, 1024)
     const uint32_t kSub = 0x64086408u;    // fp16x2 (1032, 1032)
     const uint32_t kSixteenth = 0x2C002C00u;  // fp16x2 (1/16, 1/16)
     const uint32_t kNeg72 = 0xD480D480u;  // fp16x2 (-72, -72)
-    const uint32_t w8 = w >> 8;
+    const uint32_t w8 = __umulhi(w, m.p24);  // w >> 8
     s0lo = hsub2_u32(lop3_and_or(w, 0x000F000Fu, kMagic), kSub);
     s0hi = hfma2_u32(lop3_and_or(w, 0x00F000F0u, kMagic), kSixteenth, kNeg72);
     s1lo = hsub2_u32(lop3_and_or(w8, 0x000F000Fu, kMagic), kSub);
@@ -274,9 +238,9 @@ __device__ __forceinline__ Palette palette_from_words(const uint32_t (&e)[8]) {
 
 // w: 8 nibbles (k0..k7).  Emits (k0,k1) (k2,k3) (k4,k5) (k6,k7) as f16x2.
 __device__ __forceinline__ void dec_int4km(const Palette& p, uint32_t w, uint32_t& s0lo, uint32_t& s0hi,
-                                           uint32_t& s1lo, uint32_t& s1hi) {
-  const uint32_t w4 = w << 4;
-  const uint32_t wh = w >> 16;
+                                           uint32_t& s1lo, uint32_t& s1hi, const Mul& m) {
+  const uint32_t w4 = w * m.p4;           // w << 4
+  const uint32_t wh = __umulhi(w, m.p16);  // w >> 16
   const uint32_t sel0 = w & 0x7777u;   // nibbles 0..3, bit 3 cleared
   const uint32_t sel1 = wh & 0x7777u;  // nibbles 4..7
   const uint32_t m0 = prmt(w4, w, 0xD9C8u);  // byte i = 0xFF iff bit 3 of nibble i

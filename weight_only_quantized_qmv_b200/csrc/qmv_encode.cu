@@ -184,6 +184,7 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
       const uint4 v = *reinterpret_cast<const uint4*>(codes + blk * 16);
       const uint32_t words[4] = {v.x, v.y, v.z, v.w};
       Palette pal;
+      const Mul mul = Mul::make();
       if constexpr (FMT == QMV_FMT_INT4KM) {
         const uint4* L = reinterpret_cast<const uint4*>(aux + n * 32);
         const uint4 a = L[0], c = L[1];
@@ -195,19 +196,19 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
         uint32_t s0lo, s0hi, s1lo, s1hi;
         float* o = out + 8 * q;
         if constexpr (FMT == QMV_FMT_FP4) {
-          DecFp4::run(words[q], s0lo, s0hi, s1lo, s1hi);  // (k0,k1) (k2,k3) (k4,k5) (k6,k7)
+          DecFp4::run(words[q], s0lo, s0hi, s1lo, s1hi, mul);  // (k0,k1) (k2,k3) (k4,k5) (k6,k7)
           f16x2_to_f32(s0lo, o[0], o[1]);
           f16x2_to_f32(s0hi, o[2], o[3]);
           f16x2_to_f32(s1lo, o[4], o[5]);
           f16x2_to_f32(s1hi, o[6], o[7]);
         } else if constexpr (FMT == QMV_FMT_INT4) {
-          DecInt4::run(words[q], s0lo, s0hi, s1lo, s1hi);  // (k0,k4) (k1,k5) (k2,k6) (k3,k7)
+          DecInt4::run(words[q], s0lo, s0hi, s1lo, s1hi, mul);  // (k0,k4) (k1,k5) (k2,k6) (k3,k7)
           f16x2_to_f32(s0lo, o[0], o[4]);
           f16x2_to_f32(s0hi, o[1], o[5]);
           f16x2_to_f32(s1lo, o[2], o[6]);
           f16x2_to_f32(s1hi, o[3], o[7]);
         } else {
-          dec_int4km(pal, words[q], s0lo, s0hi, s1lo, s1hi);
+          dec_int4km(pal, words[q], s0lo, s0hi, s1lo, s1hi, mul);
           f16x2_to_f32(s0lo, o[0], o[1]);
           f16x2_to_f32(s0hi, o[2], o[3]);
           f16x2_to_f32(s1lo, o[4], o[5]);

@@ -10,13 +10,24 @@
 namespace qmv {
 
 // ---- fused dequant-matvec / gather kernel -----------------------------------
-constexpr int kConsumerWarps = 8;                    // warps that decode + multiply
-constexpr int kThreads = 32 * (1 + kConsumerWarps);  // + one producer warp
-constexpr int kTileRows = 16;                        // rows per tile: one m16 step
-constexpr int kMaxCols = 16;                         // activation columns per pass
-constexpr int kMaxStages = 8;
-constexpr int kMaxPairs = 256;                       // B * topk upper bound (16 * 16)
-constexpr int kSmemLimit = 227 * 1024;               // per-block opt-in maximum on sm_100
+constexpr int kWarps = 8;                  // warps per CTA: all copy, decode and multiply
+constexpr int kThreads = 32 * kWarps;
+constexpr int kTileRows = 16;              // rows per tile: one m16 step
+constexpr int kMaxCols = 16;               // activation columns per pass
+constexpr int kStages = 3;                 // per-warp ring depth (slices in flight + 1)
+#ifndef QMV_SLICE_BYTES
+#define QMV_SLICE_BYTES 256                // bytes of codes per row in a warp's K-slice
+#endif
+#ifndef QMV_MIN_CTAS
+#define QMV_MIN_CTAS 2                     // CTAs per SM the kernel's register budget targets
+#endif
+constexpr int kSliceBytes = QMV_SLICE_BYTES;
+constexpr int kMinCtas = QMV_MIN_CTAS;
+constexpr int kMaxCtasPerSM = 4;
+constexpr int kMaxPairs = 256;             // B * topk upper bound (16 * 16)
+constexpr int kSmemLimit = 227 * 1024;     // per-block opt-in maximum on sm_100
+constexpr int kSmemPerSM = 228 * 1024;     // shared memory of one SM
+constexpr int kStaticSmem = 6 * 1024;      // the kernel's static shared memory (group table), rounded up
 
 // Aux (scale / palette) staging mode of a launch.
 enum AuxMode : int {
@@ -39,7 +50,7 @@ struct MvParams {
   int64_t tiles;           // ceil(N / 16)
   int B;                   // dense: activation rows; gather: tokens
   int topk, E, x_per_slot, gather;
-  int KC, nchunks;         // in-features per pipeline stage, stages per tile
+  int KC, nchunks;         // in-features per warp slice, slices per tile
   int RS;                  // shared-memory bytes per staged code row
   int AS;                  // shared-memory bytes per staged scale row (kAuxRows)
   int aux_mode;
@@ -48,6 +59,7 @@ struct MvParams {
   int n_xrows;             // activation rows staged
   int off_red, off_x, off_stage;  // dynamic shared-memory offsets
   int smem_bytes;
+  int ctas_per_sm;         // 1..4, by shared-memory footprint
 };
 
 // Per-format constants (bits per weight, scale bytes per 32-block).

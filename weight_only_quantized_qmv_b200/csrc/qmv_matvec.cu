@@ -9,17 +9,23 @@
 // reading only the packed codes and their block scales / row palette.
 //
 // Design (B200): the op streams ~0.5 byte of weights per multiply-add, so HBM
-// bandwidth bounds it and the instruction budget per weight is ~2-3.  Each CTA
-// (one per SM, persistent) runs one producer warp that moves 16-row weight
-// tiles into a ring of shared-memory stages with 1-D bulk async copies (TMA
-// engine, mbarrier transaction counts), and eight consumer warps that split
-// each tile along K.  A consumer turns one 32-bit word of codes into exact
-// fp16 operands in registers and lets one m16n8k16 tensor-core step do 256
-// multiply-adds (16 rows x 16 k, with the activations as the 8-column operand),
-// so the per-weight cost is the decode alone.  Block scales are applied in fp32
-// to each 32-block's partial sum; the palette format carries its scale in the
-// table and accumulates straight through.  Tile partial sums are reduced in
-// shared memory in a fixed warp order (deterministic), then written once.
+// bandwidth bounds it and the instruction budget per weight is ~2-3.  Each
+// warp of a persistent CTA is an independent pipeline over whole 16-row
+// weight tiles: it copies its tile's next K-slice (16 rows x 512 weights,
+// ~4.5 KB) with 16-byte asynchronous copies (cp.async) into a private
+// shared-memory ring while it decodes and multiplies the previous slice, and
+// it owns all of K of its tile, so no cross-warp reduction or CTA barrier
+// sits on the streaming path.  Rows land at a padded stride so the warp's
+// shared-memory reads are free of bank conflicts.  (Measured on B200: 16-byte
+// asynchronous copies and 128-bit loads both reach the ~7.0 TB/s read ceiling
+// with enough bytes in flight, while one-thread 1-D bulk copies cost ~225 ns
+// per instruction.)  The warp turns one 32-bit word of codes into exact fp16
+// operands in registers and lets one m16n8k16 tensor-core step do 256
+// multiply-adds (16 rows x 16 k, with the activations as the 8-column
+// operand), so the per-weight cost is the decode alone.  Block scales are
+// applied in fp32 to each 32-block's partial sum; the palette format carries
+// its scale in the table and accumulates straight through.  Each output is
+// accumulated by one lane in a fixed order and written once (deterministic).
 #include "qmv_device.cuh"
 
 namespace qmv {
@@ -88,53 +94,219 @@ __device__ __forceinline__ uint4 ldg_nc_128(const void* p) {
   return v;
 }
 
-// Barrier on named barrier `id` over `n` threads that also ORs a predicate.
-__device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t n, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n barrier.red.or.pred po, %2, %3, pi;\n"
-      " selp.u32 %0, 1, 0, po;\n}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most `n` (0..2) of this thread's committed copy groups are pending.
+__device__ __forceinline__ void cp_async_wait(int n) {
+  if (n <= 0)
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+  else if (n == 1)
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+  else
+    asm volatile("cp.async.wait_group 2;" ::: "memory");
 }
 
-// Block-scale of (row, block) from the staged scale region.
+// Block-scale of (row, block) from the staged scale region (fp4: the e8m0
+// scale times 2; the partial sums are halved once per tile).
 template <int FMT>
-__device__ __forceinline__ float stage_scale(uint32_t a) {
+__device__ __forceinline__ float stage_scale(uint32_t a, const Mul& m) {
   if constexpr (FMT == QMV_FMT_FP4) {
-    return e8m0_to_f32(lds_u8(a));
+    return e8m0_x2_to_f32<3>(lds_u8(a) << 24, m);
   } else {
     return __half2float(__ushort_as_half((unsigned short)lds_u16(a)));
   }
 }
 
+// fp16 scale i of a 16-byte / 8-byte group -> float
+template <int I>
+__device__ __forceinline__ float half_at(const uint4& v) {
+  const uint32_t w = (I / 2 == 0) ? v.x : (I / 2 == 1) ? v.y : (I / 2 == 2) ? v.z : v.w;
+  const __half2 h = *reinterpret_cast<const __half2*>(&w);
+  return (I % 2 == 0) ? __low2float(h) : __high2float(h);
+}
+
+// Decode one block's codes of rows g and g+8 into the two m16n8k16 A fragments.
+template <int FMT>
+__device__ __forceinline__ void decode_block(uint32_t crow_g, uint32_t crow_g8, int b, int t, const Palette& pg,
+                                             const Palette& pg8, const Mul& m, uint32_t (&a0)[4], uint32_t (&a1)[4]) {
+  uint32_t g0lo, g0hi, g1lo, g1hi, h0lo, h0hi, h1lo, h1hi;  // row g / g+8, step 0 / 1
+  if constexpr (FmtT<FMT>::kBits == 8) {
+    const uint2 vg = lds64(crow_g + 32u * b + 8u * t);
+    const uint2 vh = lds64(crow_g8 + 32u * b + 8u * t);
+    dec_int8_word(vg.x, g0lo, g0hi);
+    dec_int8_word(vg.y, g1lo, g1hi);
+    dec_int8_word(vh.x, h0lo, h0hi);
+    dec_int8_word(vh.y, h1lo, h1hi);
+  } else {
+    const uint32_t wg = lds32(crow_g + 16u * b + 4u * t);
+    const uint32_t wh = lds32(crow_g8 + 16u * b + 4u * t);
+    if constexpr (FMT == QMV_FMT_FP4) {
+      DecFp4::run(wg, g0lo, g0hi, g1lo, g1hi, m);
+      DecFp4::run(wh, h0lo, h0hi, h1lo, h1hi, m);
+    } else if constexpr (FMT == QMV_FMT_INT4) {
+      DecInt4::run(wg, g0lo, g0hi, g1lo, g1hi, m);
+      DecInt4::run(wh, h0lo, h0hi, h1lo, h1hi, m);
+    } else {
+      dec_int4km(pg, wg, g0lo, g0hi, g1lo, g1hi, m);
+      dec_int4km(pg8, wh, h0lo, h0hi, h1lo, h1hi, m);
+    }
+  }
+  a0[0] = g0lo; a0[1] = h0lo; a0[2] = g0hi; a0[3] = h0hi;
+  a1[0] = g1lo; a1[1] = h1lo; a1[2] = g1hi; a1[3] = h1hi;
+}
+
+// Multiply-accumulate one decoded block: palette formats accumulate directly,
+// block-scaled formats scale the block's exact partial in fp32.
 template <int FMT, int NT>
-__global__ void __launch_bounds__(kThreads, 1) mv_kernel(const __grid_constant__ MvParams p) {
+__device__ __forceinline__ void mac_block(float (&acc)[NT][4], const uint32_t (&a0)[4], const uint32_t (&a1)[4],
+                                          const uint4 (&xr)[NT], float sg, float sh) {
+  if constexpr (FmtT<FMT>::kLut) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      mma16816(acc[n], a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
+      mma16816(acc[n], a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
+    }
+  } else {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      mma16816(d, a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
+      mma16816(d, a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
+      acc[n][0] = fmaf(d[0], sg, acc[n][0]);
+      acc[n][1] = fmaf(d[1], sg, acc[n][1]);
+      acc[n][2] = fmaf(d[2], sh, acc[n][2]);
+      acc[n][3] = fmaf(d[3], sh, acc[n][3]);
+    }
+  }
+}
+
+// A warp's NB blocks of a full K-slice, unrolled: every shared-memory address
+// is a base plus an immediate, and the slice's scales of a row are read with
+// one or two 128-bit loads.
+template <int FMT, int NT, int NB>
+__device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g, uint32_t crow_g8, uint32_t sa_g,
+                                           uint32_t sa_g8, const uint32_t (&xb)[NT], int t, const Palette& pg,
+                                           const Palette& pg8, const Mul& m) {
+  using F = FmtT<FMT>;
+  uint4 sg0 = make_uint4(0u, 0u, 0u, 0u), sh0 = sg0, sg1 = sg0, sh1 = sg0;
+  if constexpr (!F::kLut) {
+    sg0 = lds128(sa_g);
+    sh0 = lds128(sa_g8);
+    if constexpr (NB * F::kSB == 32) {
+      sg1 = lds128(sa_g + 16u);
+      sh1 = lds128(sa_g8 + 16u);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NB; ++i) {
+    uint4 xr[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) xr[n] = lds128(xb[n] + 64u * (uint32_t)i);
+    uint32_t a0[4], a1[4];
+    decode_block<FMT>(crow_g, crow_g8, i, t, pg, pg8, m, a0, a1);
+    float sg = 0.0f, sh = 0.0f;
+    if constexpr (FMT == QMV_FMT_FP4) {
+      const uint32_t q = (uint32_t)i >> 2;
+      const uint32_t wg = q == 0 ? sg0.x : q == 1 ? sg0.y : q == 2 ? sg0.z : sg0.w;
+      const uint32_t wh = q == 0 ? sh0.x : q == 1 ? sh0.y : q == 2 ? sh0.z : sh0.w;
+      if ((i & 3) == 0) { sg = e8m0_x2_to_f32<0>(wg, m); sh = e8m0_x2_to_f32<0>(wh, m); }
+      if ((i & 3) == 1) { sg = e8m0_x2_to_f32<1>(wg, m); sh = e8m0_x2_to_f32<1>(wh, m); }
+      if ((i & 3) == 2) { sg = e8m0_x2_to_f32<2>(wg, m); sh = e8m0_x2_to_f32<2>(wh, m); }
+      if ((i & 3) == 3) { sg = e8m0_x2_to_f32<3>(wg, m); sh = e8m0_x2_to_f32<3>(wh, m); }
+    } else if constexpr (!F::kLut) {
+      const uint4& vg = (i < 8) ? sg0 : sg1;
+      const uint4& vh = (i < 8) ? sh0 : sh1;
+      switch (i & 7) {
+        case 0: sg = half_at<0>(vg); sh = half_at<0>(vh); break;
+        case 1: sg = half_at<1>(vg); sh = half_at<1>(vh); break;
+        case 2: sg = half_at<2>(vg); sh = half_at<2>(vh); break;
+        case 3: sg = half_at<3>(vg); sh = half_at<3>(vh); break;
+        case 4: sg = half_at<4>(vg); sh = half_at<4>(vh); break;
+        case 5: sg = half_at<5>(vg); sh = half_at<5>(vh); break;
+        case 6: sg = half_at<6>(vg); sh = half_at<6>(vh); break;
+        default: sg = half_at<7>(vg); sh = half_at<7>(vh); break;
+      }
+    }
+    mac_block<FMT, NT>(acc, a0, a1, xr, sg, sh);
+  }
+}
+
+__device__ __forceinline__ uint8_t ldg_u8(const uint8_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(p));
+  return (uint8_t)v;
+}
+
+// Issue one K-slice (16 rows x kc weights) of a tile into the warp's stage.
+// Lane L copies the 16-byte chunks (row 2j + L/16, column L%16) for j < 8;
+// rows past N re-read the last row (their outputs are never stored).  Scales
+// go by 16-byte copies when rows are aligned, else by plain byte loads
+// (synchronous; only for shapes whose scale rows are not 16-byte multiples).
+template <int FMT>
+__device__ __forceinline__ void issue_slice(const MvParams& p, const uint8_t* crow0, const uint8_t* arow0,
+                                            int nrows, int k0, int kc, uint32_t stage, int lane) {
+  using F = FmtT<FMT>;
+  const int cpr = kc * F::kBits / 8 / 16;  // 16-byte chunks per row of this slice (<= 16)
+  const int col = lane & 15;
+  const uint8_t* cbase = crow0 + (int64_t)k0 * F::kBits / 8 + col * 16;
+  if (col < cpr) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int row = 2 * j + (lane >> 4);
+      const int r = min(row, nrows - 1);
+      cp_async16(stage + (uint32_t)row * p.RS + (uint32_t)col * 16u, cbase + (int64_t)r * p.code_row_bytes);
+    }
+  }
+  const uint32_t auxs = stage + p.aux_off;
+  if constexpr (F::kLut) {
+    if (k0 == 0) {  // the tile's palette rides with its first slice
+      const int r = min(lane >> 1, nrows - 1);
+      cp_async16(auxs + (uint32_t)lane * 16u, arow0 + (int64_t)r * 32 + (lane & 1) * 16);
+    }
+  } else {
+    const int sbytes = (kc / 32) * F::kSB;  // scale bytes per row of this slice
+    const uint8_t* abase = arow0 + (int64_t)(k0 / 32) * F::kSB;
+    if (p.aux_mode == kAuxRows) {
+      if (sbytes >= 16) {  // 16 or 32 bytes per row: 16-byte copies
+        const int apr = sbytes / 16;
+        if (lane < kTileRows * apr) {
+          const int row = apr == 1 ? lane : (lane >> 1), c16 = apr == 1 ? 0 : (lane & 1);
+          const int r = min(row, nrows - 1);
+          cp_async16(auxs + (uint32_t)row * p.AS + (uint32_t)c16 * 16u, abase + (int64_t)r * p.aux_row_bytes + c16 * 16);
+        }
+      } else if (lane < kTileRows) {  // 8 bytes per row: 8-byte copies
+        const int r = min(lane, nrows - 1);
+        cp_async8(auxs + (uint32_t)lane * p.AS, abase + (int64_t)r * p.aux_row_bytes);
+      }
+    } else {
+      for (int i = lane; i < kTileRows * sbytes; i += 32) {
+        const int row = i / sbytes, b = i - row * sbytes;
+        const int r = min(row, nrows - 1);
+        sts_u8(auxs + (uint32_t)row * p.AS + (uint32_t)b, ldg_u8(abase + (int64_t)r * p.aux_row_bytes + b));
+      }
+    }
+  }
+}
+
+template <int FMT, int NT>
+__global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_constant__ MvParams p) {
   using F = FmtT<FMT>;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ GroupTable gt;
   __shared__ int s_ids[kMaxPairs];
-  __shared__ int s_abort;
   __shared__ int s_nvalid;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int S = p.stages;
   const uint32_t sbase = smem_addr(smem);
-  const uint32_t full0 = sbase, empty0 = sbase + 8u * S;  // mbarriers
   const int P = p.gather ? p.B * p.topk : p.B;
 
-  // ---- set-up: barriers and the column groups ------------------------------
-  if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full0 + 8u * s, 1);
-      mbar_init(empty0 + 8u * s, kConsumerWarps);
-    }
-    mbar_fence_init();
-    s_abort = 0;
-    s_nvalid = 0;
-  }
+  // ---- set-up (whole CTA): the column groups and the staged activations -----
+  if (tid == 0) s_nvalid = 0;
   if (p.gather && tid < P) s_ids[tid] = p.ids[tid];
   __syncthreads();
   if (!p.gather) {
@@ -181,119 +353,15 @@ __global__ void __launch_bounds__(kThreads, 1) mv_kernel(const __grid_constant__
         for (int64_t n = tid; n < p.N; n += blockDim.x) p.y[(int64_t)q * p.N + n] = 0.0f;
       }
     }
-    __syncthreads();
   }
-
-  const int64_t total = (int64_t)gt.ngroups * p.tiles;
-  if ((int64_t)blockIdx.x >= total) return;
-
-  if (warp == 0) {
-    // ======================= producer warp =======================
-    uint32_t it = 0;
-    bool ok = true;
-    for (int64_t u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      const int grp = (int)(u / p.tiles);
-      const int64_t tile = u - (int64_t)grp * p.tiles;
-      const int64_t row0 = tile * kTileRows;
-      const int nrows = (int)min((int64_t)kTileRows, p.N - row0);
-      const int e = gt.expert[grp];
-      const uint8_t* ce = p.codes + (int64_t)e * p.expert_code_bytes;
-      const uint8_t* ae = p.aux + (int64_t)e * p.expert_aux_bytes;
-      for (int c = 0; c < p.nchunks; ++c, ++it) {
-        const int s = (int)(it % (uint32_t)S);
-        const uint32_t ph = (it / (uint32_t)S) & 1u;
-        const uint32_t fb = full0 + 8u * s;
-        if (!mbar_wait(empty0 + 8u * s, ph ^ 1u, &s_abort, p.status)) {
-          ok = false;
-          break;
-        }
-        const int k0 = c * p.KC;
-        const int kc = min(p.KC, (int)(p.K - k0));
-        const uint32_t cbytes = (uint32_t)(kc * F::kBits / 8);
-        const uint32_t stage = sbase + p.off_stage + (uint32_t)s * p.stage_bytes;
-        const uint32_t auxs = stage + p.aux_off;
-        uint32_t tx = kTileRows * cbytes;
-        uint32_t arow = 0, lut_bytes = 0;
-        const uint8_t* bsrc = nullptr;
-        uint32_t bbytes = 0, bhead = 0, bmid = 0, bdst = 0;
-        if constexpr (F::kLut) {
-          lut_bytes = (c == 0) ? (uint32_t)nrows * 32u : 0u;
-          tx += lut_bytes;
-        } else if (p.aux_mode == kAuxRows) {
-          arow = (uint32_t)(kc / 32) * F::kSB;
-          tx += kTileRows * arow;
-        } else {
-          // whole tile scale block: bulk copy of its 16-byte-aligned middle,
-          // head/tail bytes by plain loads; staged at offset (src & 15).
-          bsrc = ae + row0 * p.aux_row_bytes;
-          bbytes = (uint32_t)nrows * (uint32_t)p.aux_row_bytes;
-          const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(bsrc) & 15u);
-          bhead = min(bbytes, (16u - mis) & 15u);
-          bmid = (bbytes - bhead) & ~15u;
-          bdst = auxs + mis;
-          tx += bmid;
-        }
-        if (lane == 0) mbar_expect_tx(fb, tx);
-        __syncwarp();
-        if (lane < kTileRows) {
-          const int r = min(lane, nrows - 1);  // rows past N re-read the last row
-          bulk_g2s(stage + (uint32_t)lane * p.RS,
-                   ce + (row0 + r) * p.code_row_bytes + (int64_t)k0 * F::kBits / 8, cbytes, fb);
-        } else {
-          const int r16 = lane - kTileRows;
-          if constexpr (F::kLut) {
-            if (r16 == 0 && lut_bytes) bulk_g2s(auxs, ae + row0 * 32, lut_bytes, fb);
-          } else {
-            if (p.aux_mode == kAuxRows) {
-              const int r = min(r16, nrows - 1);
-              bulk_g2s(auxs + (uint32_t)r16 * p.AS, ae + (row0 + r) * p.aux_row_bytes + (int64_t)(k0 / 32) * F::kSB,
-                       arow, fb);
-            } else if (r16 == 0 && bmid) {
-              bulk_g2s(bdst + bhead, bsrc + bhead, bmid, fb);
-            }
-          }
-        }
-        if constexpr (!F::kLut) {
-          if (p.aux_mode == kAuxBlock) {
-            bool wrote = false;
-            for (uint32_t i = lane; i < bhead; i += 32) {
-              sts_u8(bdst + i, bsrc[i]);
-              wrote = true;
-            }
-            for (uint32_t i = bhead + bmid + lane; i < bbytes; i += 32) {
-              sts_u8(bdst + i, bsrc[i]);
-              wrote = true;
-            }
-            if (wrote) fence_proxy_async();
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(fb);
-      }
-    }
-    // Drain: every issued stage's copies must have landed before the CTA exits.
-    if (lane == 0) {
-      const uint32_t n = it < (uint32_t)S ? it : (uint32_t)S;
-      for (uint32_t s = 0; s < n; ++s) {
-        const uint32_t last = s + (uint32_t)S * ((it - 1u - s) / (uint32_t)S);
-        mbar_wait(full0 + 8u * s, (last / (uint32_t)S) & 1u, &s_abort, p.status, /*respect_abort=*/false);
-      }
-    }
-    return;
-  }
-
-  // ======================= consumer warps =======================
-  const int cw = warp - 1;
-  const int g = lane >> 2, t = lane & 3;
+  // Activations once per CTA: row r at xbase + r * XS, in the k order the
+  // format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7) per 8), and
+  // a zero row for the columns a group does not use.
   const uint32_t xbase = sbase + p.off_x;
-
-  // Stage the activations once: row r at xbase + r * XS, in the k order the
-  // format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7) per 8).
   {
-    const int ct = tid - 32;
     const int64_t per_row = p.K / 8;
     const int64_t n16 = (int64_t)p.n_xrows * per_row;
-    for (int64_t i = ct; i < n16; i += kConsumerWarps * 32) {
+    for (int64_t i = tid; i < n16; i += kThreads) {
       const int64_t r = i / per_row, j = i - r * per_row;
       uint4 v = ldg_nc_128(p.x + r * p.K + 8 * j);
       if constexpr (F::kPermX) {
@@ -302,156 +370,165 @@ __global__ void __launch_bounds__(kThreads, 1) mv_kernel(const __grid_constant__
       }
       sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
     }
-    named_bar_sync(1, kConsumerWarps * 32);
+    for (int64_t j = tid; j < per_row; j += kThreads)
+      sts128(xbase + (uint32_t)((int64_t)p.n_xrows * p.XS + 16 * j), make_uint4(0u, 0u, 0u, 0u));
+  }
+  __syncthreads();
+
+  // ---- per-warp pipelines over whole tiles ----------------------------------
+  const int64_t total = (int64_t)gt.ngroups * p.tiles;
+  const int64_t gwarp = (int64_t)blockIdx.x * kWarps + warp, nwarps = (int64_t)gridDim.x * kWarps;
+  if (gwarp >= total) return;
+  const int S = p.stages;
+  const uint32_t ring = sbase + p.off_stage + (uint32_t)(warp * S) * p.stage_bytes;
+  const int g = lane >> 2, t = lane & 3;
+  const Mul mul = Mul::make();
+  const int KCW = p.KC;  // weights per slice
+
+  // Cursor over this warp's units (tile, group) in order, advanced without
+  // divisions: unit u = gwarp + i * nwarps, group = u / tiles.
+  struct Cursor {
+    int64_t tile;
+    int grp;
+  };
+  auto advance = [&](Cursor& cu) {
+    cu.tile += nwarps;
+    while (cu.tile >= p.tiles) {
+      cu.tile -= p.tiles;
+      ++cu.grp;
+    }
+  };
+  Cursor ci{gwarp, 0};  // issue cursor
+  while (ci.tile >= p.tiles) {
+    ci.tile -= p.tiles;
+    ++ci.grp;
+  }
+  const Cursor c_first = ci;
+  int c_issue = 0;
+  const uint8_t* crow0 = nullptr;
+  const uint8_t* arow0 = nullptr;
+  int nrows_issue = 0;
+  auto set_rows = [&]() {
+    const int64_t row0 = ci.tile * kTileRows;
+    nrows_issue = (int)min((int64_t)kTileRows, p.N - row0);
+    const int e = gt.expert[ci.grp];
+    crow0 = p.codes + (int64_t)e * p.expert_code_bytes + row0 * p.code_row_bytes;
+    arow0 = p.aux + (int64_t)e * p.expert_aux_bytes + row0 * p.aux_row_bytes;
+  };
+  set_rows();
+  auto issue_next = [&](int stage_idx) {
+    const int k0 = c_issue * KCW;
+    issue_slice<FMT>(p, crow0, arow0, nrows_issue, k0, min(KCW, (int)(p.K - k0)),
+                     ring + (uint32_t)stage_idx * p.stage_bytes, lane);
+    if (++c_issue == p.nchunks) {
+      c_issue = 0;
+      advance(ci);
+      if (ci.grp < gt.ngroups) set_rows();
+    }
+  };
+
+  // prologue: S-1 slices in flight
+  for (int j = 0; j < S - 1; ++j) {
+    if (ci.grp < gt.ngroups) issue_next(j);
+    cp_async_commit();
   }
 
-  const uint32_t red0 = sbase + p.off_red;
-  uint32_t it = 0;
-  int par = 0;
-  for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
-    const int grp = (int)(u / p.tiles);
-    const int64_t tile = u - (int64_t)grp * p.tiles;
-    const int64_t row0 = tile * kTileRows;
+  float acc[NT][4];
+  Palette pg, pg8;
+  uint32_t xa[NT];
+  int xa_grp = -1;
+  int s = 0, s_fill = S - 1;
+  for (Cursor cc = c_first; cc.grp < gt.ngroups; advance(cc)) {
+    const int grp = cc.grp;
+    const int64_t row0 = cc.tile * kTileRows;
     const int nrows = (int)min((int64_t)kTileRows, p.N - row0);
-    const int ncols = gt.count[grp], gstart = gt.start[grp];
-
-    uint32_t xa[NT];
-    bool xv[NT];
+    if (grp != xa_grp) {  // activation rows of this column group
+      xa_grp = grp;
+      const int ncols = gt.count[grp], gstart = gt.start[grp];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const int col = 8 * n + g;
-      xv[n] = col < ncols;
-      const int pair = xv[n] ? gt.sorted[gstart + col] : 0;
-      const int xrow = p.gather ? (p.x_per_slot ? pair : pair / p.topk) : pair;
-      xa[n] = xbase + (uint32_t)xrow * p.XS + (uint32_t)t * 16u;
+      for (int n = 0; n < NT; ++n) {
+        const int col = 8 * n + g;
+        int xrow = p.n_xrows;  // the zero row
+        if (col < ncols) {
+          const int pair = gt.sorted[gstart + col];
+          xrow = p.gather ? (p.x_per_slot ? pair : pair / p.topk) : pair;
+        }
+        xa[n] = xbase + (uint32_t)xrow * p.XS + (uint32_t)t * 16u;
+      }
     }
-
-    float acc[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
-    Palette pg, pg8;
-    bool tile_ok = true;
 
-    for (int c = 0; c < p.nchunks; ++c, ++it) {
-      const int s = (int)(it % (uint32_t)S);
-      const uint32_t ph = (it / (uint32_t)S) & 1u;
-      const bool ok = mbar_wait(full0 + 8u * s, ph, &s_abort, p.status);
-      if (ok) {
-        const uint32_t stage = sbase + p.off_stage + (uint32_t)s * p.stage_bytes;
-        const uint32_t auxs = stage + p.aux_off;
-        const int k0 = c * p.KC;
-        const int kc = min(p.KC, (int)(p.K - k0));
+    for (int c = 0; c < p.nchunks; ++c) {
+      // keep S-1 slices in flight: refill the stage freed by the previous slice
+      if (ci.grp < gt.ngroups) issue_next(s_fill);
+      cp_async_commit();
+      s_fill = (s_fill + 1 == S) ? 0 : s_fill + 1;
+      cp_async_wait(S - 1);  // this slice's copies (all lanes) have landed
+      __syncwarp();
+
+      const uint32_t stage = ring + (uint32_t)s * p.stage_bytes;
+      const uint32_t auxs = stage + p.aux_off;
+      const int k0 = c * KCW;
+      const int kc = min(KCW, (int)(p.K - k0));
+      if constexpr (F::kLut) {
+        if (c == 0) {
+          uint32_t e0[8], e1[8];
+          const uint4 a0 = lds128(auxs + (uint32_t)g * 32u), a1 = lds128(auxs + (uint32_t)g * 32u + 16u);
+          const uint4 b0 = lds128(auxs + (uint32_t)(g + 8) * 32u), b1 = lds128(auxs + (uint32_t)(g + 8) * 32u + 16u);
+          e0[0] = a0.x; e0[1] = a0.y; e0[2] = a0.z; e0[3] = a0.w;
+          e0[4] = a1.x; e0[5] = a1.y; e0[6] = a1.z; e0[7] = a1.w;
+          e1[0] = b0.x; e1[1] = b0.y; e1[2] = b0.z; e1[3] = b0.w;
+          e1[4] = b1.x; e1[5] = b1.y; e1[6] = b1.z; e1[7] = b1.w;
+          pg = palette_from_words(e0);
+          pg8 = palette_from_words(e1);
+        }
+      }
+      const uint32_t crow_g = stage + (uint32_t)g * p.RS, crow_g8 = stage + (uint32_t)(g + 8) * p.RS;
+      const uint32_t sa_g = auxs + (uint32_t)g * p.AS, sa_g8 = auxs + (uint32_t)(g + 8) * p.AS;
+      constexpr int kNB = kSliceBytes * 8 / F::kBits / 32;  // blocks in a full slice
+      if (kc == KCW && KCW == kNB * 32 && (F::kLut || p.aux_mode == kAuxRows)) {
+        uint32_t xb[NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
+        slice_full<FMT, NT, kNB>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
+      } else {
         const int nbc = kc / 32;
-        if constexpr (F::kLut) {
-          if (c == 0) {
-            uint32_t e0[8], e1[8];
-            const uint4 a0 = lds128(auxs + (uint32_t)g * 32u), a1 = lds128(auxs + (uint32_t)g * 32u + 16u);
-            const uint4 b0 = lds128(auxs + (uint32_t)(g + 8) * 32u), b1 = lds128(auxs + (uint32_t)(g + 8) * 32u + 16u);
-            e0[0] = a0.x; e0[1] = a0.y; e0[2] = a0.z; e0[3] = a0.w;
-            e0[4] = a1.x; e0[5] = a1.y; e0[6] = a1.z; e0[7] = a1.w;
-            e1[0] = b0.x; e1[1] = b0.y; e1[2] = b0.z; e1[3] = b0.w;
-            e1[4] = b1.x; e1[5] = b1.y; e1[6] = b1.z; e1[7] = b1.w;
-            pg = palette_from_words(e0);
-            pg8 = palette_from_words(e1);
-          }
-        }
-        // scale addresses of rows g, g+8 for block 0 of this chunk
-        uint32_t sa_g = 0, sa_g8 = 0;
-        if constexpr (!F::kLut) {
-          if (p.aux_mode == kAuxRows) {
-            sa_g = auxs + (uint32_t)g * p.AS;
-            sa_g8 = auxs + (uint32_t)(g + 8) * p.AS;
-          } else {
-            const uint8_t* bsrc = p.aux + (int64_t)gt.expert[grp] * p.expert_aux_bytes + row0 * p.aux_row_bytes;
-            const uint32_t b0a = auxs + (uint32_t)(reinterpret_cast<uintptr_t>(bsrc) & 15u) +
-                                 (uint32_t)(k0 / 32) * F::kSB;
-            sa_g = b0a + (uint32_t)g * (uint32_t)p.aux_row_bytes;
-            sa_g8 = b0a + (uint32_t)(g + 8) * (uint32_t)p.aux_row_bytes;
-          }
-        }
-        const uint32_t crow_g = stage + (uint32_t)g * p.RS, crow_g8 = stage + (uint32_t)(g + 8) * p.RS;
-        const int b_lo = cw * nbc / kConsumerWarps, b_hi = (cw + 1) * nbc / kConsumerWarps;
-#pragma unroll 2
-        for (int b = b_lo; b < b_hi; ++b) {
+        for (int b = 0; b < nbc; ++b) {
           uint4 xr[NT];
 #pragma unroll
-          for (int n = 0; n < NT; ++n)
-            xr[n] = xv[n] ? lds128(xa[n] + (uint32_t)(k0 + 32 * b) * 2u) : make_uint4(0u, 0u, 0u, 0u);
-          uint32_t g0lo, g0hi, g1lo, g1hi, h0lo, h0hi, h1lo, h1hi;  // row g / g+8, step 0 / 1
-          if constexpr (F::kBits == 8) {
-            const uint2 vg = lds64(crow_g + 32u * b + 8u * t);
-            const uint2 vh = lds64(crow_g8 + 32u * b + 8u * t);
-            dec_int8_word(vg.x, g0lo, g0hi);
-            dec_int8_word(vg.y, g1lo, g1hi);
-            dec_int8_word(vh.x, h0lo, h0hi);
-            dec_int8_word(vh.y, h1lo, h1hi);
-          } else {
-            const uint32_t wg = lds32(crow_g + 16u * b + 4u * t);
-            const uint32_t wh = lds32(crow_g8 + 16u * b + 4u * t);
-            if constexpr (FMT == QMV_FMT_FP4) {
-              DecFp4::run(wg, g0lo, g0hi, g1lo, g1hi);
-              DecFp4::run(wh, h0lo, h0hi, h1lo, h1hi);
-            } else if constexpr (FMT == QMV_FMT_INT4) {
-              DecInt4::run(wg, g0lo, g0hi, g1lo, g1hi);
-              DecInt4::run(wh, h0lo, h0hi, h1lo, h1hi);
-            } else {
-              dec_int4km(pg, wg, g0lo, g0hi, g1lo, g1hi);
-              dec_int4km(pg8, wh, h0lo, h0hi, h1lo, h1hi);
-            }
+          for (int n = 0; n < NT; ++n) xr[n] = lds128(xa[n] + (uint32_t)(k0 + 32 * b) * 2u);
+          uint32_t a0[4], a1[4];
+          decode_block<FMT>(crow_g, crow_g8, b, t, pg, pg8, mul, a0, a1);
+          float sg = 0.0f, sh = 0.0f;
+          if constexpr (!F::kLut) {
+            sg = stage_scale<FMT>(sa_g + (uint32_t)b * F::kSB, mul);
+            sh = stage_scale<FMT>(sa_g8 + (uint32_t)b * F::kSB, mul);
           }
-          if constexpr (F::kLut) {
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              mma16816(acc[n], g0lo, h0lo, g0hi, h0hi, xr[n].x, xr[n].y);
-              mma16816(acc[n], g1lo, h1lo, g1hi, h1hi, xr[n].z, xr[n].w);
-            }
-          } else {
-            const float sg = stage_scale<FMT>(sa_g + (uint32_t)b * F::kSB);
-            const float sh = stage_scale<FMT>(sa_g8 + (uint32_t)b * F::kSB);
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-              mma16816(d, g0lo, h0lo, g0hi, h0hi, xr[n].x, xr[n].y);
-              mma16816(d, g1lo, h1lo, g1hi, h1hi, xr[n].z, xr[n].w);
-              acc[n][0] = fmaf(d[0], sg, acc[n][0]);
-              acc[n][1] = fmaf(d[1], sg, acc[n][1]);
-              acc[n][2] = fmaf(d[2], sh, acc[n][2]);
-              acc[n][3] = fmaf(d[3], sh, acc[n][3]);
-            }
-          }
+          mac_block<FMT, NT>(acc, a0, a1, xr, sg, sh);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8u * s);
-      tile_ok = tile_ok && ok;
+      __syncwarp();  // all lanes are done with this stage before it is refilled
+      s = (s + 1 == S) ? 0 : s + 1;
     }
 
-    // ---- deterministic split-K reduction over the consumer warps ----
-    const uint32_t red = red0 + (uint32_t)par * (kConsumerWarps * kTileRows * kMaxCols * 4) +
-                         (uint32_t)cw * (kTileRows * kMaxCols * 4);
+    // ---- store this tile's outputs: lane (g, t) holds rows g, g+8, cols 2t, 2t+1 ----
+    const int ncols = gt.count[grp], gstart = gt.start[grp];
+    const float f = (FMT == QMV_FMT_FP4) ? 0.5f : 1.0f;  // the fp4 block scales carried a factor 2
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-      const int c0 = 8 * n + 2 * t;
-      sts_f32x2(red + (uint32_t)(g * kMaxCols + c0) * 4u, acc[n][0], acc[n][1]);
-      sts_f32x2(red + (uint32_t)((g + 8) * kMaxCols + c0) * 4u, acc[n][2], acc[n][3]);
-    }
-    const bool stop = bar_red_or(1, kConsumerWarps * 32, !tile_ok || s_abort != 0);
-    if (stop) break;
-    const int ct = tid - 32;
-    if (ct < kTileRows * ncols) {
-      const int row = ct & (kTileRows - 1), col = ct >> 4;
-      const uint32_t rp = red0 + (uint32_t)par * (kConsumerWarps * kTileRows * kMaxCols * 4) +
-                          (uint32_t)(row * kMaxCols + col) * 4u;
-      float sum = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) sum += lds_f32(rp + (uint32_t)w * (kTileRows * kMaxCols * 4));
-      if (row < nrows) {
-        const int pair = gt.sorted[gstart + col];
-        p.y[(int64_t)pair * p.N + row0 + row] = sum;
+      for (int q = 0; q < 4; ++q) {
+        const int col = 8 * n + 2 * t + (q & 1);
+        const int row = g + 8 * (q >> 1);
+        if (col < ncols && row < nrows) {
+          const int pair = gt.sorted[gstart + col];
+          p.y[(int64_t)pair * p.N + row0 + row] = acc[n][q] * f;
+        }
       }
     }
-    par ^= 1;
   }
+  cp_async_wait(0);
 }
 
 // ---------------------------------------------------------------------------
@@ -467,10 +544,12 @@ bool plan_matvec(int fmt, MvParams& p) {
   p.expert_code_bytes = p.N * p.code_row_bytes;
   p.expert_aux_bytes = p.N * p.aux_row_bytes;
   p.tiles = (p.N + kTileRows - 1) / kTileRows;
-  p.KC = (int)(p.K < fi.kc_max ? p.K : fi.kc_max);
+  // a warp's K-slice: kSliceBytes of codes per row
+  const int slice = kSliceBytes * 8 / fi.bits;
+  p.KC = (int)(p.K < slice ? p.K : slice);
   p.nchunks = (int)((p.K + p.KC - 1) / p.KC);
   const int64_t cb = (int64_t)p.KC * fi.bits / 8;
-  // Row strides chosen so the consumers' shared-memory reads are free of bank
+  // Row strides chosen so a warp's shared-memory reads are free of bank
   // conflicts: 4-bit rows at 16 mod 128 bytes (32-bit loads), 8-bit rows at
   // 32 mod 128 (64-bit loads).
   p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 16 : 32));
@@ -480,36 +559,43 @@ bool plan_matvec(int fmt, MvParams& p) {
     p.AS = 32;
     aux_region = kTileRows * 32;
   } else {
-    const int64_t chunk_sc = (int64_t)(p.KC / 32) * fi.scale_bytes;
+    const int64_t slice_sc = (int64_t)(p.KC / 32) * fi.scale_bytes;
     const int64_t last_sc = ((p.K - (int64_t)(p.nchunks - 1) * p.KC) / 32) * fi.scale_bytes;
-    const bool base16 = (reinterpret_cast<uintptr_t>(p.aux) & 15u) == 0;
-    if (base16 && p.aux_row_bytes % 16 == 0 && chunk_sc % 16 == 0 && last_sc % 16 == 0) {
+    // asynchronous scale copies (16 or 8 bytes) when every row's slice
+    // segment starts on that boundary and is a multiple of it
+    const int64_t cs = (slice_sc % 16 == 0) ? 16 : 8;
+    const bool based = (reinterpret_cast<uintptr_t>(p.aux) % cs) == 0;
+    if (based && slice_sc % 8 == 0 && slice_sc <= 32 && p.aux_row_bytes % cs == 0 && last_sc % cs == 0)
       p.aux_mode = kAuxRows;
-      int64_t j = chunk_sc / 16;
-      if (j % 2 == 0) ++j;  // odd multiple of 16 bytes: rows g = 0..7 hit distinct banks
-      p.AS = (int)(16 * j);
-      aux_region = kTileRows * p.AS;
-    } else {
+    else
       p.aux_mode = kAuxBlock;
-      p.AS = (int)p.aux_row_bytes;
-      aux_region = round_up(kTileRows * p.aux_row_bytes + 16, 16);
-    }
+    int64_t j = (slice_sc + 15) / 16;
+    if (j % 2 == 0) ++j;  // odd multiple of 16 bytes: rows g = 0..7 hit distinct banks
+    p.AS = (int)(16 * j);
+    aux_region = kTileRows * p.AS;
   }
   p.aux_off = kTileRows * p.RS;
   p.stage_bytes = (int)round_up(p.aux_off + aux_region, 128);
   p.XS = (int)(round_up(2 * p.K, 128) + 64);  // 64 mod 128: conflict-free 128-bit reads
   p.n_xrows = p.gather ? (p.x_per_slot ? p.B * p.topk : p.B) : p.B;
-  p.off_red = 128;  // mbarriers live in the first 128 bytes
-  p.off_x = p.off_red + 2 * kConsumerWarps * kTileRows * kMaxCols * 4;
-  p.off_stage = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128);
-  const int64_t static_reserve = 8 * 1024;  // the kernel's static shared memory (group table)
-  const int64_t avail = (int64_t)kSmemLimit - static_reserve - p.off_stage;
-  if (avail < 2 * (int64_t)p.stage_bytes) return false;
-  int64_t st = avail / p.stage_bytes;
-  if (st > kMaxStages) st = kMaxStages;
-  p.stages = (int)st;
-  p.smem_bytes = (int)(p.off_stage + st * p.stage_bytes);
-  return true;
+  p.off_red = 0;
+  p.off_x = 0;
+  p.off_stage = (int)round_up((int64_t)(p.n_xrows + 1) * p.XS, 128);  // + a zero row
+  const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
+  // the most CTAs per SM (up to the kernel's register budget) with the
+  // deepest ring (<= kStages slices per warp) that fits
+  for (int ctas = kMinCtas; ctas >= 1; --ctas) {
+    for (int st = kStages; st >= 2; --st) {
+      const int64_t bytes = p.off_stage + (int64_t)kWarps * st * p.stage_bytes;
+      if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
+        p.stages = st;
+        p.smem_bytes = (int)bytes;
+        p.ctas_per_sm = ctas;
+        return true;
+      }
+    }
+  }
+  return false;
 }
 
 template <int FMT, int NT>
@@ -520,12 +606,15 @@ static cudaError_t launch_t(const MvParams& p, int num_sms, cudaStream_t stream)
   if (err != cudaSuccess) return err;
   if (dev < 64 && !attr_set[dev]) {
     err = cudaFuncSetAttribute(mv_kernel<FMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kSmemLimit - 8 * 1024);
+                               kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
     attr_set[dev] = true;
   }
-  const int64_t upper = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
-  const int grid = (int)(upper < num_sms ? upper : num_sms);
+  // enough warps for every (group, tile) unit, at most ctas_per_sm CTAs per SM
+  const int64_t upper_units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
+  const int64_t want = (upper_units + kWarps - 1) / kWarps;
+  const int64_t slots = (int64_t)num_sms * p.ctas_per_sm;
+  const int grid = (int)(want < slots ? want : slots);
   mv_kernel<FMT, NT><<<grid, kThreads, p.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }

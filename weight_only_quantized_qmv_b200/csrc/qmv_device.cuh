@@ -17,21 +17,16 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
 // Loads
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
+// Loads from shared memory by 32-bit shared-window address.  Plain C++ loads
+// (not volatile asm), so the compiler may schedule them freely between the
+// barriers and fences that order them against the asynchronous copies.
+template <typename T>
+__device__ __forceinline__ const T* sptr(uint32_t a) {
+  return reinterpret_cast<const T*>(__cvta_shared_to_generic(a));
 }
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-  return v;
-}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) { return *sptr<uint32_t>(a); }
+__device__ __forceinline__ uint2 lds64(uint32_t a) { return *sptr<uint2>(a); }
+__device__ __forceinline__ uint4 lds128(uint32_t a) { return *sptr<uint4>(a); }
 
 // ---------------------------------------------------------------------------
 // Tensor-core step: D(16x8, f32) = A(16x16, f16, row) * B(16x8, f16, col) + C
@@ -45,8 +40,7 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));

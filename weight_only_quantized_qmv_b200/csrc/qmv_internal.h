@@ -21,6 +21,12 @@ constexpr int kStages = 3;                 // per-warp ring depth (slices in fli
 #ifndef QMV_MIN_CTAS
 #define QMV_MIN_CTAS 2                     // CTAs per SM the kernel's register budget targets
 #endif
+#ifndef QMV_INDEP_MMA
+#define QMV_INDEP_MMA 0                    // block-scaled formats: the block's two MMA steps independent
+#endif
+#ifndef QMV_LUT_TWO_ACC
+#define QMV_LUT_TWO_ACC 0                  // palette format: two accumulator chains
+#endif
 constexpr int kSliceBytes = QMV_SLICE_BYTES;
 constexpr int kMinCtas = QMV_MIN_CTAS;
 constexpr int kMaxCtasPerSM = 4;

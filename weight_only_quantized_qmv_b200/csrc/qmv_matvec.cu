@@ -63,16 +63,8 @@ struct GroupTable {
   int16_t sorted[kMaxPairs];  // (token, slot) pair indices ordered by expert
 };
 
-__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a) { return *sptr<uint8_t>(a); }
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) { return *sptr<uint16_t>(a); }
 __device__ __forceinline__ void sts_u8(uint32_t a, uint32_t v) {
   asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
@@ -83,10 +75,10 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
 __device__ __forceinline__ void sts_f32x2(uint32_t a, float u, float v) {
   asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(u), "f"(v) : "memory");
 }
-__device__ __forceinline__ float lds_f32(uint32_t a) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
-  return v;
+// 128-bit shared load only where `on`; elsewhere the registers keep whatever
+// they held (used for activation columns whose outputs are never stored).
+__device__ __forceinline__ void lds128_if(uint4& v, uint32_t a, uint32_t on) {
+  if (on) v = lds128(a);
 }
 __device__ __forceinline__ uint4 ldg_nc_128(const void* p) {
   uint4 v;
@@ -163,17 +155,39 @@ __device__ __forceinline__ void decode_block(uint32_t crow_g, uint32_t crow_g8, 
 // Multiply-accumulate one decoded block: palette formats accumulate directly,
 // block-scaled formats scale the block's exact partial in fp32.
 template <int FMT, int NT>
-__device__ __forceinline__ void mac_block(float (&acc)[NT][4], const uint32_t (&a0)[4], const uint32_t (&a1)[4],
-                                          const uint4 (&xr)[NT], float sg, float sh) {
+__device__ __forceinline__ void mac_block(float (&acc)[NT][4], float (&acc2)[NT][4], const uint32_t (&a0)[4],
+                                          const uint32_t (&a1)[4], const uint4 (&xr)[NT], float sg, float sh) {
   if constexpr (FmtT<FMT>::kLut) {
+#if QMV_LUT_TWO_ACC
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {  // two accumulator chains: half the dependent MMA latency
+      mma16816(acc[n], a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
+      mma16816(acc2[n], a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
+    }
+#else
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       mma16816(acc[n], a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
       mma16816(acc[n], a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
     }
+#endif
   } else {
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
+#if QMV_INDEP_MMA
+      // the block's two MMA steps into separate zero-based partials: no MMA-to-MMA dependency
+      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f}, e[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      mma16816(d, a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
+      mma16816(e, a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
+      acc[n][0] = fmaf(d[0], sg, acc[n][0]);
+      acc[n][1] = fmaf(d[1], sg, acc[n][1]);
+      acc[n][2] = fmaf(d[2], sh, acc[n][2]);
+      acc[n][3] = fmaf(d[3], sh, acc[n][3]);
+      acc2[n][0] = fmaf(e[0], sg, acc2[n][0]);
+      acc2[n][1] = fmaf(e[1], sg, acc2[n][1]);
+      acc2[n][2] = fmaf(e[2], sh, acc2[n][2]);
+      acc2[n][3] = fmaf(e[3], sh, acc2[n][3]);
+#else
       float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       mma16816(d, a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
       mma16816(d, a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
@@ -181,6 +195,7 @@ __device__ __forceinline__ void mac_block(float (&acc)[NT][4], const uint32_t (&
       acc[n][1] = fmaf(d[1], sg, acc[n][1]);
       acc[n][2] = fmaf(d[2], sh, acc[n][2]);
       acc[n][3] = fmaf(d[3], sh, acc[n][3]);
+#endif
     }
   }
 }
@@ -189,9 +204,9 @@ __device__ __forceinline__ void mac_block(float (&acc)[NT][4], const uint32_t (&
 // is a base plus an immediate, and the slice's scales of a row are read with
 // one or two 128-bit loads.
 template <int FMT, int NT, int NB>
-__device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g, uint32_t crow_g8, uint32_t sa_g,
-                                           uint32_t sa_g8, const uint32_t (&xb)[NT], int t, const Palette& pg,
-                                           const Palette& pg8, const Mul& m) {
+__device__ __forceinline__ void slice_full(float (&acc)[NT][4], float (&acc2)[NT][4], uint32_t crow_g, uint32_t crow_g8, uint32_t sa_g,
+                                           uint32_t sa_g8, const uint32_t (&xb)[NT], const uint32_t (&xon)[NT], int t,
+                                           const Palette& pg, const Palette& pg8, const Mul& m) {
   using F = FmtT<FMT>;
   uint4 sg0 = make_uint4(0u, 0u, 0u, 0u), sh0 = sg0, sg1 = sg0, sh1 = sg0;
   if constexpr (!F::kLut) {
@@ -206,7 +221,7 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g,
   for (int i = 0; i < NB; ++i) {
     uint4 xr[NT];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) xr[n] = lds128(xb[n] + 64u * (uint32_t)i);
+    for (int n = 0; n < NT; ++n) lds128_if(xr[n], xb[n] + 64u * (uint32_t)i, xon[n]);
     uint32_t a0[4], a1[4];
     decode_block<FMT>(crow_g, crow_g8, i, t, pg, pg8, m, a0, a1);
     float sg = 0.0f, sh = 0.0f;
@@ -232,7 +247,7 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g,
         default: sg = half_at<7>(vg); sh = half_at<7>(vh); break;
       }
     }
-    mac_block<FMT, NT>(acc, a0, a1, xr, sg, sh);
+    mac_block<FMT, NT>(acc, acc2, a0, a1, xr, sg, sh);
   }
 }
 
@@ -433,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
     cp_async_commit();
   }
 
-  float acc[NT][4];
+  float acc[NT][4], acc2[NT][4];  // two accumulator sets (summed once per tile)
   Palette pg, pg8;
-  uint32_t xa[NT];
+  uint32_t xa[NT], xon[NT];
   int xa_grp = -1;
   int s = 0, s_fill = S - 1;
   for (Cursor cc = c_first; cc.grp < gt.ngroups; advance(cc)) {
@@ -449,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
       for (int n = 0; n < NT; ++n) {
         const int col = 8 * n + g;
         int xrow = p.n_xrows;  // the zero row
+        xon[n] = col < ncols ? 1u : 0u;
         if (col < ncols) {
           const int pair = gt.sorted[gstart + col];
           xrow = p.gather ? (p.x_per_slot ? pair : pair / p.topk) : pair;
@@ -457,7 +473,9 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
       }
     }
 #pragma unroll
-    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[n][q] = acc2[n][q] = 0.0f;
 
     for (int c = 0; c < p.nchunks; ++c) {
       // keep S-1 slices in flight: refill the stage freed by the previous slice
@@ -491,13 +509,13 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
         uint32_t xb[NT];
 #pragma unroll
         for (int n = 0; n < NT; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
-        slice_full<FMT, NT, kNB>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
+        slice_full<FMT, NT, kNB>(acc, acc2, crow_g, crow_g8, sa_g, sa_g8, xb, xon, t, pg, pg8, mul);
       } else {
         const int nbc = kc / 32;
         for (int b = 0; b < nbc; ++b) {
           uint4 xr[NT];
 #pragma unroll
-          for (int n = 0; n < NT; ++n) xr[n] = lds128(xa[n] + (uint32_t)(k0 + 32 * b) * 2u);
+          for (int n = 0; n < NT; ++n) lds128_if(xr[n], xa[n] + (uint32_t)(k0 + 32 * b) * 2u, xon[n]);
           uint32_t a0[4], a1[4];
           decode_block<FMT>(crow_g, crow_g8, b, t, pg, pg8, mul, a0, a1);
           float sg = 0.0f, sh = 0.0f;
@@ -505,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
             sg = stage_scale<FMT>(sa_g + (uint32_t)b * F::kSB, mul);
             sh = stage_scale<FMT>(sa_g8 + (uint32_t)b * F::kSB, mul);
           }
-          mac_block<FMT, NT>(acc, a0, a1, xr, sg, sh);
+          mac_block<FMT, NT>(acc, acc2, a0, a1, xr, sg, sh);
         }
       }
       __syncwarp();  // all lanes are done with this stage before it is refilled
@@ -523,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
         const int row = g + 8 * (q >> 1);
         if (col < ncols && row < nrows) {
           const int pair = gt.sorted[gstart + col];
-          p.y[(int64_t)pair * p.N + row0 + row] = acc[n][q] * f;
+          p.y[(int64_t)pair * p.N + row0 + row] = (acc[n][q] + acc2[n][q]) * f;
         }
       }
     }

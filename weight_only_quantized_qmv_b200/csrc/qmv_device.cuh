@@ -46,6 +46,16 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same step with a zero accumulator input (no per-block zeroing of d).
+__device__ __forceinline__ void mma16816_zc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+  const float z = 0.0f;
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
+
 // ---------------------------------------------------------------------------
 // Byte/bit helpers
 // ---------------------------------------------------------------------------
@@ -149,22 +159,31 @@ struct Mul {
   }
 };
 
-// two E2M1 codes in the LOW byte of r -> f16x2 (low nibble in the low half)
-__device__ __forceinline__ uint32_t e2m1x2_lo_to_f16x2(uint32_t r) {
+// two E2M1 codes in byte I of r -> f16x2
+template <int I>
+__device__ __forceinline__ uint32_t e2m1x2_byte_to_f16x2(uint32_t r) {
   uint32_t o;
-  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b0;\n}" : "=r"(o) : "r"(r));
+  if constexpr (I == 0)
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b0;\n}" : "=r"(o) : "r"(r));
+  else if constexpr (I == 1)
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b1;\n}" : "=r"(o) : "r"(r));
+  else if constexpr (I == 2)
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b2;\n}" : "=r"(o) : "r"(r));
+  else
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, b3;\n}" : "=r"(o) : "r"(r));
   return o;
 }
 
-// FP4: pairs (k0,k1) (k2,k3) for step 0, (k4,k5) (k6,k7) for step 1.  The
-// upper bytes are brought down with multiply-high (w >> 8, w >> 16, w >> 24).
+// FP4: pairs (k0,k1) (k2,k3) for step 0, (k4,k5) (k6,k7) for step 1: one
+// hardware conversion per byte, each reading its byte of w in place.
 struct DecFp4 {
   __device__ __forceinline__ static void run(uint32_t w, uint32_t& s0lo, uint32_t& s0hi, uint32_t& s1lo,
                                              uint32_t& s1hi, const Mul& m) {
-    s0lo = e2m1x2_lo_to_f16x2(w);
-    s0hi = e2m1x2_lo_to_f16x2(__umulhi(w, m.p24));
-    s1lo = e2m1x2_lo_to_f16x2(__umulhi(w, m.p16));
-    s1hi = e2m1x2_lo_to_f16x2(__umulhi(w, m.p8));
+    (void)m;
+    s0lo = e2m1x2_byte_to_f16x2<0>(w);
+    s0hi = e2m1x2_byte_to_f16x2<1>(w);
+    s1lo = e2m1x2_byte_to_f16x2<2>(w);
+    s1hi = e2m1x2_byte_to_f16x2<3>(w);
   }
 };
 
@@ -172,11 +191,8 @@ struct DecFp4 {
 // e8m0 scale times 2.  Callers fold the factor 1/2 into their outputs.
 template <int I>
 __device__ __forceinline__ float e8m0_x2_to_f32(uint32_t u, const Mul& m) {
-  uint32_t t = u;
-  if constexpr (I == 0) t = u * m.p24;
-  if constexpr (I == 1) t = u * m.p16;
-  if constexpr (I == 2) t = u * m.p8;
-  const uint32_t byte = __umulhi(t, m.p8);  // t >> 24
+  // bytes 0..2 by a byte permute (ALU), byte 3 by a multiply-high (FMA pipe)
+  const uint32_t byte = (I < 3) ? prmt(u, 0u, 0x4440u + I) : __umulhi(u, m.p8);
   return __uint_as_float(byte * m.e23 + m.e23);
 }
 

@@ -14,18 +14,18 @@ constexpr int kWarps = 8;                  // warps per CTA: all copy, decode an
 constexpr int kThreads = 32 * kWarps;
 constexpr int kTileRows = 16;              // rows per tile: one m16 step
 constexpr int kMaxCols = 16;               // activation columns per pass
-constexpr int kStages = 3;                 // per-warp ring depth (slices in flight + 1)
+#ifndef QMV_STAGES
+#define QMV_STAGES 3                       // per-warp ring depth (slices in flight + 1)
+#endif
+constexpr int kStages = QMV_STAGES;
 #ifndef QMV_SLICE_BYTES
 #define QMV_SLICE_BYTES 256                // bytes of codes per row in a warp's K-slice
 #endif
 #ifndef QMV_MIN_CTAS
 #define QMV_MIN_CTAS 2                     // CTAs per SM the kernel's register budget targets
 #endif
-#ifndef QMV_INDEP_MMA
-#define QMV_INDEP_MMA 0                    // block-scaled formats: the block's two MMA steps independent
-#endif
-#ifndef QMV_LUT_TWO_ACC
-#define QMV_LUT_TWO_ACC 0                  // palette format: two accumulator chains
+#ifndef QMV_CTA_MAJOR
+#define QMV_CTA_MAJOR 0
 #endif
 constexpr int kSliceBytes = QMV_SLICE_BYTES;
 constexpr int kMinCtas = QMV_MIN_CTAS;
@@ -37,8 +37,8 @@ constexpr int kStaticSmem = 6 * 1024;      // the kernel's static shared memory 
 
 // Aux (scale / palette) staging mode of a launch.
 enum AuxMode : int {
-  kAuxRows = 0,   // per-row bulk copies of the chunk's scale segment (aligned shapes)
-  kAuxBlock = 1,  // the tile's whole scale block, every stage (any K % 32 == 0)
+  kAuxRows = 0,   // 8-byte asynchronous copies of each row's scale segment (8-byte granular rows)
+  kAuxBlock = 1,  // plain byte loads of the slice's scales (any K % 32 == 0)
   kAuxLut = 2     // the tile's 16 x 16 fp16 palette, first chunk only
 };
 
@@ -57,6 +57,7 @@ struct MvParams {
   int B;                   // dense: activation rows; gather: tokens
   int topk, E, x_per_slot, gather;
   int KC, nchunks;         // in-features per warp slice, slices per tile
+  int gk;                  // K granule of split units (in-features)
   int RS;                  // shared-memory bytes per staged code row
   int AS;                  // shared-memory bytes per staged scale row (kAuxRows)
   int aux_mode;

@@ -75,11 +75,6 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
 __device__ __forceinline__ void sts_f32x2(uint32_t a, float u, float v) {
   asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(u), "f"(v) : "memory");
 }
-// 128-bit shared load only where `on`; elsewhere the registers keep whatever
-// they held (used for activation columns whose outputs are never stored).
-__device__ __forceinline__ void lds128_if(uint4& v, uint32_t a, uint32_t on) {
-  if (on) v = lds128(a);
-}
 __device__ __forceinline__ uint4 ldg_nc_128(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
@@ -93,14 +88,19 @@ __device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Wait until at most `n` (0..2) of this thread's committed copy groups are pending.
+// Wait until at most `n` (0..4; larger counts wait for 4) of this thread's
+// committed copy groups are pending.
 __device__ __forceinline__ void cp_async_wait(int n) {
   if (n <= 0)
     asm volatile("cp.async.wait_group 0;" ::: "memory");
   else if (n == 1)
     asm volatile("cp.async.wait_group 1;" ::: "memory");
-  else
+  else if (n == 2)
     asm volatile("cp.async.wait_group 2;" ::: "memory");
+  else if (n == 3)
+    asm volatile("cp.async.wait_group 3;" ::: "memory");
+  else
+    asm volatile("cp.async.wait_group 4;" ::: "memory");
 }
 
 // Block-scale of (row, block) from the staged scale region (fp4: the e8m0
@@ -155,47 +155,21 @@ __device__ __forceinline__ void decode_block(uint32_t crow_g, uint32_t crow_g8, 
 // Multiply-accumulate one decoded block: palette formats accumulate directly,
 // block-scaled formats scale the block's exact partial in fp32.
 template <int FMT, int NT>
-__device__ __forceinline__ void mac_block(float (&acc)[NT][4], float (&acc2)[NT][4], const uint32_t (&a0)[4],
-                                          const uint32_t (&a1)[4], const uint4 (&xr)[NT], float sg, float sh) {
-  if constexpr (FmtT<FMT>::kLut) {
-#if QMV_LUT_TWO_ACC
+__device__ __forceinline__ void mac_block(float (&acc)[NT][4], const uint32_t (&a0)[4], const uint32_t (&a1)[4],
+                                          const uint4 (&xr)[NT], float sg, float sh) {
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {  // two accumulator chains: half the dependent MMA latency
-      mma16816(acc[n], a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
-      mma16816(acc2[n], a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
-    }
-#else
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
+  for (int n = 0; n < NT; ++n) {
+    if constexpr (FmtT<FMT>::kLut) {
       mma16816(acc[n], a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
       mma16816(acc[n], a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
-    }
-#endif
-  } else {
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-#if QMV_INDEP_MMA
-      // the block's two MMA steps into separate zero-based partials: no MMA-to-MMA dependency
-      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f}, e[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      mma16816(d, a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
-      mma16816(e, a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
-      acc[n][0] = fmaf(d[0], sg, acc[n][0]);
-      acc[n][1] = fmaf(d[1], sg, acc[n][1]);
-      acc[n][2] = fmaf(d[2], sh, acc[n][2]);
-      acc[n][3] = fmaf(d[3], sh, acc[n][3]);
-      acc2[n][0] = fmaf(e[0], sg, acc2[n][0]);
-      acc2[n][1] = fmaf(e[1], sg, acc2[n][1]);
-      acc2[n][2] = fmaf(e[2], sh, acc2[n][2]);
-      acc2[n][3] = fmaf(e[3], sh, acc2[n][3]);
-#else
-      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      mma16816(d, a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
+    } else {
+      float d[4];
+      mma16816_zc(d, a0[0], a0[1], a0[2], a0[3], xr[n].x, xr[n].y);
       mma16816(d, a1[0], a1[1], a1[2], a1[3], xr[n].z, xr[n].w);
       acc[n][0] = fmaf(d[0], sg, acc[n][0]);
       acc[n][1] = fmaf(d[1], sg, acc[n][1]);
       acc[n][2] = fmaf(d[2], sh, acc[n][2]);
       acc[n][3] = fmaf(d[3], sh, acc[n][3]);
-#endif
     }
   }
 }
@@ -204,8 +178,8 @@ __device__ __forceinline__ void mac_block(float (&acc)[NT][4], float (&acc2)[NT]
 // is a base plus an immediate, and the slice's scales of a row are read with
 // one or two 128-bit loads.
 template <int FMT, int NT, int NB>
-__device__ __forceinline__ void slice_full(float (&acc)[NT][4], float (&acc2)[NT][4], uint32_t crow_g, uint32_t crow_g8, uint32_t sa_g,
-                                           uint32_t sa_g8, const uint32_t (&xb)[NT], const uint32_t (&xon)[NT], int t,
+__device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g, uint32_t crow_g8, uint32_t sa_g,
+                                           uint32_t sa_g8, const uint32_t (&xb)[NT], int t,
                                            const Palette& pg, const Palette& pg8, const Mul& m) {
   using F = FmtT<FMT>;
   uint4 sg0 = make_uint4(0u, 0u, 0u, 0u), sh0 = sg0, sg1 = sg0, sh1 = sg0;
@@ -221,7 +195,7 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], float (&acc2)[NT
   for (int i = 0; i < NB; ++i) {
     uint4 xr[NT];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) lds128_if(xr[n], xb[n] + 64u * (uint32_t)i, xon[n]);
+    for (int n = 0; n < NT; ++n) xr[n] = lds128(xb[n] + 64u * (uint32_t)i);
     uint32_t a0[4], a1[4];
     decode_block<FMT>(crow_g, crow_g8, i, t, pg, pg8, m, a0, a1);
     float sg = 0.0f, sh = 0.0f;
@@ -247,7 +221,7 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], float (&acc2)[NT
         default: sg = half_at<7>(vg); sh = half_at<7>(vh); break;
       }
     }
-    mac_block<FMT, NT>(acc, acc2, a0, a1, xr, sg, sh);
+    mac_block<FMT, NT>(acc, a0, a1, xr, sg, sh);
   }
 }
 
@@ -255,57 +229,6 @@ __device__ __forceinline__ uint8_t ldg_u8(const uint8_t* p) {
   uint32_t v;
   asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(p));
   return (uint8_t)v;
-}
-
-// Issue one K-slice (16 rows x kc weights) of a tile into the warp's stage.
-// Lane L copies the 16-byte chunks (row 2j + L/16, column L%16) for j < 8;
-// rows past N re-read the last row (their outputs are never stored).  Scales
-// go by 16-byte copies when rows are aligned, else by plain byte loads
-// (synchronous; only for shapes whose scale rows are not 16-byte multiples).
-template <int FMT>
-__device__ __forceinline__ void issue_slice(const MvParams& p, const uint8_t* crow0, const uint8_t* arow0,
-                                            int nrows, int k0, int kc, uint32_t stage, int lane) {
-  using F = FmtT<FMT>;
-  const int cpr = kc * F::kBits / 8 / 16;  // 16-byte chunks per row of this slice (<= 16)
-  const int col = lane & 15;
-  const uint8_t* cbase = crow0 + (int64_t)k0 * F::kBits / 8 + col * 16;
-  if (col < cpr) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int row = 2 * j + (lane >> 4);
-      const int r = min(row, nrows - 1);
-      cp_async16(stage + (uint32_t)row * p.RS + (uint32_t)col * 16u, cbase + (int64_t)r * p.code_row_bytes);
-    }
-  }
-  const uint32_t auxs = stage + p.aux_off;
-  if constexpr (F::kLut) {
-    if (k0 == 0) {  // the tile's palette rides with its first slice
-      const int r = min(lane >> 1, nrows - 1);
-      cp_async16(auxs + (uint32_t)lane * 16u, arow0 + (int64_t)r * 32 + (lane & 1) * 16);
-    }
-  } else {
-    const int sbytes = (kc / 32) * F::kSB;  // scale bytes per row of this slice
-    const uint8_t* abase = arow0 + (int64_t)(k0 / 32) * F::kSB;
-    if (p.aux_mode == kAuxRows) {
-      if (sbytes >= 16) {  // 16 or 32 bytes per row: 16-byte copies
-        const int apr = sbytes / 16;
-        if (lane < kTileRows * apr) {
-          const int row = apr == 1 ? lane : (lane >> 1), c16 = apr == 1 ? 0 : (lane & 1);
-          const int r = min(row, nrows - 1);
-          cp_async16(auxs + (uint32_t)row * p.AS + (uint32_t)c16 * 16u, abase + (int64_t)r * p.aux_row_bytes + c16 * 16);
-        }
-      } else if (lane < kTileRows) {  // 8 bytes per row: 8-byte copies
-        const int r = min(lane, nrows - 1);
-        cp_async8(auxs + (uint32_t)lane * p.AS, abase + (int64_t)r * p.aux_row_bytes);
-      }
-    } else {
-      for (int i = lane; i < kTileRows * sbytes; i += 32) {
-        const int row = i / sbytes, b = i - row * sbytes;
-        const int r = min(row, nrows - 1);
-        sts_u8(auxs + (uint32_t)row * p.AS + (uint32_t)b, ldg_u8(abase + (int64_t)r * p.aux_row_bytes + b));
-      }
-    }
-  }
 }
 
 template <int FMT, int NT>
@@ -370,8 +293,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
     }
   }
   // Activations once per CTA: row r at xbase + r * XS, in the k order the
-  // format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7) per 8), and
-  // a zero row for the columns a group does not use.
+  // format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7) per 8).
   const uint32_t xbase = sbase + p.off_x;
   {
     const int64_t per_row = p.K / 8;
@@ -385,86 +307,186 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
       }
       sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
     }
-    for (int64_t j = tid; j < per_row; j += kThreads)
-      sts128(xbase + (uint32_t)((int64_t)p.n_xrows * p.XS + 16 * j), make_uint4(0u, 0u, 0u, 0u));
   }
   __syncthreads();
 
-  // ---- per-warp pipelines over whole tiles ----------------------------------
-  const int64_t total = (int64_t)gt.ngroups * p.tiles;
-  const int64_t gwarp = (int64_t)blockIdx.x * kWarps + warp, nwarps = (int64_t)gridDim.x * kWarps;
-  if (gwarp >= total) return;
+  // ---- the warp's work items ------------------------------------------------
+  // Units are (column group, 16-row tile) pairs.  With at least as many
+  // units as warps (W), each warp takes whole units round robin (all of K,
+  // one warp, no reduction).  With fewer, units are dealt to CTAs and a CTA's
+  // 8 warps split each one along K, adding their partial sums in shared
+  // memory in warp order (deterministic).  Each warp streams its items
+  // through a private ring of S slices (kc in-features of 16 rows) filled by
+  // 16-byte asynchronous copies S-1 slices ahead of the math.
+  const int ngroups = gt.ngroups;
+  const int64_t total = (int64_t)ngroups * p.tiles;
+  const int grid = (int)gridDim.x;
+  const int64_t W = (int64_t)grid * kWarps;
+  // Warps are numbered warp-major across CTAs, so the units of a partial last
+  // round land 4-5 per CTA instead of filling whole CTAs (and SMs) first.
+#if QMV_CTA_MAJOR
+  const int64_t gwarp = (int64_t)blockIdx.x * kWarps + warp;
+#else
+  const int64_t gwarp = (int64_t)warp * grid + blockIdx.x;
+#endif
+  int64_t R, tail0;
+  int T;
+  if (total >= W) {  // whole units only: this warp's units gwarp, gwarp + W, ...
+    R = (total - gwarp + W - 1) / W;
+    tail0 = total;
+    T = 0;
+  } else {  // fewer units than warps: each CTA splits its units along K
+    R = 0;
+    tail0 = 0;
+    T = total > (int64_t)blockIdx.x ? (int)((total - blockIdx.x + grid - 1) / grid) : 0;
+  }
+  const int nitems = (int)R + T;
+  // this warp's share of K in the split units: whole granules of p.gk
+  const int Kg = (int)((p.K + p.gk - 1) / p.gk);
+  const int kb_w = (int)min(p.K, (int64_t)(warp * Kg / kWarps) * p.gk);
+  const int ke_w = (int)min(p.K, (int64_t)((warp + 1) * Kg / kWarps) * p.gk);
+  const int KC = p.KC;
+  const int nsl_main = p.nchunks;
+  const int nsl_tail = ke_w > kb_w ? (ke_w - kb_w + KC - 1) / KC : 0;
+  const int n_issue = nsl_tail > 0 ? nitems : (int)R;  // items that move any bytes
+
+  struct Item {
+    int64_t tile;
+    int grp, kbeg, kend, nsl;
+    bool split;
+  };
+  auto item_at = [&](int i) {
+    Item it;
+    int64_t u;
+    if (i < R) {
+      u = gwarp + (int64_t)i * W;
+      it.kbeg = 0; it.kend = (int)p.K; it.nsl = nsl_main; it.split = false;
+    } else {
+      u = tail0 + blockIdx.x + (int64_t)(i - R) * grid;
+      it.kbeg = kb_w; it.kend = ke_w; it.nsl = nsl_tail; it.split = true;
+    }
+    if (ngroups == 1) {
+      it.grp = 0; it.tile = u;
+    } else {
+      it.grp = (int)(u / p.tiles); it.tile = u - (int64_t)it.grp * p.tiles;
+    }
+    return it;
+  };
+
   const int S = p.stages;
   const uint32_t ring = sbase + p.off_stage + (uint32_t)(warp * S) * p.stage_bytes;
+  const uint32_t ring_end = ring + (uint32_t)S * p.stage_bytes;
   const int g = lane >> 2, t = lane & 3;
+  const int cr = lane >> 1, ch = lane & 1;  // copy role: row cr of the tile, 16-byte half ch of each 32 bytes
   const Mul mul = Mul::make();
-  const int KCW = p.KC;  // weights per slice
+  const bool aux_fast = p.aux_mode != kAuxBlock;
+  constexpr int kAuxSteps = (kSliceBytes * 8 / F::kBits / 32 * F::kSB + 15) / 16;  // 16-byte steps of scales
 
-  // Cursor over this warp's units (tile, group) in order, advanced without
-  // divisions: unit u = gwarp + i * nwarps, group = u / tiles.
-  struct Cursor {
-    int64_t tile;
-    int grp;
+  // ---- issue cursor ----
+  int ii = 0, ic = 0;
+  Item iI{};
+  // Code copies: lane (cc, rp) moves 16-byte column cc of rows 2j + rp, so each
+  // instruction covers whole 128-byte lines of two rows.  Scale / palette
+  // copies: lane (cr, ch) serves row cr.
+  const int cc = lane & 15, rp = lane >> 4;
+  const int64_t rb2 = 2 * p.code_row_bytes;
+  const uint8_t* crow_base = nullptr;  // the item's tile row 0 at the next slice, + 16 * cc
+  const uint8_t* asrc = nullptr;  // row cr's scales at the next slice (+ 8 * ch) / its palette (+ 16 * ch)
+  int64_t irow0 = 0;
+  int inrows = 0;
+  auto load_issue_item = [&]() {
+    iI = item_at(ii);
+    irow0 = iI.tile * kTileRows;
+    inrows = (int)min((int64_t)kTileRows, p.N - irow0);
+    const int64_t row = min(irow0 + cr, p.N - 1);  // rows past N re-read the last row (outputs never stored)
+    const int e = gt.expert[iI.grp];
+    crow_base = p.codes + (int64_t)e * p.expert_code_bytes + irow0 * p.code_row_bytes + (int64_t)iI.kbeg * F::kBits / 8 + 16 * cc;
+    if constexpr (F::kLut)
+      asrc = p.aux + (int64_t)e * p.expert_aux_bytes + row * 32 + 16 * ch;
+    else
+      asrc = p.aux + (int64_t)e * p.expert_aux_bytes + row * p.aux_row_bytes + (int64_t)(iI.kbeg / 32) * F::kSB + 8 * ch;
   };
-  auto advance = [&](Cursor& cu) {
-    cu.tile += nwarps;
-    while (cu.tile >= p.tiles) {
-      cu.tile -= p.tiles;
-      ++cu.grp;
+  if (n_issue > 0) load_issue_item();
+  auto issue_next = [&](uint32_t stage) {
+    const int k0 = iI.kbeg + ic * KC;
+    const int kc = min(KC, iI.kend - k0);
+    // codes: rows past N re-read the last row (their outputs are never stored)
+    const int cb = kc * F::kBits / 8;  // code bytes per row, a multiple of 16
+    if (16 * cc < cb) {
+      uint32_t d = stage + (uint32_t)rp * p.RS + 16u * cc;
+      if (inrows == kTileRows) {
+        const uint8_t* q = crow_base + rp * p.code_row_bytes;
+#pragma unroll
+        for (int j = 0; j < kTileRows / 2; ++j) {
+          cp_async16(d, q);
+          q += rb2;
+          d += 2u * p.RS;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kTileRows / 2; ++j) {
+          const int r = min(2 * j + rp, inrows - 1);
+          cp_async16(d, crow_base + r * p.code_row_bytes);
+          d += 2u * p.RS;
+        }
+      }
     }
-  };
-  Cursor ci{gwarp, 0};  // issue cursor
-  while (ci.tile >= p.tiles) {
-    ci.tile -= p.tiles;
-    ++ci.grp;
-  }
-  const Cursor c_first = ci;
-  int c_issue = 0;
-  const uint8_t* crow0 = nullptr;
-  const uint8_t* arow0 = nullptr;
-  int nrows_issue = 0;
-  auto set_rows = [&]() {
-    const int64_t row0 = ci.tile * kTileRows;
-    nrows_issue = (int)min((int64_t)kTileRows, p.N - row0);
-    const int e = gt.expert[ci.grp];
-    crow0 = p.codes + (int64_t)e * p.expert_code_bytes + row0 * p.code_row_bytes;
-    arow0 = p.aux + (int64_t)e * p.expert_aux_bytes + row0 * p.aux_row_bytes;
-  };
-  set_rows();
-  auto issue_next = [&](int stage_idx) {
-    const int k0 = c_issue * KCW;
-    issue_slice<FMT>(p, crow0, arow0, nrows_issue, k0, min(KCW, (int)(p.K - k0)),
-                     ring + (uint32_t)stage_idx * p.stage_bytes, lane);
-    if (++c_issue == p.nchunks) {
-      c_issue = 0;
-      advance(ci);
-      if (ci.grp < gt.ngroups) set_rows();
+    crow_base += cb;
+    const uint32_t da = stage + p.aux_off;
+    if constexpr (F::kLut) {
+      if (ic == 0) cp_async16(da + (uint32_t)cr * 32u + 16u * ch, asrc);  // the palette rides with the first slice
+    } else if (aux_fast) {
+      const int sb = (kc / 32) * F::kSB;  // scale bytes per row, a multiple of 8
+#pragma unroll
+      for (int j = 0; j < kAuxSteps; ++j)
+        if (16 * j + 8 * ch < sb) cp_async8(da + (uint32_t)cr * p.AS + 16u * j + 8u * ch, asrc + 16 * j);
+      asrc += sb;
+    } else {
+      // scale rows that are not 8-byte granular: plain byte loads
+      const int sbytes = (kc / 32) * F::kSB;
+      const int e = gt.expert[iI.grp];
+      const uint8_t* abase = p.aux + (int64_t)e * p.expert_aux_bytes + irow0 * p.aux_row_bytes + (int64_t)(k0 / 32) * F::kSB;
+      for (int i = lane; i < kTileRows * sbytes; i += 32) {
+        const int row = i / sbytes, b = i - row * sbytes;
+        const int r = min(row, inrows - 1);
+        sts_u8(da + (uint32_t)row * p.AS + (uint32_t)b, ldg_u8(abase + (int64_t)r * p.aux_row_bytes + b));
+      }
+    }
+    if (++ic == iI.nsl) {
+      ic = 0;
+      if (++ii < n_issue) load_issue_item();
     }
   };
 
   // prologue: S-1 slices in flight
+  uint32_t fill = ring;
   for (int j = 0; j < S - 1; ++j) {
-    if (ci.grp < gt.ngroups) issue_next(j);
+    if (ii < n_issue) issue_next(fill);
     cp_async_commit();
+    fill += p.stage_bytes;
   }
 
-  float acc[NT][4], acc2[NT][4];  // two accumulator sets (summed once per tile)
+  // ---- consume ----
+  float* red = reinterpret_cast<float*>(smem + p.off_red);  // split units: [warp][NT][4][lane]
+  float acc[NT][4];
   Palette pg, pg8;
-  uint32_t xa[NT], xon[NT];
+  uint32_t xa[NT];
   int xa_grp = -1;
-  int s = 0, s_fill = S - 1;
-  for (Cursor cc = c_first; cc.grp < gt.ngroups; advance(cc)) {
-    const int grp = cc.grp;
-    const int64_t row0 = cc.tile * kTileRows;
+  uint32_t cons = ring;
+  for (int i = 0; i < nitems; ++i) {
+    const Item it = item_at(i);
+    const int grp = it.grp;
+    const int64_t row0 = it.tile * kTileRows;
     const int nrows = (int)min((int64_t)kTileRows, p.N - row0);
+    const int ncols = gt.count[grp], gstart = gt.start[grp];
     if (grp != xa_grp) {  // activation rows of this column group
       xa_grp = grp;
-      const int ncols = gt.count[grp], gstart = gt.start[grp];
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
+        // a column the group does not use reads row 0: MMA columns are
+        // independent and its outputs are never stored
         const int col = 8 * n + g;
-        int xrow = p.n_xrows;  // the zero row
-        xon[n] = col < ncols ? 1u : 0u;
+        int xrow = 0;
         if (col < ncols) {
           const int pair = gt.sorted[gstart + col];
           xrow = p.gather ? (p.x_per_slot ? pair : pair / p.topk) : pair;
@@ -475,20 +497,19 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[n][q] = acc2[n][q] = 0.0f;
+      for (int q = 0; q < 4; ++q) acc[n][q] = 0.0f;
 
-    for (int c = 0; c < p.nchunks; ++c) {
+    for (int c = 0; c < it.nsl; ++c) {
       // keep S-1 slices in flight: refill the stage freed by the previous slice
-      if (ci.grp < gt.ngroups) issue_next(s_fill);
+      if (ii < n_issue) issue_next(fill);
       cp_async_commit();
-      s_fill = (s_fill + 1 == S) ? 0 : s_fill + 1;
+      fill = (fill + p.stage_bytes == ring_end) ? ring : fill + p.stage_bytes;
       cp_async_wait(S - 1);  // this slice's copies (all lanes) have landed
       __syncwarp();
 
-      const uint32_t stage = ring + (uint32_t)s * p.stage_bytes;
-      const uint32_t auxs = stage + p.aux_off;
-      const int k0 = c * KCW;
-      const int kc = min(KCW, (int)(p.K - k0));
+      const uint32_t auxs = cons + p.aux_off;
+      const int k0 = it.kbeg + c * KC;
+      const int kc = min(KC, it.kend - k0);
       if constexpr (F::kLut) {
         if (c == 0) {
           uint32_t e0[8], e1[8];
@@ -502,20 +523,22 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
           pg8 = palette_from_words(e1);
         }
       }
-      const uint32_t crow_g = stage + (uint32_t)g * p.RS, crow_g8 = stage + (uint32_t)(g + 8) * p.RS;
+      const uint32_t crow_g = cons + (uint32_t)g * p.RS, crow_g8 = cons + (uint32_t)(g + 8) * p.RS;
       const uint32_t sa_g = auxs + (uint32_t)g * p.AS, sa_g8 = auxs + (uint32_t)(g + 8) * p.AS;
       constexpr int kNB = kSliceBytes * 8 / F::kBits / 32;  // blocks in a full slice
-      if (kc == KCW && KCW == kNB * 32 && (F::kLut || p.aux_mode == kAuxRows)) {
-        uint32_t xb[NT];
+      uint32_t xb[NT];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
-        slice_full<FMT, NT, kNB>(acc, acc2, crow_g, crow_g8, sa_g, sa_g8, xb, xon, t, pg, pg8, mul);
+      for (int n = 0; n < NT; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
+      if (kc == kNB * 32 && aux_fast) {
+        slice_full<FMT, NT, kNB>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
+      } else if (kc == kNB * 16 && aux_fast) {
+        slice_full<FMT, NT, kNB / 2>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
       } else {
         const int nbc = kc / 32;
         for (int b = 0; b < nbc; ++b) {
           uint4 xr[NT];
 #pragma unroll
-          for (int n = 0; n < NT; ++n) lds128_if(xr[n], xa[n] + (uint32_t)(k0 + 32 * b) * 2u, xon[n]);
+          for (int n = 0; n < NT; ++n) xr[n] = lds128(xb[n] + 64u * (uint32_t)b);
           uint32_t a0[4], a1[4];
           decode_block<FMT>(crow_g, crow_g8, b, t, pg, pg8, mul, a0, a1);
           float sg = 0.0f, sh = 0.0f;
@@ -523,27 +546,48 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
             sg = stage_scale<FMT>(sa_g + (uint32_t)b * F::kSB, mul);
             sh = stage_scale<FMT>(sa_g8 + (uint32_t)b * F::kSB, mul);
           }
-          mac_block<FMT, NT>(acc, acc2, a0, a1, xr, sg, sh);
+          mac_block<FMT, NT>(acc, a0, a1, xr, sg, sh);
         }
       }
       __syncwarp();  // all lanes are done with this stage before it is refilled
-      s = (s + 1 == S) ? 0 : s + 1;
+      cons = (cons + p.stage_bytes == ring_end) ? ring : cons + p.stage_bytes;
     }
 
-    // ---- store this tile's outputs: lane (g, t) holds rows g, g+8, cols 2t, 2t+1 ----
-    const int ncols = gt.count[grp], gstart = gt.start[grp];
+    // ---- outputs: lane (g, t) holds rows g, g+8, columns 2t, 2t+1 of each n-tile ----
     const float f = (FMT == QMV_FMT_FP4) ? 0.5f : 1.0f;  // the fp4 block scales carried a factor 2
+    if (!it.split) {
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
+      for (int n = 0; n < NT; ++n) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int col = 8 * n + 2 * t + (q & 1);
-        const int row = g + 8 * (q >> 1);
-        if (col < ncols && row < nrows) {
-          const int pair = gt.sorted[gstart + col];
-          p.y[(int64_t)pair * p.N + row0 + row] = (acc[n][q] + acc2[n][q]) * f;
+        for (int q = 0; q < 4; ++q) {
+          const int col = 8 * n + 2 * t + (q & 1);
+          const int row = g + 8 * (q >> 1);
+          if (col < ncols && row < nrows) {
+            const int pair = gt.sorted[gstart + col];
+            p.y[(int64_t)pair * p.N + row0 + row] = acc[n][q] * f;
+          }
         }
       }
+    } else {
+      // split unit: partial sums of all 8 warps, added in warp order
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) red[((warp * NT + n) * 4 + q) * 32 + lane] = acc[n][q];
+      __syncthreads();
+      if (tid < NT * 4 * 32) {
+        const int ln = tid & 31, q = (tid >> 5) & 3, n = tid >> 7;
+        float v = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) v += red[((w * NT + n) * 4 + q) * 32 + ln];
+        const int col = 8 * n + 2 * (ln & 3) + (q & 1);
+        const int row = (ln >> 2) + 8 * (q >> 1);
+        if (col < ncols && row < nrows) {
+          const int pair = gt.sorted[gstart + col];
+          p.y[(int64_t)pair * p.N + row0 + row] = v * f;
+        }
+      }
+      __syncthreads();
     }
   }
   cp_async_wait(0);
@@ -572,21 +616,19 @@ bool plan_matvec(int fmt, MvParams& p) {
   // 32 mod 128 (64-bit loads).
   p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 16 : 32));
   int64_t aux_region;
+  // split units divide K in granules whose code and scale segments start on
+  // 16- and 8-byte boundaries
+  p.gk = fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128);
   if (fi.lut) {
     p.aux_mode = kAuxLut;
     p.AS = 32;
     aux_region = kTileRows * 32;
   } else {
     const int64_t slice_sc = (int64_t)(p.KC / 32) * fi.scale_bytes;
-    const int64_t last_sc = ((p.K - (int64_t)(p.nchunks - 1) * p.KC) / 32) * fi.scale_bytes;
-    // asynchronous scale copies (16 or 8 bytes) when every row's slice
-    // segment starts on that boundary and is a multiple of it
-    const int64_t cs = (slice_sc % 16 == 0) ? 16 : 8;
-    const bool based = (reinterpret_cast<uintptr_t>(p.aux) % cs) == 0;
-    if (based && slice_sc % 8 == 0 && slice_sc <= 32 && p.aux_row_bytes % cs == 0 && last_sc % cs == 0)
-      p.aux_mode = kAuxRows;
-    else
-      p.aux_mode = kAuxBlock;
+    // asynchronous 8-byte scale copies when every row's scales start on an
+    // 8-byte boundary and come in whole 8-byte pieces
+    const bool based = (reinterpret_cast<uintptr_t>(p.aux) % 8) == 0;
+    p.aux_mode = (based && p.aux_row_bytes % 8 == 0) ? kAuxRows : kAuxBlock;
     int64_t j = (slice_sc + 15) / 16;
     if (j % 2 == 0) ++j;  // odd multiple of 16 bytes: rows g = 0..7 hit distinct banks
     p.AS = (int)(16 * j);
@@ -596,9 +638,10 @@ bool plan_matvec(int fmt, MvParams& p) {
   p.stage_bytes = (int)round_up(p.aux_off + aux_region, 128);
   p.XS = (int)(round_up(2 * p.K, 128) + 64);  // 64 mod 128: conflict-free 128-bit reads
   p.n_xrows = p.gather ? (p.x_per_slot ? p.B * p.topk : p.B) : p.B;
-  p.off_red = 0;
-  p.off_x = 0;
-  p.off_stage = (int)round_up((int64_t)(p.n_xrows + 1) * p.XS, 128);  // + a zero row
+  const int nt = p.B > 8 ? 2 : 1;
+  p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
+  p.off_x = (int)round_up((int64_t)kWarps * nt * 4 * 32 * 4, 128);
+  p.off_stage = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128);
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
   // the most CTAs per SM (up to the kernel's register budget) with the
   // deepest ring (<= kStages slices per warp) that fits
@@ -628,11 +671,11 @@ static cudaError_t launch_t(const MvParams& p, int num_sms, cudaStream_t stream)
     if (err != cudaSuccess) return err;
     attr_set[dev] = true;
   }
-  // enough warps for every (group, tile) unit, at most ctas_per_sm CTAs per SM
+  // one CTA per (group, tile) unit up to the resident-CTA slots: units beyond
+  // whole rounds of warps are split along K inside a CTA
   const int64_t upper_units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
-  const int64_t want = (upper_units + kWarps - 1) / kWarps;
   const int64_t slots = (int64_t)num_sms * p.ctas_per_sm;
-  const int grid = (int)(want < slots ? want : slots);
+  const int grid = (int)(upper_units < slots ? upper_units : slots);
   mv_kernel<FMT, NT><<<grid, kThreads, p.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }

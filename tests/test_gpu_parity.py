@@ -211,6 +211,37 @@ def test_matvec_one_hot_columns_bit_exact(q, fmt):
         assert np.array_equal(y[i], D[:, k]), (fmt, k)
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K", [(100, 512), (37, 2048)])
+def test_matvec_batch1_one_hot_bit_exact(q, fmt, N, K):
+    """Batch 1 with K a multiple of 256 takes the form whose MMA columns carry
+    blocks: x = e_k, one launch per k, must return column k of Wdq exactly
+    (pins the block-to-column and in-block k mapping of that form)."""
+    c_o, s_o, _ = _inputs(fmt, N, K, 1, seed=23 + K)
+    c, s = torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda()
+    D = orc.dequant(FID[fmt], c_o, s_o, N, K)
+    for k in [0, 1, 2, 3, 4, 7, 8, 9, 15, 16, 31, 32, 33, 63, 64, 100, 255, 256, 300, K - 1]:
+        x = torch.zeros((1, K), dtype=torch.float16, device="cuda")
+        x[0, k] = 1.0
+        y = q.matvec(q.__dict__["FMT_" + fmt.upper()], c, s, x).cpu().numpy()
+        assert np.array_equal(y[0], D[:, k]), (fmt, k)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_matvec_batch1_whole_units(q, fmt):
+    """Enough 16-row tiles that every warp takes whole tiles (no K split), a
+    ragged last tile, batch 1."""
+    N, K = 37905, 2048  # 2370 tiles: at least one whole tile per warp of a full grid
+    c_o, s_o, xn = _inputs(fmt, N, K, 1, seed=29)
+    y = q.matvec(q.__dict__["FMT_" + fmt.upper()], torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(),
+                 torch.from_numpy(xn).cuda()).cpu().numpy()
+    r = orc.matvec(FID[fmt], c_o, s_o, xn, N, K)
+    assert rel_err(y, r) < TOL
+    y2 = q.matvec(q.__dict__["FMT_" + fmt.upper()], torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(),
+                  torch.from_numpy(xn).cuda()).cpu().numpy()
+    assert np.array_equal(y, y2)
+
+
 def test_matvec_output_guard_bands(q):
     """Sentinels around the output rows stay untouched (no out-of-bounds
     writes on a ragged last tile)."""

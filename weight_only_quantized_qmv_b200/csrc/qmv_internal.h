@@ -33,6 +33,7 @@ constexpr int kMaxCtasPerSM = 4;
 constexpr int kMaxPairs = 256;             // B * topk upper bound (16 * 16)
 constexpr int kSmemLimit = 227 * 1024;     // per-block opt-in maximum on sm_100
 constexpr int kSmemPerSM = 228 * 1024;     // shared memory of one SM
+constexpr int kZeroBytes = 1024;           // zero activations read by the batch-1 form's idle columns
 constexpr int kStaticSmem = 6 * 1024;      // the kernel's static shared memory (group table), rounded up
 
 // Aux (scale / palette) staging mode of a launch.
@@ -58,6 +59,8 @@ struct MvParams {
   int topk, E, x_per_slot, gather;
   int KC, nchunks;         // in-features per warp slice, slices per tile
   int gk;                  // K granule of split units (in-features)
+  int one;                 // batch-1 block-column form (dense B == 1, K % 256 == 0)
+  int off_zero;            // its zero activation region
   int RS;                  // shared-memory bytes per staged code row
   int AS;                  // shared-memory bytes per staged scale row (kAuxRows)
   int aux_mode;

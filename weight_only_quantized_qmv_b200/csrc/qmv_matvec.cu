@@ -225,15 +225,109 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g,
   }
 }
 
+// Batch 1: the eight MMA columns carry eight blocks instead of eight
+// activation columns.  In a group of 8 blocks (16 MMA steps) lane (g, t)
+// decodes blocks t (steps 0-7) and t+4 (steps 8-15) of rows g and g+8, so
+// the k-slots 2t, 2t+1, 2t+8, 2t+9 of a step all belong to one block; B
+// column n holds block n's activations and zeros elsewhere (lanes whose
+// column is not their block read a zero region), so D[r][n] ends as block
+// n's partial sum for row r and takes its own scale once per group.  Codes
+// come in one 128-bit load per block and row (4-bit; two for int8).
+//   crow_g / crow_g8: rows g, g+8 of the slice + this lane's block offset
+//   sa_g / sa_g8:     their scale rows in the slice
+//   xl0 / xl1:        activations of block t / t+4 of group 0, or the zero region
+template <int FMT, int NG>
+__device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint32_t crow_g, uint32_t crow_g8,
+                                          uint32_t sa_g, uint32_t sa_g8, uint32_t xl0, uint32_t xl1, int t,
+                                          const Palette& pg, const Palette& pg8, const Mul& m) {
+  using F = FmtT<FMT>;
+  constexpr int kBB = F::kBits * 4;  // code bytes per block and row
+#pragma unroll
+  for (int gi = 0; gi < NG; ++gi) {
+    float d[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t cb = (uint32_t)((8 * gi + 4 * h) * kBB);
+      uint32_t wg[8], wh[8];
+      {
+        const uint4 u = lds128(crow_g + cb), v = lds128(crow_g8 + cb);
+        wg[0] = u.x; wg[1] = u.y; wg[2] = u.z; wg[3] = u.w;
+        wh[0] = v.x; wh[1] = v.y; wh[2] = v.z; wh[3] = v.w;
+        if constexpr (F::kBits == 8) {
+          const uint4 u2 = lds128(crow_g + cb + 16u), v2 = lds128(crow_g8 + cb + 16u);
+          wg[4] = u2.x; wg[5] = u2.y; wg[6] = u2.z; wg[7] = u2.w;
+          wh[4] = v2.x; wh[5] = v2.y; wh[6] = v2.z; wh[7] = v2.w;
+        }
+      }
+      const uint32_t xl = h ? xl1 : xl0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // word group i: in-features 8i..8i+7 of the block, MMA steps 2i and 2i+1
+        const uint4 xv = lds128(xl + (uint32_t)(64 * (8 * gi + 4 * h) + 16 * i));
+        uint32_t g0lo, g0hi, g1lo, g1hi, h0lo, h0hi, h1lo, h1hi;
+        if constexpr (F::kBits == 8) {
+          dec_int8_word(wg[2 * i], g0lo, g0hi);
+          dec_int8_word(wg[2 * i + 1], g1lo, g1hi);
+          dec_int8_word(wh[2 * i], h0lo, h0hi);
+          dec_int8_word(wh[2 * i + 1], h1lo, h1hi);
+        } else if constexpr (FMT == QMV_FMT_FP4) {
+          DecFp4::run(wg[i], g0lo, g0hi, g1lo, g1hi, m);
+          DecFp4::run(wh[i], h0lo, h0hi, h1lo, h1hi, m);
+        } else if constexpr (FMT == QMV_FMT_INT4) {
+          DecInt4::run(wg[i], g0lo, g0hi, g1lo, g1hi, m);
+          DecInt4::run(wh[i], h0lo, h0hi, h1lo, h1hi, m);
+        } else {
+          dec_int4km(pg, wg[i], g0lo, g0hi, g1lo, g1hi, m);
+          dec_int4km(pg8, wh[i], h0lo, h0hi, h1lo, h1hi, m);
+        }
+        if constexpr (F::kLut) {
+          mma16816(dl, g0lo, h0lo, g0hi, h0hi, xv.x, xv.y);
+          mma16816(dl, g1lo, h1lo, g1hi, h1hi, xv.z, xv.w);
+        } else {
+          if (h == 0 && i == 0)
+            mma16816_zc(d, g0lo, h0lo, g0hi, h0hi, xv.x, xv.y);
+          else
+            mma16816(d, g0lo, h0lo, g0hi, h0hi, xv.x, xv.y);
+          mma16816(d, g1lo, h1lo, g1hi, h1hi, xv.z, xv.w);
+        }
+      }
+    }
+    if constexpr (!F::kLut) {
+      // lane (g, t) holds blocks 2t, 2t+1 of the group for rows g and g+8
+      float s0, s1, s2, s3;
+      if constexpr (FMT == QMV_FMT_FP4) {
+        const uint32_t u = lds_u16(sa_g + (uint32_t)(8 * gi + 2 * t));
+        const uint32_t v = lds_u16(sa_g8 + (uint32_t)(8 * gi + 2 * t));
+        s0 = e8m0_x2_to_f32<0>(u, m); s1 = e8m0_x2_to_f32<1>(u, m);
+        s2 = e8m0_x2_to_f32<0>(v, m); s3 = e8m0_x2_to_f32<1>(v, m);
+      } else {
+        const uint32_t u = lds32(sa_g + (uint32_t)(2 * (8 * gi + 2 * t)));
+        const uint32_t v = lds32(sa_g8 + (uint32_t)(2 * (8 * gi + 2 * t)));
+        const __half2 hu = *reinterpret_cast<const __half2*>(&u), hv = *reinterpret_cast<const __half2*>(&v);
+        s0 = __low2float(hu); s1 = __high2float(hu);
+        s2 = __low2float(hv); s3 = __high2float(hv);
+      }
+      acc[0] = fmaf(d[0], s0, acc[0]);
+      acc[0] = fmaf(d[1], s1, acc[0]);
+      acc[1] = fmaf(d[2], s2, acc[1]);
+      acc[1] = fmaf(d[3], s3, acc[1]);
+    }
+  }
+}
+
 __device__ __forceinline__ uint8_t ldg_u8(const uint8_t* p) {
   uint32_t v;
   asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(p));
   return (uint8_t)v;
 }
 
+// NT: activation n-tiles of 8 columns (1 or 2); NT = 0 is the batch-1 form
+// whose MMA columns carry blocks (slice_one).
 template <int FMT, int NT>
 __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_constant__ MvParams p) {
   using F = FmtT<FMT>;
+  constexpr bool kOne = NT == 0;
+  constexpr int NTX = kOne ? 1 : NT;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ GroupTable gt;
   __shared__ int s_ids[kMaxPairs];
@@ -306,6 +400,9 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
                        prmt(v.y, v.w, 0x7632u));
       }
       sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
+    }
+    if constexpr (kOne) {  // the zero activations of the batch-1 form
+      for (int j = tid; j < kZeroBytes / 16; j += kThreads) sts128(sbase + p.off_zero + 16u * j, make_uint4(0u, 0u, 0u, 0u));
     }
   }
   __syncthreads();
@@ -468,9 +565,10 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
 
   // ---- consume ----
   float* red = reinterpret_cast<float*>(smem + p.off_red);  // split units: [warp][NT][4][lane]
-  float acc[NT][4];
+  float acc[NTX][4];
+  float acc1[2], dl[4];  // batch-1 form: rows g, g+8 / the palette format's running MMA sums
   Palette pg, pg8;
-  uint32_t xa[NT];
+  uint32_t xa[NTX];
   int xa_grp = -1;
   uint32_t cons = ring;
   for (int i = 0; i < nitems; ++i) {
@@ -482,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
     if (grp != xa_grp) {  // activation rows of this column group
       xa_grp = grp;
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
+      for (int n = 0; n < NTX; ++n) {
         // a column the group does not use reads row 0: MMA columns are
         // independent and its outputs are never stored
         const int col = 8 * n + g;
@@ -495,9 +593,11 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
       }
     }
 #pragma unroll
-    for (int n = 0; n < NT; ++n)
+    for (int n = 0; n < NTX; ++n)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[n][q] = 0.0f;
+    acc1[0] = acc1[1] = 0.0f;
+    dl[0] = dl[1] = dl[2] = dl[3] = 0.0f;
 
     for (int c = 0; c < it.nsl; ++c) {
       // keep S-1 slices in flight: refill the stage freed by the previous slice
@@ -526,19 +626,33 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
       const uint32_t crow_g = cons + (uint32_t)g * p.RS, crow_g8 = cons + (uint32_t)(g + 8) * p.RS;
       const uint32_t sa_g = auxs + (uint32_t)g * p.AS, sa_g8 = auxs + (uint32_t)(g + 8) * p.AS;
       constexpr int kNB = kSliceBytes * 8 / F::kBits / 32;  // blocks in a full slice
-      uint32_t xb[NT];
+      if constexpr (kOne) {
+        // slices are whole groups of 8 blocks (the host requires K % 256 == 0)
+        const uint32_t xs = xbase + (uint32_t)k0 * 2u, zb = sbase + p.off_zero;
+        const uint32_t xl0 = (g == t) ? xs + 64u * t : zb;
+        const uint32_t xl1 = (g == t + 4) ? xs + 64u * t : zb;
+        const uint32_t tb = (uint32_t)(t * F::kBits * 4);
+        if (kNB >= 16 && kc == kNB * 32)
+          slice_one<FMT, (kNB >= 16 ? kNB / 8 : 1)>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, xl0, xl1, t, pg, pg8, mul);
+        else
+          slice_one<FMT, 1>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, xl0, xl1, t, pg, pg8, mul);
+        __syncwarp();
+        cons = (cons + p.stage_bytes == ring_end) ? ring : cons + p.stage_bytes;
+        continue;
+      }
+      uint32_t xb[NTX];
 #pragma unroll
-      for (int n = 0; n < NT; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
+      for (int n = 0; n < NTX; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
       if (kc == kNB * 32 && aux_fast) {
-        slice_full<FMT, NT, kNB>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
+        slice_full<FMT, NTX, kNB>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
       } else if (kc == kNB * 16 && aux_fast) {
-        slice_full<FMT, NT, kNB / 2>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
+        slice_full<FMT, NTX, kNB / 2>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
       } else {
         const int nbc = kc / 32;
         for (int b = 0; b < nbc; ++b) {
-          uint4 xr[NT];
+          uint4 xr[NTX];
 #pragma unroll
-          for (int n = 0; n < NT; ++n) xr[n] = lds128(xb[n] + 64u * (uint32_t)b);
+          for (int n = 0; n < NTX; ++n) xr[n] = lds128(xb[n] + 64u * (uint32_t)b);
           uint32_t a0[4], a1[4];
           decode_block<FMT>(crow_g, crow_g8, b, t, pg, pg8, mul, a0, a1);
           float sg = 0.0f, sh = 0.0f;
@@ -546,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
             sg = stage_scale<FMT>(sa_g + (uint32_t)b * F::kSB, mul);
             sh = stage_scale<FMT>(sa_g8 + (uint32_t)b * F::kSB, mul);
           }
-          mac_block<FMT, NT>(acc, a0, a1, xr, sg, sh);
+          mac_block<FMT, NTX>(acc, a0, a1, xr, sg, sh);
         }
       }
       __syncwarp();  // all lanes are done with this stage before it is refilled
@@ -555,6 +669,36 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
 
     // ---- outputs: lane (g, t) holds rows g, g+8, columns 2t, 2t+1 of each n-tile ----
     const float f = (FMT == QMV_FMT_FP4) ? 0.5f : 1.0f;  // the fp4 block scales carried a factor 2
+    if constexpr (kOne) {
+      // rows g, g+8: the four lanes of a row hold disjoint blocks; add them
+      float r0 = F::kLut ? dl[0] + dl[1] : acc1[0];
+      float r1 = F::kLut ? dl[2] + dl[3] : acc1[1];
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+      const int pair = gt.sorted[gstart];
+      if (!it.split) {
+        if (t == 0) {
+          if (g < nrows) p.y[(int64_t)pair * p.N + row0 + g] = r0 * f;
+          if (g + 8 < nrows) p.y[(int64_t)pair * p.N + row0 + g + 8] = r1 * f;
+        }
+      } else {
+        if (t == 0) {
+          red[warp * 16 + g] = r0;
+          red[warp * 16 + g + 8] = r1;
+        }
+        __syncthreads();
+        if (tid < kTileRows) {
+          float v = 0.0f;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) v += red[w * 16 + tid];
+          if (tid < nrows) p.y[(int64_t)pair * p.N + row0 + tid] = v * f;
+        }
+        __syncthreads();
+      }
+      continue;
+    }
     if (!it.split) {
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
@@ -611,14 +755,21 @@ bool plan_matvec(int fmt, MvParams& p) {
   p.KC = (int)(p.K < slice ? p.K : slice);
   p.nchunks = (int)((p.K + p.KC - 1) / p.KC);
   const int64_t cb = (int64_t)p.KC * fi.bits / 8;
+  // batch 1 (dense, 4-bit formats): the block-column form, for K in whole
+  // groups of 8 blocks (int8 measured faster on the general form)
+  p.one = (!p.gather && p.B == 1 && p.K % 256 == 0 && fi.bits == 4) ? 1 : 0;
   // Row strides chosen so a warp's shared-memory reads are free of bank
   // conflicts: 4-bit rows at 16 mod 128 bytes (32-bit loads), 8-bit rows at
-  // 32 mod 128 (64-bit loads).
-  p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 16 : 32));
+  // 32 mod 128 (64-bit loads); the batch-1 form's 128-bit loads want 4-bit
+  // rows at 64 mod 128 and 8-bit rows at 16 mod 128.
+  if (p.one)
+    p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 64 : 16));
+  else
+    p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 16 : 32));
   int64_t aux_region;
   // split units divide K in granules whose code and scale segments start on
   // 16- and 8-byte boundaries
-  p.gk = fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128);
+  p.gk = p.one ? 256 : (fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128));
   if (fi.lut) {
     p.aux_mode = kAuxLut;
     p.AS = 32;
@@ -629,6 +780,7 @@ bool plan_matvec(int fmt, MvParams& p) {
     // 8-byte boundary and come in whole 8-byte pieces
     const bool based = (reinterpret_cast<uintptr_t>(p.aux) % 8) == 0;
     p.aux_mode = (based && p.aux_row_bytes % 8 == 0) ? kAuxRows : kAuxBlock;
+    if (p.aux_mode == kAuxBlock) p.one = 0;
     int64_t j = (slice_sc + 15) / 16;
     if (j % 2 == 0) ++j;  // odd multiple of 16 bytes: rows g = 0..7 hit distinct banks
     p.AS = (int)(16 * j);
@@ -641,7 +793,8 @@ bool plan_matvec(int fmt, MvParams& p) {
   const int nt = p.B > 8 ? 2 : 1;
   p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
   p.off_x = (int)round_up((int64_t)kWarps * nt * 4 * 32 * 4, 128);
-  p.off_stage = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128);
+  p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128);
+  p.off_stage = p.off_zero + (p.one ? kZeroBytes : 0);
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
   // the most CTAs per SM (up to the kernel's register budget) with the
   // deepest ring (<= kStages slices per warp) that fits
@@ -680,15 +833,21 @@ static cudaError_t launch_t(const MvParams& p, int num_sms, cudaStream_t stream)
   return cudaGetLastError();
 }
 
-cudaError_t launch_matvec(int fmt, const MvParams& p, int num_sms, cudaStream_t stream) {
+template <int FMT>
+static cudaError_t launch_f(const MvParams& p, int num_sms, cudaStream_t stream) {
   // activation columns served per pass: dense B, gather at most B pairs per
   // expert when ids are distinct per token (groups are capped at 8 * NT)
-  const bool two = p.B > 8;
+  if (p.one) return launch_t<FMT, 0>(p, num_sms, stream);
+  if (p.B > 8) return launch_t<FMT, 2>(p, num_sms, stream);
+  return launch_t<FMT, 1>(p, num_sms, stream);
+}
+
+cudaError_t launch_matvec(int fmt, const MvParams& p, int num_sms, cudaStream_t stream) {
   switch (fmt) {
-    case QMV_FMT_FP4: return two ? launch_t<QMV_FMT_FP4, 2>(p, num_sms, stream) : launch_t<QMV_FMT_FP4, 1>(p, num_sms, stream);
-    case QMV_FMT_INT4: return two ? launch_t<QMV_FMT_INT4, 2>(p, num_sms, stream) : launch_t<QMV_FMT_INT4, 1>(p, num_sms, stream);
-    case QMV_FMT_INT4KM: return two ? launch_t<QMV_FMT_INT4KM, 2>(p, num_sms, stream) : launch_t<QMV_FMT_INT4KM, 1>(p, num_sms, stream);
-    case QMV_FMT_INT8: return two ? launch_t<QMV_FMT_INT8, 2>(p, num_sms, stream) : launch_t<QMV_FMT_INT8, 1>(p, num_sms, stream);
+    case QMV_FMT_FP4: return launch_f<QMV_FMT_FP4>(p, num_sms, stream);
+    case QMV_FMT_INT4: return launch_f<QMV_FMT_INT4>(p, num_sms, stream);
+    case QMV_FMT_INT4KM: return launch_f<QMV_FMT_INT4KM>(p, num_sms, stream);
+    case QMV_FMT_INT8: return launch_f<QMV_FMT_INT8>(p, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }

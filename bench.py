@@ -10,7 +10,11 @@ shape, as no GPU palette fit exists yet); activations N(0, 1) fp16.
 
 Metric: effective weight GB/s = algorithmic bytes (codes + scales/palette +
 x + y) / kernel time, and us per matvec.  Every input (~1.1 GB per step in
-total) is larger than L2, so no flush is needed between steps.
+total) is larger than L2, so no flush is needed between steps.  The step is
+captured once as a CUDA graph (four launches on one stream) and replayed per
+step, as a decode loop runs; per-format times come from graphs of ten
+back-to-back launches of one format, and the call-by-call step time is
+reported beside them.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -172,6 +176,35 @@ def build_workload(device, formats=FORMATS):
     return x, ops, enc_ms
 
 
+def capture(fn, stream, reps):
+    """A CUDA graph of `reps` calls of fn on `stream` (fn's first calls, which
+    set kernel attributes, run outside the capture)."""
+    import torch
+    with torch.cuda.stream(stream):
+        fn()
+        fn()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                fn()
+    stream.synchronize()
+    return g
+
+
+def graph_us(g, stream, reps_per_graph, replays):
+    """Mean device time per call of a captured graph (CUDA events on its stream)."""
+    import torch
+    with torch.cuda.stream(stream):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(replays):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / (replays * reps_per_graph)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import weight_only_quantized_qmv_b200 as q
@@ -182,49 +215,49 @@ def run_ours(args, rank, world, local_rank):
     x, ops, enc_ms = build_workload(dev, formats)
     fmt_id = {"fp4": q.FMT_FP4, "int4": q.FMT_INT4, "int4km": q.FMT_INT4KM, "int8": q.FMT_INT8}
     outs = {f: torch.empty((1, N_HEAD), dtype=torch.float32, device=dev) for f in formats}
-    stream = torch.cuda.current_stream()
+    stream = torch.cuda.Stream(device=dev)
+
+    def launch(f):
+        c, a = ops[f]
+        q.matvec(fmt_id[f], c, a, x, out=outs[f], stream=stream)
 
     def step():
         for f in formats:
-            c, a = ops[f]
-            q.matvec(fmt_id[f], c, a, x, out=outs[f], stream=stream)
+            launch(f)
+
+    # A decode step runs as a CUDA graph (the deployment form): one replay =
+    # one matvec per format, back to back on one stream.
+    step_graph = capture(step, stream, 1)
 
     dist = world > 1
     if dist:
         import torch.distributed as tdist
 
-    for _ in range(args.warmup):
-        step()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step_graph.replay()
     torch.cuda.synchronize()
     if dist:
         tdist.barrier()
     torch.cuda.synchronize()
 
-    # timed region: per-step events bracket each format's kernel
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(formats) + 1)] for _ in range(args.steps)]
     cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
     gpu_index = cvd.split(",")[local_rank].strip() if cvd else str(local_rank)
     with ClockSampler(gpu_index) as clk:
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for s in range(args.steps):
-            e = evs[s]
-            e[0].record(stream)
-            for i, f in enumerate(formats):
-                c, a = ops[f]
-                q.matvec(fmt_id[f], c, a, x, out=outs[f], stream=stream)
-                e[i + 1].record(stream)
-        t_end.record(stream)
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            for _ in range(args.steps):
+                step_graph.replay()
+            t_end.record(stream)
         torch.cuda.synchronize()
     if dist:
         tdist.barrier()
     torch.cuda.synchronize()
     clocks = clk.summary()
     total_ms = t_start.elapsed_time(t_end)
-    per_fmt_ms = {f: [evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)]
-                  for i, f in enumerate(formats)}
-    flags = q.status_fetch()
+    flags = q.status_fetch(stream)
     if flags:
         raise RuntimeError(f"kernel status flags 0x{flags:x}")
 
@@ -236,20 +269,34 @@ def run_ours(args, rank, world, local_rank):
     bytes_step = sum(algorithmic_bytes(f, N_HEAD, K_HEAD, 1) for f in formats)
     value = bytes_step * world / (ms_step * 1e-3) / 1e9
 
+    # per-format kernel time: a graph of 10 back-to-back launches of one format
     peak, peak_src = hbm_peak()
     per_fmt = {}
+    replays = max(3, min(30, args.steps // 100))
     for f in formats:
-        us = statistics.mean(per_fmt_ms[f]) * 1e3
+        g = capture(lambda f=f: launch(f), stream, 10)
+        us = graph_us(g, stream, 10, replays)
+        del g
         gbs = algorithmic_bytes(f, N_HEAD, K_HEAD, 1) / (us * 1e-6) / 1e9
-        per_fmt[f] = {"us": round(us, 3), "us_median": round(statistics.median(per_fmt_ms[f]) * 1e3, 3),
-                      "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
-                      "frac_of_8tbs": round(gbs / 8000.0, 4),
-                      "bytes": algorithmic_bytes(f, N_HEAD, K_HEAD, 1)}
+        per_fmt[f] = {"us": round(us, 3), "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
+                      "frac_of_8tbs": round(gbs / 8000.0, 4), "bytes": algorithmic_bytes(f, N_HEAD, K_HEAD, 1)}
     dom = max(formats, key=lambda f: per_fmt[f]["us"])
     roof = {"bound": "hbm", "kernel": f"mv_kernel<{dom}> lm_head 248320x2048 B=1",
             "achieved": per_fmt[dom]["gbs"], "peak": peak, "unit": "GB/s",
             "frac": round(per_fmt[dom]["gbs"] / peak, 4), "peak_source": f"{peak_src} (hbm copy)",
-            "traffic": profiled_traffic(dom), "algorithmic_bytes": per_fmt[dom]["bytes"]}
+            "traffic": profiled_traffic(dom), "algorithmic_bytes": per_fmt[dom]["bytes"],
+            "timing": "CUDA events around replays of a graph of 10 launches"}
+
+    # the same step launched call by call (no graph), for context
+    with torch.cuda.stream(stream):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_plain = max(10, min(300, args.steps // 10))
+        e0.record(stream)
+        for _ in range(n_plain):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    plain_us = e0.elapsed_time(e1) * 1e3 / n_plain
 
     # extra measurements (outside the timed region): batch 4 / 16 verify
     extra = measure_batches(q, ops, dev, stream) if not args.no_extras and "fp4" in formats else None
@@ -261,30 +308,22 @@ def run_ours(args, rank, world, local_rank):
     return {
         "ms_per_step": ms_step, "value": value, "per_fmt": per_fmt, "roofline": roof, "clocks": clocks,
         "encode_ms": enc_ms, "batches": extra, "e2e": e2e, "bytes_step": bytes_step,
-        "gpu_launches": len(formats) * args.steps,
+        "gpu_launches": len(formats) * args.steps, "step_us_without_graph": round(plain_us, 2),
     }
 
 
-def measure_batches(q, ops, dev, stream, reps=30):
+def measure_batches(q, ops, dev, stream):
     import torch
     from weight_only_quantized_qmv_b200 import synth
-    g = synth.generator(7, dev)
+    g0 = synth.generator(7, dev)
     res = {}
     for B in (4, 16):
-        x = synth.activations(B, K_HEAD, g)
+        x = synth.activations(B, K_HEAD, g0)
         out = torch.empty((B, N_HEAD), dtype=torch.float32, device=dev)
         c, a = ops["fp4"]
-        for _ in range(3):
-            q.matvec_fp4(c, a, x, out=out, stream=stream)
-        ts = []
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            q.matvec_fp4(c, a, x, out=out, stream=stream)
-            e1.record(stream)
-            ts.append((e0, e1))
-        torch.cuda.synchronize()
-        us = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+        g = capture(lambda: q.matvec_fp4(c, a, x, out=out, stream=stream), stream, 10)
+        us = graph_us(g, stream, 10, 5)
+        del g
         res[f"fp4_b{B}"] = {"us": round(us, 3),
                             "gbs": round(algorithmic_bytes("fp4", N_HEAD, K_HEAD, B) / (us * 1e-6) / 1e9, 1)}
     return res
@@ -481,8 +520,10 @@ def main():
             "config": {"workload": "lm_head 248320x2048 batch 1; one matvec per format per step "
                                    f"({', '.join(args.formats)})",
                        "l2": "inputs larger than L2 (~1.1 GB read per step), no flush",
+                       "launch": "the step is a CUDA graph replayed once per step",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "per_format": r["per_fmt"], "roofline": r["roofline"], "cpu_baseline": cpu, "e2e": r["e2e"],
+            "step_us_without_graph": r["step_us_without_graph"],
             "gpu_launches": r["gpu_launches"] * world, "clocks": r["clocks"], "encode_ms": r["encode_ms"],
             "batch_verify": r["batches"],
         }

@@ -386,26 +386,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
       }
     }
   }
-  // Activations once per CTA: row r at xbase + r * XS, in the k order the
-  // format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7) per 8).
   const uint32_t xbase = sbase + p.off_x;
-  {
-    const int64_t per_row = p.K / 8;
-    const int64_t n16 = (int64_t)p.n_xrows * per_row;
-    for (int64_t i = tid; i < n16; i += kThreads) {
-      const int64_t r = i / per_row, j = i - r * per_row;
-      uint4 v = ldg_nc_128(p.x + r * p.K + 8 * j);
-      if constexpr (F::kPermX) {
-        v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
-                       prmt(v.y, v.w, 0x7632u));
-      }
-      sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
-    }
-    if constexpr (kOne) {  // the zero activations of the batch-1 form
-      for (int j = tid; j < kZeroBytes / 16; j += kThreads) sts128(sbase + p.off_zero + 16u * j, make_uint4(0u, 0u, 0u, 0u));
-    }
-  }
-  __syncthreads();
+  __syncthreads();  // the group table
 
   // ---- the warp's work items ------------------------------------------------
   // Units are (column group, 16-row tile) pairs.  With at least as many
@@ -562,6 +544,27 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
     cp_async_commit();
     fill += p.stage_bytes;
   }
+
+  // The activations are staged while the first weight slices are in flight.
+  // Activations once per CTA: row r at xbase + r * XS, in the k order the
+  // format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7) per 8).
+  {
+    const int64_t per_row = p.K / 8;
+    const int64_t n16 = (int64_t)p.n_xrows * per_row;
+    for (int64_t i = tid; i < n16; i += kThreads) {
+      const int64_t r = i / per_row, j = i - r * per_row;
+      uint4 v = ldg_nc_128(p.x + r * p.K + 8 * j);
+      if constexpr (F::kPermX) {
+        v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
+                       prmt(v.y, v.w, 0x7632u));
+      }
+      sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
+    }
+    if constexpr (kOne) {  // the zero activations of the batch-1 form
+      for (int j = tid; j < kZeroBytes / 16; j += kThreads) sts128(sbase + p.off_zero + 16u * j, make_uint4(0u, 0u, 0u, 0u));
+    }
+  }
+  __syncthreads();
 
   // ---- consume ----
   float* red = reinterpret_cast<float*>(smem + p.off_red);  // split units: [warp][NT][4][lane]
@@ -793,8 +796,10 @@ bool plan_matvec(int fmt, MvParams& p) {
   const int nt = p.B > 8 ? 2 : 1;
   p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
   p.off_x = (int)round_up((int64_t)kWarps * nt * 4 * 32 * 4, 128);
-  p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128);
-  p.off_stage = p.off_zero + (p.one ? kZeroBytes : 0);
+  // the zero region starts 32 bytes past a 128-byte line: its reads and the
+  // activation reads of the same instruction fall in different banks
+  p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
+  p.off_stage = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
   // the most CTAs per SM (up to the kernel's register budget) with the
   // deepest ring (<= kStages slices per warp) that fits

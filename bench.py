@@ -14,7 +14,9 @@ total) is larger than L2, so no flush is needed between steps.  The step is
 captured once as a CUDA graph (four launches on one stream) and replayed per
 step, as a decode loop runs; per-format times come from graphs of ten
 back-to-back launches of one format, and the call-by-call step time is
-reported beside them.
+reported beside them.  The weights are fixed, so launches may stream them
+while the preceding launch drains (qmv_set_weight_prefetch; --no-prefetch
+turns that off).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -213,6 +215,10 @@ def run_ours(args, rank, world, local_rank):
     q.lib()
     formats = tuple(args.formats)
     x, ops, enc_ms = build_workload(dev, formats)
+    torch.cuda.synchronize()
+    # the decode loop's weights are fixed: let each launch stream its weights
+    # while its predecessor drains (no work in the timed region writes them)
+    q.set_weight_prefetch(not args.no_prefetch)
     fmt_id = {"fp4": q.FMT_FP4, "int4": q.FMT_INT4, "int4km": q.FMT_INT4KM, "int8": q.FMT_INT8}
     outs = {f: torch.empty((1, N_HEAD), dtype=torch.float32, device=dev) for f in formats}
     stream = torch.cuda.Stream(device=dev)
@@ -478,6 +484,8 @@ def main():
     ap.add_argument("--formats", nargs="+", choices=FORMATS, default=list(FORMATS),
                     help="weight formats in the step (default: all four, the benchmark workload)")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e and batch-4/16 measurements")
+    ap.add_argument("--no-prefetch", action="store_true",
+                    help="keep weight reads behind the preceding launch (qmv_set_weight_prefetch(0))")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -521,6 +529,7 @@ def main():
                                    f"({', '.join(args.formats)})",
                        "l2": "inputs larger than L2 (~1.1 GB read per step), no flush",
                        "launch": "the step is a CUDA graph replayed once per step",
+                       "weight_prefetch": not args.no_prefetch,
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "per_format": r["per_fmt"], "roofline": r["roofline"], "cpu_baseline": cpu, "e2e": r["e2e"],
             "step_us_without_graph": r["step_us_without_graph"],

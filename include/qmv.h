@@ -165,6 +165,19 @@ qmv_status qmv_dequant(int fmt, const void* codes, const void* aux, int64_t N, i
  * set, QMV_OK otherwise, QMV_ERR_CUDA if the stream reported an error. */
 qmv_status qmv_status_fetch(void* stream, uint32_t* flags);
 
+/* Overlap of consecutive matvec launches.  Every matvec / gather launch
+ * lets the next one in its stream become resident during its last blocks
+ * (programmatic dependent launch) and waits for the preceding work before
+ * it reads activations or expert ids or writes outputs.  With
+ * enable = 1, dense matvec launches made afterwards (any stream, any
+ * thread) also start streaming their weight codes, scales and palettes
+ * BEFORE that wait, so a kernel's pipeline fill hides under its
+ * predecessor's tail.  Enable it only when no work still in flight on the
+ * stream writes those weights (a decode loop over fixed weights); after an
+ * encoder call on the same stream, synchronize or keep it off.  Default 0.
+ * Returns QMV_ERR_ARG if enable is not 0 or 1. */
+qmv_status qmv_set_weight_prefetch(int enable);
+
 /* Text of the last error of this host thread ("" if none). */
 const char* qmv_last_error(void);
 

@@ -101,6 +101,14 @@ def test_encoder_argument_checks(L):
     assert L.qmv_status_fetch(None, None) == q.ERR_ARG
 
 
+def test_weight_prefetch_option(L):
+    import weight_only_quantized_qmv_b200 as q
+    assert L.qmv_set_weight_prefetch(2) == q.ERR_ARG
+    assert L.qmv_set_weight_prefetch(-1) == q.ERR_ARG
+    assert L.qmv_set_weight_prefetch(1) == q.OK
+    assert L.qmv_set_weight_prefetch(0) == q.OK
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     import weight_only_quantized_qmv_b200 as q

@@ -242,6 +242,45 @@ def test_matvec_batch1_whole_units(q, fmt):
     assert np.array_equal(y, y2)
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_weight_prefetch_same_results_and_ordering(q, fmt):
+    """With early weight reads on, results are bit-identical, and each launch
+    still sees activations (and weights) written by the work just before it
+    on the same stream."""
+    N, K = 3000, 2048
+    f = q.__dict__["FMT_" + fmt.upper()]
+    c_o, s_o, xn = _inputs(fmt, N, K, 1, seed=31)
+    c, s = torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda()
+    xs = [torch.from_numpy(synth.activations(1, K, synth.generator(40 + i, "cpu")).numpy()).cuda() for i in range(4)]
+    ref = [q.matvec(f, c, s, x) for x in xs]
+    torch.cuda.synchronize()
+    st = torch.cuda.Stream()
+    xbuf = torch.empty_like(xs[0])
+    outs = [torch.empty((1, N), dtype=torch.float32, device="cuda") for _ in xs]
+    try:
+        q.set_weight_prefetch(True)
+        with torch.cuda.stream(st):
+            for _ in range(3):
+                for i, x in enumerate(xs):
+                    xbuf.copy_(x)  # a kernel on the same stream writes the activations
+                    q.matvec(f, c, s, xbuf, out=outs[i], stream=st)
+        st.synchronize()
+    finally:
+        q.set_weight_prefetch(False)
+    for r, o in zip(ref, outs):
+        assert torch.equal(r, o)
+    # weights rewritten right before the call (prefetch off, the default)
+    c2 = torch.zeros_like(c) if fmt != "int4km" else c.clone()
+    s2 = s.clone()
+    with torch.cuda.stream(st):
+        c2.copy_(c)
+        s2.copy_(s)
+        y = q.matvec(f, c2, s2, xs[0], stream=st)
+    st.synchronize()
+    assert torch.equal(y, ref[0])
+    assert q.status_fetch() == 0
+
+
 def test_matvec_output_guard_bands(q):
     """Sentinels around the output rows stay untouched (no out-of-bounds
     writes on a ragged last tile)."""

@@ -53,6 +53,7 @@ SIGNATURES = {
     "qmv_gather_matvec": [_I32, _P, _P, _I32, _I64, _I64, _P, _I32, _I32, _P, _I32, _P, _P],
     "qmv_dequant": [_I32, _P, _P, _I64, _I64, _P, _P],
     "qmv_status_fetch": [_P, ctypes.POINTER(ctypes.c_uint32)],
+    "qmv_set_weight_prefetch": [_I32],
     "qmv_last_error": [],
     "qmv_version": [],
 }
@@ -215,6 +216,13 @@ def dequant(fmt: int, codes: torch.Tensor, aux: torch.Tensor, stream=None) -> to
     out = torch.empty((N, K), dtype=torch.float32, device=codes.device)
     _call("qmv_dequant", fmt, _ptr(codes), _ptr(aux), N, K, _ptr(out), _stream(stream))
     return out
+
+
+def set_weight_prefetch(enable: bool) -> None:
+    """Let dense matvec launches start streaming weights before the preceding
+    work in their stream completes (only while nothing in flight writes the
+    weights; see qmv_set_weight_prefetch in include/qmv.h)."""
+    _call("qmv_set_weight_prefetch", int(bool(enable)))
 
 
 def status_fetch(stream=None) -> int:

@@ -1,6 +1,7 @@
 // qmv_abi.cu -- the extern "C" entry points of libqmv (declared in qmv.h):
 // host-side argument validation, the per-device status word, last-error text
 // and the kernel launches on the caller's stream.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -10,6 +11,7 @@
 namespace {
 
 thread_local char g_err[512] = "";
+std::atomic<int> g_weight_prefetch{0};  // qmv_set_weight_prefetch
 
 qmv_status fail(qmv_status code, const char* fmt, ...) {
   va_list ap;
@@ -139,6 +141,7 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
   int sms;
   QMV_TRY(device_ctx(&st, &sms));
   p.status = st;
+  p.prefetch = (!gather && g_weight_prefetch.load(std::memory_order_relaxed)) ? 1 : 0;
   cudaError_t e = qmv::launch_matvec(fmt, p, sms, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "matvec launch");
   return QMV_OK;
@@ -235,6 +238,12 @@ qmv_status qmv_status_fetch(void* stream, uint32_t* flags) {
 }
 
 const char* qmv_last_error(void) { return g_err; }
+
+qmv_status qmv_set_weight_prefetch(int enable) {
+  if (enable != 0 && enable != 1) return fail(QMV_ERR_ARG, "enable must be 0 or 1 (got %d)", enable);
+  g_weight_prefetch.store(enable, std::memory_order_relaxed);
+  return QMV_OK;
+}
 
 const char* qmv_version(void) { return "0.1.0"; }
 

@@ -61,6 +61,8 @@ struct MvParams {
   int gk;                  // K granule of split units (in-features)
   int one;                 // batch-1 block-column form (dense B == 1, K % 256 == 0)
   int off_zero;            // its zero activation region
+  int off_xsum;            // its per-block activation sums (int4)
+  int prefetch;            // dense: weights may be read before the preceding grid completes
   int RS;                  // shared-memory bytes per staged code row
   int AS;                  // shared-memory bytes per staged scale row (kAuxRows)
   int aux_mode;

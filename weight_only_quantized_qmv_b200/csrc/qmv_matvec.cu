@@ -236,15 +236,23 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g,
 //   crow_g / crow_g8: rows g, g+8 of the slice + this lane's block offset
 //   sa_g / sa_g8:     their scale rows in the slice
 //   xl0 / xl1:        activations of block t / t+4 of group 0, or the zero region
+//
+// int4 in this form: a nibble masked into the low bits of an fp16 is the
+// subnormal n * 2^-24 (n * 2^-20 for the upper nibble of a byte), so the
+// decode is one AND per two weights.  The two nibble positions accumulate
+// in separate MMA sums (dlo, dhi); per block, 2^20 * (16 * dlo + dhi) is the
+// exact sum of n * x, and the offset 8 is removed with the block's sum of
+// activations (xsum, exact in fp64, rounded once to fp32).
 template <int FMT, int NG>
 __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint32_t crow_g, uint32_t crow_g8,
-                                          uint32_t sa_g, uint32_t sa_g8, uint32_t xl0, uint32_t xl1, int t,
-                                          const Palette& pg, const Palette& pg8, const Mul& m) {
+                                          uint32_t sa_g, uint32_t sa_g8, uint32_t xl0, uint32_t xl1, uint32_t xs_t,
+                                          int t, const Palette& pg, const Palette& pg8, const Mul& m) {
   using F = FmtT<FMT>;
   constexpr int kBB = F::kBits * 4;  // code bytes per block and row
+  constexpr bool kSub = FMT == QMV_FMT_INT4;  // the subnormal int4 decode
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi) {
-    float d[4];
+    float d[4], dh[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const uint32_t cb = (uint32_t)((8 * gi + 4 * h) * kBB);
@@ -265,6 +273,22 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
         // word group i: in-features 8i..8i+7 of the block, MMA steps 2i and 2i+1
         const uint4 xv = lds128(xl + (uint32_t)(64 * (8 * gi + 4 * h) + 16 * i));
         uint32_t g0lo, g0hi, g1lo, g1hi, h0lo, h0hi, h1lo, h1hi;
+        if constexpr (kSub) {
+          // step 2i: (k0,k4), (k2,k6) as n * 2^-24; step 2i+1: (k1,k5), (k3,k7) as n * 2^-20
+          const uint32_t g8 = __umulhi(wg[i], m.p24), h8 = __umulhi(wh[i], m.p24);  // w >> 8
+          const uint32_t gl0 = wg[i] & 0x000F000Fu, gl1 = g8 & 0x000F000Fu;
+          const uint32_t hl0 = wh[i] & 0x000F000Fu, hl1 = h8 & 0x000F000Fu;
+          const uint32_t gu0 = wg[i] & 0x00F000F0u, gu1 = g8 & 0x00F000F0u;
+          const uint32_t hu0 = wh[i] & 0x00F000F0u, hu1 = h8 & 0x00F000F0u;
+          if (h == 0 && i == 0) {
+            mma16816_zc(d, gl0, hl0, gl1, hl1, xv.x, xv.y);
+            mma16816_zc(dh, gu0, hu0, gu1, hu1, xv.z, xv.w);
+          } else {
+            mma16816(d, gl0, hl0, gl1, hl1, xv.x, xv.y);
+            mma16816(dh, gu0, hu0, gu1, hu1, xv.z, xv.w);
+          }
+          continue;
+        }
         if constexpr (F::kBits == 8) {
           dec_int8_word(wg[2 * i], g0lo, g0hi);
           dec_int8_word(wg[2 * i + 1], g1lo, g1hi);
@@ -307,6 +331,14 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
         s0 = __low2float(hu); s1 = __high2float(hu);
         s2 = __low2float(hv); s3 = __high2float(hv);
       }
+      if constexpr (kSub) {
+        // block partial = 2^20 * (16 * dlo + dhi) - 8 * sum(x), one rounding each
+        const float2 xs = *sptr<float2>(xs_t + (uint32_t)(4 * 8 * gi));  // blocks 2t, 2t+1 of the group
+        d[0] = fmaf(fmaf(d[0], 16.0f, dh[0]), 1048576.0f, -8.0f * xs.x);
+        d[1] = fmaf(fmaf(d[1], 16.0f, dh[1]), 1048576.0f, -8.0f * xs.y);
+        d[2] = fmaf(fmaf(d[2], 16.0f, dh[2]), 1048576.0f, -8.0f * xs.x);
+        d[3] = fmaf(fmaf(d[3], 16.0f, dh[3]), 1048576.0f, -8.0f * xs.y);
+      }
       acc[0] = fmaf(d[0], s0, acc[0]);
       acc[0] = fmaf(d[1], s1, acc[0]);
       acc[1] = fmaf(d[2], s2, acc[1]);
@@ -314,6 +346,9 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
     }
   }
 }
+
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_wait_preceding() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint8_t ldg_u8(const uint8_t* p) {
   uint32_t v;
@@ -336,6 +371,12 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_addr(smem);
   const int P = p.gather ? p.B * p.topk : p.B;
+
+  // Programmatic dependent launch: the next grid in the stream may become
+  // resident as this one's blocks finish; this grid reads activations / ids
+  // and writes outputs only after the preceding grid has completed.
+  grid_launch_dependents();
+  if (!p.prefetch) grid_wait_preceding();
 
   // ---- set-up (whole CTA): the column groups and the staged activations -----
   if (tid == 0) s_nvalid = 0;
@@ -545,6 +586,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
     fill += p.stage_bytes;
   }
 
+  if (p.prefetch) grid_wait_preceding();  // weights only before this point
+
   // The activations are staged while the first weight slices are in flight.
   // Activations once per CTA: row r at xbase + r * XS, in the k order the
   // format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7) per 8).
@@ -554,11 +597,31 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
     for (int64_t i = tid; i < n16; i += kThreads) {
       const int64_t r = i / per_row, j = i - r * per_row;
       uint4 v = ldg_nc_128(p.x + r * p.K + 8 * j);
-      if constexpr (F::kPermX) {
+      if constexpr (F::kPermX && kOne) {  // (k0,k4), (k2,k6), (k1,k5), (k3,k7)
+        v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.y, v.w, 0x5410u), prmt(v.x, v.z, 0x7632u),
+                       prmt(v.y, v.w, 0x7632u));
+      } else if constexpr (F::kPermX) {  // (k0,k4), (k1,k5), (k2,k6), (k3,k7)
         v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
                        prmt(v.y, v.w, 0x7632u));
       }
       sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
+    }
+    if constexpr (kOne && FMT == QMV_FMT_INT4) {
+      // per-block activation sums: exact in fp64 (32 fp16 terms), one rounding to fp32
+      for (int64_t b = tid; b < p.K / 32; b += kThreads) {
+        double sum = 0.0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = ldg_nc_128(p.x + 32 * b + 8 * q);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 hv = *reinterpret_cast<const __half2*>(&w4[e]);
+            sum += (double)__low2float(hv) + (double)__high2float(hv);
+          }
+        }
+        *reinterpret_cast<float*>(smem + p.off_xsum + 4 * b) = (float)sum;
+      }
     }
     if constexpr (kOne) {  // the zero activations of the batch-1 form
       for (int j = tid; j < kZeroBytes / 16; j += kThreads) sts128(sbase + p.off_zero + 16u * j, make_uint4(0u, 0u, 0u, 0u));
@@ -635,10 +698,12 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
         const uint32_t xl0 = (g == t) ? xs + 64u * t : zb;
         const uint32_t xl1 = (g == t + 4) ? xs + 64u * t : zb;
         const uint32_t tb = (uint32_t)(t * F::kBits * 4);
+        const uint32_t xs_t = sbase + p.off_xsum + 4u * (uint32_t)(k0 / 32 + 2 * t);  // block sums of this lane
         if (kNB >= 16 && kc == kNB * 32)
-          slice_one<FMT, (kNB >= 16 ? kNB / 8 : 1)>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, xl0, xl1, t, pg, pg8, mul);
+          slice_one<FMT, (kNB >= 16 ? kNB / 8 : 1)>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, xl0, xl1, xs_t, t,
+                                                    pg, pg8, mul);
         else
-          slice_one<FMT, 1>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, xl0, xl1, t, pg, pg8, mul);
+          slice_one<FMT, 1>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, xl0, xl1, xs_t, t, pg, pg8, mul);
         __syncwarp();
         cons = (cons + p.stage_bytes == ring_end) ? ring : cons + p.stage_bytes;
         continue;
@@ -799,7 +864,8 @@ bool plan_matvec(int fmt, MvParams& p) {
   // the zero region starts 32 bytes past a 128-byte line: its reads and the
   // activation reads of the same instruction fall in different banks
   p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
-  p.off_stage = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
+  p.off_xsum = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
+  p.off_stage = (int)round_up(p.off_xsum + ((p.one && fmt == QMV_FMT_INT4) ? 4 * (p.K / 32) : 0), 128);
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
   // the most CTAs per SM (up to the kernel's register budget) with the
   // deepest ring (<= kStages slices per warp) that fits
@@ -834,8 +900,17 @@ static cudaError_t launch_t(const MvParams& p, int num_sms, cudaStream_t stream)
   const int64_t upper_units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
   const int64_t slots = (int64_t)num_sms * p.ctas_per_sm;
   const int grid = (int)(upper_units < slots ? upper_units : slots);
-  mv_kernel<FMT, NT><<<grid, kThreads, p.smem_bytes, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)p.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT>, p);
 }
 
 template <int FMT>

@@ -133,7 +133,8 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t byte) {
 // Per-format decoders: one 32-bit word of a row's codes (8 weights, k = 8t..8t+7
 // of one 32-block for the 4-bit formats; 4 weights for int8) -> fp16 operands
 // for the two m16n8k16 steps of that block.  The k order the decoder emits is
-// the order the activations are staged in shared memory (kXPerm below).
+// the order the activations are staged in shared memory (see the kernel's
+// activation staging).
 // ---------------------------------------------------------------------------
 
 // A 32-bit constant the compiler cannot fold, so that multiplies by powers of
@@ -145,14 +146,12 @@ __device__ __forceinline__ uint32_t opaque(uint32_t c) {
   return r;
 }
 
-// Multipliers the decoders use to move bytes with integer multiply-high.
+// Multipliers kept opaque so the decoders' shifts-by-multiply stay integer
+// multiply-adds on the FMA pipe.
 struct Mul {
-  uint32_t p8, p16, p24, p4, e23;  // 2^8, 2^16, 2^24, 2^4, 2^23
+  uint32_t p4, e23;  // 2^4, 2^23
   __device__ __forceinline__ static Mul make() {
     Mul m;
-    m.p8 = opaque(1u << 8);
-    m.p16 = opaque(1u << 16);
-    m.p24 = opaque(1u << 24);
     m.p4 = opaque(1u << 4);
     m.e23 = opaque(1u << 23);
     return m;
@@ -192,7 +191,7 @@ struct DecFp4 {
 template <int I>
 __device__ __forceinline__ float e8m0_x2_to_f32(uint32_t u, const Mul& m) {
   // bytes 0..2 by a byte permute (ALU), byte 3 by a multiply-high (FMA pipe)
-  const uint32_t byte = (I < 3) ? prmt(u, 0u, 0x4440u + I) : __umulhi(u, m.p8);
+  const uint32_t byte = (I < 3) ? prmt(u, 0u, 0x4440u + I) : (u >> 24);
   return __uint_as_float(byte * m.e23 + m.e23);
 }
 
@@ -207,7 +206,7 @@ struct DecInt4 {
     const uint32_t kSub = 0x64086408u;    // fp16x2 (1032, 1032)
     const uint32_t kSixteenth = 0x2C002C00u;  // fp16x2 (1/16, 1/16)
     const uint32_t kNeg72 = 0xD480D480u;  // fp16x2 (-72, -72)
-    const uint32_t w8 = __umulhi(w, m.p24);  // w >> 8
+    const uint32_t w8 = w >> 8;
     s0lo = hsub2_u32(lop3_and_or(w, 0x000F000Fu, kMagic), kSub);
     s0hi = hfma2_u32(lop3_and_or(w, 0x00F000F0u, kMagic), kSixteenth, kNeg72);
     s1lo = hsub2_u32(lop3_and_or(w8, 0x000F000Fu, kMagic), kSub);
@@ -249,8 +248,8 @@ __device__ __forceinline__ Palette palette_from_words(const uint32_t (&e)[8]) {
 // w: 8 nibbles (k0..k7).  Emits (k0,k1) (k2,k3) (k4,k5) (k6,k7) as f16x2.
 __device__ __forceinline__ void dec_int4km(const Palette& p, uint32_t w, uint32_t& s0lo, uint32_t& s0hi,
                                            uint32_t& s1lo, uint32_t& s1hi, const Mul& m) {
-  const uint32_t w4 = w * m.p4;           // w << 4
-  const uint32_t wh = __umulhi(w, m.p16);  // w >> 16
+  const uint32_t w4 = w * m.p4;  // w << 4 on the multiply pipe (the lookups load the ALU)
+  const uint32_t wh = w >> 16;
   const uint32_t sel0 = w & 0x7777u;   // nibbles 0..3, bit 3 cleared
   const uint32_t sel1 = wh & 0x7777u;  // nibbles 4..7
   const uint32_t m0 = prmt(w4, w, 0xD9C8u);  // byte i = 0xFF iff bit 3 of nibble i

@@ -24,9 +24,6 @@ constexpr int kStages = QMV_STAGES;
 #ifndef QMV_MIN_CTAS
 #define QMV_MIN_CTAS 2                     // CTAs per SM the kernel's register budget targets
 #endif
-#ifndef QMV_CTA_MAJOR
-#define QMV_CTA_MAJOR 0
-#endif
 constexpr int kSliceBytes = QMV_SLICE_BYTES;
 constexpr int kMinCtas = QMV_MIN_CTAS;
 constexpr int kMaxCtasPerSM = 4;

@@ -275,7 +275,7 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
         uint32_t g0lo, g0hi, g1lo, g1hi, h0lo, h0hi, h1lo, h1hi;
         if constexpr (kSub) {
           // step 2i: (k0,k4), (k2,k6) as n * 2^-24; step 2i+1: (k1,k5), (k3,k7) as n * 2^-20
-          const uint32_t g8 = __umulhi(wg[i], m.p24), h8 = __umulhi(wh[i], m.p24);  // w >> 8
+          const uint32_t g8 = wg[i] >> 8, h8 = wh[i] >> 8;
           const uint32_t gl0 = wg[i] & 0x000F000Fu, gl1 = g8 & 0x000F000Fu;
           const uint32_t hl0 = wh[i] & 0x000F000Fu, hl1 = h8 & 0x000F000Fu;
           const uint32_t gu0 = wg[i] & 0x00F000F0u, gu1 = g8 & 0x00F000F0u;
@@ -444,11 +444,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
   const int64_t W = (int64_t)grid * kWarps;
   // Warps are numbered warp-major across CTAs, so the units of a partial last
   // round land 4-5 per CTA instead of filling whole CTAs (and SMs) first.
-#if QMV_CTA_MAJOR
-  const int64_t gwarp = (int64_t)blockIdx.x * kWarps + warp;
-#else
   const int64_t gwarp = (int64_t)warp * grid + blockIdx.x;
-#endif
   int64_t R, tail0;
   int T;
   if (total >= W) {  // whole units only: this warp's units gwarp, gwarp + W, ...

@@ -134,15 +134,15 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
     p.E = 1;
     p.topk = 1;
   }
-  if (!qmv::plan_matvec(fmt, p))
-    return fail(QMV_ERR_UNSUPPORTED, "activations (%d rows x %lld) do not fit the on-chip staging", p.n_xrows,
-                (long long)K);
   uint32_t* st;
   int sms;
   QMV_TRY(device_ctx(&st, &sms));
+  if (!qmv::plan_matvec(fmt, p, sms))
+    return fail(QMV_ERR_UNSUPPORTED, "activations (%d rows x %lld) do not fit the on-chip staging", p.n_xrows,
+                (long long)K);
   p.status = st;
   p.prefetch = (!gather && g_weight_prefetch.load(std::memory_order_relaxed)) ? 1 : 0;
-  cudaError_t e = qmv::launch_matvec(fmt, p, sms, (cudaStream_t)stream);
+  cudaError_t e = qmv::launch_matvec(fmt, p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "matvec launch");
   return QMV_OK;
 }

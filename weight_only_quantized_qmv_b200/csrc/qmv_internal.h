@@ -10,7 +10,7 @@
 namespace qmv {
 
 // ---- fused dequant-matvec / gather kernel -----------------------------------
-constexpr int kWarps = 8;                  // warps per CTA: all copy, decode and multiply
+constexpr int kWarps = 8;                  // warps per CTA (16 for one-CTA-per-SM launches)
 constexpr int kThreads = 32 * kWarps;
 constexpr int kTileRows = 16;              // rows per tile: one m16 step
 constexpr int kMaxCols = 16;               // activation columns per pass
@@ -31,7 +31,7 @@ constexpr int kMaxPairs = 256;             // B * topk upper bound (16 * 16)
 constexpr int kSmemLimit = 227 * 1024;     // per-block opt-in maximum on sm_100
 constexpr int kSmemPerSM = 228 * 1024;     // shared memory of one SM
 constexpr int kZeroBytes = 1024;           // zero activations read by the batch-1 form's idle columns
-constexpr int kStaticSmem = 6 * 1024;      // the kernel's static shared memory (group table), rounded up
+constexpr int kStaticSmem = 5 * 1024;      // the kernel's static shared memory (group table), rounded up
 
 // Aux (scale / palette) staging mode of a launch.
 enum AuxMode : int {
@@ -68,7 +68,9 @@ struct MvParams {
   int n_xrows;             // activation rows staged
   int off_red, off_x, off_stage;  // dynamic shared-memory offsets
   int smem_bytes;
-  int ctas_per_sm;         // 1..4, by shared-memory footprint
+  int ctas_per_sm;         // 1..2, by shared-memory footprint
+  int warps;               // warps per CTA (8 or 16)
+  int grid;                // CTAs of the launch
 };
 
 // Per-format constants (bits per weight, scale bytes per 32-block).
@@ -85,11 +87,12 @@ inline FmtInfo fmt_info(int fmt) {
   }
 }
 
-// Fills the geometry of `p` (shapes and pointers already set).  Returns false
-// when the activations plus a two-stage ring do not fit in shared memory.
-bool plan_matvec(int fmt, MvParams& p);
+// Fills the geometry and the launch shape of `p` (shapes and pointers
+// already set) for a device with `num_sms` SMs.  Returns false when the
+// activations plus a two-stage ring do not fit in shared memory.
+bool plan_matvec(int fmt, MvParams& p, int num_sms);
 
-cudaError_t launch_matvec(int fmt, const MvParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_matvec(int fmt, const MvParams& p, cudaStream_t stream);
 
 // ---- encoders / dequant ------------------------------------------------------
 struct ClipList {

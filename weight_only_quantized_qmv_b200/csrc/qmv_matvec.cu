@@ -62,6 +62,8 @@ struct GroupTable {
   int count[kMaxPairs];
   int16_t sorted[kMaxPairs];  // (token, slot) pair indices ordered by expert
 };
+// the kernel's static shared memory: the group table, the ids, a counter
+static_assert(sizeof(GroupTable) + kMaxPairs * sizeof(int) + 16 <= kStaticSmem, "static shared memory reserve");
 
 __device__ __forceinline__ uint32_t lds_u8(uint32_t a) { return *sptr<uint8_t>(a); }
 __device__ __forceinline__ uint32_t lds_u16(uint32_t a) { return *sptr<uint16_t>(a); }
@@ -358,11 +360,14 @@ __device__ __forceinline__ uint8_t ldg_u8(const uint8_t* p) {
 
 // NT: activation n-tiles of 8 columns (1 or 2); NT = 0 is the batch-1 form
 // whose MMA columns carry blocks (slice_one).
-template <int FMT, int NT>
-__global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_constant__ MvParams p) {
+// WARPS: warps per CTA (8, two CTAs per SM; or 16, one CTA per SM, when the
+// staged activations leave room for only one 8-warp CTA).
+template <int FMT, int NT, int WARPS>
+__global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kernel(const __grid_constant__ MvParams p) {
   using F = FmtT<FMT>;
   constexpr bool kOne = NT == 0;
   constexpr int NTX = kOne ? 1 : NT;
+  constexpr int kT = 32 * WARPS;  // threads per CTA
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ GroupTable gt;
   __shared__ int s_ids[kMaxPairs];
@@ -441,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
   const int ngroups = gt.ngroups;
   const int64_t total = (int64_t)ngroups * p.tiles;
   const int grid = (int)gridDim.x;
-  const int64_t W = (int64_t)grid * kWarps;
+  const int64_t W = (int64_t)grid * WARPS;
   // Warps are numbered warp-major across CTAs, so the units of a partial last
   // round land 4-5 per CTA instead of filling whole CTAs (and SMs) first.
   const int64_t gwarp = (int64_t)warp * grid + blockIdx.x;
@@ -459,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
   const int nitems = (int)R + T;
   // this warp's share of K in the split units: whole granules of p.gk
   const int Kg = (int)((p.K + p.gk - 1) / p.gk);
-  const int kb_w = (int)min(p.K, (int64_t)(warp * Kg / kWarps) * p.gk);
-  const int ke_w = (int)min(p.K, (int64_t)((warp + 1) * Kg / kWarps) * p.gk);
+  const int kb_w = (int)min(p.K, (int64_t)(warp * Kg / WARPS) * p.gk);
+  const int ke_w = (int)min(p.K, (int64_t)((warp + 1) * Kg / WARPS) * p.gk);
   const int KC = p.KC;
   const int nsl_main = p.nchunks;
   const int nsl_tail = ke_w > kb_w ? (ke_w - kb_w + KC - 1) / KC : 0;
@@ -590,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
   {
     const int64_t per_row = p.K / 8;
     const int64_t n16 = (int64_t)p.n_xrows * per_row;
-    for (int64_t i = tid; i < n16; i += kThreads) {
+    for (int64_t i = tid; i < n16; i += kT) {
       const int64_t r = i / per_row, j = i - r * per_row;
       uint4 v = ldg_nc_128(p.x + r * p.K + 8 * j);
       if constexpr (F::kPermX && kOne) {  // (k0,k4), (k2,k6), (k1,k5), (k3,k7)
@@ -604,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
     }
     if constexpr (kOne && FMT == QMV_FMT_INT4) {
       // per-block activation sums: exact in fp64 (32 fp16 terms), one rounding to fp32
-      for (int64_t b = tid; b < p.K / 32; b += kThreads) {
+      for (int64_t b = tid; b < p.K / 32; b += kT) {
         double sum = 0.0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -620,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
       }
     }
     if constexpr (kOne) {  // the zero activations of the batch-1 form
-      for (int j = tid; j < kZeroBytes / 16; j += kThreads) sts128(sbase + p.off_zero + 16u * j, make_uint4(0u, 0u, 0u, 0u));
+      for (int j = tid; j < kZeroBytes / 16; j += kT) sts128(sbase + p.off_zero + 16u * j, make_uint4(0u, 0u, 0u, 0u));
     }
   }
   __syncthreads();
@@ -756,7 +761,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
         if (tid < kTileRows) {
           float v = 0.0f;
 #pragma unroll
-          for (int w = 0; w < kWarps; ++w) v += red[w * 16 + tid];
+          for (int w = 0; w < WARPS; ++w) v += red[w * 16 + tid];
           if (tid < nrows) p.y[(int64_t)pair * p.N + row0 + tid] = v * f;
         }
         __syncthreads();
@@ -787,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
         const int ln = tid & 31, q = (tid >> 5) & 3, n = tid >> 7;
         float v = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) v += red[((w * NT + n) * 4 + q) * 32 + ln];
+        for (int w = 0; w < WARPS; ++w) v += red[((w * NT + n) * 4 + q) * 32 + ln];
         const int col = 8 * n + 2 * (ln & 3) + (q & 1);
         const int row = (ln >> 2) + 8 * (q >> 1);
         if (col < ncols && row < nrows) {
@@ -807,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) mv_kernel(const __grid_con
 
 static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
-bool plan_matvec(int fmt, MvParams& p) {
+bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   const FmtInfo fi = fmt_info(fmt);
   p.code_row_bytes = p.K * fi.bits / 8;
   p.aux_row_bytes = fi.lut ? 32 : (p.K / 32) * fi.scale_bytes;
@@ -846,7 +851,10 @@ bool plan_matvec(int fmt, MvParams& p) {
     p.aux_mode = (based && p.aux_row_bytes % 8 == 0) ? kAuxRows : kAuxBlock;
     if (p.aux_mode == kAuxBlock) p.one = 0;
     int64_t j = (slice_sc + 15) / 16;
-    if (j % 2 == 0) ++j;  // odd multiple of 16 bytes: rows g = 0..7 hit distinct banks
+    // the batch-1 form reads 4 bytes of rows g = 0..7 per load: an odd
+    // multiple of 16 bytes puts them in distinct banks (elsewhere the scale
+    // loads are a few per slice and the tighter rows let more warps fit)
+    if (p.one && j % 2 == 0) ++j;
     p.AS = (int)(16 * j);
     aux_region = kTileRows * p.AS;
   }
@@ -855,19 +863,32 @@ bool plan_matvec(int fmt, MvParams& p) {
   p.XS = (int)(round_up(2 * p.K, 128) + 64);  // 64 mod 128: conflict-free 128-bit reads
   p.n_xrows = p.gather ? (p.x_per_slot ? p.B * p.topk : p.B) : p.B;
   const int nt = p.B > 8 ? 2 : 1;
-  p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
-  p.off_x = (int)round_up((int64_t)kWarps * nt * 4 * 32 * 4, 128);
-  // the zero region starts 32 bytes past a 128-byte line: its reads and the
-  // activation reads of the same instruction fall in different banks
-  p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
-  p.off_xsum = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
-  p.off_stage = (int)round_up(p.off_xsum + ((p.one && fmt == QMV_FMT_INT4) ? 4 * (p.K / 32) : 0), 128);
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
-  // the most CTAs per SM (up to the kernel's register budget) with the
-  // deepest ring (<= kStages slices per warp) that fits
-  for (int ctas = kMinCtas; ctas >= 1; --ctas) {
+  // Layouts in order of preference: two 8-warp CTAs per SM, else one 16-warp
+  // CTA (the staged activations shared by 16 warps), else one 8-warp CTA;
+  // within each the deepest ring (<= kStages slices per warp) that fits.
+  const int cand[3][2] = {{kWarps, kMinCtas}, {2 * kWarps, 1}, {kWarps, 1}};
+  // one CTA per (group, tile) unit up to the resident-CTA slots
+  const int64_t upper_units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
+  for (int ci = 0; ci < 3; ++ci) {
+    const int warps = cand[ci][0], ctas = cand[ci][1];
+    if (warps != kWarps && p.one) continue;  // the batch-1 form fits two 8-warp CTAs
+    p.warps = warps;
+    const int64_t slots = (int64_t)num_sms * ctas;
+    p.grid = (int)(upper_units < slots ? upper_units : slots);
+    // Units are split along K (partial sums meet in shared memory) only when
+    // there are fewer than the grid's warps; a (group, tile) count of at
+    // least p.tiles means that can happen only if p.tiles is below it.
+    const bool may_split = p.tiles < (int64_t)p.grid * warps;
+    p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
+    p.off_x = may_split ? (int)round_up((int64_t)warps * nt * 4 * 32 * 4, 128) : 0;
+    // the zero region starts 32 bytes past a 128-byte line: its reads and the
+    // activation reads of the same instruction fall in different banks
+    p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
+    p.off_xsum = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
+    p.off_stage = (int)round_up(p.off_xsum + ((p.one && fmt == QMV_FMT_INT4) ? 4 * (p.K / 32) : 0), 128);
     for (int st = kStages; st >= 2; --st) {
-      const int64_t bytes = p.off_stage + (int64_t)kWarps * st * p.stage_bytes;
+      const int64_t bytes = p.off_stage + (int64_t)warps * st * p.stage_bytes;
       if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
         p.stages = st;
         p.smem_bytes = (int)bytes;
@@ -879,26 +900,21 @@ bool plan_matvec(int fmt, MvParams& p) {
   return false;
 }
 
-template <int FMT, int NT>
-static cudaError_t launch_t(const MvParams& p, int num_sms, cudaStream_t stream) {
+template <int FMT, int NT, int WARPS>
+static cudaError_t launch_t(const MvParams& p, cudaStream_t stream) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 64 && !attr_set[dev]) {
-    err = cudaFuncSetAttribute(mv_kernel<FMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(mv_kernel<FMT, NT, WARPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
     attr_set[dev] = true;
   }
-  // one CTA per (group, tile) unit up to the resident-CTA slots: units beyond
-  // whole rounds of warps are split along K inside a CTA
-  const int64_t upper_units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
-  const int64_t slots = (int64_t)num_sms * p.ctas_per_sm;
-  const int grid = (int)(upper_units < slots ? upper_units : slots);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.gridDim = dim3((unsigned)p.grid);
+  cfg.blockDim = dim3(32 * WARPS);
   cfg.dynamicSmemBytes = (size_t)p.smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -906,24 +922,25 @@ static cudaError_t launch_t(const MvParams& p, int num_sms, cudaStream_t stream)
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT>, p);
+  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT, WARPS>, p);
 }
 
 template <int FMT>
-static cudaError_t launch_f(const MvParams& p, int num_sms, cudaStream_t stream) {
+static cudaError_t launch_f(const MvParams& p, cudaStream_t stream) {
   // activation columns served per pass: dense B, gather at most B pairs per
   // expert when ids are distinct per token (groups are capped at 8 * NT)
-  if (p.one) return launch_t<FMT, 0>(p, num_sms, stream);
-  if (p.B > 8) return launch_t<FMT, 2>(p, num_sms, stream);
-  return launch_t<FMT, 1>(p, num_sms, stream);
+  if (p.one) return launch_t<FMT, 0, kWarps>(p, stream);
+  const bool wide = p.warps == 2 * kWarps;
+  if (p.B > 8) return wide ? launch_t<FMT, 2, 2 * kWarps>(p, stream) : launch_t<FMT, 2, kWarps>(p, stream);
+  return wide ? launch_t<FMT, 1, 2 * kWarps>(p, stream) : launch_t<FMT, 1, kWarps>(p, stream);
 }
 
-cudaError_t launch_matvec(int fmt, const MvParams& p, int num_sms, cudaStream_t stream) {
+cudaError_t launch_matvec(int fmt, const MvParams& p, cudaStream_t stream) {
   switch (fmt) {
-    case QMV_FMT_FP4: return launch_f<QMV_FMT_FP4>(p, num_sms, stream);
-    case QMV_FMT_INT4: return launch_f<QMV_FMT_INT4>(p, num_sms, stream);
-    case QMV_FMT_INT4KM: return launch_f<QMV_FMT_INT4KM>(p, num_sms, stream);
-    case QMV_FMT_INT8: return launch_f<QMV_FMT_INT8>(p, num_sms, stream);
+    case QMV_FMT_FP4: return launch_f<QMV_FMT_FP4>(p, stream);
+    case QMV_FMT_INT4: return launch_f<QMV_FMT_INT4>(p, stream);
+    case QMV_FMT_INT4KM: return launch_f<QMV_FMT_INT4KM>(p, stream);
+    case QMV_FMT_INT8: return launch_f<QMV_FMT_INT8>(p, stream);
   }
   return cudaErrorInvalidValue;
 }

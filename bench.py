@@ -304,8 +304,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     plain_us = e0.elapsed_time(e1) * 1e3 / n_plain
 
-    # extra measurements (outside the timed region): batch 4 / 16 verify
+    # extra measurements (outside the timed region): batch 4 / 16 verify, the int4km decode step
     extra = measure_batches(q, ops, dev, stream) if not args.no_extras and "fp4" in formats else None
+    dstep = (measure_decode_step(q, ops["int4km"][0], ops["int4km"][1], dev, stream)
+             if not args.no_extras and "int4km" in formats else None)
+    amax = None if args.no_extras else measure_argmax(q, ops, fmt_id, x, dev, stream, formats)
 
     # end to end through the C ABI with host buffers: H2D x, the matvecs, D2H y
     e2e = None if args.no_extras else measure_e2e(q, ops, fmt_id, x, dev, stream, formats,
@@ -315,6 +318,7 @@ def run_ours(args, rank, world, local_rank):
         "ms_per_step": ms_step, "value": value, "per_fmt": per_fmt, "roofline": roof, "clocks": clocks,
         "encode_ms": enc_ms, "batches": extra, "e2e": e2e, "bytes_step": bytes_step,
         "gpu_launches": len(formats) * args.steps, "step_us_without_graph": round(plain_us, 2),
+        "decode_step_int4km": dstep, "argmax_b1": amax,
     }
 
 
@@ -332,6 +336,91 @@ def measure_batches(q, ops, dev, stream):
         del g
         res[f"fp4_b{B}"] = {"us": round(us, 3),
                             "gbs": round(algorithmic_bytes("fp4", N_HEAD, K_HEAD, B) / (us * 1e-6) / 1e9, 1)}
+    return res
+
+
+def measure_argmax(q, ops, fmt_id, x, dev, stream, formats):
+    """Greedy next token from the head: the fused matvec + argmax against the
+    matvec followed by torch.argmax, per format at batch 1 (graphs of 10)."""
+    import torch
+    ws = q.argmax_workspace(dev)
+    res = {}
+    for f in formats:
+        c, a = ops[f]
+        idx = torch.empty(1, dtype=torch.int32, device=dev)
+        val = torch.empty(1, dtype=torch.float32, device=dev)
+        y = torch.empty((1, N_HEAD), dtype=torch.float32, device=dev)
+        g1 = capture(lambda: q.matvec_argmax(fmt_id[f], c, a, x, ws, idx=idx, val=val, stream=stream), stream, 10)
+        fused = graph_us(g1, stream, 10, 5)
+        del g1
+
+        def unfused():
+            q.matvec(fmt_id[f], c, a, x, out=y, stream=stream)
+            torch.argmax(y, dim=1)
+
+        g2 = capture(unfused, stream, 10)
+        plain = graph_us(g2, stream, 10, 5)
+        del g2
+        with torch.cuda.stream(stream):
+            ref = int(torch.argmax(q.matvec(fmt_id[f], c, a, x, stream=stream), dim=1).item())
+        res[f] = {"fused_us": round(fused, 2), "matvec_then_argmax_us": round(plain, 2),
+                  "same_index": int(idx.item()) == ref}
+    return res
+
+
+def measure_decode_step(q, lm_idx, lm_lut, dev, stream, reps=20):
+    """The int4km decode step of the workload list, timed as one CUDA graph per
+    batch size: the 248320x2048 lm_head, 10 layers of q (4096x2048) and o
+    (2048x4096), and one routed-expert layer (256 experts; gate and up
+    512x2048, down 2048x512; top-8 uniform routing).  Random palettes and
+    indices of the fitted shapes; each launch reads fixed synthetic
+    activations (the step's data flow between layers is not modelled)."""
+    import torch
+    from weight_only_quantized_qmv_b200 import synth
+    g = synth.generator(11, dev)
+    E, topk, H, I = 256, 8, 2048, 512
+    layers = []
+    for _ in range(10):
+        ql, qi = synth.palette_tables(4096, H, g)
+        ol, oi = synth.palette_tables(H, 4096, g)
+        layers.append((qi, ql, oi, ol))
+    gl, gi = synth.palette_tables(E * I, H, g)
+    ul, ui = synth.palette_tables(E * I, H, g)
+    dl, di = synth.palette_tables(E * H, I, g)
+    gi, gl = gi.view(E, I, H // 2), gl.view(E, I, 16)
+    ui, ul = ui.view(E, I, H // 2), ul.view(E, I, 16)
+    di, dl = di.view(E, H, I // 2), dl.view(E, H, 16)
+    res = {}
+    for B in (1, 8):
+        x_h = synth.activations(B, H, g)
+        x_o = synth.activations(B, 4096, g)
+        x_d = synth.activations(B, I, g, extra_shape=(topk,))
+        ids = synth.routing(B, topk, E, g).to(dev)
+        y_lm = torch.empty((B, N_HEAD), dtype=torch.float32, device=dev)
+        y_q = torch.empty((B, 4096), dtype=torch.float32, device=dev)
+        y_o = torch.empty((B, H), dtype=torch.float32, device=dev)
+        y_g = torch.empty((B, topk, I), dtype=torch.float32, device=dev)
+        y_u = torch.empty((B, topk, I), dtype=torch.float32, device=dev)
+        y_d = torch.empty((B, topk, H), dtype=torch.float32, device=dev)
+
+        def step():
+            for qi, ql, oi, ol in layers:
+                q.matvec_int4km(qi, ql, x_h, out=y_q, stream=stream)
+                q.matvec_int4km(oi, ol, x_o, out=y_o, stream=stream)
+            q.gather_matvec(q.FMT_INT4KM, gi, gl, ids, x_h, out=y_g, stream=stream)
+            q.gather_matvec(q.FMT_INT4KM, ui, ul, ids, x_h, out=y_u, stream=stream)
+            q.gather_matvec(q.FMT_INT4KM, di, dl, ids, x_d, x_per_slot=True, out=y_d, stream=stream)
+            q.matvec_int4km(lm_idx, lm_lut, x_h, out=y_lm, stream=stream)
+
+        gph = capture(step, stream, 1)
+        us = graph_us(gph, stream, 1, reps)
+        del gph
+        n_exp = len(set(ids.flatten().tolist()))
+        dense = (algorithmic_bytes("int4km", N_HEAD, H, B)
+                 + 10 * (algorithmic_bytes("int4km", 4096, H, B) + algorithmic_bytes("int4km", H, 4096, B)))
+        expert = n_exp * (2 * (I * H // 2 + I * 32) + (H * I // 2 + H * 32))
+        res[f"b{B}"] = {"us": round(us, 2), "launches": 24, "distinct_experts": n_exp,
+                        "bytes": dense + expert, "gbs": round((dense + expert) / (us * 1e-6) / 1e9, 1)}
     return res
 
 
@@ -532,7 +621,8 @@ def main():
                        "weight_prefetch": not args.no_prefetch,
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "per_format": r["per_fmt"], "roofline": r["roofline"], "cpu_baseline": cpu, "e2e": r["e2e"],
-            "step_us_without_graph": r["step_us_without_graph"],
+            "step_us_without_graph": r["step_us_without_graph"], "decode_step_int4km": r["decode_step_int4km"],
+            "argmax_b1": r["argmax_b1"],
             "gpu_launches": r["gpu_launches"] * world, "clocks": r["clocks"], "encode_ms": r["encode_ms"],
             "batch_verify": r["batches"],
         }

@@ -47,6 +47,7 @@
 #ifndef QMV_H
 #define QMV_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -131,6 +132,31 @@ qmv_status qmv_matvec_int4km(const uint8_t* idx, const uint16_t* lut, const uint
 /* codes [N, K] int8; scales [N, K/32] fp16. */
 qmv_status qmv_matvec_int8(const int8_t* codes, const uint16_t* scales, const uint16_t* x,
                            int B, int64_t N, int64_t K, float* y, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Fused matvec + argmax (greedy next token from the lm_head; the pages'
+ * fused head+argmax kernel: "coreai-optimization (coreai-opt) reference",
+ * sec. "The LM head + embeddings").  For each activation row b computes
+ * y[b, :] = x[b, :] Wdq^T exactly as qmv_matvec_* does, without writing y,
+ * and returns
+ *     idx[b] = the lowest n with y[b, n] = max_n y[b, n]     (int32, device)
+ *     val[b] = y[b, idx[b]]                                   (float32, device)
+ * Values are ordered as floats with -0 == +0 (a NaN with the sign bit clear
+ * ranks above +Inf, one with it set below -Inf).
+ *   fmt        QMV_FMT_*; codes / aux as for the format's qmv_matvec_* call.
+ *   N          < 2^31.
+ *   workspace  device buffer of at least qmv_argmax_workspace_bytes() bytes,
+ *              16-byte aligned, zero-filled before its first use; every call
+ *              leaves it zero-filled again.  One call at a time per
+ *              workspace (calls on other streams need their own).
+ * Errors as for qmv_matvec_*; QMV_ERR_ARG also for a short or misaligned
+ * workspace or misaligned idx / val. */
+qmv_status qmv_matvec_argmax(int fmt, const void* codes, const void* aux, const uint16_t* x, int B,
+                             int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                             int32_t* idx, float* val, void* stream);
+
+/* Bytes of workspace qmv_matvec_argmax needs on the current device. */
+qmv_status qmv_argmax_workspace_bytes(size_t* bytes);
 
 /* ---------------------------------------------------------------------
  * Routed-expert gather matvec ([P1] sec. 1 gather formats; [P2] sec. 3:

@@ -315,6 +315,76 @@ def test_matvec_is_deterministic(q):
 
 
 # ---------------------------------------------------------------------------
+# fused matvec + argmax
+# ---------------------------------------------------------------------------
+
+def _first_argmax(y):
+    """Lowest index of the maximum per row (values compared with -0 == +0)."""
+    y = np.asarray(y, np.float64) + 0.0
+    m = y.max(axis=1, keepdims=True)
+    return (y == m).argmax(axis=1), m[:, 0]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K,B", [(17, 96, 1), (1000, 2048, 1), (1000, 2048, 3), (300, 544, 16), (37905, 2048, 1),
+                                   (37905, 2048, 9)])
+def test_matvec_argmax_matches_unfused(q, fmt, N, K, B):
+    """The fused argmax equals the argmax of the same kernel's materialised y
+    (bit-identical outputs, lowest index on ties) and is within tolerance of
+    the fp64 oracle's maximum."""
+    f = q.__dict__["FMT_" + fmt.upper()]
+    c_o, s_o, xn = _inputs(fmt, N, K, B, seed=N + K + B)
+    c, s, x = torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(), torch.from_numpy(xn).cuda()
+    ws = q.argmax_workspace()
+    idx, val = q.matvec_argmax(f, c, s, x, ws)
+    y = q.matvec(f, c, s, x).cpu().numpy()
+    want_i, want_v = _first_argmax(y)
+    assert np.array_equal(idx.cpu().numpy(), want_i)
+    assert np.array_equal(val.cpu().numpy(), want_v.astype(np.float32))
+    r = orc.matvec(FID[fmt], c_o, s_o, xn, N, K)
+    got = r[np.arange(B), idx.cpu().numpy()]
+    assert np.all(got >= r.max(axis=1) - TOL * np.abs(r).max(axis=1))
+    assert int(ws.count_nonzero()) == 0  # left zero-filled for the next call
+    assert q.status_fetch() == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_matvec_argmax_planted_and_ties(q, fmt):
+    """A planted maximum is found exactly; two identical rows holding the
+    maximum resolve to the lower index; repeated calls reuse the workspace."""
+    N, K, B = 3000, 1024, 2
+    f = q.__dict__["FMT_" + fmt.upper()]
+    g = synth.generator(77, "cpu")
+    W, _ = synth.weights(N, K, g, n_outlier_cols=0)
+    x = synth.activations(B, K, g).numpy()
+    Wn = W.numpy()
+    # row 2321 aligned with x[0]; rows 777 and 2900 identical and aligned with x[1]
+    Wn[2321] = np.sign(x[0].astype(np.float32)) * 0.05
+    Wn[777] = np.sign(x[1].astype(np.float32)) * 0.05
+    Wn[2900] = Wn[777]
+    c_o, s_o, _ = encode_orc(fmt, Wn)
+    c, s, xg = torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(), torch.from_numpy(x).cuda()
+    ws = q.argmax_workspace()
+    r = orc.matvec(FID[fmt], c_o, s_o, x, N, K)
+    for _ in range(3):
+        idx, val = q.matvec_argmax(f, c, s, xg, ws)
+        got = idx.cpu().numpy()
+        assert got[0] == 2321 and r[0].argmax() == 2321
+        assert got[1] == 777 and r[1, 777] == r[1, 2900] and r[1].argmax() == 777
+
+
+def test_matvec_argmax_rejects_short_workspace(q):
+    N, K = 64, 256
+    c = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((N, K // 32), dtype=torch.uint8, device="cuda")
+    x = torch.zeros((1, K), dtype=torch.float16, device="cuda")
+    ws = torch.zeros(q.argmax_workspace_bytes() - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(q.QmvError) as ei:
+        q.matvec_argmax(q.FMT_FP4, c, s, x, ws)
+    assert ei.value.status == q.ERR_ARG
+
+
+# ---------------------------------------------------------------------------
 # gather over routed experts
 # ---------------------------------------------------------------------------
 

@@ -51,6 +51,8 @@ SIGNATURES = {
     "qmv_matvec_int4km": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int8": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_gather_matvec": [_I32, _P, _P, _I32, _I64, _I64, _P, _I32, _I32, _P, _I32, _P, _P],
+    "qmv_matvec_argmax": [_I32, _P, _P, _P, _I32, _I64, _I64, _P, ctypes.c_size_t, _P, _P, _P],
+    "qmv_argmax_workspace_bytes": [ctypes.POINTER(ctypes.c_size_t)],
     "qmv_dequant": [_I32, _P, _P, _I64, _I64, _P, _P],
     "qmv_status_fetch": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "qmv_set_weight_prefetch": [_I32],
@@ -184,6 +186,42 @@ def matvec_int4km(idx, lut, x, out=None, stream=None):
 
 def matvec_int8(codes, scales, x, out=None, stream=None):
     return matvec(FMT_INT8, codes, scales, x, out, stream)
+
+
+def argmax_workspace_bytes() -> int:
+    """Workspace bytes matvec_argmax needs on the current device."""
+    n = ctypes.c_size_t(0)
+    _call("qmv_argmax_workspace_bytes", ctypes.byref(n))
+    return int(n.value)
+
+
+def argmax_workspace(device=None) -> torch.Tensor:
+    """A zero-filled workspace for matvec_argmax (reusable, one call at a time)."""
+    return torch.zeros(argmax_workspace_bytes(), dtype=torch.uint8, device=device or "cuda")
+
+
+def matvec_argmax(fmt: int, codes: torch.Tensor, aux: torch.Tensor, x: torch.Tensor, workspace: torch.Tensor,
+                  idx=None, val=None, stream=None):
+    """Per activation row b: (idx int32 [B], val float32 [B]) = the lowest n
+    with y[b, n] maximal and that maximum, y = x Wdq^T (not materialised)."""
+    _need(codes, "codes", _CODES[fmt])
+    _need(aux, "scales/lut", _AUX[fmt])
+    _need(workspace, "workspace", torch.uint8)
+    N, K = _nk(fmt, codes)
+    xx = x.unsqueeze(0) if x.dim() == 1 else x
+    _need(xx, "x", torch.float16)
+    B = xx.shape[0]
+    if xx.shape[1] != K:
+        raise ValueError(f"x has {xx.shape[1]} features, weights have {K}")
+    if idx is None:
+        idx = torch.empty(B, dtype=torch.int32, device=codes.device)
+    if val is None:
+        val = torch.empty(B, dtype=torch.float32, device=codes.device)
+    _need(idx, "idx", torch.int32, (B,))
+    _need(val, "val", torch.float32, (B,))
+    _call("qmv_matvec_argmax", fmt, _ptr(codes), _ptr(aux), _ptr(xx), B, N, K, _ptr(workspace),
+          workspace.numel(), _ptr(idx), _ptr(val), _stream(stream))
+    return idx, val
 
 
 def gather_matvec(fmt: int, codes_stack: torch.Tensor, aux_stack: torch.Tensor, expert_ids: torch.Tensor,

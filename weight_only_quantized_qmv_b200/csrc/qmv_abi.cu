@@ -98,9 +98,16 @@ qmv_status encode_int(int qmax, const float* W, int64_t N, int64_t K, const floa
   return QMV_OK;
 }
 
+struct ArgmaxOut {
+  void* ws;
+  size_t ws_bytes;
+  int32_t* idx;
+  float* val;
+};
+
 qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
                          int64_t K, float* y, void* stream, bool gather, int E, const int32_t* ids, int topk,
-                         int x_per_slot) {
+                         int x_per_slot, const ArgmaxOut* am = nullptr) {
   if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
   QMV_TRY(check_ptr(codes, "codes"));
   if (!aux) return fail(QMV_ERR_ARG, "scales/lut is null");
@@ -109,7 +116,7 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
   if (fmt == QMV_FMT_INT4KM) QMV_TRY(check_ptr(aux, "lut"));
   if (fmt != QMV_FMT_FP4 && (reinterpret_cast<uintptr_t>(aux) & 1u)) return fail(QMV_ERR_ARG, "fp16 scales misaligned");
   QMV_TRY(check_ptr(x, "x"));
-  if (!y || (reinterpret_cast<uintptr_t>(y) & 3u)) return fail(QMV_ERR_ARG, "y null or misaligned");
+  if (!am && (!y || (reinterpret_cast<uintptr_t>(y) & 3u))) return fail(QMV_ERR_ARG, "y null or misaligned");
   QMV_TRY(check_shape(N, K));
   if (B < 1 || B > 16) return fail(QMV_ERR_UNSUPPORTED, "B must be in [1, 16] (got %d)", B);
   qmv::MvParams p{};
@@ -142,6 +149,19 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
                 (long long)K);
   p.status = st;
   p.prefetch = (!gather && g_weight_prefetch.load(std::memory_order_relaxed)) ? 1 : 0;
+  if (am) {
+    if (N >= (int64_t(1) << 31)) return fail(QMV_ERR_SHAPE, "argmax needs N < 2^31");
+    if (!am->ws || (reinterpret_cast<uintptr_t>(am->ws) & 15u)) return fail(QMV_ERR_ARG, "workspace null or not 16-byte aligned");
+    if (am->ws_bytes < qmv::argmax_workspace_bytes(sms))
+      return fail(QMV_ERR_ARG, "workspace has %zu bytes, needs %zu", am->ws_bytes, qmv::argmax_workspace_bytes(sms));
+    if (!am->idx || (reinterpret_cast<uintptr_t>(am->idx) & 3u)) return fail(QMV_ERR_ARG, "idx null or misaligned");
+    if (!am->val || (reinterpret_cast<uintptr_t>(am->val) & 3u)) return fail(QMV_ERR_ARG, "val null or misaligned");
+    p.argmax = 1;
+    p.am_ticket = static_cast<uint32_t*>(am->ws);
+    p.am_part = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(am->ws) + 16);
+    p.am_idx = am->idx;
+    p.am_val = am->val;
+  }
   cudaError_t e = qmv::launch_matvec(fmt, p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "matvec launch");
   return QMV_OK;
@@ -192,6 +212,22 @@ qmv_status qmv_matvec_int4km(const uint8_t* idx, const uint16_t* lut, const uint
 qmv_status qmv_matvec_int8(const int8_t* codes, const uint16_t* scales, const uint16_t* x, int B, int64_t N,
                            int64_t K, float* y, void* stream) {
   return matvec_common(QMV_FMT_INT8, codes, scales, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
+}
+
+qmv_status qmv_matvec_argmax(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
+                             int64_t K, void* workspace, size_t workspace_bytes, int32_t* idx, float* val,
+                             void* stream) {
+  const ArgmaxOut am{workspace, workspace_bytes, idx, val};
+  return matvec_common(fmt, codes, aux, x, B, N, K, nullptr, stream, false, 0, nullptr, 0, 0, &am);
+}
+
+qmv_status qmv_argmax_workspace_bytes(size_t* bytes) {
+  if (!bytes) return fail(QMV_ERR_ARG, "bytes is null");
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  *bytes = qmv::argmax_workspace_bytes(sms);
+  return QMV_OK;
 }
 
 qmv_status qmv_gather_matvec(int fmt, const void* codes_stack, const void* aux_stack, int E, int64_t N, int64_t K,

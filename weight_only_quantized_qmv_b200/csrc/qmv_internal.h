@@ -71,6 +71,11 @@ struct MvParams {
   int ctas_per_sm;         // 1..2, by shared-memory footprint
   int warps;               // warps per CTA (8 or 16)
   int grid;                // CTAs of the launch
+  int argmax;              // fused argmax: outputs go to am_* instead of y
+  uint32_t* am_ticket;     // workspace: CTA counter, then [grid][kMaxCols] partial keys
+  unsigned long long* am_part;
+  int32_t* am_idx;
+  float* am_val;
 };
 
 // Per-format constants (bits per weight, scale bytes per 32-block).
@@ -91,6 +96,12 @@ inline FmtInfo fmt_info(int fmt) {
 // already set) for a device with `num_sms` SMs.  Returns false when the
 // activations plus a two-stage ring do not fit in shared memory.
 bool plan_matvec(int fmt, MvParams& p, int num_sms);
+
+// Workspace bytes of the fused argmax for a device with `num_sms` SMs: a
+// 16-byte counter block and one partial key per (CTA, activation row).
+inline size_t argmax_workspace_bytes(int num_sms) {
+  return 16 + (size_t)num_sms * 2 * kMaxCols * sizeof(unsigned long long);
+}
 
 cudaError_t launch_matvec(int fmt, const MvParams& p, cudaStream_t stream);
 

@@ -63,7 +63,8 @@ struct GroupTable {
   int16_t sorted[kMaxPairs];  // (token, slot) pair indices ordered by expert
 };
 // the kernel's static shared memory: the group table, the ids, a counter
-static_assert(sizeof(GroupTable) + kMaxPairs * sizeof(int) + 16 <= kStaticSmem, "static shared memory reserve");
+static_assert(sizeof(GroupTable) + kMaxPairs * sizeof(int) + kMaxCols * 8 + 32 <= kStaticSmem,
+              "static shared memory reserve");
 
 __device__ __forceinline__ uint32_t lds_u8(uint32_t a) { return *sptr<uint8_t>(a); }
 __device__ __forceinline__ uint32_t lds_u16(uint32_t a) { return *sptr<uint16_t>(a); }
@@ -349,6 +350,18 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
   }
 }
 
+// Fused argmax: an output y[b, n] as a 64-bit key whose unsigned order is
+// (value as a float with -0 == +0, then lower n first).
+__device__ __forceinline__ unsigned long long argmax_key(float v, int64_t n) {
+  const uint32_t u = __float_as_uint(v + 0.0f);  // -0 -> +0
+  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)k << 32) | (unsigned long long)(~(uint32_t)n);
+}
+__device__ __forceinline__ float argmax_key_value(unsigned long long key) {
+  const uint32_t k = (uint32_t)(key >> 32);
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void grid_wait_preceding() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -362,7 +375,8 @@ __device__ __forceinline__ uint8_t ldg_u8(const uint8_t* p) {
 // whose MMA columns carry blocks (slice_one).
 // WARPS: warps per CTA (8, two CTAs per SM; or 16, one CTA per SM, when the
 // staged activations leave room for only one 8-warp CTA).
-template <int FMT, int NT, int WARPS>
+// AM: fused argmax (outputs folded into per-row maxima instead of stored).
+template <int FMT, int NT, int WARPS, bool AM>
 __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kernel(const __grid_constant__ MvParams p) {
   using F = FmtT<FMT>;
   constexpr bool kOne = NT == 0;
@@ -372,6 +386,8 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   __shared__ GroupTable gt;
   __shared__ int s_ids[kMaxPairs];
   __shared__ int s_nvalid;
+  __shared__ unsigned long long s_best[kMaxCols];  // fused argmax: this CTA's best key per activation row
+  __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_addr(smem);
@@ -385,6 +401,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
 
   // ---- set-up (whole CTA): the column groups and the staged activations -----
   if (tid == 0) s_nvalid = 0;
+  if (tid < kMaxCols) s_best[tid] = 0ull;
   if (p.gather && tid < P) s_ids[tid] = p.ids[tid];
   __syncthreads();
   if (!p.gather) {
@@ -632,6 +649,30 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
 
   // ---- consume ----
   float* red = reinterpret_cast<float*>(smem + p.off_red);  // split units: [warp][NT][4][lane]
+  // One output y[pair, n]: stored, or folded into this thread's running
+  // argmax for one of its columns (slot: a thread's columns are fixed for the
+  // whole launch, and threads with the same t share them).
+  unsigned long long best[2 * NTX];
+  int bcol[2 * NTX];
+#pragma unroll
+  for (int i = 0; i < 2 * NTX; ++i) {
+    best[i] = 0ull;
+    bcol[i] = -1;
+  }
+  auto emit = [&](int slot, int pair, int64_t n, float v) {
+    if constexpr (AM) {
+      const unsigned long long k = argmax_key(v, n);
+#pragma unroll
+      for (int i = 0; i < 2 * NTX; ++i) {
+        if (i == slot) {
+          best[i] = k > best[i] ? k : best[i];
+          bcol[i] = pair;
+        }
+      }
+    } else {
+      p.y[(int64_t)pair * p.N + n] = v;
+    }
+  };
   float acc[NTX][4];
   float acc1[2], dl[4];  // batch-1 form: rows g, g+8 / the palette format's running MMA sums
   Palette pg, pg8;
@@ -749,8 +790,8 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       const int pair = gt.sorted[gstart];
       if (!it.split) {
         if (t == 0) {
-          if (g < nrows) p.y[(int64_t)pair * p.N + row0 + g] = r0 * f;
-          if (g + 8 < nrows) p.y[(int64_t)pair * p.N + row0 + g + 8] = r1 * f;
+          if (g < nrows) emit(0, pair, row0 + g, r0 * f);
+          if (g + 8 < nrows) emit(0, pair, row0 + g + 8, r1 * f);
         }
       } else {
         if (t == 0) {
@@ -762,7 +803,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
           float v = 0.0f;
 #pragma unroll
           for (int w = 0; w < WARPS; ++w) v += red[w * 16 + tid];
-          if (tid < nrows) p.y[(int64_t)pair * p.N + row0 + tid] = v * f;
+          if (tid < nrows) emit(0, pair, row0 + tid, v * f);
         }
         __syncthreads();
       }
@@ -777,7 +818,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
           const int row = g + 8 * (q >> 1);
           if (col < ncols && row < nrows) {
             const int pair = gt.sorted[gstart + col];
-            p.y[(int64_t)pair * p.N + row0 + row] = acc[n][q] * f;
+            emit(2 * n + (q & 1), pair, row0 + row, acc[n][q] * f);
           }
         }
       }
@@ -797,13 +838,62 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
         const int row = (ln >> 2) + 8 * (q >> 1);
         if (col < ncols && row < nrows) {
           const int pair = gt.sorted[gstart + col];
-          p.y[(int64_t)pair * p.N + row0 + row] = v * f;
+          emit(0, pair, row0 + row, v * f);
         }
       }
       __syncthreads();
     }
   }
   cp_async_wait(0);
+
+  if constexpr (AM) {
+    // the lanes sharing t (and so their columns) combine, then one shared
+    // atomic per column and warp
+#pragma unroll
+    for (int i = 0; i < 2 * NTX; ++i) {
+      unsigned long long k = best[i];
+      int c = bcol[i];
+#pragma unroll
+      for (int m = 4; m < 32; m *= 2) {
+        const unsigned long long k2 = __shfl_xor_sync(0xffffffffu, k, m);
+        const int c2 = __shfl_xor_sync(0xffffffffu, c, m);
+        k = k2 > k ? k2 : k;
+        c = c2 > c ? c2 : c;
+      }
+      if (lane < 4 && c >= 0) atomicMax(&s_best[c], k);
+    }
+    // CTA partials to the workspace; the last CTA to finish (counter) takes
+    // the maximum over all CTAs for each row and resets the counter.
+    __syncthreads();
+    if (tid < p.B) p.am_part[(int64_t)blockIdx.x * kMaxCols + tid] = s_best[tid];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(p.am_ticket, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (s_last) {
+      // all threads: thread tid folds entries (CTA c, row tid % 16) -- the
+      // stride is a multiple of 16 -- and the rows meet in s_best (which
+      // already holds this CTA's own partials)
+      __threadfence();
+      const int b = tid & (kMaxCols - 1);
+      const int nent = (int)gridDim.x * kMaxCols;
+      unsigned long long mine = 0ull;
+#pragma unroll 4
+      for (int e = tid; e < nent; e += kT) {
+        const unsigned long long k = __ldcg(p.am_part + e);
+        mine = k > mine ? k : mine;
+        p.am_part[e] = 0ull;  // the workspace is left zero-filled
+      }
+      if (b < p.B) atomicMax(&s_best[b], mine);
+      __syncthreads();
+      if (tid < p.B) {
+        const unsigned long long best = s_best[tid];
+        p.am_idx[tid] = (int32_t)(~(uint32_t)best);
+        p.am_val[tid] = argmax_key_value(best);
+      }
+      if (tid == 0) *p.am_ticket = 0u;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -900,14 +990,14 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   return false;
 }
 
-template <int FMT, int NT, int WARPS>
+template <int FMT, int NT, int WARPS, bool AM>
 static cudaError_t launch_t(const MvParams& p, cudaStream_t stream) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 64 && !attr_set[dev]) {
-    err = cudaFuncSetAttribute(mv_kernel<FMT, NT, WARPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(mv_kernel<FMT, NT, WARPS, AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
     attr_set[dev] = true;
@@ -922,17 +1012,22 @@ static cudaError_t launch_t(const MvParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT, WARPS>, p);
+  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT, WARPS, AM>, p);
+}
+
+template <int FMT, bool AM>
+static cudaError_t launch_fa(const MvParams& p, cudaStream_t stream) {
+  // activation columns served per pass: dense B, gather at most B pairs per
+  // expert when ids are distinct per token (groups are capped at 8 * NT)
+  if (p.one) return launch_t<FMT, 0, kWarps, AM>(p, stream);
+  const bool wide = p.warps == 2 * kWarps;
+  if (p.B > 8) return wide ? launch_t<FMT, 2, 2 * kWarps, AM>(p, stream) : launch_t<FMT, 2, kWarps, AM>(p, stream);
+  return wide ? launch_t<FMT, 1, 2 * kWarps, AM>(p, stream) : launch_t<FMT, 1, kWarps, AM>(p, stream);
 }
 
 template <int FMT>
 static cudaError_t launch_f(const MvParams& p, cudaStream_t stream) {
-  // activation columns served per pass: dense B, gather at most B pairs per
-  // expert when ids are distinct per token (groups are capped at 8 * NT)
-  if (p.one) return launch_t<FMT, 0, kWarps>(p, stream);
-  const bool wide = p.warps == 2 * kWarps;
-  if (p.B > 8) return wide ? launch_t<FMT, 2, 2 * kWarps>(p, stream) : launch_t<FMT, 2, kWarps>(p, stream);
-  return wide ? launch_t<FMT, 1, 2 * kWarps>(p, stream) : launch_t<FMT, 1, kWarps>(p, stream);
+  return p.argmax ? launch_fa<FMT, true>(p, stream) : launch_fa<FMT, false>(p, stream);
 }
 
 cudaError_t launch_matvec(int fmt, const MvParams& p, cudaStream_t stream) {

@@ -158,6 +158,16 @@ qmv_status qmv_matvec_argmax(int fmt, const void* codes, const void* aux, const 
 /* Bytes of workspace qmv_matvec_argmax needs on the current device. */
 qmv_status qmv_argmax_workspace_bytes(size_t* bytes);
 
+/* qmv_matvec_argmax with a library-owned scratch instead of a caller
+ * workspace: a static device array (zero at load, left zero by every call),
+ * located once per device; nothing is allocated.  One call at a time per
+ * device (calls on several streams at once need qmv_matvec_argmax with
+ * their own workspaces).  QMV_ERR_UNSUPPORTED when the device needs more
+ * scratch than the array holds (more than 512 SMs); otherwise arguments and
+ * errors as for qmv_matvec_argmax. */
+qmv_status qmv_matvec_argmax_static(int fmt, const void* codes, const void* aux, const uint16_t* x, int B,
+                                    int64_t N, int64_t K, int32_t* idx, float* val, void* stream);
+
 /* ---------------------------------------------------------------------
  * Routed-expert gather matvec ([P1] sec. 1 gather formats; [P2] sec. 3:
  * only the selected experts' weights are read).  For token b and slot j,

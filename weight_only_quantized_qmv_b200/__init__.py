@@ -53,6 +53,7 @@ SIGNATURES = {
     "qmv_gather_matvec": [_I32, _P, _P, _I32, _I64, _I64, _P, _I32, _I32, _P, _I32, _P, _P],
     "qmv_matvec_argmax": [_I32, _P, _P, _P, _I32, _I64, _I64, _P, ctypes.c_size_t, _P, _P, _P],
     "qmv_argmax_workspace_bytes": [ctypes.POINTER(ctypes.c_size_t)],
+    "qmv_matvec_argmax_static": [_I32, _P, _P, _P, _I32, _I64, _I64, _P, _P, _P],
     "qmv_dequant": [_I32, _P, _P, _I64, _I64, _P, _P],
     "qmv_status_fetch": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "qmv_set_weight_prefetch": [_I32],
@@ -221,6 +222,29 @@ def matvec_argmax(fmt: int, codes: torch.Tensor, aux: torch.Tensor, x: torch.Ten
     _need(val, "val", torch.float32, (B,))
     _call("qmv_matvec_argmax", fmt, _ptr(codes), _ptr(aux), _ptr(xx), B, N, K, _ptr(workspace),
           workspace.numel(), _ptr(idx), _ptr(val), _stream(stream))
+    return idx, val
+
+
+def matvec_argmax_static(fmt: int, codes: torch.Tensor, aux: torch.Tensor, x: torch.Tensor, idx=None, val=None,
+                         stream=None):
+    """matvec_argmax on the library's own static scratch (no workspace, no
+    allocation; one call at a time per device)."""
+    _need(codes, "codes", _CODES[fmt])
+    _need(aux, "scales/lut", _AUX[fmt])
+    N, K = _nk(fmt, codes)
+    xx = x.unsqueeze(0) if x.dim() == 1 else x
+    _need(xx, "x", torch.float16)
+    B = xx.shape[0]
+    if xx.shape[1] != K:
+        raise ValueError(f"x has {xx.shape[1]} features, weights have {K}")
+    if idx is None:
+        idx = torch.empty(B, dtype=torch.int32, device=codes.device)
+    if val is None:
+        val = torch.empty(B, dtype=torch.float32, device=codes.device)
+    _need(idx, "idx", torch.int32, (B,))
+    _need(val, "val", torch.float32, (B,))
+    _call("qmv_matvec_argmax_static", fmt, _ptr(codes), _ptr(aux), _ptr(xx), B, N, K, _ptr(idx), _ptr(val),
+          _stream(stream))
     return idx, val
 
 

@@ -98,6 +98,28 @@ qmv_status encode_int(int qmax, const float* W, int64_t N, int64_t K, const floa
   return QMV_OK;
 }
 
+// Scratch of qmv_matvec_argmax_static: room for 512 SMs (two CTAs each),
+// zero at module load; every call leaves it zero.  Its address is looked up
+// once per device.
+constexpr size_t kStaticArgmaxBytes = 16 + 512 * 2 * qmv::kMaxCols * sizeof(unsigned long long);
+__device__ __align__(256) unsigned char g_argmax_scratch[kStaticArgmaxBytes];
+void* g_argmax_scratch_ptr[kMaxDevices] = {};
+
+qmv_status static_argmax_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(QMV_ERR_UNSUPPORTED, "device %d out of range", dev);
+  if (!g_argmax_scratch_ptr[dev]) {
+    void* a = nullptr;
+    e = cudaGetSymbolAddress(&a, g_argmax_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(argmax scratch)");
+    g_argmax_scratch_ptr[dev] = a;
+  }
+  *ptr = g_argmax_scratch_ptr[dev];
+  return QMV_OK;
+}
+
 struct ArgmaxOut {
   void* ws;
   size_t ws_bytes;
@@ -218,6 +240,20 @@ qmv_status qmv_matvec_argmax(int fmt, const void* codes, const void* aux, const 
                              int64_t K, void* workspace, size_t workspace_bytes, int32_t* idx, float* val,
                              void* stream) {
   const ArgmaxOut am{workspace, workspace_bytes, idx, val};
+  return matvec_common(fmt, codes, aux, x, B, N, K, nullptr, stream, false, 0, nullptr, 0, 0, &am);
+}
+
+qmv_status qmv_matvec_argmax_static(int fmt, const void* codes, const void* aux, const uint16_t* x, int B,
+                                    int64_t N, int64_t K, int32_t* idx, float* val, void* stream) {
+  void* ws = nullptr;
+  QMV_TRY(static_argmax_scratch(&ws));
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  if (qmv::argmax_workspace_bytes(sms) > kStaticArgmaxBytes)
+    return fail(QMV_ERR_UNSUPPORTED, "device needs %zu bytes of argmax scratch, the library holds %zu",
+                qmv::argmax_workspace_bytes(sms), kStaticArgmaxBytes);
+  const ArgmaxOut am{ws, kStaticArgmaxBytes, idx, val};
   return matvec_common(fmt, codes, aux, x, B, N, K, nullptr, stream, false, 0, nullptr, 0, 0, &am);
 }
 

@@ -290,9 +290,12 @@ int oracle_encode_int_sym(const float* W, int64_t N, int64_t K, int qmax,
 /*  grouping; P2 sec.8: per-output-row 16-entry codebook]             */
 /* ------------------------------------------------------------------ */
 
+/* Ascending, -0 before +0: a total order on finite floats, so the sorted
+ * row (and the initial centres read from it) is fully determined. */
 static int orc_cmp_float(const void* a, const void* b) {
   float x = *(const float*)a, y = *(const float*)b;
-  return (x > y) - (x < y);
+  if (x != y) return (x > y) - (x < y);
+  return (int)(signbit(y) != 0) - (int)(signbit(x) != 0);
 }
 
 /* Nearest of the 16 centres to v, distance |v - c| in double, ties to the
@@ -311,7 +314,7 @@ static int orc_nearest16(const double* c, double v) {
 }
 
 /* Per row (n = K weights), readings where no page fixes the details:
- *  1. sort the row ascending;
+ *  1. sort the row ascending (-0 before +0);
  *  2. centre k starts at sorted[floor((2k+1) n / 32)], the (k+1/2)/16
  *     quantile without interpolation;
  *  3. `iters` Lloyd steps: assign each weight to the nearest centre (double

@@ -324,6 +324,21 @@ def test_relerr_ordering_and_page_band(orc):
 # int4km k-means (LUT values: parity unpinned; invariants pinned)
 # --------------------------------------------------------------------------
 
+def test_kmeans_signed_zero_order(orc):
+    """Sorting puts -0 before +0 (a total order), so initial centres read from
+    a run of signed zeros are fixed: 16 x -0 then 16 x +0 give centres 1..7 at
+    -0 and 8..15 at +0; centre 0 takes every point (ties to the lower index)
+    and its double sum starting at +0 stays +0."""
+    W = np.array([[-0.0] * 16 + [0.0] * 16], np.float32)
+    rng = np.random.default_rng(3)
+    W = W[:, rng.permutation(32)]
+    lut, idx, flags = orc.kmeans_int4km(W)
+    assert flags == 0
+    bits = lut.view(np.uint16)[0].tolist()
+    assert bits == [0x0000] + [0x8000] * 7 + [0x0000] * 8
+    assert (idx == 0).all()
+
+
 def test_kmeans_exact_on_few_distinct_values(orc):
     """A row of <= 16 fp16-representable values, each occurring at least
     n/16 times, is a fixed point of Lloyd from the quantile start (every

@@ -111,6 +111,26 @@ qmv_status qmv_encode_int4(const float* W, int64_t N, int64_t K, const float* cl
 qmv_status qmv_encode_int8(const float* W, int64_t N, int64_t K, const float* clips,
                            int n_clips, int8_t* codes, uint16_t* scales, void* stream);
 
+/* int4km encode: per row a 16-entry fp16 palette by scalar 1-D k-means and
+ * the packed 4-bit index of each weight ([P3] "Palettization": scalar
+ * k-means, 2^n_bits centroids, per-channel grouping; [P2] sec. 8: per-row
+ * 16-entry codebook).  Per row of K weights: sort ascending (-0 before +0);
+ * centre k starts at sorted[floor((2k+1) K / 32)]; `iters` Lloyd steps (each
+ * weight to the nearest centre by double distance, ties to the lower index;
+ * a non-empty centre becomes float(double sum of its members in ascending
+ * order / count), an empty one keeps its value); palette = fp16 RNE of the
+ * centres; index = nearest palette entry (double distance, ties to the
+ * lower index).  A row with Inf/NaN is written as zeros and sets
+ * QMV_FLAG_NONFINITE.
+ *   W      [N, K] float32 (device)
+ *   K      multiple of 32, at most 16384
+ *   iters  0 .. 1000 (the workloads use 20)
+ *   lut    [N, 16] fp16 (out);  idx [N, K/2] uint8, element 2j in the low nibble (out)
+ * Errors: QMV_ERR_ARG (pointers, iters), QMV_ERR_SHAPE (N, K % 32),
+ * QMV_ERR_UNSUPPORTED (K > 16384). */
+qmv_status qmv_encode_int4km(const float* W, int64_t N, int64_t K, int iters, uint16_t* lut, uint8_t* idx,
+                             void* stream);
+
 /* ---------------------------------------------------------------------
  * Fused dequantize + matvec, y = x Wdq^T with fp32 accumulation
  * ([P2] sec. 1-3, 8).  x: [B, K] fp16; y: [B, N] float32 (overwritten).

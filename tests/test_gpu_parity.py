@@ -315,6 +315,73 @@ def test_matvec_is_deterministic(q):
 
 
 # ---------------------------------------------------------------------------
+# int4km encoder (GPU palette fit) against the oracle's k-means
+# ---------------------------------------------------------------------------
+
+def _km_rows(K, seed):
+    """Rows that stress the fit: synthetic weights with outliers, few distinct
+    values, signed zeros, constant, two values, duplicated quantile values."""
+    g = synth.generator(seed, "cpu")
+    W, _ = synth.weights(40, K, g, n_outlier_cols=2)
+    W = W.numpy().copy()
+    rng = np.random.default_rng(seed)
+    W[1] = rng.choice(np.array([-0.03, -0.01, 0.0, 0.02, 0.05], np.float32), K)
+    W[2] = np.where(rng.random(K) < 0.5, -0.0, 0.0).astype(np.float32)
+    W[3] = 0.0125
+    W[4] = np.where(rng.random(K) < 0.3, -0.02, 0.04).astype(np.float32)
+    W[5, : K // 2] = 0.01
+    W[6] = np.round(W[6] * 64) / 64  # coarse grid: many ties
+    W[7] = rng.standard_normal(K).astype(np.float32) * 1e-6
+    W[8] = (rng.standard_normal(K) * 30.0).astype(np.float32)
+    return W
+
+
+@pytest.mark.parametrize("K", [32, 96, 544, 2048, 4096])
+@pytest.mark.parametrize("iters", [0, 1, 20])
+def test_encode_int4km_bit_exact(q, K, iters):
+    W = _km_rows(K, seed=K + iters)
+    lut_o, idx_o, fl_o = orc.kmeans_int4km(W, iters=iters)
+    idx, lut = q.encode_int4km(torch.from_numpy(W).cuda(), iters=iters)
+    assert np.array_equal(lut.cpu().numpy().view(np.uint16), lut_o.view(np.uint16))
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert q.status_fetch() == fl_o == 0
+
+
+def test_encode_int4km_nonfinite_rows(q):
+    W = _km_rows(256, seed=5)
+    W[3, 7] = np.inf
+    W[9, 100] = np.nan
+    lut_o, idx_o, fl_o = orc.kmeans_int4km(W)
+    idx, lut = q.encode_int4km(torch.from_numpy(W).cuda())
+    assert np.array_equal(lut.cpu().numpy().view(np.uint16), lut_o.view(np.uint16))
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert fl_o == q.FLAG_NONFINITE
+    assert q.status_fetch() == q.FLAG_NONFINITE
+
+
+def test_encode_int4km_then_matvec(q):
+    """GPU palette fit -> GPU matvec against the oracle's fit -> fp64 matvec."""
+    N, K, B = 1000, 2048, 2
+    g = synth.generator(13, "cpu")
+    W, _ = synth.weights(N, K, g, n_outlier_cols=2)
+    x = synth.activations(B, K, g).numpy()
+    idx, lut = q.encode_int4km(W.cuda())
+    y = q.matvec_int4km(idx, lut, torch.from_numpy(x).cuda()).cpu().numpy()
+    lut_o, idx_o, _ = orc.kmeans_int4km(W.numpy())
+    assert rel_err(y, orc.matvec(orc.FMT_INT4KM, idx_o, lut_o, x, N, K)) < TOL
+
+
+def test_encode_int4km_argument_checks(q):
+    W = torch.zeros((4, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(q.QmvError) as ei:
+        q.encode_int4km(W, iters=-1)
+    assert ei.value.status == q.ERR_ARG
+    with pytest.raises(q.QmvError) as ei:
+        q.encode_int4km(torch.zeros((4, 32768), dtype=torch.float32, device="cuda"))
+    assert ei.value.status == q.ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------
 # fused matvec + argmax
 # ---------------------------------------------------------------------------
 

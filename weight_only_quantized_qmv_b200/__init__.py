@@ -46,6 +46,7 @@ SIGNATURES = {
     "qmv_encode_fp4": [_P, _I64, _I64, _P, _P, _P],
     "qmv_encode_int4": [_P, _I64, _I64, _P, _I32, _P, _P, _P],
     "qmv_encode_int8": [_P, _I64, _I64, _P, _I32, _P, _P, _P],
+    "qmv_encode_int4km": [_P, _I64, _I64, _I32, _P, _P, _P],
     "qmv_matvec_fp4": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int4": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int4km": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
@@ -139,6 +140,20 @@ def encode_int4(W: torch.Tensor, clips=INT4_CLIPS, stream=None):
 def encode_int8(W: torch.Tensor, clips=INT8_CLIPS, stream=None):
     """-> (codes int8 [N, K], scales float16 [N, K/32])."""
     return _encode_int("qmv_encode_int8", W, clips, 8, stream)
+
+
+KMEANS_ITERS = 20  # Lloyd steps of the int4km workloads
+
+
+def encode_int4km(W: torch.Tensor, iters: int = KMEANS_ITERS, stream=None):
+    """W float32 [N, K] -> (idx uint8 [N, K/2], lut float16 [N, 16]): per-row
+    16-entry k-means palette and packed indices."""
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    idx = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    lut = torch.empty((N, 16), dtype=torch.float16, device=W.device)
+    _call("qmv_encode_int4km", _ptr(W), N, K, int(iters), _ptr(lut), _ptr(idx), _stream(stream))
+    return idx, lut
 
 
 # ---------------------------------------------------------------- matvec

@@ -216,6 +216,22 @@ qmv_status qmv_encode_int8(const float* W, int64_t N, int64_t K, const float* cl
   return encode_int(127, W, N, K, clips, n_clips, reinterpret_cast<uint8_t*>(codes), scales, stream);
 }
 
+qmv_status qmv_encode_int4km(const float* W, int64_t N, int64_t K, int iters, uint16_t* lut, uint8_t* idx,
+                             void* stream) {
+  QMV_TRY(check_ptr(W, "W"));
+  QMV_TRY(check_ptr(idx, "idx"));
+  if (!lut || (reinterpret_cast<uintptr_t>(lut) & 1u)) return fail(QMV_ERR_ARG, "lut null or misaligned");
+  if (iters < 0 || iters > 1000) return fail(QMV_ERR_ARG, "iters must be in [0, 1000] (got %d)", iters);
+  QMV_TRY(check_shape(N, K));
+  if (K > 16384) return fail(QMV_ERR_UNSUPPORTED, "K must be <= 16384 for the palette fit (got %lld)", (long long)K);
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  cudaError_t e = qmv::launch_encode_int4km(W, N, K, iters, lut, idx, st, sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "encode_int4km launch");
+  return QMV_OK;
+}
+
 qmv_status qmv_matvec_fp4(const uint8_t* codes, const uint8_t* scales, const uint16_t* x, int B, int64_t N,
                           int64_t K, float* y, void* stream) {
   return matvec_common(QMV_FMT_FP4, codes, scales, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);

@@ -116,6 +116,8 @@ cudaError_t launch_encode_fp4(const float* W, int64_t N, int64_t K, uint8_t* cod
 cudaError_t launch_encode_int(int qmax, const float* W, int64_t N, int64_t K, const ClipList& clips,
                               uint8_t* codes, uint16_t* scales, uint32_t* status, int num_sms,
                               cudaStream_t stream);
+cudaError_t launch_encode_int4km(const float* W, int64_t N, int64_t K, int iters, uint16_t* lut, uint8_t* idx,
+                                 uint32_t* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_dequant(int fmt, const uint8_t* codes, const uint8_t* aux, int64_t N, int64_t K, float* Wdq,
                            int num_sms, cudaStream_t stream);
 

@@ -249,9 +249,9 @@ __device__ __forceinline__ Palette palette_from_words(const uint32_t (&e)[8]) {
 __device__ __forceinline__ void dec_int4km(const Palette& p, uint32_t w, uint32_t& s0lo, uint32_t& s0hi,
                                            uint32_t& s1lo, uint32_t& s1hi, const Mul& m) {
   const uint32_t w4 = w * m.p4;  // w << 4 on the multiply pipe (the lookups load the ALU)
-  const uint32_t wh = w >> 16;
-  const uint32_t sel0 = w & 0x7777u;   // nibbles 0..3, bit 3 cleared
-  const uint32_t sel1 = wh & 0x7777u;  // nibbles 4..7
+  // byte permutes read only the low 16 bits of their selector
+  const uint32_t sel0 = w & 0x77777777u;  // bit 3 of every nibble cleared; nibbles 0..3 in the low half
+  const uint32_t sel1 = sel0 >> 16;       // nibbles 4..7
   const uint32_t m0 = prmt(w4, w, 0xD9C8u);  // byte i = 0xFF iff bit 3 of nibble i
   const uint32_t m1 = prmt(w4, w, 0xFBEAu);  // nibbles 4..7
   const uint32_t lo_a = lop3_mux(prmt(p.lo0, p.lo1, sel0), prmt(p.lo2, p.lo3, sel0), m0);

@@ -87,6 +87,24 @@ def profiled_traffic(kernel_fmt: str):
     return int(m.group(1)) if m else None
 
 
+# ----------------------------------------------------------------- ranks
+
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's time: every rank takes the job's pace from it
+    (all-reduce MAX on the process group; gloo on CPU tensors, NCCL on GPU)."""
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank_step: int, world: int, ms_step: float) -> float:
+    """Whole-job throughput: every replica moves bytes_per_rank_step per step,
+    all of them at the slowest rank's step time."""
+    return bytes_per_rank_step * world / (ms_step * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -268,11 +286,9 @@ def run_ours(args, rank, world, local_rank):
 
     ms_step = total_ms / args.steps
     if dist:
-        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms_step = float(t.item())
+        ms_step = max_over_ranks(ms_step, dev)
     bytes_step = sum(algorithmic_bytes(f, N_HEAD, K_HEAD, 1) for f in formats)
-    value = bytes_step * world / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(bytes_step, world, ms_step)
 
     # per-format kernel time: a graph of 10 back-to-back launches of one format
     peak, peak_src = hbm_peak()

@@ -16,7 +16,7 @@ import numpy as np
 
 from . import build as _build
 
-FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8 = 0, 1, 2, 3
+FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8, FMT_INT4AFF = 0, 1, 2, 3, 4
 FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT = 1, 2, 4
 
 # Clip lists: the int4 list of the int4 lm_head workload (1.00 down to 0.50
@@ -47,12 +47,16 @@ def lib():
         L.oracle_encode_fp4.argtypes = [P, I64, I64, P, P, U32P]
         L.oracle_encode_int_sym.argtypes = [P, I64, I64, I32, P, I32, P, P, U32P]
         L.oracle_kmeans_int4km.argtypes = [P, I64, I64, I32, P, P, P, U32P]
+        L.oracle_encode_int4aff.argtypes = [P, I64, I64, P, P, U32P]
+        L.oracle_int4aff_aux_row_bytes.argtypes = [I64]
+        L.oracle_int4aff_aux_row_bytes.restype = I64
         L.oracle_dequant.argtypes = [I32, P, P, I64, I64, P]
         L.oracle_matvec_rows.argtypes = [I32, P, P, P, I32, I64, I64, P, I64, P]
         L.oracle_gather_matvec.argtypes = [I32, P, P, I32, I64, I64, P, I32, I32, P, I32, P, U32P]
         L.oracle_num_threads.restype = I32
         L.oracle_set_num_threads.argtypes = [I32]
-        for f in ("oracle_encode_fp4", "oracle_encode_int_sym", "oracle_kmeans_int4km", "oracle_dequant",
+        for f in ("oracle_encode_fp4", "oracle_encode_int_sym", "oracle_kmeans_int4km", "oracle_encode_int4aff",
+                  "oracle_dequant",
                   "oracle_matvec_rows", "oracle_gather_matvec"):
             getattr(L, f).restype = I32
         _lib = L
@@ -127,6 +131,22 @@ def encode_int4(W, clips=INT4_CLIPS):
 def encode_int8(W, clips=INT8_CLIPS):
     """-> (codes int8 [N, K], scales float16 [N, K/32], flags)."""
     return _encode_sym(W, 127, clips)
+
+
+def int4aff_aux_row_bytes(K):
+    return int(lib().oracle_int4aff_aux_row_bytes(int(K)))
+
+
+def encode_int4aff(W):
+    """-> (codes uint8 [N, K/2] (q nibbles), aux uint8 [N, row bytes] (fp16
+    scales [K/32] then zero-point nibbles), flags)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    codes = np.zeros((N, K // 2), np.uint8)
+    aux = np.zeros((N, int4aff_aux_row_bytes(K)), np.uint8)
+    fl = ctypes.c_uint32(0)
+    _check(lib().oracle_encode_int4aff(_p(W), N, K, _p(codes), _p(aux), ctypes.byref(fl)), "encode_int4aff")
+    return codes, aux, fl.value
 
 
 def kmeans_int4km(W, iters=KMEANS_ITERS, want_sse=False):

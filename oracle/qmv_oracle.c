@@ -46,6 +46,7 @@
 #define ORC_FMT_INT4 1
 #define ORC_FMT_INT4KM 2
 #define ORC_FMT_INT8 3
+#define ORC_FMT_INT4AFF 4
 
 /* ------------------------------------------------------------------ */
 /* IEEE binary16 <-> binary32, written from the format definition.     */
@@ -386,6 +387,82 @@ int oracle_kmeans_int4km(const float* W, int64_t N, int64_t K, int iters,
 }
 
 /* ------------------------------------------------------------------ */
+/* int4 affine (asymmetric) per block of 32                           */
+/* [P3 "Quantization": symmetric vs asymmetric scheme; "Theoretical     */
+/*  size": an fp16 scale and an n_bits zero point per group]; [P1 sec.1:*/
+/*  the gather format int4aff, affine int4, block 32]                  */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of one row's aux for int4aff: fp16 scales [K/32], then the zero
+ * points, two per byte (block 2j in the low nibble). */
+int64_t oracle_int4aff_aux_row_bytes(int64_t K) { return 2 * (K / 32) + (K / 32 + 1) / 2; }
+
+/* Readings where no page fixes the details, per block of 32 weights:
+ *  range [lo, hi] = [min(min w, 0), max(max w, 0)] (zero inside, so the
+ *  zero point is an integer of [0, 15]);
+ *  s = fp16_RNE((hi - lo) / 15), computed in float;
+ *  z = clamp(rint(-lo / s), 0, 15) with the stored s (float);
+ *  q = clamp(rint(w / s) + z, 0, 15) (float);  Wdq = s * (q - z).
+ * An all-zero block has s = 0, q = z = 0.  An fp16 overflow of s zeroes the
+ * block and raises SCALE_OVERFLOW; Inf/NaN zeroes it and raises NONFINITE. */
+int oracle_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes,
+                          uint8_t* aux, uint32_t* flags_out) {
+  if (K % 32 != 0 || N < 0) return -2;
+  uint32_t flags = 0;
+  int64_t nb = K / 32, arow = oracle_int4aff_aux_row_bytes(K);
+#pragma omp parallel for reduction(| : flags) schedule(static)
+  for (int64_t n = 0; n < N; n++) {
+    uint8_t* ar = aux + n * arow;
+    uint16_t* sc = (uint16_t*)ar;
+    uint8_t* zp = ar + 2 * nb;
+    memset(zp, 0, (size_t)((nb + 1) / 2));
+    for (int64_t b = 0; b < nb; b++) {
+      const float* w = W + n * K + b * 32;
+      float lo = 0.0f, hi = 0.0f;
+      int finite = 1;
+      for (int i = 0; i < 32; i++) {
+        if (!isfinite(w[i])) finite = 0;
+        if (w[i] < lo) lo = w[i];
+        if (w[i] > hi) hi = w[i];
+      }
+      int q[32] = {0};
+      uint16_t sh = 0;
+      int z = 0;
+      if (!finite) {
+        flags |= ORC_FLAG_NONFINITE;
+      } else {
+        sh = orc_f32_to_f16((hi - lo) / 15.0f);
+        if ((sh & 0x7C00) == 0x7C00) {
+          flags |= ORC_FLAG_SCALE_OVERFLOW;
+          sh = 0;
+        } else {
+          float s = orc_f16_to_f32(sh);
+          if (s != 0.0f) {
+            float zf = rintf(-lo / s);
+            if (zf < 0.0f) zf = 0.0f;
+            if (zf > 15.0f) zf = 15.0f;
+            z = (int)zf;
+            for (int i = 0; i < 32; i++) {
+              float r = rintf(w[i] / s) + (float)z;
+              if (r < 0.0f) r = 0.0f;
+              if (r > 15.0f) r = 15.0f;
+              q[i] = (int)r;
+            }
+          }
+        }
+      }
+      sc[b] = sh;
+      zp[b / 2] |= (uint8_t)(z << ((b % 2) * 4));
+      uint8_t* cb = codes + n * (K / 2) + b * 16;
+      for (int i = 0; i < 32; i += 2) cb[i / 2] = (uint8_t)(q[i] | (q[i + 1] << 4));
+    }
+  }
+  if (flags_out) *flags_out = flags;
+  return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Dequantization (exact in float) and the fp64 matvec                *//* ------------------------------------------------------------------ */
 /* Dequantization (exact in float) and the fp64 matvec                */
 /* ------------------------------------------------------------------ */
 
@@ -417,13 +494,23 @@ static float orc_wdq(int fmt, const void* codes, const void* aux, int64_t K,
       float s = orc_f16_to_f32(((const uint16_t*)aux)[n * nb + k / 32]);
       return (float)q * s;
     }
+    case ORC_FMT_INT4AFF: {
+      uint8_t byte = ((const uint8_t*)codes)[n * (K / 2) + k / 2];
+      int q = (k % 2) ? (byte >> 4) : (byte & 15);
+      const uint8_t* ar = (const uint8_t*)aux + n * oracle_int4aff_aux_row_bytes(K);
+      int64_t b = k / 32;
+      float s = orc_f16_to_f32(((const uint16_t*)ar)[b]);
+      uint8_t zb = ar[2 * nb + b / 2];
+      int z = (b % 2) ? (zb >> 4) : (zb & 15);
+      return (float)(q - z) * s;
+    }
   }
   return NAN;
 }
 
 int oracle_dequant(int fmt, const void* codes, const void* aux, int64_t N,
                    int64_t K, float* Wdq) {
-  if (K % 32 != 0 || N < 0 || fmt < 0 || fmt > 3) return -2;
+  if (K % 32 != 0 || N < 0 || fmt < 0 || fmt > 4) return -2;
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; n++)
     for (int64_t k = 0; k < K; k++) Wdq[n * K + k] = orc_wdq(fmt, codes, aux, K, n, k);
@@ -437,7 +524,7 @@ int oracle_dequant(int fmt, const void* codes, const void* aux, int64_t N,
 int oracle_matvec_rows(int fmt, const void* codes, const void* aux,
                        const uint16_t* x, int B, int64_t N, int64_t K,
                        const int64_t* rows, int64_t nrows, double* r) {
-  if (K % 32 != 0 || N < 0 || B < 1 || fmt < 0 || fmt > 3) return -2;
+  if (K % 32 != 0 || N < 0 || B < 1 || fmt < 0 || fmt > 4) return -2;
   int64_t R = rows ? nrows : N;
   double* xd = (double*)malloc((size_t)(B * K) * sizeof(double));
   for (int64_t i = 0; i < (int64_t)B * K; i++) xd[i] = (double)orc_f16_to_f32(x[i]);
@@ -469,11 +556,12 @@ int oracle_gather_matvec(int fmt, const void* codes, const void* aux, int E,
                          int64_t N, int64_t K, const int32_t* ids, int B,
                          int topk, const uint16_t* x, int x_per_slot,
                          double* y, uint32_t* flags_out) {
-  if (K % 32 != 0 || N < 0 || B < 1 || topk < 1 || fmt < 0 || fmt > 3) return -2;
+  if (K % 32 != 0 || N < 0 || B < 1 || topk < 1 || fmt < 0 || fmt > 4) return -2;
   int64_t code_bytes = (fmt == ORC_FMT_INT8) ? N * K : N * (K / 2);
   int64_t aux_bytes = (fmt == ORC_FMT_FP4) ? N * (K / 32)
                       : (fmt == ORC_FMT_INT4KM) ? N * 16 * 2
-                                                : N * (K / 32) * 2;
+                      : (fmt == ORC_FMT_INT4AFF) ? N * oracle_int4aff_aux_row_bytes(K)
+                                                 : N * (K / 32) * 2;
   uint32_t flags = 0;
   for (int b = 0; b < B; b++) {
     for (int j = 0; j < topk; j++) {

@@ -26,6 +26,10 @@ MUTANTS = {
                                       "if (cnt[k] > 0 && 0) c[k] = (double)(float)(sum[k] / (double)cnt[k]);"),
     "fp16 ties away from zero": ("double m = nearbyint(ldexp(a, 10 - E));", "double m = round(ldexp(a, 10 - E));"),
     "int8 clamp at 126": ("if (r > (float)qmax) r = (float)qmax;", "if (r > (float)qmax - 1) r = (float)qmax - 1;"),
+    "int4aff zero point dropped in dequant": ("return (float)(q - z) * s;", "return (float)(q) * s;"),
+    "int4aff range without zero": ("float lo = 0.0f, hi = 0.0f;", "float lo = w[0], hi = w[0];"),
+    "int4aff zero-point nibble order": ("zp[b / 2] |= (uint8_t)(z << ((b % 2) * 4));",
+                                        "zp[b / 2] |= (uint8_t)(z << ((1 - b % 2) * 4));"),
 }
 
 

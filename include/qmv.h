@@ -68,7 +68,8 @@ enum {
   QMV_FMT_FP4 = 0,    /* E2M1 codes + e8m0 scale byte per 32-block      */
   QMV_FMT_INT4 = 1,   /* symmetric int4 (nibble = q + 8) + fp16 scale   */
   QMV_FMT_INT4KM = 2, /* 4-bit index into a per-row 16-entry fp16 LUT   */
-  QMV_FMT_INT8 = 3    /* symmetric int8 (two's complement) + fp16 scale */
+  QMV_FMT_INT8 = 3,   /* symmetric int8 (two's complement) + fp16 scale */
+  QMV_FMT_INT4AFF = 4 /* affine int4 (q, zero point) + fp16 scale      */
 };
 
 /* Device status bits (qmv_status_fetch). */
@@ -111,6 +112,24 @@ qmv_status qmv_encode_int4(const float* W, int64_t N, int64_t K, const float* cl
 qmv_status qmv_encode_int8(const float* W, int64_t N, int64_t K, const float* clips,
                            int n_clips, int8_t* codes, uint16_t* scales, void* stream);
 
+/* Affine (asymmetric) int4 encode per block of 32 ([P3] "Quantization":
+ * asymmetric scheme; "Theoretical size": an fp16 scale and an n_bits zero
+ * point per group; [P1] sec. 1: the gather format int4aff).  Per block:
+ * range [lo, hi] = [min(min w, 0), max(max w, 0)]; s = fp16_RNE((hi - lo) /
+ * 15); z = clamp(rint(-lo / s), 0, 15); q = clamp(rint(w / s) + z, 0, 15),
+ * float arithmetic with the stored s; Wdq = s * (q - z).  An all-zero block
+ * has s = 0, q = z = 0; an fp16 overflow of s zeroes the block with
+ * QMV_FLAG_SCALE_OVERFLOW; Inf/NaN zeroes it with QMV_FLAG_NONFINITE.
+ *   codes  [N, K/2] uint8, q nibbles, element 2j in the low nibble (out)
+ *   aux    [N, qmv_int4aff_aux_row_bytes(K)] uint8 (out): per row the fp16
+ *          scales [K/32], then the zero points two per byte (block 2j in the
+ *          low nibble; a last odd block leaves the high nibble 0). */
+qmv_status qmv_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* aux,
+                              void* stream);
+
+/* Bytes of one int4aff aux row: 2 * (K/32) + ceil(K/64). */
+int64_t qmv_int4aff_aux_row_bytes(int64_t K);
+
 /* int4km encode: per row a 16-entry fp16 palette by scalar 1-D k-means and
  * the packed 4-bit index of each weight ([P3] "Palettization": scalar
  * k-means, 2^n_bits centroids, per-channel grouping; [P2] sec. 8: per-row
@@ -152,6 +171,15 @@ qmv_status qmv_matvec_int4km(const uint8_t* idx, const uint16_t* lut, const uint
 /* codes [N, K] int8; scales [N, K/32] fp16. */
 qmv_status qmv_matvec_int8(const int8_t* codes, const uint16_t* scales, const uint16_t* x,
                            int B, int64_t N, int64_t K, float* y, void* stream);
+
+/* codes [N, K/2] uint8 (q nibbles); aux [N, qmv_int4aff_aux_row_bytes(K)]
+ * (fp16 scales, then zero-point nibbles), as qmv_encode_int4aff writes them;
+ * y[b, n] = sum_k s(n, k/32) * (q[n, k] - z(n, k/32)) * x[b, k].  aux may
+ * have any alignment; with aux 8-byte aligned and K % 512 == 0 the scales
+ * and zero points are copied asynchronously, otherwise byte by byte (slower,
+ * same result). */
+qmv_status qmv_matvec_int4aff(const uint8_t* codes, const uint8_t* aux, const uint16_t* x,
+                              int B, int64_t N, int64_t K, float* y, void* stream);
 
 /* ---------------------------------------------------------------------
  * Fused matvec + argmax (greedy next token from the lm_head; the pages'

@@ -16,7 +16,7 @@ from weight_only_quantized_qmv_b200 import synth
 pytestmark = pytest.mark.gpu
 
 TOL = 1e-3
-FMTS = ("fp4", "int4", "int4km", "int8")
+FMTS = ("fp4", "int4", "int4km", "int8", "int4aff")
 
 
 @pytest.fixture(scope="module")
@@ -54,6 +54,8 @@ def encode_gpu(q, fmt, W, W_np=None):
         return q.encode_int4(W)
     if fmt == "int8":
         return q.encode_int8(W)
+    if fmt == "int4aff":
+        return q.encode_int4aff(W)
     lut, idx, _ = orc.kmeans_int4km(W.cpu().numpy() if W_np is None else W_np)
     return torch.from_numpy(idx).cuda(), torch.from_numpy(lut).cuda()
 
@@ -65,12 +67,15 @@ def encode_orc(fmt, Wn):
         c, s, f = orc.encode_int4(Wn)
     elif fmt == "int8":
         c, s, f = orc.encode_int8(Wn)
+    elif fmt == "int4aff":
+        c, s, f = orc.encode_int4aff(Wn)
     else:
         s, c, f = orc.kmeans_int4km(Wn)
     return c, s, f
 
 
-FID = {"fp4": orc.FMT_FP4, "int4": orc.FMT_INT4, "int4km": orc.FMT_INT4KM, "int8": orc.FMT_INT8}
+FID = {"fp4": orc.FMT_FP4, "int4": orc.FMT_INT4, "int4km": orc.FMT_INT4KM, "int8": orc.FMT_INT8,
+       "int4aff": orc.FMT_INT4AFF}
 
 
 def np_bits(t):
@@ -111,7 +116,7 @@ def test_e2m1_hardware_conversion_matches_oracle_table(q):
     assert q.status_fetch() == 0
 
 
-@pytest.mark.parametrize("fmt", ["fp4", "int4", "int8"])
+@pytest.mark.parametrize("fmt", ["fp4", "int4", "int8", "int4aff"])
 @pytest.mark.parametrize("N,K", [(1, 32), (40, 96), (300, 544), (64, 2080), (33, 4096)])
 def test_encoder_bit_exact(q, fmt, N, K):
     W, _ = gen_w(N, K, seed=N + K, n_out=max(1, K // 1000))
@@ -124,7 +129,50 @@ def test_encoder_bit_exact(q, fmt, N, K):
     c_o, s_o, f = encode_orc(fmt, Wn)
     assert f == 0
     assert np.array_equal(np_bits(c_g), c_o.view(np.uint8))
-    assert np.array_equal(np_bits(s_g), s_o.view(np.uint8) if fmt == "fp4" else s_o.view(np.uint16))
+    assert np.array_equal(np_bits(s_g), s_o.view(np.uint8) if fmt in ("fp4", "int4aff") else s_o.view(np.uint16))
+    assert q.status_fetch() == 0
+
+
+def test_encode_int4aff_special_blocks(q):
+    """Blocks of one sign (zero point at an end of the range), a constant
+    block, a block whose range gives an fp16-subnormal scale, halfway cases
+    of w / s, and a last odd block (its zero-point byte's high nibble stays 0)."""
+    K = 96
+    W = np.zeros((6, K), np.float32)
+    rng = np.random.default_rng(5)
+    W[0] = np.abs(rng.standard_normal(K)).astype(np.float32) * 0.02  # all >= 0: z = 0
+    W[1] = -np.abs(rng.standard_normal(K)).astype(np.float32) * 0.02  # all <= 0: z = 15
+    W[2] = 0.375  # constant block
+    W[3] = rng.standard_normal(K).astype(np.float32) * 1e-7  # scale in the fp16 subnormal range
+    W[4] = (np.arange(K) % 31 - 15).astype(np.float32) * 0.5 / 15.0  # w / s on halfway points
+    W[5] = rng.standard_normal(K).astype(np.float32)
+    c_g, a_g = q.encode_int4aff(torch.from_numpy(W).cuda())
+    c_o, a_o, f = orc.encode_int4aff(W)
+    assert f == 0 and q.status_fetch() == 0
+    assert np.array_equal(c_g.cpu().numpy(), c_o)
+    assert np.array_equal(a_g.cpu().numpy(), a_o)
+    assert (a_o[:, -1] >> 4 == 0).all()  # K / 32 = 3 blocks: the last byte holds one zero point
+
+
+def test_int4aff_unaligned_aux(q):
+    """An aux plane starting at an odd byte (and one at 4 mod 8) takes the
+    bytewise staging path on a shape that is otherwise copied asynchronously."""
+    N, K = 70, 2048
+    for B in (1, 3):
+        c_o, a_o, xn = _inputs("int4aff", N, K, B, seed=19 + B)
+        r = orc.matvec(orc.FMT_INT4AFF, c_o, a_o, xn, N, K)
+        c, x = torch.from_numpy(c_o).cuda(), torch.from_numpy(xn).cuda()
+        y0 = q.matvec_int4aff(c, torch.from_numpy(a_o).cuda(), x)
+        for off in (1, 4):
+            ab = torch.zeros(a_o.size + off, dtype=torch.uint8, device="cuda")
+            ab[off:] = torch.from_numpy(a_o.reshape(-1)).cuda()
+            y = q.matvec_int4aff(c, ab[off:].view(N, -1), x)
+            assert rel_err(y.cpu().numpy(), r) < TOL
+            if B == 1:
+                # batch 1 leaves the block-column form for the general one: same tolerance
+                assert rel_err(y.cpu().numpy(), y0.cpu().numpy().astype(np.float64)) < TOL
+            else:
+                assert torch.equal(y, y0)  # same form, same summation order
     assert q.status_fetch() == 0
 
 
@@ -514,7 +562,7 @@ def test_nonfinite_weights_flag_and_zero_blocks(q):
     W[3, 40] = float("nan")
     W[5, 100] = float("inf")
     Wn = W.cpu().numpy()
-    for fmt in ("fp4", "int4", "int8"):
+    for fmt in ("fp4", "int4", "int8", "int4aff"):
         c, s = encode_gpu(q, fmt, W)
         flags = q.status_fetch()
         assert flags & q.FLAG_NONFINITE, fmt
@@ -531,6 +579,12 @@ def test_scale_overflow_flag(q):
     c_o, s_o, f = orc.encode_int4(W.cpu().numpy(), np.array([1.0], np.float32))
     assert f & orc.FLAG_SCALE_OVERFLOW
     assert np.array_equal(c.cpu().numpy(), c_o) and np.array_equal(np_bits(s), s_o.view(np.uint16))
+    # affine int4: (1e6 - 0) / 15 > 65504
+    c, a = q.encode_int4aff(W)
+    assert q.status_fetch() & q.FLAG_SCALE_OVERFLOW
+    c_o, a_o, f = orc.encode_int4aff(W.cpu().numpy())
+    assert f & orc.FLAG_SCALE_OVERFLOW
+    assert np.array_equal(c.cpu().numpy(), c_o) and np.array_equal(a.cpu().numpy(), a_o)
 
 
 def test_argument_errors_raise(q):
@@ -561,7 +615,7 @@ def _full_encode_check(q, fmt, W, rows):
     c_o, s_o, f = encode_orc(fmt, W[torch.from_numpy(rows).cuda()].cpu().numpy())
     assert f == 0
     assert np.array_equal(np_bits(c)[rows], c_o.view(np.uint8))
-    assert np.array_equal(np_bits(s)[rows], s_o.view(np.uint8) if fmt == "fp4" else s_o.view(np.uint16))
+    assert np.array_equal(np_bits(s)[rows], s_o.view(np.uint8) if fmt in ("fp4", "int4aff") else s_o.view(np.uint16))
     return c, s, c_o, s_o
 
 
@@ -587,8 +641,8 @@ def test_full_int8_head_130560x2048(q):
 
 @pytest.mark.slow
 def test_full_int4_and_fp4_head_248320x2048(q):
-    """int4 (11 clips) and fp4 on the same outlier-bearing head; fp4 at
-    batch 1, 4 and 16."""
+    """int4 (11 clips), affine int4 and fp4 on the same outlier-bearing head;
+    affine int4 at batch 1 and 16, fp4 at batch 1, 4 and 16."""
     N, K = 248320, 2048
     g = synth.generator(0, "cuda")
     W, _ = synth.weights(N, K, g, n_outlier_cols=2)
@@ -596,6 +650,10 @@ def test_full_int4_and_fp4_head_248320x2048(q):
     rows = sample_rows(N)
     c, s, c_o, s_o = _full_encode_check(q, "int4", W, rows)
     _sampled_matvec(q, "int4", c, s, c_o, s_o, x16[:1], rows, K)
+    del c, s
+    c, s, c_o, s_o = _full_encode_check(q, "int4aff", W, rows)
+    for B in (1, 16):
+        _sampled_matvec(q, "int4aff", c, s, c_o, s_o, x16[:B], rows, K)
     del c, s
     c, s, c_o, s_o = _full_encode_check(q, "fp4", W, rows)
     for B in (1, 4, 16):

@@ -21,8 +21,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqmv.so")
 
-FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8 = 0, 1, 2, 3
-FMT_NAMES = {FMT_FP4: "fp4", FMT_INT4: "int4", FMT_INT4KM: "int4km", FMT_INT8: "int8"}
+FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8, FMT_INT4AFF = 0, 1, 2, 3, 4
+FMT_NAMES = {FMT_FP4: "fp4", FMT_INT4: "int4", FMT_INT4KM: "int4km", FMT_INT8: "int8", FMT_INT4AFF: "int4aff"}
 FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT = 1, 2, 4
 OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_DATA, ERR_CUDA = 0, -1, -2, -3, -4, -5
 
@@ -47,10 +47,13 @@ SIGNATURES = {
     "qmv_encode_int4": [_P, _I64, _I64, _P, _I32, _P, _P, _P],
     "qmv_encode_int8": [_P, _I64, _I64, _P, _I32, _P, _P, _P],
     "qmv_encode_int4km": [_P, _I64, _I64, _I32, _P, _P, _P],
+    "qmv_encode_int4aff": [_P, _I64, _I64, _P, _P, _P],
+    "qmv_int4aff_aux_row_bytes": [_I64],
     "qmv_matvec_fp4": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int4": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int4km": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int8": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
+    "qmv_matvec_int4aff": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_gather_matvec": [_I32, _P, _P, _I32, _I64, _I64, _P, _I32, _I32, _P, _I32, _P, _P],
     "qmv_matvec_argmax": [_I32, _P, _P, _P, _I32, _I64, _I64, _P, ctypes.c_size_t, _P, _P, _P],
     "qmv_argmax_workspace_bytes": [ctypes.POINTER(ctypes.c_size_t)],
@@ -74,7 +77,8 @@ def lib() -> ctypes.CDLL:
         for name, args in SIGNATURES.items():
             f = getattr(L, name)
             f.argtypes = args
-            f.restype = ctypes.c_char_p if name in ("qmv_last_error", "qmv_version") else ctypes.c_int
+            f.restype = (ctypes.c_char_p if name in ("qmv_last_error", "qmv_version")
+                         else ctypes.c_int64 if name == "qmv_int4aff_aux_row_bytes" else ctypes.c_int)
         _lib = L
     return _lib
 
@@ -156,12 +160,30 @@ def encode_int4km(W: torch.Tensor, iters: int = KMEANS_ITERS, stream=None):
     return idx, lut
 
 
+def int4aff_aux_row_bytes(K: int) -> int:
+    """Bytes of one int4aff aux row: fp16 scales [K/32], then zero points two per byte."""
+    return int(lib().qmv_int4aff_aux_row_bytes(int(K)))
+
+
+def encode_int4aff(W: torch.Tensor, stream=None):
+    """W float32 [N, K] -> (codes uint8 [N, K/2] (q nibbles), aux uint8 [N,
+    int4aff_aux_row_bytes(K)]): affine int4 per block of 32."""
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    aux = torch.empty((N, int4aff_aux_row_bytes(K)), dtype=torch.uint8, device=W.device)
+    _call("qmv_encode_int4aff", _ptr(W), N, K, _ptr(codes), _ptr(aux), _stream(stream))
+    return codes, aux
+
+
 # ---------------------------------------------------------------- matvec
 
-_AUX = {FMT_FP4: torch.uint8, FMT_INT4: torch.float16, FMT_INT4KM: torch.float16, FMT_INT8: torch.float16}
-_CODES = {FMT_FP4: torch.uint8, FMT_INT4: torch.uint8, FMT_INT4KM: torch.uint8, FMT_INT8: torch.int8}
+_AUX = {FMT_FP4: torch.uint8, FMT_INT4: torch.float16, FMT_INT4KM: torch.float16, FMT_INT8: torch.float16,
+        FMT_INT4AFF: torch.uint8}
+_CODES = {FMT_FP4: torch.uint8, FMT_INT4: torch.uint8, FMT_INT4KM: torch.uint8, FMT_INT8: torch.int8,
+          FMT_INT4AFF: torch.uint8}
 _ENTRY = {FMT_FP4: "qmv_matvec_fp4", FMT_INT4: "qmv_matvec_int4", FMT_INT4KM: "qmv_matvec_int4km",
-          FMT_INT8: "qmv_matvec_int8"}
+          FMT_INT8: "qmv_matvec_int8", FMT_INT4AFF: "qmv_matvec_int4aff"}
 
 
 def _nk(fmt, codes):
@@ -202,6 +224,10 @@ def matvec_int4km(idx, lut, x, out=None, stream=None):
 
 def matvec_int8(codes, scales, x, out=None, stream=None):
     return matvec(FMT_INT8, codes, scales, x, out, stream)
+
+
+def matvec_int4aff(codes, aux, x, out=None, stream=None):
+    return matvec(FMT_INT4AFF, codes, aux, x, out, stream)
 
 
 def argmax_workspace_bytes() -> int:

@@ -63,6 +63,10 @@ qmv_status check_ptr(const void* p, const char* name) {
   return QMV_OK;
 }
 
+// formats whose aux is fp16 scales at every row start (int4aff rows may have
+// an odd byte count and are read bytewise where they are not 8-byte granular)
+bool has_fp16_scale_rows(int fmt) { return fmt == QMV_FMT_INT4 || fmt == QMV_FMT_INT8; }
+
 qmv_status check_shape(int64_t N, int64_t K) {
   if (N < 1) return fail(QMV_ERR_SHAPE, "N must be >= 1 (got %lld)", (long long)N);
   if (K < 32 || K % 32 != 0)
@@ -130,13 +134,14 @@ struct ArgmaxOut {
 qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
                          int64_t K, float* y, void* stream, bool gather, int E, const int32_t* ids, int topk,
                          int x_per_slot, const ArgmaxOut* am = nullptr) {
-  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
+  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT4AFF) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
   QMV_TRY(check_ptr(codes, "codes"));
   if (!aux) return fail(QMV_ERR_ARG, "scales/lut is null");
   // the staged scale block copies handle any byte alignment; the palette and
   // row-aligned scale copies need 16-byte alignment
   if (fmt == QMV_FMT_INT4KM) QMV_TRY(check_ptr(aux, "lut"));
-  if (fmt != QMV_FMT_FP4 && (reinterpret_cast<uintptr_t>(aux) & 1u)) return fail(QMV_ERR_ARG, "fp16 scales misaligned");
+  if (has_fp16_scale_rows(fmt) && (reinterpret_cast<uintptr_t>(aux) & 1u))
+    return fail(QMV_ERR_ARG, "fp16 scales misaligned");
   QMV_TRY(check_ptr(x, "x"));
   if (!am && (!y || (reinterpret_cast<uintptr_t>(y) & 3u))) return fail(QMV_ERR_ARG, "y null or misaligned");
   QMV_TRY(check_shape(N, K));
@@ -232,6 +237,21 @@ qmv_status qmv_encode_int4km(const float* W, int64_t N, int64_t K, int iters, ui
   return QMV_OK;
 }
 
+qmv_status qmv_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* aux, void* stream) {
+  QMV_TRY(check_ptr(W, "W"));
+  QMV_TRY(check_ptr(codes, "codes"));
+  if (!aux) return fail(QMV_ERR_ARG, "aux is null");
+  QMV_TRY(check_shape(N, K));
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  cudaError_t e = qmv::launch_encode_int4aff(W, N, K, codes, aux, st, sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "encode_int4aff launch");
+  return QMV_OK;
+}
+
+int64_t qmv_int4aff_aux_row_bytes(int64_t K) { return K >= 32 ? qmv::int4aff_aux_row_bytes(K) : 0; }
+
 qmv_status qmv_matvec_fp4(const uint8_t* codes, const uint8_t* scales, const uint16_t* x, int B, int64_t N,
                           int64_t K, float* y, void* stream) {
   return matvec_common(QMV_FMT_FP4, codes, scales, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
@@ -250,6 +270,11 @@ qmv_status qmv_matvec_int4km(const uint8_t* idx, const uint16_t* lut, const uint
 qmv_status qmv_matvec_int8(const int8_t* codes, const uint16_t* scales, const uint16_t* x, int B, int64_t N,
                            int64_t K, float* y, void* stream) {
   return matvec_common(QMV_FMT_INT8, codes, scales, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
+}
+
+qmv_status qmv_matvec_int4aff(const uint8_t* codes, const uint8_t* aux, const uint16_t* x, int B, int64_t N,
+                              int64_t K, float* y, void* stream) {
+  return matvec_common(QMV_FMT_INT4AFF, codes, aux, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
 }
 
 qmv_status qmv_matvec_argmax(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
@@ -290,11 +315,12 @@ qmv_status qmv_gather_matvec(int fmt, const void* codes_stack, const void* aux_s
 }
 
 qmv_status qmv_dequant(int fmt, const void* codes, const void* aux, int64_t N, int64_t K, float* Wdq, void* stream) {
-  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
+  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT4AFF) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
   QMV_TRY(check_ptr(codes, "codes"));
   if (!aux) return fail(QMV_ERR_ARG, "aux is null");
   if (fmt == QMV_FMT_INT4KM) QMV_TRY(check_ptr(aux, "lut"));
-  if (fmt != QMV_FMT_FP4 && (reinterpret_cast<uintptr_t>(aux) & 1u)) return fail(QMV_ERR_ARG, "fp16 scales misaligned");
+  if (has_fp16_scale_rows(fmt) && (reinterpret_cast<uintptr_t>(aux) & 1u))
+    return fail(QMV_ERR_ARG, "fp16 scales misaligned");
   QMV_TRY(check_ptr(Wdq, "Wdq"));
   QMV_TRY(check_shape(N, K));
   uint32_t* st;

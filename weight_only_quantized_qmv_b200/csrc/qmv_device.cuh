@@ -202,17 +202,27 @@ __device__ __forceinline__ float e8m0_x2_to_f32(uint32_t u, const Mul& m) {
 struct DecInt4 {
   __device__ __forceinline__ static void run(uint32_t w, uint32_t& s0lo, uint32_t& s0hi, uint32_t& s1lo,
                                              uint32_t& s1hi, const Mul& m) {
-    const uint32_t kMagic = 0x64006400u;  // fp16x2 (1024, 1024)
-    const uint32_t kSub = 0x64086408u;    // fp16x2 (1032, 1032)
+    (void)m;
+    // zero point 8: subtract 1032 from the low nibbles, -72 after the 1/16 scaling of the high ones
+    run_z(w, s0lo, s0hi, s1lo, s1hi, 0x64086408u, 0xD480D480u);
+  }
+  // Any zero point z (affine int4): sub = fp16x2 (1024 + z), neg = fp16x2 -(64 + z);
+  // the results n - z are small integers, exact in fp16.
+  __device__ __forceinline__ static void run_z(uint32_t w, uint32_t& s0lo, uint32_t& s0hi, uint32_t& s1lo,
+                                               uint32_t& s1hi, uint32_t sub, uint32_t neg) {
+    const uint32_t kMagic = 0x64006400u;      // fp16x2 (1024, 1024)
     const uint32_t kSixteenth = 0x2C002C00u;  // fp16x2 (1/16, 1/16)
-    const uint32_t kNeg72 = 0xD480D480u;  // fp16x2 (-72, -72)
     const uint32_t w8 = w >> 8;
-    s0lo = hsub2_u32(lop3_and_or(w, 0x000F000Fu, kMagic), kSub);
-    s0hi = hfma2_u32(lop3_and_or(w, 0x00F000F0u, kMagic), kSixteenth, kNeg72);
-    s1lo = hsub2_u32(lop3_and_or(w8, 0x000F000Fu, kMagic), kSub);
-    s1hi = hfma2_u32(lop3_and_or(w8, 0x00F000F0u, kMagic), kSixteenth, kNeg72);
+    s0lo = hsub2_u32(lop3_and_or(w, 0x000F000Fu, kMagic), sub);
+    s0hi = hfma2_u32(lop3_and_or(w, 0x00F000F0u, kMagic), kSixteenth, neg);
+    s1lo = hsub2_u32(lop3_and_or(w8, 0x000F000Fu, kMagic), sub);
+    s1hi = hfma2_u32(lop3_and_or(w8, 0x00F000F0u, kMagic), kSixteenth, neg);
   }
 };
+// The run_z constants of zero point z (0..15): fp16 1024 + z is 0x6400 + z,
+// fp16 -(64 + z) is 0xD400 + 16 z (ulp 1/16 at 64).
+__device__ __forceinline__ uint32_t int4_zp_sub(uint32_t z) { return (0x6400u + z) * 0x00010001u; }
+__device__ __forceinline__ uint32_t int4_zp_neg(uint32_t z) { return (0xD400u + 16u * z) * 0x00010001u; }
 
 // INT8: one word holds 4 weights (k0..k3).  Bias each byte by 128, splice it
 // under 0x64 (fp16 1024 + u), subtract 1152: exact q.  Pairs (k0,k1) (k2,k3).

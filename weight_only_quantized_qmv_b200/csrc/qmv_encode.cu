@@ -149,6 +149,68 @@ __global__ void enc_int_kernel(const float* __restrict__ W, int64_t nblocks, Cli
   }
 }
 
+// Affine (asymmetric) int4 per block of 32, in the oracle's float order
+// ([P3] "Quantization" / "Theoretical size"; [P1] sec. 1 int4aff): one thread
+// per pair of blocks, so each thread owns whole zero-point bytes.
+//   range [lo, hi] = [min(min w, 0), max(max w, 0)]; s = fp16((hi - lo) / 15);
+//   z = clamp(rint(-lo / s), 0, 15); q = clamp(rint(w / s) + z, 0, 15).
+__global__ void enc_aff_kernel(const float* __restrict__ W, int64_t N, int64_t K, uint8_t* __restrict__ codes,
+                               uint8_t* __restrict__ aux, uint32_t* status) {
+  const int64_t nb = K / 32, npair = (nb + 1) / 2, arow = int4aff_aux_row_bytes(K);
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < N * npair;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = t / npair, pr = t - n * npair;
+    uint8_t* ar = aux + n * arow;
+    uint32_t zbyte = 0, flags = 0;
+    for (int half = 0; half < 2; ++half) {
+      const int64_t b = 2 * pr + half;
+      if (b >= nb) break;
+      const float* w = W + n * K + b * 32;
+      float v[32];
+      float lo = 0.0f, hi = 0.0f;
+      bool finite = true;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        v[i] = w[i];
+        finite = finite && isfinite(v[i]);
+        if (v[i] < lo) lo = v[i];
+        if (v[i] > hi) hi = v[i];
+      }
+      uint16_t sh = 0;
+      uint32_t z = 0;
+      uint32_t q[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) q[i] = 0;
+      if (!finite) {
+        flags |= QMV_FLAG_NONFINITE;
+      } else {
+        sh = __half_as_ushort(__float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f)));
+        if ((sh & 0x7C00u) == 0x7C00u) {
+          flags |= QMV_FLAG_SCALE_OVERFLOW;
+          sh = 0;
+        } else {
+          const float s = __half2float(__ushort_as_half(sh));
+          if (s != 0.0f) {
+            const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.0f), 15.0f);
+            z = (uint32_t)zf;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              q[i] = (uint32_t)fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v[i], s)), zf), 0.0f), 15.0f);
+          }
+        }
+      }
+      ar[2 * b] = (uint8_t)(sh & 0xFFu);  // rows of an odd byte count: byte stores
+      ar[2 * b + 1] = (uint8_t)(sh >> 8);
+      zbyte |= z << (4 * half);
+      uint8_t* cb = codes + n * (K / 2) + b * 16;
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) cb[i / 2] = (uint8_t)(q[i] | (q[i + 1] << 4));
+    }
+    ar[2 * nb + pr] = (uint8_t)zbyte;
+    if (flags) atomicOr(status, flags);
+  }
+}
+
 // Test-only dequantizer built on the matvec kernels' own decoders, so that
 // its bit-exact comparison with the oracle also checks those decoders.
 __device__ __forceinline__ void f16x2_to_f32(uint32_t v, float& lo, float& hi) {
@@ -201,6 +263,14 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
           f16x2_to_f32(s0hi, o[2], o[3]);
           f16x2_to_f32(s1lo, o[4], o[5]);
           f16x2_to_f32(s1hi, o[6], o[7]);
+        } else if constexpr (FMT == QMV_FMT_INT4AFF) {
+          const uint8_t* ar = aux + n * int4aff_aux_row_bytes(K);
+          const uint32_t z = (ar[2 * nb_row + b / 2] >> (4 * (b & 1))) & 15u;
+          DecInt4::run_z(words[q], s0lo, s0hi, s1lo, s1hi, int4_zp_sub(z), int4_zp_neg(z));  // q - z
+          f16x2_to_f32(s0lo, o[0], o[4]);
+          f16x2_to_f32(s0hi, o[1], o[5]);
+          f16x2_to_f32(s1lo, o[2], o[6]);
+          f16x2_to_f32(s1hi, o[3], o[7]);
         } else if constexpr (FMT == QMV_FMT_INT4) {
           DecInt4::run(words[q], s0lo, s0hi, s1lo, s1hi, mul);  // (k0,k4) (k1,k5) (k2,k6) (k3,k7)
           f16x2_to_f32(s0lo, o[0], o[4]);
@@ -221,6 +291,11 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
         for (int i = 0; i < 32; ++i) out[i] = __fmul_rn(out[i], s);
       } else if constexpr (FMT == QMV_FMT_INT4) {
         const float s = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(aux)[blk]));
+#pragma unroll
+        for (int i = 0; i < 32; ++i) out[i] = __fmul_rn(out[i], s);
+      } else if constexpr (FMT == QMV_FMT_INT4AFF) {
+        const uint8_t* ar = aux + n * int4aff_aux_row_bytes(K);  // rows may have an odd byte count
+        const float s = __half2float(__ushort_as_half((unsigned short)(ar[2 * b] | (ar[2 * b + 1] << 8))));
 #pragma unroll
         for (int i = 0; i < 32; ++i) out[i] = __fmul_rn(out[i], s);
       }
@@ -257,6 +332,13 @@ cudaError_t launch_encode_int(int qmax, const float* W, int64_t N, int64_t K, co
   return cudaGetLastError();
 }
 
+cudaError_t launch_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* aux,
+                                  uint32_t* status, int num_sms, cudaStream_t stream) {
+  const int64_t npairs = N * ((K / 32 + 1) / 2);
+  enc_aff_kernel<<<grid_for(npairs, 128, num_sms), 128, 0, stream>>>(W, N, K, codes, aux, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dequant(int fmt, const uint8_t* codes, const uint8_t* aux, int64_t N, int64_t K, float* Wdq,
                            int num_sms, cudaStream_t stream) {
   const int64_t nb = N * (K / 32);
@@ -266,6 +348,7 @@ cudaError_t launch_dequant(int fmt, const uint8_t* codes, const uint8_t* aux, in
     case QMV_FMT_INT4: dequant_kernel<QMV_FMT_INT4><<<grid, 128, 0, stream>>>(codes, aux, N, K, Wdq); break;
     case QMV_FMT_INT4KM: dequant_kernel<QMV_FMT_INT4KM><<<grid, 128, 0, stream>>>(codes, aux, N, K, Wdq); break;
     case QMV_FMT_INT8: dequant_kernel<QMV_FMT_INT8><<<grid, 128, 0, stream>>>(codes, aux, N, K, Wdq); break;
+    case QMV_FMT_INT4AFF: dequant_kernel<QMV_FMT_INT4AFF><<<grid, 128, 0, stream>>>(codes, aux, N, K, Wdq); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

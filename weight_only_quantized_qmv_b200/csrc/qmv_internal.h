@@ -58,7 +58,9 @@ struct MvParams {
   int gk;                  // K granule of split units (in-features)
   int one;                 // batch-1 block-column form (dense B == 1, K % 256 == 0)
   int off_zero;            // its zero activation region
-  int off_xsum;            // its per-block activation sums (int4)
+  int off_xsum;            // its per-block activation sums (int4, int4aff)
+  int64_t zplane;          // int4aff: byte offset of the zero points in an aux row
+  int zoff;                // int4aff: byte offset of the slice's zero points in a staged aux row
   int prefetch;            // dense: weights may be read before the preceding grid completes
   int RS;                  // shared-memory bytes per staged code row
   int AS;                  // shared-memory bytes per staged scale row (kAuxRows)
@@ -82,15 +84,19 @@ struct MvParams {
 struct FmtInfo {
   int bits, scale_bytes, kc_max;
   bool lut;
+  bool zp;  // per-block zero points after the scales (int4aff)
 };
 inline FmtInfo fmt_info(int fmt) {
   switch (fmt) {
-    case QMV_FMT_FP4: return {4, 1, 2048, false};
-    case QMV_FMT_INT4: return {4, 2, 2048, false};
-    case QMV_FMT_INT4KM: return {4, 0, 2048, true};
-    default: return {8, 2, 1024, false};
+    case QMV_FMT_FP4: return {4, 1, 2048, false, false};
+    case QMV_FMT_INT4: return {4, 2, 2048, false, false};
+    case QMV_FMT_INT4KM: return {4, 0, 2048, true, false};
+    case QMV_FMT_INT4AFF: return {4, 2, 2048, false, true};
+    default: return {8, 2, 1024, false, false};
   }
 }
+// Bytes of one int4aff aux row: fp16 scales, then zero points two per byte.
+__host__ __device__ inline int64_t int4aff_aux_row_bytes(int64_t K) { return 2 * (K / 32) + (K / 32 + 1) / 2; }
 
 // Fills the geometry and the launch shape of `p` (shapes and pointers
 // already set) for a device with `num_sms` SMs.  Returns false when the
@@ -116,6 +122,8 @@ cudaError_t launch_encode_fp4(const float* W, int64_t N, int64_t K, uint8_t* cod
 cudaError_t launch_encode_int(int qmax, const float* W, int64_t N, int64_t K, const ClipList& clips,
                               uint8_t* codes, uint16_t* scales, uint32_t* status, int num_sms,
                               cudaStream_t stream);
+cudaError_t launch_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* aux,
+                                  uint32_t* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_encode_int4km(const float* W, int64_t N, int64_t K, int iters, uint16_t* lut, uint8_t* idx,
                                  uint32_t* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_dequant(int fmt, const uint8_t* codes, const uint8_t* aux, int64_t N, int64_t K, float* Wdq,

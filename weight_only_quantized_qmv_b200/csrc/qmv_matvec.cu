@@ -35,22 +35,29 @@ struct FmtT;
 template <>
 struct FmtT<QMV_FMT_FP4> {
   static constexpr int kBits = 4, kSB = 1;
-  static constexpr bool kLut = false, kPermX = false;
+  static constexpr bool kLut = false, kPermX = false, kZp = false;
 };
 template <>
 struct FmtT<QMV_FMT_INT4> {
   static constexpr int kBits = 4, kSB = 2;
-  static constexpr bool kLut = false, kPermX = true;  // decoder emits (k0,k4),(k1,k5),...
+  static constexpr bool kLut = false, kPermX = true, kZp = false;  // decoder emits (k0,k4),(k1,k5),...
 };
 template <>
 struct FmtT<QMV_FMT_INT4KM> {
   static constexpr int kBits = 4, kSB = 0;
-  static constexpr bool kLut = true, kPermX = false;
+  static constexpr bool kLut = true, kPermX = false, kZp = false;
 };
 template <>
 struct FmtT<QMV_FMT_INT8> {
   static constexpr int kBits = 8, kSB = 2;
-  static constexpr bool kLut = false, kPermX = false;
+  static constexpr bool kLut = false, kPermX = false, kZp = false;
+};
+// affine int4: the int4 decoder with the block's own zero point instead of 8;
+// a slice's zero points are staged after its scales, two per byte
+template <>
+struct FmtT<QMV_FMT_INT4AFF> {
+  static constexpr int kBits = 4, kSB = 2;
+  static constexpr bool kLut = false, kPermX = true, kZp = true;
 };
 
 // Column groups: the activation rows served by one pass over one expert's
@@ -86,6 +93,9 @@ __device__ __forceinline__ uint4 ldg_nc_128(const void* p) {
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
@@ -125,10 +135,12 @@ __device__ __forceinline__ float half_at(const uint4& v) {
   return (I % 2 == 0) ? __low2float(h) : __high2float(h);
 }
 
-// Decode one block's codes of rows g and g+8 into the two m16n8k16 A fragments.
+// Decode one block's codes of rows g and g+8 into the two m16n8k16 A fragments
+// (zg / zh: the block's zero points of rows g / g+8, affine int4 only).
 template <int FMT>
 __device__ __forceinline__ void decode_block(uint32_t crow_g, uint32_t crow_g8, int b, int t, const Palette& pg,
-                                             const Palette& pg8, const Mul& m, uint32_t (&a0)[4], uint32_t (&a1)[4]) {
+                                             const Palette& pg8, const Mul& m, uint32_t (&a0)[4], uint32_t (&a1)[4],
+                                             uint32_t zg = 0u, uint32_t zh = 0u) {
   uint32_t g0lo, g0hi, g1lo, g1hi, h0lo, h0hi, h1lo, h1hi;  // row g / g+8, step 0 / 1
   if constexpr (FmtT<FMT>::kBits == 8) {
     const uint2 vg = lds64(crow_g + 32u * b + 8u * t);
@@ -146,6 +158,9 @@ __device__ __forceinline__ void decode_block(uint32_t crow_g, uint32_t crow_g8, 
     } else if constexpr (FMT == QMV_FMT_INT4) {
       DecInt4::run(wg, g0lo, g0hi, g1lo, g1hi, m);
       DecInt4::run(wh, h0lo, h0hi, h1lo, h1hi, m);
+    } else if constexpr (FMT == QMV_FMT_INT4AFF) {
+      DecInt4::run_z(wg, g0lo, g0hi, g1lo, g1hi, int4_zp_sub(zg), int4_zp_neg(zg));
+      DecInt4::run_z(wh, h0lo, h0hi, h1lo, h1hi, int4_zp_sub(zh), int4_zp_neg(zh));
     } else {
       dec_int4km(pg, wg, g0lo, g0hi, g1lo, g1hi, m);
       dec_int4km(pg8, wh, h0lo, h0hi, h1lo, h1hi, m);
@@ -179,10 +194,10 @@ __device__ __forceinline__ void mac_block(float (&acc)[NT][4], const uint32_t (&
 
 // A warp's NB blocks of a full K-slice, unrolled: every shared-memory address
 // is a base plus an immediate, and the slice's scales of a row are read with
-// one or two 128-bit loads.
+// one or two 128-bit loads (zo: offset of the zero points from the scales).
 template <int FMT, int NT, int NB>
 __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g, uint32_t crow_g8, uint32_t sa_g,
-                                           uint32_t sa_g8, const uint32_t (&xb)[NT], int t,
+                                           uint32_t sa_g8, uint32_t zo, const uint32_t (&xb)[NT], int t,
                                            const Palette& pg, const Palette& pg8, const Mul& m) {
   using F = FmtT<FMT>;
   uint4 sg0 = make_uint4(0u, 0u, 0u, 0u), sh0 = sg0, sg1 = sg0, sh1 = sg0;
@@ -194,13 +209,29 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g,
       sh1 = lds128(sa_g8 + 16u);
     }
   }
+  uint2 zwg = make_uint2(0u, 0u), zwh = zwg;  // the slice's zero-point nibbles of rows g, g+8
+  if constexpr (F::kZp) {
+    static_assert(NB == 8 || NB == 16, "zero points come in 4- or 8-byte pieces");
+    if constexpr (NB == 16) {
+      zwg = lds64(sa_g + zo);
+      zwh = lds64(sa_g8 + zo);
+    } else {
+      zwg.x = lds32(sa_g + zo);
+      zwh.x = lds32(sa_g8 + zo);
+    }
+  }
 #pragma unroll
   for (int i = 0; i < NB; ++i) {
     uint4 xr[NT];
 #pragma unroll
     for (int n = 0; n < NT; ++n) xr[n] = lds128(xb[n] + 64u * (uint32_t)i);
     uint32_t a0[4], a1[4];
-    decode_block<FMT>(crow_g, crow_g8, i, t, pg, pg8, m, a0, a1);
+    uint32_t zg = 0u, zh = 0u;
+    if constexpr (F::kZp) {
+      zg = ((i < 8 ? zwg.x : zwg.y) >> (4 * (i & 7))) & 15u;
+      zh = ((i < 8 ? zwh.x : zwh.y) >> (4 * (i & 7))) & 15u;
+    }
+    decode_block<FMT>(crow_g, crow_g8, i, t, pg, pg8, m, a0, a1, zg, zh);
     float sg = 0.0f, sh = 0.0f;
     if constexpr (FMT == QMV_FMT_FP4) {
       const uint32_t q = (uint32_t)i >> 2;
@@ -244,15 +275,16 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g,
 // subnormal n * 2^-24 (n * 2^-20 for the upper nibble of a byte), so the
 // decode is one AND per two weights.  The two nibble positions accumulate
 // in separate MMA sums (dlo, dhi); per block, 2^20 * (16 * dlo + dhi) is the
-// exact sum of n * x, and the offset 8 is removed with the block's sum of
-// activations (xsum, exact in fp64, rounded once to fp32).
+// exact sum of n * x, and the offset (8, or the block's zero point z for
+// affine int4, staged zo bytes after the scales) is removed with the block's
+// sum of activations (xsum, exact in fp64, rounded once to fp32).
 template <int FMT, int NG>
 __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint32_t crow_g, uint32_t crow_g8,
-                                          uint32_t sa_g, uint32_t sa_g8, uint32_t xl0, uint32_t xl1, uint32_t xs_t,
-                                          int t, const Palette& pg, const Palette& pg8, const Mul& m) {
+                                          uint32_t sa_g, uint32_t sa_g8, uint32_t zo, uint32_t xl0, uint32_t xl1,
+                                          uint32_t xs_t, int t, const Palette& pg, const Palette& pg8, const Mul& m) {
   using F = FmtT<FMT>;
   constexpr int kBB = F::kBits * 4;  // code bytes per block and row
-  constexpr bool kSub = FMT == QMV_FMT_INT4;  // the subnormal int4 decode
+  constexpr bool kSub = FMT == QMV_FMT_INT4 || FMT == QMV_FMT_INT4AFF;  // the subnormal int4 decode
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi) {
     float d[4], dh[4];
@@ -334,13 +366,28 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
         s0 = __low2float(hu); s1 = __high2float(hu);
         s2 = __low2float(hv); s3 = __high2float(hv);
       }
-      if constexpr (kSub) {
+      if constexpr (FMT == QMV_FMT_INT4) {
         // block partial = 2^20 * (16 * dlo + dhi) - 8 * sum(x), one rounding each
         const float2 xs = *sptr<float2>(xs_t + (uint32_t)(4 * 8 * gi));  // blocks 2t, 2t+1 of the group
         d[0] = fmaf(fmaf(d[0], 16.0f, dh[0]), 1048576.0f, -8.0f * xs.x);
         d[1] = fmaf(fmaf(d[1], 16.0f, dh[1]), 1048576.0f, -8.0f * xs.y);
         d[2] = fmaf(fmaf(d[2], 16.0f, dh[2]), 1048576.0f, -8.0f * xs.x);
         d[3] = fmaf(fmaf(d[3], 16.0f, dh[3]), 1048576.0f, -8.0f * xs.y);
+      } else if constexpr (kSub) {
+        // block partial = 2^20 * (16 * dlo + dhi) - z * sum(x): the scaling by
+        // 2^20 is exact, so one rounding for the sum and one for the fma
+        const float2 xs = *sptr<float2>(xs_t + (uint32_t)(4 * 8 * gi));
+        const uint32_t zg = lds_u8(sa_g + zo + (uint32_t)(4 * gi + t));  // blocks 2t (low), 2t+1 (high)
+        const uint32_t zh = lds_u8(sa_g8 + zo + (uint32_t)(4 * gi + t));
+        // z as a float: 2^23 + z spliced into the mantissa, minus 2^23 (exact)
+        const float z0 = __uint_as_float(0x4B000000u | (zg & 15u)) - 8388608.0f;
+        const float z1 = __uint_as_float(0x4B000000u | (zg >> 4)) - 8388608.0f;
+        const float z2 = __uint_as_float(0x4B000000u | (zh & 15u)) - 8388608.0f;
+        const float z3 = __uint_as_float(0x4B000000u | (zh >> 4)) - 8388608.0f;
+        d[0] = fmaf(-z0, xs.x, fmaf(d[0], 16.0f, dh[0]) * 1048576.0f);
+        d[1] = fmaf(-z1, xs.y, fmaf(d[1], 16.0f, dh[1]) * 1048576.0f);
+        d[2] = fmaf(-z2, xs.x, fmaf(d[2], 16.0f, dh[2]) * 1048576.0f);
+        d[3] = fmaf(-z3, xs.y, fmaf(d[3], 16.0f, dh[3]) * 1048576.0f);
       }
       acc[0] = fmaf(d[0], s0, acc[0]);
       acc[0] = fmaf(d[1], s1, acc[0]);
@@ -530,6 +577,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   const int64_t rb2 = 2 * p.code_row_bytes;
   const uint8_t* crow_base = nullptr;  // the item's tile row 0 at the next slice, + 16 * cc
   const uint8_t* asrc = nullptr;  // row cr's scales at the next slice (+ 8 * ch) / its palette (+ 16 * ch)
+  const uint8_t* zsrc = nullptr;  // affine int4: row cr's zero points at the next slice (+ 4 * ch)
   int64_t irow0 = 0;
   int inrows = 0;
   auto load_issue_item = [&]() {
@@ -543,6 +591,8 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       asrc = p.aux + (int64_t)e * p.expert_aux_bytes + row * 32 + 16 * ch;
     else
       asrc = p.aux + (int64_t)e * p.expert_aux_bytes + row * p.aux_row_bytes + (int64_t)(iI.kbeg / 32) * F::kSB + 8 * ch;
+    if constexpr (F::kZp)
+      zsrc = p.aux + (int64_t)e * p.expert_aux_bytes + row * p.aux_row_bytes + p.zplane + iI.kbeg / 64 + 4 * ch;
   };
   if (n_issue > 0) load_issue_item();
   auto issue_next = [&](uint32_t stage) {
@@ -579,6 +629,11 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       for (int j = 0; j < kAuxSteps; ++j)
         if (16 * j + 8 * ch < sb) cp_async8(da + (uint32_t)cr * p.AS + 16u * j + 8u * ch, asrc + 16 * j);
       asrc += sb;
+      if constexpr (F::kZp) {
+        const int zb = kc / 64;  // zero-point bytes per row, a multiple of 4
+        if (4 * ch < zb) cp_async4(da + (uint32_t)cr * p.AS + (uint32_t)p.zoff + 4u * ch, zsrc);
+        zsrc += zb;
+      }
     } else {
       // scale rows that are not 8-byte granular: plain byte loads
       const int sbytes = (kc / 32) * F::kSB;
@@ -588,6 +643,17 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
         const int row = i / sbytes, b = i - row * sbytes;
         const int r = min(row, inrows - 1);
         sts_u8(da + (uint32_t)row * p.AS + (uint32_t)b, ldg_u8(abase + (int64_t)r * p.aux_row_bytes + b));
+      }
+      if constexpr (F::kZp) {
+        // slices start on even blocks: the slice's zero points are whole bytes
+        const int zbytes = (kc / 32 + 1) / 2;
+        const uint8_t* zbase = p.aux + (int64_t)e * p.expert_aux_bytes + irow0 * p.aux_row_bytes + p.zplane + k0 / 64;
+        for (int i = lane; i < kTileRows * zbytes; i += 32) {
+          const int row = i / zbytes, b = i - row * zbytes;
+          const int r = min(row, inrows - 1);
+          sts_u8(da + (uint32_t)row * p.AS + (uint32_t)p.zoff + (uint32_t)b,
+                 ldg_u8(zbase + (int64_t)r * p.aux_row_bytes + b));
+        }
       }
     }
     if (++ic == iI.nsl) {
@@ -624,7 +690,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       }
       sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
     }
-    if constexpr (kOne && FMT == QMV_FMT_INT4) {
+    if constexpr (kOne && (FMT == QMV_FMT_INT4 || FMT == QMV_FMT_INT4AFF)) {
       // per-block activation sums: exact in fp64 (32 fp16 terms), one rounding to fp32
       for (int64_t b = tid; b < p.K / 32; b += kT) {
         double sum = 0.0;
@@ -734,6 +800,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       const uint32_t crow_g = cons + (uint32_t)g * p.RS, crow_g8 = cons + (uint32_t)(g + 8) * p.RS;
       const uint32_t sa_g = auxs + (uint32_t)g * p.AS, sa_g8 = auxs + (uint32_t)(g + 8) * p.AS;
       constexpr int kNB = kSliceBytes * 8 / F::kBits / 32;  // blocks in a full slice
+      const uint32_t zo = (uint32_t)p.zoff;
       if constexpr (kOne) {
         // slices are whole groups of 8 blocks (the host requires K % 256 == 0)
         const uint32_t xs = xbase + (uint32_t)k0 * 2u, zb = sbase + p.off_zero;
@@ -742,10 +809,10 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
         const uint32_t tb = (uint32_t)(t * F::kBits * 4);
         const uint32_t xs_t = sbase + p.off_xsum + 4u * (uint32_t)(k0 / 32 + 2 * t);  // block sums of this lane
         if (kNB >= 16 && kc == kNB * 32)
-          slice_one<FMT, (kNB >= 16 ? kNB / 8 : 1)>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, xl0, xl1, xs_t, t,
-                                                    pg, pg8, mul);
+          slice_one<FMT, (kNB >= 16 ? kNB / 8 : 1)>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, zo, xl0, xl1,
+                                                    xs_t, t, pg, pg8, mul);
         else
-          slice_one<FMT, 1>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, xl0, xl1, xs_t, t, pg, pg8, mul);
+          slice_one<FMT, 1>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, zo, xl0, xl1, xs_t, t, pg, pg8, mul);
         __syncwarp();
         cons = (cons + p.stage_bytes == ring_end) ? ring : cons + p.stage_bytes;
         continue;
@@ -754,9 +821,9 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
 #pragma unroll
       for (int n = 0; n < NTX; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
       if (kc == kNB * 32 && aux_fast) {
-        slice_full<FMT, NTX, kNB>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
+        slice_full<FMT, NTX, kNB>(acc, crow_g, crow_g8, sa_g, sa_g8, zo, xb, t, pg, pg8, mul);
       } else if (kc == kNB * 16 && aux_fast) {
-        slice_full<FMT, NTX, kNB / 2>(acc, crow_g, crow_g8, sa_g, sa_g8, xb, t, pg, pg8, mul);
+        slice_full<FMT, NTX, kNB / 2>(acc, crow_g, crow_g8, sa_g, sa_g8, zo, xb, t, pg, pg8, mul);
       } else {
         const int nbc = kc / 32;
         for (int b = 0; b < nbc; ++b) {
@@ -764,7 +831,12 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
 #pragma unroll
           for (int n = 0; n < NTX; ++n) xr[n] = lds128(xb[n] + 64u * (uint32_t)b);
           uint32_t a0[4], a1[4];
-          decode_block<FMT>(crow_g, crow_g8, b, t, pg, pg8, mul, a0, a1);
+          uint32_t zg = 0u, zh = 0u;
+          if constexpr (F::kZp) {
+            zg = (lds_u8(sa_g + zo + (uint32_t)(b >> 1)) >> (4 * (b & 1))) & 15u;
+            zh = (lds_u8(sa_g8 + zo + (uint32_t)(b >> 1)) >> (4 * (b & 1))) & 15u;
+          }
+          decode_block<FMT>(crow_g, crow_g8, b, t, pg, pg8, mul, a0, a1, zg, zh);
           float sg = 0.0f, sh = 0.0f;
           if constexpr (!F::kLut) {
             sg = stage_scale<FMT>(sa_g + (uint32_t)b * F::kSB, mul);
@@ -905,7 +977,8 @@ static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   const FmtInfo fi = fmt_info(fmt);
   p.code_row_bytes = p.K * fi.bits / 8;
-  p.aux_row_bytes = fi.lut ? 32 : (p.K / 32) * fi.scale_bytes;
+  p.aux_row_bytes = fi.lut ? 32 : fi.zp ? int4aff_aux_row_bytes(p.K) : (p.K / 32) * fi.scale_bytes;
+  p.zplane = fi.zp ? 2 * (p.K / 32) : 0;
   p.expert_code_bytes = p.N * p.code_row_bytes;
   p.expert_aux_bytes = p.N * p.aux_row_bytes;
   p.tiles = (p.N + kTileRows - 1) / kTileRows;
@@ -928,7 +1001,9 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   int64_t aux_region;
   // split units divide K in granules whose code and scale segments start on
   // 16- and 8-byte boundaries
-  p.gk = p.one ? 256 : (fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128));
+  // (affine int4: 256, so a granule's zero points start on a 4-byte boundary)
+  p.gk = (p.one || fi.zp) ? 256 : (fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128));
+  p.zoff = 0;
   if (fi.lut) {
     p.aux_mode = kAuxLut;
     p.AS = 32;
@@ -936,11 +1011,16 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   } else {
     const int64_t slice_sc = (int64_t)(p.KC / 32) * fi.scale_bytes;
     // asynchronous 8-byte scale copies when every row's scales start on an
-    // 8-byte boundary and come in whole 8-byte pieces
+    // 8-byte boundary and come in whole 8-byte pieces (affine int4: and the
+    // zero points of every slice in whole 4-byte pieces)
     const bool based = (reinterpret_cast<uintptr_t>(p.aux) % 8) == 0;
-    p.aux_mode = (based && p.aux_row_bytes % 8 == 0) ? kAuxRows : kAuxBlock;
+    const bool zp_ok = !fi.zp || (p.zplane % 4 == 0 && p.K % 256 == 0);
+    p.aux_mode = (based && p.aux_row_bytes % 8 == 0 && zp_ok) ? kAuxRows : kAuxBlock;
     if (p.aux_mode == kAuxBlock) p.one = 0;
-    int64_t j = (slice_sc + 15) / 16;
+    // a staged row: the slice's scales, then (affine int4) its zero points
+    p.zoff = fi.zp ? (int)round_up(slice_sc, 8) : 0;
+    const int64_t row_bytes = fi.zp ? p.zoff + (p.KC / 32 + 1) / 2 : slice_sc;
+    int64_t j = (row_bytes + 15) / 16;
     // the batch-1 form reads 4 bytes of rows g = 0..7 per load: an odd
     // multiple of 16 bytes puts them in distinct banks (elsewhere the scale
     // loads are a few per slice and the tighter rows let more warps fit)
@@ -976,7 +1056,8 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
     // activation reads of the same instruction fall in different banks
     p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
     p.off_xsum = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
-    p.off_stage = (int)round_up(p.off_xsum + ((p.one && fmt == QMV_FMT_INT4) ? 4 * (p.K / 32) : 0), 128);
+    const bool xsum = p.one && (fmt == QMV_FMT_INT4 || fmt == QMV_FMT_INT4AFF);
+    p.off_stage = (int)round_up(p.off_xsum + (xsum ? 4 * (p.K / 32) : 0), 128);
     for (int st = kStages; st >= 2; --st) {
       const int64_t bytes = p.off_stage + (int64_t)warps * st * p.stage_bytes;
       if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
@@ -1036,6 +1117,7 @@ cudaError_t launch_matvec(int fmt, const MvParams& p, cudaStream_t stream) {
     case QMV_FMT_INT4: return launch_f<QMV_FMT_INT4>(p, stream);
     case QMV_FMT_INT4KM: return launch_f<QMV_FMT_INT4KM>(p, stream);
     case QMV_FMT_INT8: return launch_f<QMV_FMT_INT8>(p, stream);
+    case QMV_FMT_INT4AFF: return launch_f<QMV_FMT_INT4AFF>(p, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -16,7 +16,8 @@ import numpy as np
 
 from . import build as _build
 
-FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8, FMT_INT4AFF = 0, 1, 2, 3, 4
+FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8, FMT_INT4AFF, FMT_INT8KM = 0, 1, 2, 3, 4, 5
+KM8_GROUP = 32  # int8km: output rows sharing one 256-entry LUT
 FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT = 1, 2, 4
 
 # Clip lists: the int4 list of the int4 lm_head workload (1.00 down to 0.50
@@ -50,12 +51,16 @@ def lib():
         L.oracle_encode_int4aff.argtypes = [P, I64, I64, P, P, U32P]
         L.oracle_int4aff_aux_row_bytes.argtypes = [I64]
         L.oracle_int4aff_aux_row_bytes.restype = I64
+        L.oracle_kmeans_int8km.argtypes = [P, I64, I64, I32, P, P, P, U32P]
+        L.oracle_int8km_groups.argtypes = [I64]
+        L.oracle_int8km_groups.restype = I64
         L.oracle_dequant.argtypes = [I32, P, P, I64, I64, P]
         L.oracle_matvec_rows.argtypes = [I32, P, P, P, I32, I64, I64, P, I64, P]
         L.oracle_gather_matvec.argtypes = [I32, P, P, I32, I64, I64, P, I32, I32, P, I32, P, U32P]
         L.oracle_num_threads.restype = I32
         L.oracle_set_num_threads.argtypes = [I32]
         for f in ("oracle_encode_fp4", "oracle_encode_int_sym", "oracle_kmeans_int4km", "oracle_encode_int4aff",
+                  "oracle_kmeans_int8km",
                   "oracle_dequant",
                   "oracle_matvec_rows", "oracle_gather_matvec"):
             getattr(L, f).restype = I32
@@ -159,6 +164,24 @@ def kmeans_int4km(W, iters=KMEANS_ITERS, want_sse=False):
     fl = ctypes.c_uint32(0)
     _check(lib().oracle_kmeans_int4km(_p(W), N, K, iters, _p(lut), _p(idx),
                                       _p(sse) if want_sse else None, ctypes.byref(fl)), "kmeans")
+    return (lut, idx, fl.value, sse) if want_sse else (lut, idx, fl.value)
+
+
+def int8km_groups(N):
+    return int(lib().oracle_int8km_groups(int(N)))
+
+
+def kmeans_int8km(W, iters=KMEANS_ITERS, want_sse=False):
+    """-> (lut float16 [ceil(N/32), 256], idx uint8 [N, K], flags[, sse double [ceil(N/32), iters+1]])."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    G = int8km_groups(N)
+    lut = np.zeros((G, 256), np.float16)
+    idx = np.zeros((N, K), np.uint8)
+    sse = np.zeros((G, iters + 1), np.float64) if want_sse else None
+    fl = ctypes.c_uint32(0)
+    _check(lib().oracle_kmeans_int8km(_p(W), N, K, iters, _p(lut), _p(idx),
+                                      _p(sse) if want_sse else None, ctypes.byref(fl)), "kmeans8")
     return (lut, idx, fl.value, sse) if want_sse else (lut, idx, fl.value)
 
 

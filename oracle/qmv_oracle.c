@@ -19,8 +19,9 @@
  *        palettization", sections "Quantization" (symmetric, per-block 32),
  *        "Palettization" (scalar 1-D k-means, 2^n_bits LUT, per-channel
  *        grouping) and "Theoretical size" (fp16 scales, LUT bytes).
- *   [P5] "Compression (palettization & quantization)", section "Per-channel
- *        int8 on a big-vocab LM head: use per-block-32".
+ *   [P5] "Compression (palettization & quantization)", sections "Per-channel
+ *        int8 on a big-vocab LM head: use per-block-32" and "int8 k-means >
+ *        whole-model int4" (the recommended recipe: 8-bit k-means, group 32).
  *
  * Where the pages leave a step open, the reading taken is stated at the
  * function.  Every floating-point step is written so that its rounding is
@@ -28,10 +29,11 @@
  * no contraction: build with -ffp-contract=off, never -ffast-math).
  *
  * Parity status: every function here is pinned by tests under
- * tests/test_oracle_pins.py except oracle_kmeans_int4km's LUT *values*,
- * which no page fixes (see its comment): "parity unpinned" for those values;
- * its invariants (exact reconstruction of <=16 distinct values, monotone
- * SSE, nearest-entry indices) are pinned.
+ * tests/test_oracle_pins.py except the k-means LUT *values* (int4km and
+ * int8km), which no page fixes (see orc_kmeans_fit): "parity unpinned" for
+ * those values; their invariants (exact reconstruction of <= 16 / 256
+ * distinct values, monotone SSE, nearest-entry indices, group boundaries)
+ * are pinned.
  */
 #include <math.h>
 #include <stdint.h>
@@ -47,6 +49,8 @@
 #define ORC_FMT_INT4KM 2
 #define ORC_FMT_INT8 3
 #define ORC_FMT_INT4AFF 4
+#define ORC_FMT_INT8KM 5
+#define ORC_KM8_GROUP 32 /* int8km: output rows sharing one 256-entry LUT */
 
 /* ------------------------------------------------------------------ */
 /* IEEE binary16 <-> binary32, written from the format definition.     */
@@ -286,9 +290,12 @@ int oracle_encode_int_sym(const float* W, int64_t N, int64_t K, int qmax,
 }
 
 /* ------------------------------------------------------------------ */
-/* int4km: per-row 16-entry LUT by scalar 1-D k-means                 */
-/* [P3 "Palettization": scalar k-means, 2^n_bits centroids, per-channel */
-/*  grouping; P2 sec.8: per-output-row 16-entry codebook]             */
+/* Palettization: scalar 1-D k-means LUTs                             */
+/* [P3 "Palettization": scalar k-means, 2^n_bits centroids, per-tensor */
+/*  or per-grouped-channel granularity (group_size output channels     */
+/*  share one LUT); P2 sec.8: per-output-row 16-entry codebook (int4km);*/
+/*  P5 "int8 k-means > whole-model int4" / P1 sec.1: int8km, 8-bit    */
+/*  k-means with group 32]                                             */
 /* ------------------------------------------------------------------ */
 
 /* Ascending, -0 before +0: a total order on finite floats, so the sorted
@@ -299,12 +306,12 @@ static int orc_cmp_float(const void* a, const void* b) {
   return (int)(signbit(y) != 0) - (int)(signbit(x) != 0);
 }
 
-/* Nearest of the 16 centres to v, distance |v - c| in double, ties to the
+/* Nearest of the nc centres to v, distance |v - c| in double, ties to the
  * lower index. */
-static int orc_nearest16(const double* c, double v) {
+static int orc_nearest(const double* c, int nc, double v) {
   int best = 0;
   double bd = fabs(v - c[0]);
-  for (int k = 1; k < 16; k++) {
+  for (int k = 1; k < nc; k++) {
     double d = fabs(v - c[k]);
     if (d < bd) {
       bd = d;
@@ -314,20 +321,62 @@ static int orc_nearest16(const double* c, double v) {
   return best;
 }
 
-/* Per row (n = K weights), readings where no page fixes the details:
- *  1. sort the row ascending (-0 before +0);
- *  2. centre k starts at sorted[floor((2k+1) n / 32)], the (k+1/2)/16
+/* The fit of one group of n finite weights into nc centres, readings where
+ * no page fixes the details:
+ *  1. sort the values ascending (-0 before +0);
+ *  2. centre k starts at sorted[floor((2k+1) n / (2 nc))], the (k+1/2)/nc
  *     quantile without interpolation;
- *  3. `iters` Lloyd steps: assign each weight to the nearest centre (double
+ *  3. `iters` Lloyd steps: assign each value to the nearest centre (double
  *     distance, ties to the lower index); each non-empty centre becomes
  *     float(double sum of its members, added in ascending value order /
- *     count); an empty centre keeps its value;
- *  4. LUT = fp16_RNE(centres);
- *  5. indices = nearest LUT entry (double distance, ties to lower index).
+ *     count); an empty centre keeps its value.
+ * s: the n values (sorted in place); c: the nc centres (out);
+ * sse (optional, [iters+1]): the SSE against the centres before each step
+ * and after the last. */
+static void orc_kmeans_fit(float* s, int64_t n, int nc, int iters, double* c, double* sse_out) {
+  qsort(s, (size_t)n, sizeof(float), orc_cmp_float);
+  for (int k = 0; k < nc; k++) c[k] = (double)s[((2 * k + 1) * n) / (2 * nc)];
+  double* sum = (double*)malloc((size_t)nc * sizeof(double));
+  int64_t* cnt = (int64_t*)malloc((size_t)nc * sizeof(int64_t));
+  for (int it = 0; it <= iters; it++) {
+    double sse = 0.0;
+    for (int k = 0; k < nc; k++) {
+      sum[k] = 0.0;
+      cnt[k] = 0;
+    }
+    for (int64_t i = 0; i < n; i++) {
+      double v = (double)s[i];
+      int j = orc_nearest(c, nc, v);
+      double d = v - c[j];
+      sse += d * d;
+      sum[j] += v;
+      cnt[j]++;
+    }
+    if (sse_out) sse_out[it] = sse;
+    if (it == iters) break;
+    for (int k = 0; k < nc; k++)
+      if (cnt[k] > 0) c[k] = (double)(float)(sum[k] / (double)cnt[k]);
+  }
+  free(sum);
+  free(cnt);
+}
+
+/* LUT = fp16_RNE(centres): writes the bits and returns the entries' values
+ * in cl. */
+static void orc_lut_from_centres(const double* c, int nc, uint16_t* lut, double* cl) {
+  for (int k = 0; k < nc; k++) {
+    uint16_t h = orc_f32_to_f16((float)c[k]);
+    lut[k] = h;
+    cl[k] = (double)orc_f16_to_f32(h);
+  }
+}
+
+/* int4km, one group per output row (n = K weights, 16 centres): the fit
+ * above, LUT = fp16_RNE(centres), indices = nearest LUT entry (double
+ * distance, ties to the lower index).
  * idx: uint8 [N, K/2] (element 2j low nibble); lut: fp16 bits [N, 16].
  * A row holding Inf/NaN is written as zeros and raises a flag.
- * sse_trace (optional, [N, iters+1]): the SSE against the centres before
- * each step and after the last, for the monotonicity pin. */
+ * sse_trace (optional, [N, iters+1]) for the monotonicity pin. */
 int oracle_kmeans_int4km(const float* W, int64_t N, int64_t K, int iters,
                          uint16_t* lut, uint8_t* idx, double* sse_trace,
                          uint32_t* flags_out) {
@@ -349,38 +398,62 @@ int oracle_kmeans_int4km(const float* W, int64_t N, int64_t K, int iters,
     }
     float* s = (float*)malloc((size_t)K * sizeof(float));
     memcpy(s, w, (size_t)K * sizeof(float));
-    qsort(s, (size_t)K, sizeof(float), orc_cmp_float);
-    double c[16];
-    for (int k = 0; k < 16; k++) c[k] = (double)s[((2 * k + 1) * K) / 32];
-    for (int it = 0; it <= iters; it++) {
-      double sum[16] = {0}, sse = 0.0;
-      int64_t cnt[16] = {0};
-      for (int64_t i = 0; i < K; i++) {
-        double v = (double)s[i];
-        int j = orc_nearest16(c, v);
-        double d = v - c[j];
-        sse += d * d;
-        sum[j] += v;
-        cnt[j]++;
-      }
-      if (sse_trace) sse_trace[n * (iters + 1) + it] = sse;
-      if (it == iters) break;
-      for (int k = 0; k < 16; k++)
-        if (cnt[k] > 0) c[k] = (double)(float)(sum[k] / (double)cnt[k]);
-    }
+    double c[16], cl[16];
+    orc_kmeans_fit(s, K, 16, iters, c, sse_trace ? sse_trace + n * (iters + 1) : NULL);
     free(s);
-    double cl[16];
-    for (int k = 0; k < 16; k++) {
-      uint16_t h = orc_f32_to_f16((float)c[k]);
-      lut[n * 16 + k] = h;
-      cl[k] = (double)orc_f16_to_f32(h);
-    }
+    orc_lut_from_centres(c, 16, lut + n * 16, cl);
     uint8_t* ib = idx + n * (K / 2);
     for (int64_t i = 0; i < K; i += 2) {
-      int a = orc_nearest16(cl, (double)w[i]);
-      int b = orc_nearest16(cl, (double)w[i + 1]);
+      int a = orc_nearest(cl, 16, (double)w[i]);
+      int b = orc_nearest(cl, 16, (double)w[i + 1]);
       ib[i / 2] = (uint8_t)(a | (b << 4));
     }
+  }
+  if (flags_out) *flags_out = flags;
+  return 0;
+}
+
+/* Number of int8km LUT groups of N rows: ceil(N / 32).  A last group of
+ * fewer rows (N % 32 != 0) is fitted on the rows it has, so no row is left
+ * uncompressed. */
+int64_t oracle_int8km_groups(int64_t N) { return (N + ORC_KM8_GROUP - 1) / ORC_KM8_GROUP; }
+
+/* int8km: per group of 32 consecutive output rows (n = rows * K weights),
+ * the same fit with 256 centres; LUT = fp16_RNE(centres); each weight's
+ * index = nearest LUT entry (double distance, ties to the lower index).
+ * idx: uint8 [N, K]; lut: fp16 bits [ceil(N/32), 256].  A group holding
+ * Inf/NaN is written as zeros and raises a flag.
+ * sse_trace (optional, [ceil(N/32), iters+1]). */
+int oracle_kmeans_int8km(const float* W, int64_t N, int64_t K, int iters,
+                         uint16_t* lut, uint8_t* idx, double* sse_trace,
+                         uint32_t* flags_out) {
+  if (K % 32 != 0 || N < 0 || iters < 0) return -2;
+  uint32_t flags = 0;
+  int64_t G = oracle_int8km_groups(N);
+#pragma omp parallel for reduction(| : flags) schedule(dynamic, 1)
+  for (int64_t g = 0; g < G; g++) {
+    int64_t r0 = g * ORC_KM8_GROUP;
+    int64_t rows = N - r0 < ORC_KM8_GROUP ? N - r0 : ORC_KM8_GROUP;
+    int64_t n = rows * K;
+    const float* w = W + r0 * K;
+    int finite = 1;
+    for (int64_t i = 0; i < n; i++)
+      if (!isfinite(w[i])) finite = 0;
+    if (!finite) {
+      flags |= ORC_FLAG_NONFINITE;
+      memset(lut + g * 256, 0, 512);
+      memset(idx + r0 * K, 0, (size_t)n);
+      if (sse_trace)
+        for (int t = 0; t <= iters; t++) sse_trace[g * (iters + 1) + t] = NAN;
+      continue;
+    }
+    float* s = (float*)malloc((size_t)n * sizeof(float));
+    memcpy(s, w, (size_t)n * sizeof(float));
+    double c[256], cl[256];
+    orc_kmeans_fit(s, n, 256, iters, c, sse_trace ? sse_trace + g * (iters + 1) : NULL);
+    free(s);
+    orc_lut_from_centres(c, 256, lut + g * 256, cl);
+    for (int64_t i = 0; i < n; i++) idx[r0 * K + i] = (uint8_t)orc_nearest(cl, 256, (double)w[i]);
   }
   if (flags_out) *flags_out = flags;
   return 0;
@@ -412,8 +485,7 @@ int oracle_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes,
   int64_t nb = K / 32, arow = oracle_int4aff_aux_row_bytes(K);
 #pragma omp parallel for reduction(| : flags) schedule(static)
   for (int64_t n = 0; n < N; n++) {
-    uint8_t* ar = aux + n * arow;
-    uint16_t* sc = (uint16_t*)ar;
+    uint8_t* ar = aux + n * arow; /* rows may have an odd byte count: byte access */
     uint8_t* zp = ar + 2 * nb;
     memset(zp, 0, (size_t)((nb + 1) / 2));
     for (int64_t b = 0; b < nb; b++) {
@@ -451,7 +523,8 @@ int oracle_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes,
           }
         }
       }
-      sc[b] = sh;
+      ar[2 * b] = (uint8_t)(sh & 0xFF);
+      ar[2 * b + 1] = (uint8_t)(sh >> 8);
       zp[b / 2] |= (uint8_t)(z << ((b % 2) * 4));
       uint8_t* cb = codes + n * (K / 2) + b * 16;
       for (int i = 0; i < 32; i += 2) cb[i / 2] = (uint8_t)(q[i] | (q[i + 1] << 4));
@@ -462,13 +535,14 @@ int oracle_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes,
 }
 
 /* ------------------------------------------------------------------ */
-/* Dequantization (exact in float) and the fp64 matvec                *//* ------------------------------------------------------------------ */
+/* ------------------------------------------------------------------ */
 /* Dequantization (exact in float) and the fp64 matvec                */
 /* ------------------------------------------------------------------ */
 
 /* Dequantized weight (row n, column k) of one format.  aux is the scale
- * plane (fp4: uint8 [N,K/32]; int4/int8: fp16 bits [N,K/32]) or the LUT
- * (int4km: fp16 bits [N,16]). */
+ * plane (fp4: uint8 [N,K/32]; int4/int8: fp16 bits [N,K/32]), the LUT
+ * (int4km: fp16 bits [N,16]; int8km: fp16 bits [ceil(N/32),256]) or the
+ * int4aff rows (fp16 scales then zero points). */
 static float orc_wdq(int fmt, const void* codes, const void* aux, int64_t K,
                      int64_t n, int64_t k) {
   int64_t nb = K / 32;
@@ -499,10 +573,14 @@ static float orc_wdq(int fmt, const void* codes, const void* aux, int64_t K,
       int q = (k % 2) ? (byte >> 4) : (byte & 15);
       const uint8_t* ar = (const uint8_t*)aux + n * oracle_int4aff_aux_row_bytes(K);
       int64_t b = k / 32;
-      float s = orc_f16_to_f32(((const uint16_t*)ar)[b]);
+      float s = orc_f16_to_f32((uint16_t)(ar[2 * b] | (ar[2 * b + 1] << 8)));
       uint8_t zb = ar[2 * nb + b / 2];
       int z = (b % 2) ? (zb >> 4) : (zb & 15);
       return (float)(q - z) * s;
+    }
+    case ORC_FMT_INT8KM: {
+      uint8_t j = ((const uint8_t*)codes)[n * K + k];
+      return orc_f16_to_f32(((const uint16_t*)aux)[(n / ORC_KM8_GROUP) * 256 + j]);
     }
   }
   return NAN;
@@ -510,7 +588,7 @@ static float orc_wdq(int fmt, const void* codes, const void* aux, int64_t K,
 
 int oracle_dequant(int fmt, const void* codes, const void* aux, int64_t N,
                    int64_t K, float* Wdq) {
-  if (K % 32 != 0 || N < 0 || fmt < 0 || fmt > 4) return -2;
+  if (K % 32 != 0 || N < 0 || fmt < 0 || fmt > 5) return -2;
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; n++)
     for (int64_t k = 0; k < K; k++) Wdq[n * K + k] = orc_wdq(fmt, codes, aux, K, n, k);
@@ -524,7 +602,7 @@ int oracle_dequant(int fmt, const void* codes, const void* aux, int64_t N,
 int oracle_matvec_rows(int fmt, const void* codes, const void* aux,
                        const uint16_t* x, int B, int64_t N, int64_t K,
                        const int64_t* rows, int64_t nrows, double* r) {
-  if (K % 32 != 0 || N < 0 || B < 1 || fmt < 0 || fmt > 4) return -2;
+  if (K % 32 != 0 || N < 0 || B < 1 || fmt < 0 || fmt > 5) return -2;
   int64_t R = rows ? nrows : N;
   double* xd = (double*)malloc((size_t)(B * K) * sizeof(double));
   for (int64_t i = 0; i < (int64_t)B * K; i++) xd[i] = (double)orc_f16_to_f32(x[i]);
@@ -556,10 +634,11 @@ int oracle_gather_matvec(int fmt, const void* codes, const void* aux, int E,
                          int64_t N, int64_t K, const int32_t* ids, int B,
                          int topk, const uint16_t* x, int x_per_slot,
                          double* y, uint32_t* flags_out) {
-  if (K % 32 != 0 || N < 0 || B < 1 || topk < 1 || fmt < 0 || fmt > 4) return -2;
-  int64_t code_bytes = (fmt == ORC_FMT_INT8) ? N * K : N * (K / 2);
+  if (K % 32 != 0 || N < 0 || B < 1 || topk < 1 || fmt < 0 || fmt > 5) return -2;
+  int64_t code_bytes = (fmt == ORC_FMT_INT8 || fmt == ORC_FMT_INT8KM) ? N * K : N * (K / 2);
   int64_t aux_bytes = (fmt == ORC_FMT_FP4) ? N * (K / 32)
                       : (fmt == ORC_FMT_INT4KM) ? N * 16 * 2
+                      : (fmt == ORC_FMT_INT8KM) ? oracle_int8km_groups(N) * 256 * 2
                       : (fmt == ORC_FMT_INT4AFF) ? N * oracle_int4aff_aux_row_bytes(K)
                                                  : N * (K / 32) * 2;
   uint32_t flags = 0;

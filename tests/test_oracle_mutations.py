@@ -30,6 +30,12 @@ MUTANTS = {
     "int4aff range without zero": ("float lo = 0.0f, hi = 0.0f;", "float lo = w[0], hi = w[0];"),
     "int4aff zero-point nibble order": ("zp[b / 2] |= (uint8_t)(z << ((b % 2) * 4));",
                                         "zp[b / 2] |= (uint8_t)(z << ((1 - b % 2) * 4));"),
+    "k-means start at the lower quantile edge": ("c[k] = (double)s[((2 * k + 1) * n) / (2 * nc)];",
+                                                 "c[k] = (double)s[(k * n) / nc];"),
+    "int8km indices against unrounded centres": ("(uint8_t)orc_nearest(cl, 256, (double)w[i]);",
+                                                 "(uint8_t)orc_nearest(c, 256, (double)w[i]);"),
+    "int8km last partial group dropped": ("return (N + ORC_KM8_GROUP - 1) / ORC_KM8_GROUP;",
+                                          "return N / ORC_KM8_GROUP;"),
 }
 
 

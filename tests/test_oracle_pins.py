@@ -503,6 +503,113 @@ def test_kmeans_quantile_start(orc):
 
 
 # --------------------------------------------------------------------------
+# int8km: 256-entry LUT per group of 32 output rows
+# --------------------------------------------------------------------------
+
+def _km8_nearest(W, lut):
+    """Brute-force nearest LUT entry of every weight (lowest index on ties),
+    the LUT of row n being lut[n // 32]."""
+    N, K = W.shape
+    L = lut.astype(np.float64)[np.arange(N) // 32]  # [N, 256]
+    d = np.abs(W.astype(np.float64)[:, :, None] - L[:, None, :])
+    return np.argmin(d, axis=2)
+
+
+def test_int8km_quantile_start_and_groups(orc):
+    """iters = 0: each group's LUT is fp16 of its sorted values at the
+    (k + 1/2)/256 quantiles; N = 70 makes groups of 32, 32 and a last one of 6
+    rows; indices are the nearest entry of the row's own group."""
+    N, K = 70, 96
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[32:64] *= 10.0  # a group on another scale: a mix-up of groups shows
+    lut, idx, flags = orc.kmeans_int8km(W, iters=0)
+    assert flags == 0 and lut.shape == (3, 256) and idx.shape == (N, K)
+    for g, (r0, r1) in enumerate([(0, 32), (32, 64), (64, 70)]):
+        s = np.sort(W[r0:r1].reshape(-1))
+        n = s.size
+        want = s[[((2 * k + 1) * n) // 512 for k in range(256)]].astype(np.float16)
+        assert np.array_equal(lut[g], want), g
+    assert np.array_equal(idx.astype(np.int64), _km8_nearest(W, lut))
+
+
+def test_int8km_exact_on_few_distinct_values(orc):
+    """A group of <= 256 fp16-representable values, each at least n/256 times,
+    is a fixed point of Lloyd from the quantile start: exact reconstruction."""
+    N, K = 64, 256
+    W = np.zeros((N, K), np.float32)
+    for g in range(2):
+        nd = int(RNG.integers(100, 257))
+        vals = np.unique(np.float16(RNG.standard_normal(nd) * 0.05)).astype(np.float32)
+        nd = len(vals)
+        n = 32 * K
+        counts = np.full(nd, n // 256)
+        counts += np.bincount(RNG.integers(0, nd, n - counts.sum()), minlength=nd)
+        W[32 * g:32 * g + 32] = RNG.permutation(np.repeat(vals, counts)).reshape(32, K)
+    lut, idx, flags = orc.kmeans_int8km(W)
+    assert flags == 0
+    D = orc.dequant(orc.FMT_INT8KM, idx, lut, N, K)
+    assert np.array_equal(D, W)
+    assert np.array_equal(idx.astype(np.int64), _km8_nearest(W, lut))
+
+
+def test_int8km_sse_monotone_nearest_and_independent_groups(orc):
+    N, K = 40, 128
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[:, 5] *= 20
+    lut, idx, flags, sse = orc.kmeans_int8km(W, want_sse=True)
+    assert flags == 0 and sse.shape == (2, 21)
+    assert np.all(np.diff(sse, axis=1) <= 1e-18)
+    assert np.array_equal(idx.astype(np.int64), _km8_nearest(W, lut))
+    assert np.all(np.diff(lut.astype(np.float64), axis=1) >= 0)
+    # a change in the second group leaves the first group's fit untouched
+    W2 = W.copy()
+    W2[35:] = (RNG.standard_normal((5, K)) * 0.5).astype(np.float32)
+    lut2, idx2, _ = orc.kmeans_int8km(W2)
+    assert np.array_equal(lut2[0], lut[0]) and np.array_equal(idx2[:32], idx[:32])
+    assert not np.array_equal(lut2[1], lut[1])
+
+
+def test_int8km_nonfinite_group(orc):
+    W = (RNG.standard_normal((64, 64)) * 0.02).astype(np.float32)
+    W[40, 7] = np.inf
+    lut, idx, flags = orc.kmeans_int8km(W)
+    assert flags & orc.FLAG_NONFINITE
+    assert not lut[1].view(np.uint16).any() and not idx[32:].any()
+    lut0, idx0, f0 = orc.kmeans_int8km(W[:32])
+    assert f0 == 0 and np.array_equal(lut0[0], lut[0]) and np.array_equal(idx0, idx[:32])
+
+
+def test_int8km_matches_sklearn_lloyd(orc):
+    """Same quantile start, 20 Lloyd steps on one group: scikit-learn's
+    KMeans (float64 centres) lands within fp16 rounding of most entries."""
+    from sklearn.cluster import KMeans
+    N, K = 32, 64
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    lut, _, _ = orc.kmeans_int8km(W)
+    v = np.sort(W.reshape(-1))
+    init = v[[((2 * k + 1) * v.size) // 512 for k in range(256)]].astype(np.float64)[:, None]
+    km = KMeans(256, init=init, n_init=1, max_iter=20, tol=0.0, algorithm="lloyd")
+    km.fit(W.reshape(-1).astype(np.float64)[:, None])
+    ref = np.sort(km.cluster_centers_[:, 0]).astype(np.float16)
+    assert np.mean(ref == lut[0]) >= 0.9
+
+
+def test_int8km_error_below_int4km_page_band(orc):
+    """The pages measure the 4-bit schemes' weight error at 3.6x int8km's on a
+    real head.  On Gaussian weights int8km's relative error is below
+    int4km's / 3.6 (measured ratio ~6).  (Heavy tails are another matter:
+    20 Lloyd steps from the quantile start do not yet spread 256 centres
+    over a group's far tail.)"""
+    g = np.random.default_rng(11)
+    W = (g.standard_normal((64, 512)) * 0.02).astype(np.float32)
+    lut8, idx8, _ = orc.kmeans_int8km(W)
+    lut4, idx4, _ = orc.kmeans_int4km(W)
+    e8 = np.linalg.norm(orc.dequant(orc.FMT_INT8KM, idx8, lut8, 64, 512) - W) / np.linalg.norm(W)
+    e4 = np.linalg.norm(orc.dequant(orc.FMT_INT4KM, idx4, lut4, 64, 512) - W) / np.linalg.norm(W)
+    assert e8 * 3.6 < e4, (e8, e4)
+
+
+# --------------------------------------------------------------------------
 # matvec and gather
 # --------------------------------------------------------------------------
 
@@ -517,6 +624,10 @@ def _encode_all(orc, W):
     out[orc.FMT_INT4KM] = (idx, lut)
     c, s, _ = orc.encode_int8(W)
     out[orc.FMT_INT8] = (c, s)
+    c, a, _ = orc.encode_int4aff(W)
+    out[orc.FMT_INT4AFF] = (c, a)
+    lut8, idx8, _ = orc.kmeans_int8km(W)
+    out[orc.FMT_INT8KM] = (idx8, lut8)
     return out
 
 

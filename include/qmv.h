@@ -17,6 +17,9 @@
  *        palettization": per-block symmetric quantization, 1-D k-means
  *        palettes, fp16 scales, and the pitfall that layers whose dimension
  *        does not divide the block are silently skipped (here: rejected).
+ *   [P5] "Compression (palettization & quantization)": "int8 k-means >
+ *        whole-model int4" (the recommended recipe, 8-bit k-means with
+ *        group 32).
  *
  * Conventions for every call below
  *  - All array pointers are DEVICE pointers owned by the caller, 16-byte
@@ -69,7 +72,8 @@ enum {
   QMV_FMT_INT4 = 1,   /* symmetric int4 (nibble = q + 8) + fp16 scale   */
   QMV_FMT_INT4KM = 2, /* 4-bit index into a per-row 16-entry fp16 LUT   */
   QMV_FMT_INT8 = 3,   /* symmetric int8 (two's complement) + fp16 scale */
-  QMV_FMT_INT4AFF = 4 /* affine int4 (q, zero point) + fp16 scale      */
+  QMV_FMT_INT4AFF = 4, /* affine int4 (q, zero point) + fp16 scale     */
+  QMV_FMT_INT8KM = 5   /* 8-bit index into a 256-entry fp16 LUT per 32 rows */
 };
 
 /* Device status bits (qmv_status_fetch). */
@@ -180,6 +184,18 @@ qmv_status qmv_matvec_int8(const int8_t* codes, const uint16_t* scales, const ui
  * same result). */
 qmv_status qmv_matvec_int4aff(const uint8_t* codes, const uint8_t* aux, const uint16_t* x,
                               int B, int64_t N, int64_t K, float* y, void* stream);
+
+/* int8km matvec ([P3] "Palettization": per-grouped-channel LUTs, 2^n_bits
+ * entries; [P5] "int8 k-means > whole-model int4": 8-bit k-means, group 32;
+ * [P1] sec. 1: the gather format int8km):
+ *   y[b, n] = sum_k x[b, k] * lut[n / 32][idx[n, k]]
+ *   idx  [N, K] uint8 (16-byte aligned)
+ *   lut  [ceil(N/32), 256] fp16 bits (2-byte aligned); rows 32g..32g+31
+ *        share lut[g] (a last group may have fewer rows)
+ * Other arguments and errors as qmv_matvec_fp4.  The LUTs come from the
+ * caller (a k-means fit; no encoder in this library). */
+qmv_status qmv_matvec_int8km(const uint8_t* idx, const uint16_t* lut, const uint16_t* x, int B,
+                             int64_t N, int64_t K, float* y, void* stream);
 
 /* ---------------------------------------------------------------------
  * Fused matvec + argmax (greedy next token from the lm_head; the pages'

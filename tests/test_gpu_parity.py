@@ -16,7 +16,8 @@ from weight_only_quantized_qmv_b200 import synth
 pytestmark = pytest.mark.gpu
 
 TOL = 1e-3
-FMTS = ("fp4", "int4", "int4km", "int8", "int4aff")
+FMTS = ("fp4", "int4", "int4km", "int8", "int4aff", "int8km")
+KM8_ITERS = 3  # Lloyd steps of the int8km test fits (256 centres per 32 rows: the fit dominates test time)
 
 
 @pytest.fixture(scope="module")
@@ -69,13 +70,15 @@ def encode_orc(fmt, Wn):
         c, s, f = orc.encode_int8(Wn)
     elif fmt == "int4aff":
         c, s, f = orc.encode_int4aff(Wn)
+    elif fmt == "int8km":
+        s, c, f = orc.kmeans_int8km(Wn, iters=KM8_ITERS)
     else:
         s, c, f = orc.kmeans_int4km(Wn)
     return c, s, f
 
 
 FID = {"fp4": orc.FMT_FP4, "int4": orc.FMT_INT4, "int4km": orc.FMT_INT4KM, "int8": orc.FMT_INT8,
-       "int4aff": orc.FMT_INT4AFF}
+       "int4aff": orc.FMT_INT4AFF, "int8km": orc.FMT_INT8KM}
 
 
 def np_bits(t):
@@ -176,6 +179,23 @@ def test_int4aff_unaligned_aux(q):
     assert q.status_fetch() == 0
 
 
+def test_int8km_lut_checks_and_unaligned_lut(q):
+    """The binding rejects a LUT of the wrong group count; a LUT plane that
+    starts 2 bytes past a 16-byte boundary gives the same outputs."""
+    N, K, B = 70, 2080, 3
+    c_o, s_o, xn = _inputs("int8km", N, K, B, seed=41)
+    c, x = torch.from_numpy(c_o).cuda(), torch.from_numpy(xn).cuda()
+    y0 = q.matvec_int8km(c, torch.from_numpy(s_o).cuda(), x)
+    with pytest.raises(ValueError):
+        q.matvec_int8km(c, torch.from_numpy(s_o[:2].copy()).cuda(), x)
+    lb = torch.zeros(s_o.size + 1, dtype=torch.float16, device="cuda")
+    lb[1:] = torch.from_numpy(s_o.reshape(-1)).cuda()
+    y = q.matvec_int8km(c, lb[1:].view(s_o.shape), x)
+    assert torch.equal(y, y0)
+    assert rel_err(y.cpu().numpy(), orc.matvec(orc.FMT_INT8KM, c_o, s_o, xn, N, K)) < TOL
+    assert q.status_fetch() == 0
+
+
 def test_c1_tiny_fp4_round_trip_and_matvec(q):
     """512x1024 fp4, 8 outlier columns x20, x ~N(0,1) fp16, seed 0."""
     g = synth.generator(0, "cpu")
@@ -216,9 +236,10 @@ def _inputs(fmt, N, K, B, seed):
     W, _ = synth.weights(N, K, g, n_outlier_cols=2)
     x = synth.activations(B, K, g)
     Wn = W.numpy()
-    c_o, s_o, _ = encode_orc(fmt, Wn) if fmt != "int4km" or N * K <= 2_000_000 else (None, None, 0)
-    if c_o is None:
-        lut, idx = synth.palette_tables(N, K, g)
+    big = (fmt == "int4km" and N * K > 2_000_000) or (fmt == "int8km" and N * K > 600_000)
+    c_o, s_o, _ = encode_orc(fmt, Wn) if not big else (None, None, 0)
+    if c_o is None:  # stand-in tables where the CPU fit is too slow
+        lut, idx = (synth.palette_tables8 if fmt == "int8km" else synth.palette_tables)(N, K, g)
         c_o, s_o = idx.numpy(), lut.numpy()
     return c_o, s_o, x.numpy()
 
@@ -473,10 +494,12 @@ def test_matvec_argmax_planted_and_ties(q, fmt):
     W, _ = synth.weights(N, K, g, n_outlier_cols=0)
     x = synth.activations(B, K, g).numpy()
     Wn = W.numpy()
-    # row 2321 aligned with x[0]; rows 777 and 2900 identical and aligned with x[1]
+    # row 2321 aligned with x[0]; rows 777 and 2900 identical and aligned with
+    # x[1] (int8km: 777 and 778, one LUT group, so their weights stay equal)
+    tw = 778 if fmt == "int8km" else 2900
     Wn[2321] = np.sign(x[0].astype(np.float32)) * 0.05
     Wn[777] = np.sign(x[1].astype(np.float32)) * 0.05
-    Wn[2900] = Wn[777]
+    Wn[tw] = Wn[777]
     c_o, s_o, _ = encode_orc(fmt, Wn)
     c, s, xg = torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(), torch.from_numpy(x).cuda()
     ws = q.argmax_workspace()
@@ -485,7 +508,7 @@ def test_matvec_argmax_planted_and_ties(q, fmt):
         idx, val = q.matvec_argmax(f, c, s, xg, ws)
         got = idx.cpu().numpy()
         assert got[0] == 2321 and r[0].argmax() == 2321
-        assert got[1] == 777 and r[1, 777] == r[1, 2900] and r[1].argmax() == 777
+        assert got[1] == 777 and r[1, 777] == r[1, tw] and r[1].argmax() == 777
 
 
 def test_matvec_argmax_rejects_short_workspace(q):

@@ -21,8 +21,10 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqmv.so")
 
-FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8, FMT_INT4AFF = 0, 1, 2, 3, 4
-FMT_NAMES = {FMT_FP4: "fp4", FMT_INT4: "int4", FMT_INT4KM: "int4km", FMT_INT8: "int8", FMT_INT4AFF: "int4aff"}
+FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8, FMT_INT4AFF, FMT_INT8KM = 0, 1, 2, 3, 4, 5
+FMT_NAMES = {FMT_FP4: "fp4", FMT_INT4: "int4", FMT_INT4KM: "int4km", FMT_INT8: "int8", FMT_INT4AFF: "int4aff",
+             FMT_INT8KM: "int8km"}
+KM8_GROUP = 32  # int8km: output rows sharing one 256-entry LUT
 FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT = 1, 2, 4
 OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_DATA, ERR_CUDA = 0, -1, -2, -3, -4, -5
 
@@ -54,6 +56,7 @@ SIGNATURES = {
     "qmv_matvec_int4km": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int8": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int4aff": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
+    "qmv_matvec_int8km": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_gather_matvec": [_I32, _P, _P, _I32, _I64, _I64, _P, _I32, _I32, _P, _I32, _P, _P],
     "qmv_matvec_argmax": [_I32, _P, _P, _P, _I32, _I64, _I64, _P, ctypes.c_size_t, _P, _P, _P],
     "qmv_argmax_workspace_bytes": [ctypes.POINTER(ctypes.c_size_t)],
@@ -179,17 +182,41 @@ def encode_int4aff(W: torch.Tensor, stream=None):
 # ---------------------------------------------------------------- matvec
 
 _AUX = {FMT_FP4: torch.uint8, FMT_INT4: torch.float16, FMT_INT4KM: torch.float16, FMT_INT8: torch.float16,
-        FMT_INT4AFF: torch.uint8}
+        FMT_INT4AFF: torch.uint8, FMT_INT8KM: torch.float16}
 _CODES = {FMT_FP4: torch.uint8, FMT_INT4: torch.uint8, FMT_INT4KM: torch.uint8, FMT_INT8: torch.int8,
-          FMT_INT4AFF: torch.uint8}
+          FMT_INT4AFF: torch.uint8, FMT_INT8KM: torch.uint8}
 _ENTRY = {FMT_FP4: "qmv_matvec_fp4", FMT_INT4: "qmv_matvec_int4", FMT_INT4KM: "qmv_matvec_int4km",
-          FMT_INT8: "qmv_matvec_int8", FMT_INT4AFF: "qmv_matvec_int4aff"}
+          FMT_INT8: "qmv_matvec_int8", FMT_INT4AFF: "qmv_matvec_int4aff", FMT_INT8KM: "qmv_matvec_int8km"}
+
+
+def int8km_groups(N: int) -> int:
+    """LUT groups of an int8km matrix of N rows: ceil(N / 32)."""
+    return (int(N) + KM8_GROUP - 1) // KM8_GROUP
 
 
 def _nk(fmt, codes):
     N = codes.shape[-2]
-    K = codes.shape[-1] * (1 if fmt == FMT_INT8 else 2)
+    K = codes.shape[-1] * (1 if fmt in (FMT_INT8, FMT_INT8KM) else 2)
     return N, K
+
+
+def aux_shape(fmt: int, N: int, K: int):
+    """Shape of one matrix's scales / palette / aux rows in format fmt."""
+    if fmt in (FMT_FP4, FMT_INT4, FMT_INT8):
+        return (N, K // 32)
+    if fmt == FMT_INT4KM:
+        return (N, 16)
+    if fmt == FMT_INT4AFF:
+        return (N, int4aff_aux_row_bytes(K))
+    if fmt == FMT_INT8KM:
+        return (int8km_groups(N), 256)
+    raise ValueError(f"unknown format {fmt}")
+
+
+def _need_aux(fmt, aux, N, K, lead=()):
+    want = tuple(lead) + aux_shape(fmt, N, K)
+    if tuple(aux.shape) != want:
+        raise ValueError(f"{FMT_NAMES[fmt]} aux must have shape {want}, got {tuple(aux.shape)}")
 
 
 def matvec(fmt: int, codes: torch.Tensor, aux: torch.Tensor, x: torch.Tensor, out=None, stream=None):
@@ -197,6 +224,7 @@ def matvec(fmt: int, codes: torch.Tensor, aux: torch.Tensor, x: torch.Tensor, ou
     _need(codes, "codes", _CODES[fmt])
     _need(aux, "scales/lut", _AUX[fmt])
     N, K = _nk(fmt, codes)
+    _need_aux(fmt, aux, N, K)
     squeeze = x.dim() == 1
     xx = x.unsqueeze(0) if squeeze else x
     _need(xx, "x", torch.float16)
@@ -230,6 +258,11 @@ def matvec_int4aff(codes, aux, x, out=None, stream=None):
     return matvec(FMT_INT4AFF, codes, aux, x, out, stream)
 
 
+def matvec_int8km(idx, lut, x, out=None, stream=None):
+    """idx uint8 [N, K], lut float16 [ceil(N/32), 256] -> y float32 [B, N]."""
+    return matvec(FMT_INT8KM, idx, lut, x, out, stream)
+
+
 def argmax_workspace_bytes() -> int:
     """Workspace bytes matvec_argmax needs on the current device."""
     n = ctypes.c_size_t(0)
@@ -250,6 +283,7 @@ def matvec_argmax(fmt: int, codes: torch.Tensor, aux: torch.Tensor, x: torch.Ten
     _need(aux, "scales/lut", _AUX[fmt])
     _need(workspace, "workspace", torch.uint8)
     N, K = _nk(fmt, codes)
+    _need_aux(fmt, aux, N, K)
     xx = x.unsqueeze(0) if x.dim() == 1 else x
     _need(xx, "x", torch.float16)
     B = xx.shape[0]
@@ -273,6 +307,7 @@ def matvec_argmax_static(fmt: int, codes: torch.Tensor, aux: torch.Tensor, x: to
     _need(codes, "codes", _CODES[fmt])
     _need(aux, "scales/lut", _AUX[fmt])
     N, K = _nk(fmt, codes)
+    _need_aux(fmt, aux, N, K)
     xx = x.unsqueeze(0) if x.dim() == 1 else x
     _need(xx, "x", torch.float16)
     B = xx.shape[0]
@@ -299,6 +334,9 @@ def gather_matvec(fmt: int, codes_stack: torch.Tensor, aux_stack: torch.Tensor, 
     _need(x, "x", torch.float16)
     E = codes_stack.shape[0]
     N, K = _nk(fmt, codes_stack)
+    if codes_stack.dim() != 3:
+        raise ValueError("codes_stack must be [E, N, ...]")
+    _need_aux(fmt, aux_stack, N, K, lead=(E,))
     B, topk = expert_ids.shape
     want = (B, topk, K) if x_per_slot else (B, K)
     if tuple(x.shape) != want:
@@ -316,6 +354,7 @@ def dequant(fmt: int, codes: torch.Tensor, aux: torch.Tensor, stream=None) -> to
     _need(codes, "codes", _CODES[fmt])
     _need(aux, "aux", _AUX[fmt])
     N, K = _nk(fmt, codes)
+    _need_aux(fmt, aux, N, K)
     out = torch.empty((N, K), dtype=torch.float32, device=codes.device)
     _call("qmv_dequant", fmt, _ptr(codes), _ptr(aux), N, K, _ptr(out), _stream(stream))
     return out

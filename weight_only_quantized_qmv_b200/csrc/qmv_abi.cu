@@ -65,7 +65,7 @@ qmv_status check_ptr(const void* p, const char* name) {
 
 // formats whose aux is fp16 scales at every row start (int4aff rows may have
 // an odd byte count and are read bytewise where they are not 8-byte granular)
-bool has_fp16_scale_rows(int fmt) { return fmt == QMV_FMT_INT4 || fmt == QMV_FMT_INT8; }
+bool has_fp16_scale_rows(int fmt) { return fmt == QMV_FMT_INT4 || fmt == QMV_FMT_INT8 || fmt == QMV_FMT_INT8KM; }
 
 qmv_status check_shape(int64_t N, int64_t K) {
   if (N < 1) return fail(QMV_ERR_SHAPE, "N must be >= 1 (got %lld)", (long long)N);
@@ -134,7 +134,7 @@ struct ArgmaxOut {
 qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
                          int64_t K, float* y, void* stream, bool gather, int E, const int32_t* ids, int topk,
                          int x_per_slot, const ArgmaxOut* am = nullptr) {
-  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT4AFF) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
+  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8KM) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
   QMV_TRY(check_ptr(codes, "codes"));
   if (!aux) return fail(QMV_ERR_ARG, "scales/lut is null");
   // the staged scale block copies handle any byte alignment; the palette and
@@ -171,7 +171,8 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
   uint32_t* st;
   int sms;
   QMV_TRY(device_ctx(&st, &sms));
-  if (!qmv::plan_matvec(fmt, p, sms))
+  const bool km8 = fmt == QMV_FMT_INT8KM;
+  if (!(km8 ? qmv::plan_km8(p, sms) : qmv::plan_matvec(fmt, p, sms)))
     return fail(QMV_ERR_UNSUPPORTED, "activations (%d rows x %lld) do not fit the on-chip staging", p.n_xrows,
                 (long long)K);
   p.status = st;
@@ -189,7 +190,7 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
     p.am_idx = am->idx;
     p.am_val = am->val;
   }
-  cudaError_t e = qmv::launch_matvec(fmt, p, (cudaStream_t)stream);
+  cudaError_t e = km8 ? qmv::launch_km8(p, (cudaStream_t)stream) : qmv::launch_matvec(fmt, p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "matvec launch");
   return QMV_OK;
 }
@@ -277,6 +278,11 @@ qmv_status qmv_matvec_int4aff(const uint8_t* codes, const uint8_t* aux, const ui
   return matvec_common(QMV_FMT_INT4AFF, codes, aux, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
 }
 
+qmv_status qmv_matvec_int8km(const uint8_t* idx, const uint16_t* lut, const uint16_t* x, int B, int64_t N,
+                             int64_t K, float* y, void* stream) {
+  return matvec_common(QMV_FMT_INT8KM, idx, lut, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
+}
+
 qmv_status qmv_matvec_argmax(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
                              int64_t K, void* workspace, size_t workspace_bytes, int32_t* idx, float* val,
                              void* stream) {
@@ -315,7 +321,7 @@ qmv_status qmv_gather_matvec(int fmt, const void* codes_stack, const void* aux_s
 }
 
 qmv_status qmv_dequant(int fmt, const void* codes, const void* aux, int64_t N, int64_t K, float* Wdq, void* stream) {
-  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT4AFF) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
+  if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8KM) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
   QMV_TRY(check_ptr(codes, "codes"));
   if (!aux) return fail(QMV_ERR_ARG, "aux is null");
   if (fmt == QMV_FMT_INT4KM) QMV_TRY(check_ptr(aux, "lut"));

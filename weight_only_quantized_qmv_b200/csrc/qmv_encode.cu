@@ -228,7 +228,13 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
        blk += (int64_t)gridDim.x * blockDim.x) {
     const int64_t n = blk / nb_row, b = blk - n * nb_row;
     float out[32];
-    if constexpr (FMT == QMV_FMT_INT8) {
+    if constexpr (FMT == QMV_FMT_INT8KM) {
+      // one LUT of 256 fp16 entries per 32 rows
+      const uint16_t* L = reinterpret_cast<const uint16_t*>(aux) + (n / 32) * 256;
+      const uint8_t* src = codes + blk * 32;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) out[i] = __half2float(__ushort_as_half(L[src[i]]));
+    } else if constexpr (FMT == QMV_FMT_INT8) {
       const uint4* src = reinterpret_cast<const uint4*>(codes + blk * 32);
       const float s = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(aux)[blk]));
       const uint4 v0 = src[0], v1 = src[1];
@@ -349,6 +355,7 @@ cudaError_t launch_dequant(int fmt, const uint8_t* codes, const uint8_t* aux, in
     case QMV_FMT_INT4KM: dequant_kernel<QMV_FMT_INT4KM><<<grid, 128, 0, stream>>>(codes, aux, N, K, Wdq); break;
     case QMV_FMT_INT8: dequant_kernel<QMV_FMT_INT8><<<grid, 128, 0, stream>>>(codes, aux, N, K, Wdq); break;
     case QMV_FMT_INT4AFF: dequant_kernel<QMV_FMT_INT4AFF><<<grid, 128, 0, stream>>>(codes, aux, N, K, Wdq); break;
+    case QMV_FMT_INT8KM: dequant_kernel<QMV_FMT_INT8KM><<<grid, 128, 0, stream>>>(codes, aux, N, K, Wdq); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -61,6 +61,7 @@ struct MvParams {
   int off_xsum;            // its per-block activation sums (int4, int4aff)
   int64_t zplane;          // int4aff: byte offset of the zero points in an aux row
   int zoff;                // int4aff: byte offset of the slice's zero points in a staged aux row
+  int off_tab;             // int8km: the replicated LUT (32 KB)
   int prefetch;            // dense: weights may be read before the preceding grid completes
   int RS;                  // shared-memory bytes per staged code row
   int AS;                  // shared-memory bytes per staged scale row (kAuxRows)
@@ -110,6 +111,9 @@ inline size_t argmax_workspace_bytes(int num_sms) {
 }
 
 cudaError_t launch_matvec(int fmt, const MvParams& p, cudaStream_t stream);
+// int8km (dense or gather; p.argmax for the fused argmax): geometry, launch.
+bool plan_km8(MvParams& p, int num_sms);
+cudaError_t launch_km8(const MvParams& p, cudaStream_t stream);
 
 // ---- encoders / dequant ------------------------------------------------------
 struct ClipList {

@@ -27,6 +27,7 @@
 // its scale in the table and accumulates straight through.  Each output is
 // accumulated by one lane in a fixed order and written once (deterministic).
 #include "qmv_device.cuh"
+#include "qmv_kernel_common.cuh"
 
 namespace qmv {
 
@@ -60,36 +61,6 @@ struct FmtT<QMV_FMT_INT4AFF> {
   static constexpr bool kLut = false, kPermX = true, kZp = true;
 };
 
-// Column groups: the activation rows served by one pass over one expert's
-// weights (dense: one group of all B rows).
-struct GroupTable {
-  int ngroups;
-  int expert[kMaxPairs];
-  int start[kMaxPairs];
-  int count[kMaxPairs];
-  int16_t sorted[kMaxPairs];  // (token, slot) pair indices ordered by expert
-};
-// the kernel's static shared memory: the group table, the ids, a counter
-static_assert(sizeof(GroupTable) + kMaxPairs * sizeof(int) + kMaxCols * 8 + 32 <= kStaticSmem,
-              "static shared memory reserve");
-
-__device__ __forceinline__ uint32_t lds_u8(uint32_t a) { return *sptr<uint8_t>(a); }
-__device__ __forceinline__ uint32_t lds_u16(uint32_t a) { return *sptr<uint16_t>(a); }
-__device__ __forceinline__ void sts_u8(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ void sts_f32x2(uint32_t a, float u, float v) {
-  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(u), "f"(v) : "memory");
-}
-__device__ __forceinline__ uint4 ldg_nc_128(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -397,26 +368,6 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
   }
 }
 
-// Fused argmax: an output y[b, n] as a 64-bit key whose unsigned order is
-// (value as a float with -0 == +0, then lower n first).
-__device__ __forceinline__ unsigned long long argmax_key(float v, int64_t n) {
-  const uint32_t u = __float_as_uint(v + 0.0f);  // -0 -> +0
-  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return ((unsigned long long)k << 32) | (unsigned long long)(~(uint32_t)n);
-}
-__device__ __forceinline__ float argmax_key_value(unsigned long long key) {
-  const uint32_t k = (uint32_t)(key >> 32);
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void grid_wait_preceding() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-__device__ __forceinline__ uint8_t ldg_u8(const uint8_t* p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(p));
-  return (uint8_t)v;
-}
 
 // NT: activation n-tiles of 8 columns (1 or 2); NT = 0 is the batch-1 form
 // whose MMA columns carry blocks (slice_one).
@@ -438,7 +389,6 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_addr(smem);
-  const int P = p.gather ? p.B * p.topk : p.B;
 
   // Programmatic dependent launch: the next grid in the stream may become
   // resident as this one's blocks finish; this grid reads activations / ids
@@ -446,58 +396,9 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   grid_launch_dependents();
   if (!p.prefetch) grid_wait_preceding();
 
-  // ---- set-up (whole CTA): the column groups and the staged activations -----
-  if (tid == 0) s_nvalid = 0;
-  if (tid < kMaxCols) s_best[tid] = 0ull;
-  if (p.gather && tid < P) s_ids[tid] = p.ids[tid];
-  __syncthreads();
-  if (!p.gather) {
-    if (tid == 0) {
-      gt.ngroups = 1;
-      gt.expert[0] = 0;
-      gt.start[0] = 0;
-      gt.count[0] = p.B;
-    }
-    if (tid < P) gt.sorted[tid] = (int16_t)tid;
-  } else if (tid < P) {
-    const int e = s_ids[tid];
-    if (e >= 0 && e < p.E) {
-      int rank = 0;  // stable rank of this pair among valid pairs ordered by expert id
-      for (int j = 0; j < P; ++j) {
-        const int f = s_ids[j];
-        rank += (f >= 0 && f < p.E && (f < e || (f == e && j < tid))) ? 1 : 0;
-      }
-      gt.sorted[rank] = (int16_t)tid;
-      atomicAdd(&s_nvalid, 1);
-    }
-  }
-  __syncthreads();
-  if (p.gather) {
-    if (tid == 0) {
-      int ng = 0;
-      for (int i = 0; i < s_nvalid; ++i) {
-        const int e = s_ids[gt.sorted[i]];
-        if (ng == 0 || gt.expert[ng - 1] != e || gt.count[ng - 1] == 8 * NT) {
-          gt.expert[ng] = e;
-          gt.start[ng] = i;
-          gt.count[ng] = 0;
-          ++ng;
-        }
-        gt.count[ng - 1]++;
-      }
-      gt.ngroups = ng;
-    }
-    // a pair with an out-of-range expert id gets a zero output row (one CTA per pair)
-    for (int q = 0; q < P; ++q) {
-      const int e = s_ids[q];
-      if ((e < 0 || e >= p.E) && (q % (int)gridDim.x) == (int)blockIdx.x) {
-        if (tid == 0) atomicOr(p.status, QMV_FLAG_BAD_EXPERT);
-        for (int64_t n = tid; n < p.N; n += blockDim.x) p.y[(int64_t)q * p.N + n] = 0.0f;
-      }
-    }
-  }
+  // ---- set-up (whole CTA): the column groups -----
+  setup_groups<8 * NTX>(p, gt, s_ids, s_nvalid, s_best, tid);
   const uint32_t xbase = sbase + p.off_x;
-  __syncthreads();  // the group table
 
   // ---- the warp's work items ------------------------------------------------
   // Units are (column group, 16-row tile) pairs.  With at least as many
@@ -918,54 +819,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   }
   cp_async_wait(0);
 
-  if constexpr (AM) {
-    // the lanes sharing t (and so their columns) combine, then one shared
-    // atomic per column and warp
-#pragma unroll
-    for (int i = 0; i < 2 * NTX; ++i) {
-      unsigned long long k = best[i];
-      int c = bcol[i];
-#pragma unroll
-      for (int m = 4; m < 32; m *= 2) {
-        const unsigned long long k2 = __shfl_xor_sync(0xffffffffu, k, m);
-        const int c2 = __shfl_xor_sync(0xffffffffu, c, m);
-        k = k2 > k ? k2 : k;
-        c = c2 > c ? c2 : c;
-      }
-      if (lane < 4 && c >= 0) atomicMax(&s_best[c], k);
-    }
-    // CTA partials to the workspace; the last CTA to finish (counter) takes
-    // the maximum over all CTAs for each row and resets the counter.
-    __syncthreads();
-    if (tid < p.B) p.am_part[(int64_t)blockIdx.x * kMaxCols + tid] = s_best[tid];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(p.am_ticket, 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (s_last) {
-      // all threads: thread tid folds entries (CTA c, row tid % 16) -- the
-      // stride is a multiple of 16 -- and the rows meet in s_best (which
-      // already holds this CTA's own partials)
-      __threadfence();
-      const int b = tid & (kMaxCols - 1);
-      const int nent = (int)gridDim.x * kMaxCols;
-      unsigned long long mine = 0ull;
-#pragma unroll 4
-      for (int e = tid; e < nent; e += kT) {
-        const unsigned long long k = __ldcg(p.am_part + e);
-        mine = k > mine ? k : mine;
-        p.am_part[e] = 0ull;  // the workspace is left zero-filled
-      }
-      if (b < p.B) atomicMax(&s_best[b], mine);
-      __syncthreads();
-      if (tid < p.B) {
-        const unsigned long long best = s_best[tid];
-        p.am_idx[tid] = (int32_t)(~(uint32_t)best);
-        p.am_val[tid] = argmax_key_value(best);
-      }
-      if (tid == 0) *p.am_ticket = 0u;
-    }
-  }
+  if constexpr (AM) argmax_finish<2 * NTX, kT>(best, bcol, s_best, s_last, p, tid, lane);
 }
 
 // ---------------------------------------------------------------------------

@@ -62,6 +62,18 @@ def palette_tables(N: int, K: int, gen: torch.Generator, std: float = WEIGHT_STD
     return lut, idx
 
 
+def palette_tables8(N: int, K: int, gen: torch.Generator, std: float = WEIGHT_STD, device=None):
+    """Stand-in int8km inputs (as palette_tables, 8-bit): per group of 32 rows
+    a sorted 256-entry fp16 table drawn ~N(0, std) and uniformly random index
+    bytes [N, K].  Same shapes and bytes as a fitted int8km palette."""
+    device = device or gen.device
+    G = (N + 31) // 32
+    lut = torch.randn(G, 256, generator=gen, device=device, dtype=torch.float32).mul_(std)
+    lut = torch.sort(lut, dim=1).values.to(torch.float16)
+    idx = torch.randint(0, 256, (N, K), generator=gen, device=device, dtype=torch.int32).to(torch.uint8)
+    return lut, idx
+
+
 def int_codes(N: int, K: int, bits: int, gen: torch.Generator, device=None):
     """Uniform random packed codes (uint8 [N, K*bits/8]) for edge-case tests."""
     device = device or gen.device

@@ -545,13 +545,15 @@ def test_gather_parity(q, fmt, B, topk, x_per_slot):
     r, fl = orc.gather_matvec(FID[fmt], cs, aus, E, N, K, ids, x, x_per_slot)
     assert fl == 0
     assert rel_err(y.reshape(-1, N), r.reshape(-1, N)) < TOL
-    # identical to the dense kernel on the chosen expert's weights, bit for bit
+    # identical, bit for bit, to the dense kernel on the chosen expert's
+    # weights taking the same tensor-core path: a batch of two (dense batch 1
+    # may take a batch-1 form with another summation order)
     for b in range(B):
         for j in range(topk):
             e = ids[b, j]
             xb = x[b, j] if x_per_slot else x[b]
             yd = q.matvec(F, torch.from_numpy(cs[e]).cuda(), torch.from_numpy(aus[e]).cuda(),
-                          torch.from_numpy(xb[None].copy()).cuda()).cpu().numpy()[0]
+                          torch.from_numpy(np.stack([xb, xb])).cuda()).cpu().numpy()[0]
             assert np.array_equal(yd, y[b, j]), (b, j)
     assert q.status_fetch() == 0
 

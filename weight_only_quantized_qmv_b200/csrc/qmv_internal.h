@@ -61,7 +61,8 @@ struct MvParams {
   int off_xsum;            // its per-block activation sums (int4, int4aff)
   int64_t zplane;          // int4aff: byte offset of the zero points in an aux row
   int zoff;                // int4aff: byte offset of the slice's zero points in a staged aux row
-  int off_tab;             // int8km: the replicated LUT (32 KB)
+  int off_tab;             // int8km: the replicated LUT table (64 KB, two buffers)
+  int red_bufs;            // int8km: partial-sum buffers (2, or 1 where shared memory is short)
   int prefetch;            // dense: weights may be read before the preceding grid completes
   int RS;                  // shared-memory bytes per staged code row
   int AS;                  // shared-memory bytes per staged scale row (kAuxRows)

@@ -13,8 +13,9 @@
 //    parts, and the 8 partial sums meet in shared memory in part order, so a
 //    result does not depend on the CTA size.
 //  * The unit's LUT is written to shared memory with each entry repeated in
-//    all 32 banks (word e * 32 + lane), so the lookup of lane l reads bank l:
-//    one conflict-free 32-bit load per weight whatever the indices.
+//    all 32 banks, so the lookup of lane l reads bank l: one conflict-free
+//    32-bit load per weight whatever the indices.  Two table buffers: the
+//    next unit's LUT is written while this one is read.
 //  * Index bytes go from global memory straight to registers (one 16-byte
 //    load per row and chunk, one chunk ahead); the next unit's index rows are
 //    prefetched into L2 (128-byte lines, spread over the CTA's threads)
@@ -41,27 +42,104 @@ __device__ __forceinline__ uint4 ldg_stream_128(const void* p) {
 // L2 prefetch of the line holding p
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
-// Lookup of byte J of w in the replicated table (tab_l = table + 4 * lane):
-// the entry's fp16 value in both halves of the returned word.
+// The LUT table: 256 rows of 256 bytes at the start of the dynamic shared
+// memory; row c holds entry c of buffer 0 in words 0..31 and of buffer 1 in
+// words 32..63 (each word: the fp16 value in both halves).  A lookup's byte
+// offset c * 256 + buffer * 128 + lane * 4 is one byte permute of the index
+// byte and lb = buffer * 128 + lane * 4, and the table's base is a constant,
+// so a lookup is one permute and one conflict-free 32-bit shared load.
+extern __shared__ __align__(1024) uint8_t km8_smem[];
+
 template <int J>
-__device__ __forceinline__ uint32_t km8_lookup(uint32_t w, uint32_t tab_l) {
-  const uint32_t c = (J == 3) ? (w >> 24) : prmt(w, 0u, 0x4440u + J);
-  return lds32(tab_l + (c << 7));
+__device__ __forceinline__ uint32_t km8_lookup(uint32_t w, uint32_t lb, uint32_t tb) {
+  const uint32_t off = prmt(w, lb, 0x5504u + 16u * J);  // bytes: lb.0, w.J, 0, 0
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(tb + off));  // tb: the table's shared address
+  return v;
 }
 // the A operand pair (byte J, byte J + 1) of w: low half from J
 template <int J>
-__device__ __forceinline__ uint32_t km8_pair(uint32_t w, uint32_t tab_l) {
-  return prmt(km8_lookup<J>(w, tab_l), km8_lookup<J + 1>(w, tab_l), 0x5410u);
+__device__ __forceinline__ uint32_t km8_pair(uint32_t w, uint32_t lb, uint32_t tb) {
+  return prmt(km8_lookup<J>(w, lb, tb), km8_lookup<J + 1>(w, lb, tb), 0x5410u);
 }
 
-// NT: activation n-tiles of 8 columns (1 or 2).  WARPS: 8 (two CTAs per SM)
-// or 16 (one CTA per SM, when the staged activations are large).
+// One 64-wide chunk of a warp's rows g, g+8 (index words cg, ch of this
+// lane's 16 in-features) against the staged activations xa[n] + 128 c.
+// PARTIAL: the chunk ends at K after 32 in-features; lanes t >= 2 hold no
+// weights and contribute exact zeros.
+template <int NT, bool PARTIAL>
+__device__ __forceinline__ void km8_chunk(float (&acc)[NT][4], const uint4& cg, const uint4& ch, const uint32_t (&xa)[NT],
+                                          const bool (&xon)[NT], int64_t c, uint32_t lb, uint32_t tb, int t) {
+  uint4 xr0[NT], xr1[NT];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    xr0[n] = make_uint4(0u, 0u, 0u, 0u);
+    xr1[n] = xr0[n];
+    if (xon[n]) {
+      xr0[n] = lds128(xa[n] + 128u * (uint32_t)c);
+      xr1[n] = lds128(xa[n] + 128u * (uint32_t)c + 16u);
+    }
+  }
+  const uint32_t wg[4] = {cg.x, cg.y, cg.z, cg.w}, wh[4] = {ch.x, ch.y, ch.z, ch.w};
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    uint32_t a0 = km8_pair<0>(wg[s], lb, tb), a2 = km8_pair<2>(wg[s], lb, tb);
+    uint32_t a1 = km8_pair<0>(wh[s], lb, tb), a3 = km8_pair<2>(wh[s], lb, tb);
+    if (PARTIAL && t >= 2) a0 = a1 = a2 = a3 = 0u;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const uint32_t b0 = s == 0 ? xr0[n].x : s == 1 ? xr0[n].z : s == 2 ? xr1[n].x : xr1[n].z;
+      const uint32_t b1 = s == 0 ? xr0[n].y : s == 1 ? xr0[n].w : s == 2 ? xr1[n].y : xr1[n].w;
+      mma16816(acc[n], a0, a1, a2, a3, b0, b1);
+    }
+  }
+}
+
+// Batch 1 (dense): no tensor cores.  The table holds fp32 values and the
+// activations are staged as fp32, 16 per lane and chunk (chunk c of the
+// staged row: 256 bytes, the 16 bytes of lane quarter t and word i at
+// 64 i + 16 t, so the four quarters of a load are conflict-free).  Each
+// weight is one byte permute, one shared load and one fp32 fma; the even
+// and odd in-features of a row accumulate separately (shorter chains).
+template <bool PARTIAL>
+__device__ __forceinline__ void km8_chunk_b1(float (&ag)[2], float (&ah)[2], const uint4& cg, const uint4& ch,
+                                             uint32_t xa, int64_t c, uint32_t lb, uint32_t tb, int t) {
+  if (PARTIAL && t >= 2) return;
+  const uint32_t wg[4] = {cg.x, cg.y, cg.z, cg.w}, wh[4] = {ch.x, ch.y, ch.z, ch.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 xv = lds128(xa + 256u * (uint32_t)c + 64u * (uint32_t)i);
+    const float x0 = __uint_as_float(xv.x), x1 = __uint_as_float(xv.y);
+    const float x2 = __uint_as_float(xv.z), x3 = __uint_as_float(xv.w);
+    ag[0] = fmaf(__uint_as_float(km8_lookup<0>(wg[i], lb, tb)), x0, ag[0]);
+    ah[0] = fmaf(__uint_as_float(km8_lookup<0>(wh[i], lb, tb)), x0, ah[0]);
+    ag[1] = fmaf(__uint_as_float(km8_lookup<1>(wg[i], lb, tb)), x1, ag[1]);
+    ah[1] = fmaf(__uint_as_float(km8_lookup<1>(wh[i], lb, tb)), x1, ah[1]);
+    ag[0] = fmaf(__uint_as_float(km8_lookup<2>(wg[i], lb, tb)), x2, ag[0]);
+    ah[0] = fmaf(__uint_as_float(km8_lookup<2>(wh[i], lb, tb)), x2, ah[0]);
+    ag[1] = fmaf(__uint_as_float(km8_lookup<3>(wg[i], lb, tb)), x3, ag[1]);
+    ah[1] = fmaf(__uint_as_float(km8_lookup<3>(wh[i], lb, tb)), x3, ah[1]);
+  }
+}
+
+// NT: activation n-tiles of 8 columns (1 or 2), or 0: dense batch 1 on the
+// fp32 path above.  WARPS: 8 (two CTAs per SM) or 16 (one CTA per SM, when
+// the staged activations are large).
+//
+// Per unit, with one barrier: the next unit's LUT entries are requested at
+// the start (registers) and written to the other table buffer at the end;
+// the partial sums alternate between two buffers (one buffer and a second
+// barrier where shared memory is short); a warp's index loads run one chunk
+// ahead straight across unit boundaries.
 template <int NT, int WARPS, bool AM>
 __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(const __grid_constant__ MvParams p) {
   constexpr int kT = 32 * WARPS;
-  constexpr int KP = 8;                 // K parts per unit
+  constexpr int KP = 8;                  // K parts per unit
   constexpr int PPW = KP / (WARPS / 2);  // parts per warp
-  extern __shared__ __align__(1024) uint8_t smem[];
+  constexpr bool kF = NT == 0;           // the batch-1 fp32 path
+  constexpr int NTX = kF ? 1 : NT;
+  constexpr int EPW = 256 / WARPS;       // LUT entries per warp in a table build
+  constexpr int kRedFloats = kF ? KP * 2 * 2 * 32 : KP * 2 * NTX * 4 * 32;  // one partial-sum buffer
   __shared__ GroupTable gt;
   __shared__ int s_ids[kMaxPairs];
   __shared__ int s_nvalid;
@@ -70,19 +148,19 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const uint32_t sbase = smem_addr(smem);
-  const uint32_t tab = sbase + p.off_tab;  // [256][32] words
-  const uint32_t tab_l = tab + 4u * (uint32_t)lane;
+  const uint32_t sbase = smem_addr(km8_smem);  // the LUT table: [256][2 buffers][32] words
   const uint32_t xbase = sbase + p.off_x;
-  float* red = reinterpret_cast<float*>(smem + p.off_red);  // [KP][2 tiles][NT][4][32]
+  // partial sums, two buffers of [KP][2 tiles][NT][4][32] (batch-1 path: [KP][2 tiles][2 rows][32])
+  float* red0 = reinterpret_cast<float*>(km8_smem + p.off_red);
   const int64_t K = p.K;
   const int64_t G = p.tiles;  // row groups of 32
 
   grid_launch_dependents();
   if (!p.prefetch) grid_wait_preceding();
-  setup_groups<8 * NT>(p, gt, s_ids, s_nvalid, s_best, tid);
+  setup_groups<8 * NTX>(p, gt, s_ids, s_nvalid, s_best, tid);
   const int ngroups = gt.ngroups;
   const int64_t total = (int64_t)ngroups * G;
+  const int64_t grid = gridDim.x;
 
   // a unit's index rows: expert e, rows [32 rg, min(32 rg + 32, N))
   auto unit_codes = [&](int64_t u, int64_t& rg, int& grp, const uint8_t*& base, int& nrows) {
@@ -104,11 +182,62 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
     const int64_t bytes = min((int64_t)nrows * K, (int64_t)1 << 18);
     for (int64_t off = 128 * (int64_t)tid; off < bytes; off += 128 * kT) prefetch_l2(base + off);
   };
+  // this thread's LUT entry of unit u (lanes < EPW), in the table's word format
+  auto lut_entry = [&](int64_t u) -> uint32_t {
+    int64_t rg;
+    int grp, nrows;
+    const uint8_t* base;
+    unit_codes(u, rg, grp, base, nrows);
+    const uint16_t* lut =
+        reinterpret_cast<const uint16_t*>(p.aux + (int64_t)gt.expert[grp] * p.expert_aux_bytes) + rg * 256;
+    uint32_t v = 0u;
+    if (lane < EPW) {
+      const uint32_t h = lut[warp * EPW + lane];
+      v = kF ? __float_as_uint(__half2float(__ushort_as_half((unsigned short)h))) : (h | (h << 16));
+    }
+    return v;
+  };
+  // whole CTA: the entries (from lut_entry) into table buffer b
+  auto write_table = [&](uint32_t v, int b) {
+#pragma unroll
+    for (int j = 0; j < EPW / 4; ++j) {
+      // rows 4j .. 4j+3 of this warp's entries, 8 lanes x 16 bytes per row
+      const int r = 4 * j + (lane >> 3);
+      const uint32_t w = __shfl_sync(0xffffffffu, v, r);
+      sts128(sbase + (uint32_t)(warp * EPW + r) * 256u + 128u * (uint32_t)b + 16u * (uint32_t)(lane & 7),
+             make_uint4(w, w, w, w));
+    }
+  };
   if ((int64_t)blockIdx.x < total) prefetch_unit(blockIdx.x);  // weights only
+  if ((int64_t)blockIdx.x + grid < total) prefetch_unit(blockIdx.x + grid);
 
   if (p.prefetch) grid_wait_preceding();
-  // activations in natural order, each row zero-padded to whole 64-wide chunks
-  {
+  if constexpr (kF) {
+    // one fp32 row: in-features 64c + 16t + 4i .. +3 at byte 256c + 64i + 16t,
+    // zero-padded to whole chunks
+    const int64_t n8 = p.XS / 32;  // 8-feature pieces of the padded row
+    for (int64_t j = tid; j < n8; j += kT) {
+      float f[8];
+      if (j < K / 8) {
+        const uint4 v = ldg_nc_128(p.x + 8 * j);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __half2 h = *reinterpret_cast<const __half2*>(&w4[e]);
+          f[2 * e] = __low2float(h);
+          f[2 * e + 1] = __high2float(h);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+      }
+      const int64_t k = 8 * j, c = k / 64, tq = (k % 64) / 16, i = (k % 16) / 4;  // i even
+      const uint32_t a = xbase + (uint32_t)(256 * c + 64 * i + 16 * tq);
+      sts128(a, make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3])));
+      sts128(a + 64u, make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]), __float_as_uint(f[6]), __float_as_uint(f[7])));
+    }
+  } else {
+    // activations in natural order, each row zero-padded to whole 64-wide chunks
     const int64_t per_row = p.XS / 16;  // 16-byte pieces of a staged row
     const int64_t k16 = K / 8;          // pieces holding activations
     const int64_t n16 = (int64_t)p.n_xrows * per_row;
@@ -118,55 +247,61 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
       sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
     }
   }
+  if ((int64_t)blockIdx.x < total) write_table(lut_entry(blockIdx.x), 0);
+  __syncthreads();  // the first table and the activations
 
   const int tile = warp & 1;
-  const int64_t nch = (K + 63) / 64;
+  const int nch = (int)((K + 63) / 64);
+  const int kp0 = (warp >> 1) * PPW;
+  const int cA = kp0 * nch / KP, cB = (kp0 + PPW) * nch / KP;  // this warp's chunks, every unit
+  const int rgi = tile * 16 + g;  // row g of this warp's tile within a unit
 
-  unsigned long long best[NT];
-  int bcol[NT];
+  unsigned long long best[NTX];
+  int bcol[NTX];
 #pragma unroll
-  for (int i = 0; i < NT; ++i) {
+  for (int i = 0; i < NTX; ++i) {
     best[i] = 0ull;
     bcol[i] = -1;
   }
 
-  for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
+  // the first chunk of this warp in unit u (zero where past K)
+  auto first_chunk = [&](int64_t u, uint4& cg, uint4& ch) {
+    cg = make_uint4(0u, 0u, 0u, 0u);
+    ch = cg;
+    if (u < total && cA < cB && 64 * (int64_t)cA + 16 * t < K) {
+      int64_t rg;
+      int grp, nrows;
+      const uint8_t* base;
+      unit_codes(u, rg, grp, base, nrows);
+      cg = ldg_stream_128(base + (int64_t)min(rgi, nrows - 1) * K + 64 * cA + 16 * t);
+      ch = ldg_stream_128(base + (int64_t)min(rgi + 8, nrows - 1) * K + 64 * cA + 16 * t);
+    }
+  };
+  uint4 cg, ch;
+  first_chunk(blockIdx.x, cg, ch);
+
+  int buf = 0;
+  for (int64_t u = blockIdx.x; u < total; u += grid, buf ^= 1) {
     int64_t rg;
     int grp, nrows;
     const uint8_t* ubase;
     unit_codes(u, rg, grp, ubase, nrows);
     const int ncols = gt.count[grp], gstart = gt.start[grp];
+    const bool has_next = u + grid < total;
+    float* red = red0 + (p.red_bufs == 2 ? buf : 0) * kRedFloats;
+    if (p.red_bufs == 1) __syncthreads();  // one partial-sum buffer: the previous unit's sums have been read
 
-    // ---- the unit's LUT, replicated across the banks ----
-    __syncthreads();  // the previous unit's lookups and partial sums are done (and the staged activations)
-    {
-      constexpr int EPW = 256 / WARPS;  // entries per warp
-      const uint16_t* lut = reinterpret_cast<const uint16_t*>(p.aux + (int64_t)gt.expert[grp] * p.expert_aux_bytes) +
-                            rg * 256;
-      uint32_t v = 0u;
-      if (lane < EPW) {
-        const uint32_t h = lut[warp * EPW + lane];
-        v = h | (h << 16);
-      }
-#pragma unroll
-      for (int j = 0; j < EPW / 4; ++j) {
-        // rows 4j .. 4j+3 of this warp's entries, 8 lanes x 16 bytes per row
-        const int r = 4 * j + (lane >> 3);
-        const uint32_t w = __shfl_sync(0xffffffffu, v, r);
-        sts128(tab + (uint32_t)(warp * EPW + r) * 128u + 16u * (uint32_t)(lane & 7), make_uint4(w, w, w, w));
-      }
-    }
-    if (u + (int64_t)gridDim.x < total) prefetch_unit(u + gridDim.x);
-    __syncthreads();
+    // the next unit's LUT entries, written to the other buffer after this unit's lookups
+    const uint32_t lutv = has_next ? lut_entry(u + grid) : 0u;
+    if (u + 2 * grid < total) prefetch_unit(u + 2 * grid);
 
-    // ---- this warp's rows and K part ----
-    const int rgi = tile * 16 + g;  // row g of the tile within the unit
     const uint8_t* row_g = ubase + (int64_t)min(rgi, nrows - 1) * K + 16 * t;
     const uint8_t* row_h = ubase + (int64_t)min(rgi + 8, nrows - 1) * K + 16 * t;
-    uint32_t xa[NT];
-    bool xon[NT];
+    const uint32_t lb = 128u * (uint32_t)buf + 4u * (uint32_t)lane;
+    uint32_t xa[NTX];
+    bool xon[NTX];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
+    for (int n = 0; n < NTX; ++n) {
       const int col = 8 * n + g;
       xon[n] = col < ncols;
       int xrow = 0;
@@ -176,79 +311,99 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
       }
       xa[n] = xbase + (uint32_t)xrow * p.XS + 32u * (uint32_t)t;
     }
-    // this warp's parts are contiguous in K: chunks [cA, cB), one chunk ahead
-    const int kp0 = (warp >> 1) * PPW;
-    const int64_t cA = kp0 * nch / KP, cB = (kp0 + PPW) * nch / KP;
-    uint4 cg = make_uint4(0u, 0u, 0u, 0u), ch = cg;
-    if (cA < cB && 64 * cA + 16 * t < K) {
-      cg = ldg_stream_128(row_g + 64 * cA);
-      ch = ldg_stream_128(row_h + 64 * cA);
-    }
+    if constexpr (kF) xa[0] = xbase + 16u * (uint32_t)t;
+
 #pragma unroll 1
     for (int part = 0; part < PPW; ++part) {
       const int kp = kp0 + part;
-      const int64_t c0 = kp * nch / KP, c1 = (kp + 1) * nch / KP;
-      float acc[NT][4];
+      const int c0 = kp * nch / KP, c1 = (kp + 1) * nch / KP;
+      float acc[NTX][4];  // batch-1 path: acc[0][0..1] row g, acc[0][2..3] row g+8
 #pragma unroll
-      for (int n = 0; n < NT; ++n)
+      for (int n = 0; n < NTX; ++n)
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[n][q] = 0.0f;
-
-      for (int64_t c = c0; c < c1; ++c) {
-        uint4 ng = make_uint4(0u, 0u, 0u, 0u), nh = ng;
-        if (c + 1 < cB && 64 * (c + 1) + 16 * t < K) {
-          ng = ldg_stream_128(row_g + 64 * (c + 1));
-          nh = ldg_stream_128(row_h + 64 * (c + 1));
+      for (int c = c0; c < c1; ++c) {
+        // the next chunk: this unit's, or the next unit's first
+        uint4 ng, nh;
+        if (c + 1 < cB) {
+          ng = make_uint4(0u, 0u, 0u, 0u);
+          nh = ng;
+          if (64 * (int64_t)(c + 1) + 16 * t < K) {
+            ng = ldg_stream_128(row_g + 64 * (int64_t)(c + 1));
+            nh = ldg_stream_128(row_h + 64 * (int64_t)(c + 1));
+          }
+        } else {
+          first_chunk(u + grid, ng, nh);
         }
-        const bool live = 64 * c + 16 * t < K;  // in-features past K (a last half chunk) stay zero
-        uint4 xr0[NT], xr1[NT];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          xr0[n] = make_uint4(0u, 0u, 0u, 0u);
-          xr1[n] = xr0[n];
-          if (xon[n]) {
-            xr0[n] = lds128(xa[n] + 128u * (uint32_t)c);
-            xr1[n] = lds128(xa[n] + 128u * (uint32_t)c + 16u);
-          }
-        }
-        const uint32_t wg[4] = {cg.x, cg.y, cg.z, cg.w}, wh[4] = {ch.x, ch.y, ch.z, ch.w};
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          uint32_t a0 = 0u, a1 = 0u, a2 = 0u, a3 = 0u;
-          if (live) {
-            a0 = km8_pair<0>(wg[s], tab_l);
-            a2 = km8_pair<2>(wg[s], tab_l);
-            a1 = km8_pair<0>(wh[s], tab_l);
-            a3 = km8_pair<2>(wh[s], tab_l);
-          }
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const uint32_t b0 = s == 0 ? xr0[n].x : s == 1 ? xr0[n].z : s == 2 ? xr1[n].x : xr1[n].z;
-            const uint32_t b1 = s == 0 ? xr0[n].y : s == 1 ? xr0[n].w : s == 2 ? xr1[n].y : xr1[n].w;
-            mma16816(acc[n], a0, a1, a2, a3, b0, b1);
-          }
+        const bool full = 64 * (int64_t)c + 64 <= K;
+        if constexpr (kF) {
+          float ag[2] = {acc[0][0], acc[0][1]}, ah[2] = {acc[0][2], acc[0][3]};
+          if (full)
+            km8_chunk_b1<false>(ag, ah, cg, ch, xa[0], c, lb, sbase, t);
+          else
+            km8_chunk_b1<true>(ag, ah, cg, ch, xa[0], c, lb, sbase, t);
+          acc[0][0] = ag[0];
+          acc[0][1] = ag[1];
+          acc[0][2] = ah[0];
+          acc[0][3] = ah[1];
+        } else {
+          if (full)
+            km8_chunk<NTX, false>(acc, cg, ch, xa, xon, c, lb, sbase, t);
+          else
+            km8_chunk<NTX, true>(acc, cg, ch, xa, xon, c, lb, sbase, t);
         }
         cg = ng;
         ch = nh;
       }
-      // this part's partial sums
+      if constexpr (kF) {
+        red[((kp * 2 + tile) * 2 + 0) * 32 + lane] = acc[0][0] + acc[0][1];
+        red[((kp * 2 + tile) * 2 + 1) * 32 + lane] = acc[0][2] + acc[0][3];
+      } else {
 #pragma unroll
-      for (int n = 0; n < NT; ++n)
+        for (int n = 0; n < NTX; ++n)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) red[(((kp * 2 + tile) * NT + n) * 4 + q) * 32 + lane] = acc[n][q];
+          for (int q = 0; q < 4; ++q)
+            red[(((kp * 2 + tile) * NTX + n) * 4 + q) * 32 + lane] = acc[n][q];
+      }
     }
+    if (cA >= cB) first_chunk(u + grid, cg, ch);  // (no chunks: nothing was loaded ahead)
 
-    // ---- the K parts meet in shared memory, in order ----
+    // The next unit's LUT into the other buffer (its last reader, the
+    // previous unit, passed the previous barrier), then one barrier: this
+    // unit's partial sums and the next table are complete.
+    if (has_next) write_table(lutv, buf ^ 1);
     __syncthreads();
-    if (tid < 256) {
+
+    // ---- the K parts meet, in order (read while the next unit runs) ----
+    if (kF) {
+      if (tid < 32) {
+        // row tid of the unit: tile tid / 16, lanes (g, 0..3) of rows g (rr 0) / g+8 (rr 1)
+        const int tl = tid >> 4, rw = tid & 15, gg = rw & 7, rr = rw >> 3;
+        float v = 0.0f;
+#pragma unroll
+        for (int k = 0; k < KP; ++k)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) v += red[((k * 2 + tl) * 2 + rr) * 32 + gg * 4 + q];  // part, lane order
+        if (tid < nrows) {
+          const int64_t nrow = rg * 32 + tid;
+          if constexpr (AM) {
+            const unsigned long long key = argmax_key(v, nrow);
+            best[0] = key > best[0] ? key : best[0];
+            bcol[0] = 0;
+          } else {
+            p.y[nrow] = v;
+          }
+        }
+      }
+    } else if (tid < 256) {
       // thread: tile tid / 128, accumulator q, lane ln; its column of n-tile n is 8n + 2(ln % 4) + q % 2
       const int tl = tid >> 7, q = (tid >> 5) & 3, ln = tid & 31;
       const int row = tl * 16 + (ln >> 2) + 8 * (q >> 1);
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
+      for (int n = 0; n < NTX; ++n) {
         float v = 0.0f;
 #pragma unroll
-        for (int k = 0; k < KP; ++k) v += red[(((2 * k + tl) * NT + n) * 4 + q) * 32 + ln];  // part order
+        for (int k = 0; k < KP; ++k) v += red[(((2 * k + tl) * NTX + n) * 4 + q) * 32 + ln];  // part order
         const int col = 8 * n + 2 * (ln & 3) + (q & 1);
         if (col < ncols && row < nrows) {
           const int pair = gt.sorted[gstart + col];
@@ -265,7 +420,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
     }
   }
 
-  if constexpr (AM) argmax_finish<NT, kT>(best, bcol, s_best, s_last, p, tid, lane);
+  if constexpr (AM) argmax_finish<NTX, kT>(best, bcol, s_best, s_last, p, tid, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -286,15 +441,22 @@ bool plan_km8(MvParams& p, int num_sms) {
   p.XS = (int)(round_up8(2 * round_up8(p.K, 64), 128) + 16);
   p.n_xrows = p.gather ? (p.x_per_slot ? p.B * p.topk : p.B) : p.B;
   const int nt = p.B > 8 ? 2 : 1;
+  // dense batch 1: the fp32 path (one fp32 row, in its own chunk layout)
+  p.one = (!p.gather && p.B == 1) ? 1 : 0;
+  if (p.one) p.XS = (int)(256 * ((p.K + 63) / 64));
+  const int64_t red_one = p.one ? (int64_t)8 * 2 * 2 * 32 * 4 : (int64_t)8 * 2 * nt * 4 * 32 * 4;  // one buffer
   const int64_t units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
-  const int cand[2][2] = {{8, 2}, {16, 1}};
-  for (int ci = 0; ci < 2; ++ci) {
+  // layouts in order of preference: two 8-warp CTAs per SM, one 16-warp CTA;
+  // two partial-sum buffers, else one
+  const int cand[4][3] = {{8, 2, 2}, {16, 1, 2}, {8, 2, 1}, {16, 1, 1}};
+  for (int ci = 0; ci < 4; ++ci) {
     const int warps = cand[ci][0], ctas = cand[ci][1];
     p.warps = warps;
-    p.off_tab = 0;  // 32 KB
-    p.off_red = 256 * 128;
-    p.off_x = (int)round_up8(p.off_red + (int64_t)8 * 2 * nt * 4 * 32 * 4, 128);  // 8 parts x 2 tiles
+    p.red_bufs = cand[ci][2];
+    p.off_tab = 0;  // 64 KB: 256 rows x 2 buffers x 128 bytes
+    p.off_red = 256 * 256;
+    p.off_x = (int)round_up8(p.off_red + p.red_bufs * red_one, 128);
     const int64_t bytes = p.off_x + (int64_t)p.n_xrows * p.XS;
     if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
       p.smem_bytes = (int)bytes;
@@ -335,6 +497,7 @@ static cudaError_t launch_km8_t(const MvParams& p, cudaStream_t stream) {
 template <bool AM>
 static cudaError_t launch_km8_a(const MvParams& p, cudaStream_t stream) {
   const bool wide = p.warps == 16;
+  if (p.one) return wide ? launch_km8_t<0, 16, AM>(p, stream) : launch_km8_t<0, 8, AM>(p, stream);
   if (p.B > 8) return wide ? launch_km8_t<2, 16, AM>(p, stream) : launch_km8_t<2, 8, AM>(p, stream);
   return wide ? launch_km8_t<1, 16, AM>(p, stream) : launch_km8_t<1, 8, AM>(p, stream);
 }

@@ -52,6 +52,10 @@ def lib():
         L.oracle_int4aff_aux_row_bytes.argtypes = [I64]
         L.oracle_int4aff_aux_row_bytes.restype = I64
         L.oracle_kmeans_int8km.argtypes = [P, I64, I64, I32, P, P, P, U32P]
+        L.oracle_outlier_columns.argtypes = [P, I64, I64, I64, P]
+        L.oracle_encode_int4km_o8.argtypes = [P, I64, I64, I64, I32, P, P, P, P, P, U32P]
+        L.oracle_dequant_int4km_o8.argtypes = [P, P, P, P, P, I64, I64, I64, P]
+        L.oracle_matvec_int4km_o8.argtypes = [P, P, P, P, P, P, I32, I64, I64, I64, P]
         L.oracle_int8km_groups.argtypes = [I64]
         L.oracle_int8km_groups.restype = I64
         L.oracle_dequant.argtypes = [I32, P, P, I64, I64, P]
@@ -60,7 +64,8 @@ def lib():
         L.oracle_num_threads.restype = I32
         L.oracle_set_num_threads.argtypes = [I32]
         for f in ("oracle_encode_fp4", "oracle_encode_int_sym", "oracle_kmeans_int4km", "oracle_encode_int4aff",
-                  "oracle_kmeans_int8km",
+                  "oracle_kmeans_int8km", "oracle_outlier_columns", "oracle_encode_int4km_o8",
+                  "oracle_dequant_int4km_o8", "oracle_matvec_int4km_o8",
                   "oracle_dequant",
                   "oracle_matvec_rows", "oracle_gather_matvec"):
             getattr(L, f).restype = I32
@@ -183,6 +188,54 @@ def kmeans_int8km(W, iters=KMEANS_ITERS, want_sse=False):
     _check(lib().oracle_kmeans_int8km(_p(W), N, K, iters, _p(lut), _p(idx),
                                       _p(sse) if want_sse else None, ctypes.byref(fl)), "kmeans8")
     return (lut, idx, fl.value, sse) if want_sse else (lut, idx, fl.value)
+
+
+def outlier_columns(W, C):
+    """The C columns (ascending, int32) with the largest max |w| (ties: lower index)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    cols = np.zeros(C, np.int32)
+    _check(lib().oracle_outlier_columns(_p(W), N, K, int(C), _p(cols)), "outlier_columns")
+    return cols
+
+
+def encode_int4km_o8(W, C, iters=KMEANS_ITERS, cols=None):
+    """Mixed int4km + int8 outlier columns.  -> (cols int32 [C], lut float16 [N, 16],
+    idx uint8 [N, (K-C)/2], ocodes int8 [N, C], oscales float16 [N, C/32], flags)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    cols = outlier_columns(W, C) if cols is None else _c(cols, np.int32)
+    lut = np.zeros((N, 16), np.float16)
+    idx = np.zeros((N, (K - C) // 2), np.uint8)
+    oc = np.zeros((N, C), np.int8)
+    osc = np.zeros((N, C // 32), np.float16)
+    fl = ctypes.c_uint32(0)
+    _check(lib().oracle_encode_int4km_o8(_p(W), N, K, int(C), int(iters), _p(cols), _p(lut), _p(idx), _p(oc),
+                                         _p(osc), ctypes.byref(fl)), "encode_int4km_o8")
+    return cols, lut, idx, oc, osc, fl.value
+
+
+def dequant_int4km_o8(cols, lut, idx, oc, osc, N, K):
+    C = len(cols)
+    out = np.zeros((N, K), np.float32)
+    args = [_c(a, t) for a, t in ((lut, np.float16), (idx, np.uint8), (oc, np.int8), (osc, np.float16),
+                                  (cols, np.int32))]
+    _check(lib().oracle_dequant_int4km_o8(*[_p(a) for a in args], N, K, C, _p(out)), "dequant_int4km_o8")
+    return out
+
+
+def matvec_int4km_o8(cols, lut, idx, oc, osc, x, N, K):
+    """fp64 r = x Wdq^T for the mixed format.  x float16 [B, K] -> float64 [B, N]."""
+    C = len(cols)
+    x = _c(x, np.float16)
+    if x.ndim == 1:
+        x = x[None]
+    B = x.shape[0]
+    out = np.zeros((B, N), np.float64)
+    args = [_c(a, t) for a, t in ((lut, np.float16), (idx, np.uint8), (oc, np.int8), (osc, np.float16),
+                                  (cols, np.int32))]
+    _check(lib().oracle_matvec_int4km_o8(*[_p(a) for a in args], _p(x), B, N, K, C, _p(out)), "matvec_int4km_o8")
+    return out
 
 
 def dequant(fmt, codes, aux, N, K):

@@ -536,6 +536,139 @@ int oracle_encode_int4aff(const float* W, int64_t N, int64_t K, uint8_t* codes,
 
 /* ------------------------------------------------------------------ */
 /* ------------------------------------------------------------------ */
+/* Mixed int4km + int8 outlier columns                                */
+/* ["Stream D" next steps: a mixed int4 + int8-outlier matvec that     */
+/*  extends the int4km linear, to bridge the 4-bit quality cliff at    */
+/*  about int4 bandwidth; the pages leave the format open]             */
+/* ------------------------------------------------------------------ */
+
+/* Readings where the pages are silent: the outliers are whole input
+ * columns (in-features); the C columns (C % 32 == 0, C < K) with the
+ * largest max_n |W[n, k]| are kept as symmetric int8 (per-block-32 fp16
+ * scales along the C outlier columns, clip list {1.0}); the other K - C
+ * columns, in ascending order, form an int4km matrix (per-row 16-entry
+ * palette).  A column holding Inf/NaN counts as the most outlying.  Ties in
+ * the column maximum go to the lower column index.  cols: the C outlier
+ * columns in ascending order. */
+typedef struct {
+  float m;
+  int64_t k;
+} orc_colmax;
+static int orc_cmp_colmax(const void* a, const void* b) {
+  const orc_colmax* x = (const orc_colmax*)a;
+  const orc_colmax* y = (const orc_colmax*)b;
+  if (x->m != y->m) return (x->m > y->m) ? -1 : 1; /* larger first */
+  return (x->k > y->k) - (x->k < y->k);           /* then lower column */
+}
+static int orc_cmp_i32(const void* a, const void* b) {
+  int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+  return (x > y) - (x < y);
+}
+
+int oracle_outlier_columns(const float* W, int64_t N, int64_t K, int64_t C, int32_t* cols) {
+  if (K % 32 != 0 || N < 1 || C < 0 || C % 32 != 0 || C >= K) return -2;
+  orc_colmax* cm = (orc_colmax*)malloc((size_t)K * sizeof(orc_colmax));
+  for (int64_t k = 0; k < K; k++) {
+    float m = 0.0f;
+    for (int64_t n = 0; n < N; n++) {
+      float a = fabsf(W[n * K + k]);
+      if (!(a <= m)) m = isnan(a) ? INFINITY : a; /* NaN and Inf: the largest */
+    }
+    cm[k].m = m;
+    cm[k].k = k;
+  }
+  qsort(cm, (size_t)K, sizeof(orc_colmax), orc_cmp_colmax);
+  for (int64_t i = 0; i < C; i++) cols[i] = (int32_t)cm[i].k;
+  qsort(cols, (size_t)C, sizeof(int32_t), orc_cmp_i32);
+  free(cm);
+  return 0;
+}
+
+/* Is column k an outlier column (cols ascending, C entries)? */
+static int orc_is_outlier(const int32_t* cols, int64_t C, int64_t k) {
+  int64_t lo = 0, hi = C;
+  while (lo < hi) {
+    int64_t mid = (lo + hi) / 2;
+    if (cols[mid] < k) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo < C && cols[lo] == k;
+}
+
+/* Encode with the given outlier columns: lut fp16 bits [N, 16], idx uint8
+ * [N, (K-C)/2] (the int4km fit of the K-C main columns), ocodes int8 [N, C]
+ * and oscales fp16 bits [N, C/32] (the int8 encode of the outlier
+ * columns). */
+int oracle_encode_int4km_o8(const float* W, int64_t N, int64_t K, int64_t C, int iters,
+                            const int32_t* cols, uint16_t* lut, uint8_t* idx, int8_t* ocodes,
+                            uint16_t* oscales, uint32_t* flags_out) {
+  if (K % 32 != 0 || N < 1 || C < 0 || C % 32 != 0 || C >= K || iters < 0) return -2;
+  int64_t M = K - C;
+  float* Wm = (float*)malloc((size_t)(N * M) * sizeof(float));
+  float* Wo = (float*)malloc((size_t)((N * C) > 0 ? N * C : 1) * sizeof(float));
+  for (int64_t n = 0; n < N; n++) {
+    int64_t jm = 0, jo = 0;
+    for (int64_t k = 0; k < K; k++) {
+      if (orc_is_outlier(cols, C, k)) Wo[n * C + jo++] = W[n * K + k];
+      else Wm[n * M + jm++] = W[n * K + k];
+    }
+  }
+  uint32_t f1 = 0, f2 = 0;
+  int rc = oracle_kmeans_int4km(Wm, N, M, iters, lut, idx, NULL, &f1);
+  if (rc == 0 && C > 0) {
+    const float one = 1.0f;
+    rc = oracle_encode_int_sym(Wo, N, C, 127, &one, 1, (uint8_t*)ocodes, oscales, &f2);
+  }
+  free(Wm);
+  free(Wo);
+  if (flags_out) *flags_out = f1 | f2;
+  return rc;
+}
+
+/* Wdq fp32 [N, K]: main columns from the palette, outlier columns q * s. */
+int oracle_dequant_int4km_o8(const uint16_t* lut, const uint8_t* idx, const int8_t* ocodes,
+                             const uint16_t* oscales, const int32_t* cols, int64_t N, int64_t K,
+                             int64_t C, float* Wdq) {
+  if (K % 32 != 0 || N < 0 || C < 0 || C % 32 != 0 || C >= K) return -2;
+  int64_t M = K - C;
+  for (int64_t n = 0; n < N; n++) {
+    int64_t jm = 0, jo = 0;
+    for (int64_t k = 0; k < K; k++) {
+      if (orc_is_outlier(cols, C, k)) {
+        float s = orc_f16_to_f32(oscales[n * (C / 32) + jo / 32]);
+        Wdq[n * K + k] = (float)ocodes[n * C + jo] * s;
+        jo++;
+      } else {
+        uint8_t byte = idx[n * (M / 2) + jm / 2];
+        int e = (jm % 2) ? (byte >> 4) : (byte & 15);
+        Wdq[n * K + k] = orc_f16_to_f32(lut[n * 16 + e]);
+        jm++;
+      }
+    }
+  }
+  return 0;
+}
+
+/* r[b, n] = sum_k double(x[b, k]) * double(Wdq[n, k]), k ascending. */
+int oracle_matvec_int4km_o8(const uint16_t* lut, const uint8_t* idx, const int8_t* ocodes,
+                            const uint16_t* oscales, const int32_t* cols, const uint16_t* x, int B,
+                            int64_t N, int64_t K, int64_t C, double* r) {
+  if (K % 32 != 0 || N < 0 || B < 1 || C < 0 || C % 32 != 0 || C >= K) return -2;
+  float* Wdq = (float*)malloc((size_t)(N > 0 ? N * K : 1) * sizeof(float));
+  int rc = oracle_dequant_int4km_o8(lut, idx, ocodes, oscales, cols, N, K, C, Wdq);
+  for (int64_t n = 0; rc == 0 && n < N; n++) {
+    for (int b = 0; b < B; b++) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; k++)
+        acc += (double)orc_f16_to_f32(x[(int64_t)b * K + k]) * (double)Wdq[n * K + k];
+      r[(int64_t)b * N + n] = acc;
+    }
+  }
+  free(Wdq);
+  return rc;
+}
+
+/* ------------------------------------------------------------------ */
 /* Dequantization (exact in float) and the fp64 matvec                */
 /* ------------------------------------------------------------------ */
 

@@ -36,6 +36,9 @@ MUTANTS = {
                                                  "(uint8_t)orc_nearest(c, 256, (double)w[i]);"),
     "int8km last partial group dropped": ("return (N + ORC_KM8_GROUP - 1) / ORC_KM8_GROUP;",
                                           "return N / ORC_KM8_GROUP;"),
+    "outlier columns by the smallest maximum": ("if (x->m != y->m) return (x->m > y->m) ? -1 : 1;",
+                                                "if (x->m != y->m) return (x->m > y->m) ? 1 : -1;"),
+    "outlier dequant with the first scale only": ("oscales[n * (C / 32) + jo / 32]", "oscales[n * (C / 32)]"),
 }
 
 

@@ -610,6 +610,79 @@ def test_int8km_error_below_int4km_page_band(orc):
 
 
 # --------------------------------------------------------------------------
+# mixed int4km + int8 outlier columns
+# --------------------------------------------------------------------------
+
+def _outlier_weights(N, K, cols, seed):
+    g = np.random.default_rng(seed)
+    W = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[:, cols] *= 20.0
+    return W
+
+
+def test_outlier_columns_brute_force_and_planted(orc):
+    N, K = 24, 256
+    g = np.random.default_rng(3)
+    W = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[:, 17] = W[:, 200]  # equal column maxima: the lower index goes first
+    W[5, 99] = np.nan     # a non-finite column counts as the most outlying
+    for C in (0, 32, 64):
+        got = orc.outlier_columns(W, C)
+        m = np.abs(W.astype(np.float64)).max(axis=0)
+        m = np.where(np.isnan(np.abs(W)).any(axis=0), np.inf, m)
+        order = np.lexsort((np.arange(K), -m))  # largest maximum first, then lower index
+        assert np.array_equal(got, np.sort(order[:C]).astype(np.int32)), C
+    planted = np.sort(np.random.default_rng(4).choice(K, 32, replace=False))
+    Wp = _outlier_weights(N, K, planted, 5)
+    assert np.array_equal(orc.outlier_columns(Wp, 32), planted)
+
+
+def test_int4km_o8_parts_and_special_cases(orc):
+    """The main part is the int4km fit of the remaining columns in order, the
+    outlier part the int8 encode of the outlier columns in order; C = 0 is
+    plain int4km; the dequantized matrix puts each part back in its columns."""
+    N, K, C = 40, 320, 64
+    cols = np.sort(np.random.default_rng(6).choice(K, C, replace=False)).astype(np.int32)
+    W = _outlier_weights(N, K, cols, 7)
+    c, lut, idx, oc, osc, fl = orc.encode_int4km_o8(W, C)
+    assert fl == 0 and np.array_equal(c, cols)
+    main = np.setdiff1d(np.arange(K), cols)
+    lut_m, idx_m, _ = orc.kmeans_int4km(W[:, main])
+    assert np.array_equal(lut, lut_m) and np.array_equal(idx, idx_m)
+    oc_r, osc_r, _ = orc.encode_int8(W[:, cols])
+    assert np.array_equal(oc, oc_r) and np.array_equal(osc.view(np.uint16), osc_r.view(np.uint16))
+    D = orc.dequant_int4km_o8(c, lut, idx, oc, osc, N, K)
+    e = np.empty((N, K - C), np.int64)
+    e[:, 0::2], e[:, 1::2] = idx & 15, idx >> 4
+    assert np.array_equal(D[:, main], lut.astype(np.float32)[np.arange(N)[:, None], e])
+    sc = np.repeat(osc.astype(np.float32), 32, axis=1)
+    assert np.array_equal(D[:, cols], oc.astype(np.float32) * sc)
+    # no outliers: plain int4km
+    c0, lut0, idx0, _, _, _ = orc.encode_int4km_o8(W, 0)
+    lut4, idx4, _ = orc.kmeans_int4km(W)
+    assert len(c0) == 0 and np.array_equal(lut0, lut4) and np.array_equal(idx0, idx4)
+    D0 = orc.dequant_int4km_o8(c0, lut0, idx0, np.zeros((N, 0), np.int8), np.zeros((N, 0), np.float16), N, K)
+    assert np.array_equal(D0, orc.dequant(orc.FMT_INT4KM, idx4, lut4, N, K))
+
+
+def test_int4km_o8_matvec_and_error(orc):
+    """The matvec is x Wdq^T; on weights with 32 outlier columns (x20) the
+    mixed format's weight error is far below plain int4km's."""
+    N, K, C = 64, 512, 32
+    cols = np.sort(np.random.default_rng(8).choice(K, C, replace=False)).astype(np.int32)
+    W = _outlier_weights(N, K, cols, 9)
+    c, lut, idx, oc, osc, _ = orc.encode_int4km_o8(W, C)
+    D = orc.dequant_int4km_o8(c, lut, idx, oc, osc, N, K).astype(np.float64)
+    x = RNG.standard_normal((3, K)).astype(np.float16)
+    r = orc.matvec_int4km_o8(c, lut, idx, oc, osc, x, N, K)
+    assert np.allclose(r, x.astype(np.float64) @ D.T, rtol=1e-12, atol=1e-15)
+    lut4, idx4, _ = orc.kmeans_int4km(W)
+    e_mixed = np.linalg.norm(D - W) / np.linalg.norm(W)
+    e_km = np.linalg.norm(orc.dequant(orc.FMT_INT4KM, idx4, lut4, N, K) - W) / np.linalg.norm(W)
+    assert e_mixed * 3 < e_km, (e_mixed, e_km)
+
+
+# --------------------------------------------------------------------------
 # matvec and gather
 # --------------------------------------------------------------------------
 

@@ -198,6 +198,45 @@ qmv_status qmv_matvec_int8km(const uint8_t* idx, const uint16_t* lut, const uint
                              int64_t N, int64_t K, float* y, void* stream);
 
 /* ---------------------------------------------------------------------
+ * Mixed int4km + int8 outlier columns ("Stream D", next steps: a mixed
+ * int4 + int8-outlier matvec extending the int4km linear; the format is
+ * the pages' open question, the reading taken here):
+ *   the C input columns (C % 32 == 0, 0 <= C < K) with the largest
+ *   max_n |W[n, k]| (Inf/NaN the largest; ties to the lower column) are
+ *   symmetric int8 with per-block-32 fp16 scales along the outlier columns
+ *   (clip 1.0); the other K - C columns, ascending, are an int4km matrix.
+ *   y[b, n] = sum_{k main} x[b, k] lut[n][idx] + sum_{k outlier} x[b, k] q s
+ * Arrays: cols int32 [C] (ascending), lut fp16 [N, 16], idx uint8
+ * [N, (K-C)/2], ocodes int8 [N, C], oscales fp16 [N, C/32].  Workspaces
+ * are caller-owned device memory (16-byte aligned) of the sizes below.
+ * --------------------------------------------------------------------- */
+
+/* Bytes of the workspace of qmv_encode_int4km_o8 / qmv_matvec_int4km_o8. */
+int64_t qmv_int4km_o8_encode_workspace_bytes(int64_t N, int64_t K, int64_t C);
+int64_t qmv_int4km_o8_matvec_workspace_bytes(int B, int64_t K, int64_t C);
+
+/* The C outlier columns of W fp32 [N, K] into cols (ascending).
+ * workspace: at least 8 * K bytes. */
+qmv_status qmv_outlier_columns(const float* W, int64_t N, int64_t K, int64_t C, int32_t* cols,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Encode: the outlier columns (written to cols), the int4km fit of the main
+ * columns (qmv_encode_int4km, `iters` Lloyd steps) and the int8 encode of
+ * the outlier columns.  K - C <= 16384. */
+qmv_status qmv_encode_int4km_o8(const float* W, int64_t N, int64_t K, int64_t C, int iters,
+                                int32_t* cols, uint16_t* lut, uint8_t* idx, int8_t* ocodes,
+                                uint16_t* oscales, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* y fp32 [B, N] for x fp16 [B, K]: the activations are split by column
+ * (workspace), the int4km kernel writes y from the main columns and the
+ * int8 kernel adds the outlier columns.  Three launches on `stream`. */
+qmv_status qmv_matvec_int4km_o8(const uint8_t* idx, const uint16_t* lut, const int8_t* ocodes,
+                                const uint16_t* oscales, const int32_t* cols, const uint16_t* x,
+                                int B, int64_t N, int64_t K, int64_t C, void* workspace,
+                                size_t workspace_bytes, float* y, void* stream);
+
+/* ---------------------------------------------------------------------
  * Fused matvec + argmax (greedy next token from the lm_head; the pages'
  * fused head+argmax kernel: "coreai-optimization (coreai-opt) reference",
  * sec. "The LM head + embeddings").  For each activation row b computes

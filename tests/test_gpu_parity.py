@@ -731,3 +731,103 @@ def test_full_decode_step_int4km(q, B):
                                len(rows), K)
                 assert rel_err(y[b, j][rows][None], r) < TOL, (name, b, j)
     assert q.status_fetch() == 0
+
+
+# ---------------------------------------------------------------------------
+# mixed int4km + int8 outlier columns
+# ---------------------------------------------------------------------------
+
+def _outlier_w(N, K, C, seed):
+    g = np.random.default_rng(seed)
+    W = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    cols = np.sort(g.choice(K, C, replace=False))
+    W[:, cols] *= 20.0
+    return W
+
+
+@pytest.mark.parametrize("N,K,C", [(3000, 256, 32), (40, 4096, 64), (7, 1088, 96), (300, 2048, 0)])
+def test_outlier_columns_exact(q, N, K, C):
+    """The GPU column choice equals the oracle's, with ties, a NaN column and
+    several blocks of the rank kernel."""
+    W = _outlier_w(N, K, max(C, 32), seed=N + K)
+    W[:, 5] = W[:, K - 3]  # equal maxima: the lower column first
+    W[N // 2, 9] = np.nan
+    got = q.outlier_columns(torch.from_numpy(W).cuda(), C).cpu().numpy()
+    assert np.array_equal(got, orc.outlier_columns(W, C))
+    assert q.status_fetch() == 0
+
+
+@pytest.mark.parametrize("N,K,C", [(200, 1088, 64), (33, 544, 32), (64, 2048, 0)])
+def test_encode_int4km_o8_bit_exact(q, N, K, C):
+    W = _outlier_w(N, K, max(C, 32), seed=3 * N + K)
+    cols, lut, idx, oc, osc = q.encode_int4km_o8(torch.from_numpy(W).cuda(), C)
+    c_o, lut_o, idx_o, oc_o, osc_o, f = orc.encode_int4km_o8(W, C)
+    assert f == 0 and q.status_fetch() == 0
+    assert np.array_equal(cols.cpu().numpy(), c_o)
+    assert np.array_equal(lut.cpu().numpy().view(np.uint16), lut_o.view(np.uint16))
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert np.array_equal(oc.cpu().numpy(), oc_o)
+    assert np.array_equal(osc.cpu().numpy().view(np.uint16), osc_o.view(np.uint16))
+
+
+@pytest.mark.parametrize("N,K,C", [(70, 544, 32), (600, 2048, 64), (130, 4096, 128), (17, 96, 64)])
+@pytest.mark.parametrize("B", [1, 3, 9, 16])
+def test_matvec_int4km_o8_parity(q, N, K, C, B):
+    W = _outlier_w(N, K, C, seed=7 * N + K + B)
+    c_o, lut_o, idx_o, oc_o, osc_o, _ = orc.encode_int4km_o8(W, C)
+    x = synth.activations(B, K, synth.generator(N + B, "cpu")).numpy()
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    y = q.matvec_int4km_o8(t(c_o), t(lut_o), t(idx_o), t(oc_o), t(osc_o), t(x)).cpu().numpy()
+    r = orc.matvec_int4km_o8(c_o, lut_o, idx_o, oc_o, osc_o, x, N, K)
+    assert rel_err(y, r) < TOL
+    assert q.status_fetch() == 0
+
+
+def test_matvec_int4km_o8_no_outliers_is_int4km(q):
+    N, K, B = 300, 2048, 2
+    W = _outlier_w(N, K, 32, seed=51)
+    c_o, lut_o, idx_o, oc_o, osc_o, _ = orc.encode_int4km_o8(W, 0)
+    x = torch.from_numpy(synth.activations(B, K, synth.generator(52, "cpu")).numpy()).cuda()
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    y = q.matvec_int4km_o8(t(c_o), t(lut_o), t(idx_o), t(oc_o), t(osc_o), x)
+    assert torch.equal(y, q.matvec_int4km(t(idx_o), t(lut_o), x))
+
+
+@pytest.mark.slow
+def test_matvec_int4km_o8_full_head_sampled(q):
+    """The 248320 x 2048 head with 64 outlier columns, GPU-encoded (bit-exact
+    with the oracle per row, checked on sampled rows) at batch 1 and 16."""
+    N, K, C = 248320, 2048, 64
+    g = synth.generator(0, "cuda")
+    W, _ = synth.weights(N, K, g, n_outlier_cols=2)
+    cols, lut, idx, oc, osc = q.encode_int4km_o8(W, C)
+    rows = sample_rows(N, n_rand=256)
+    Wr = W[torch.from_numpy(rows).cuda()].cpu().numpy()
+    c_o = orc.outlier_columns(W.cpu().numpy(), C)
+    assert np.array_equal(cols.cpu().numpy(), c_o)
+    _, lut_o, idx_o, oc_o, osc_o, _ = orc.encode_int4km_o8(Wr, C, cols=c_o)
+    assert np.array_equal(lut.cpu().numpy()[rows].view(np.uint16), lut_o.view(np.uint16))
+    assert np.array_equal(idx.cpu().numpy()[rows], idx_o) and np.array_equal(oc.cpu().numpy()[rows], oc_o)
+    x16 = synth.activations(16, K, g)
+    for B in (1, 16):
+        y = q.matvec_int4km_o8(cols, lut, idx, oc, osc, x16[:B]).cpu().numpy()[:, rows]
+        r = orc.matvec_int4km_o8(c_o, lut_o, idx_o, oc_o, osc_o, x16[:B].cpu().numpy(), len(rows), K)
+        assert rel_err(y, r) < TOL
+    assert q.status_fetch() == 0
+
+
+def test_int4km_o8_argument_errors(q):
+    W = torch.zeros(64, 256, device="cuda")
+    with pytest.raises(q.QmvError) as ei:
+        q.outlier_columns(W, 48)  # C % 32 != 0
+    assert ei.value.status == q.ERR_SHAPE
+    with pytest.raises(q.QmvError) as ei:
+        q.outlier_columns(W, 256)  # C == K
+    assert ei.value.status == q.ERR_SHAPE
+    cols, lut, idx, oc, osc = q.encode_int4km_o8(W, 32)
+    x = torch.zeros(1, 256, dtype=torch.float16, device="cuda")
+    ws = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(q.QmvError) as ei:
+        q.matvec_int4km_o8(cols, lut, idx, oc, osc, x, workspace=ws)
+    assert ei.value.status == q.ERR_ARG
+    assert q.status_fetch() == 0

@@ -57,6 +57,11 @@ SIGNATURES = {
     "qmv_matvec_int8": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int4aff": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int8km": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
+    "qmv_int4km_o8_encode_workspace_bytes": [_I64, _I64, _I64],
+    "qmv_int4km_o8_matvec_workspace_bytes": [_I32, _I64, _I64],
+    "qmv_outlier_columns": [_P, _I64, _I64, _I64, _P, _P, ctypes.c_size_t, _P],
+    "qmv_encode_int4km_o8": [_P, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "qmv_matvec_int4km_o8": [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P],
     "qmv_gather_matvec": [_I32, _P, _P, _I32, _I64, _I64, _P, _I32, _I32, _P, _I32, _P, _P],
     "qmv_matvec_argmax": [_I32, _P, _P, _P, _I32, _I64, _I64, _P, ctypes.c_size_t, _P, _P, _P],
     "qmv_argmax_workspace_bytes": [ctypes.POINTER(ctypes.c_size_t)],
@@ -81,7 +86,8 @@ def lib() -> ctypes.CDLL:
             f = getattr(L, name)
             f.argtypes = args
             f.restype = (ctypes.c_char_p if name in ("qmv_last_error", "qmv_version")
-                         else ctypes.c_int64 if name == "qmv_int4aff_aux_row_bytes" else ctypes.c_int)
+                         else ctypes.c_int64 if name.endswith("_bytes") and name != "qmv_argmax_workspace_bytes"
+                         else ctypes.c_int)
         _lib = L
     return _lib
 
@@ -358,6 +364,71 @@ def dequant(fmt: int, codes: torch.Tensor, aux: torch.Tensor, stream=None) -> to
     out = torch.empty((N, K), dtype=torch.float32, device=codes.device)
     _call("qmv_dequant", fmt, _ptr(codes), _ptr(aux), N, K, _ptr(out), _stream(stream))
     return out
+
+
+# ---------------------------------------------------------------- mixed int4km + int8 outlier columns
+
+def outlier_columns(W: torch.Tensor, C: int, stream=None) -> torch.Tensor:
+    """int32 [C]: the C columns of W (float32 [N, K]) with the largest max |w|, ascending."""
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    cols = torch.empty(C, dtype=torch.int32, device=W.device)
+    ws = torch.empty(max(8 * K, 16), dtype=torch.uint8, device=W.device)
+    _call("qmv_outlier_columns", _ptr(W), N, K, int(C), _ptr(cols), _ptr(ws), ws.numel(), _stream(stream))
+    return cols
+
+
+def encode_int4km_o8(W: torch.Tensor, C: int, iters: int = KMEANS_ITERS, stream=None):
+    """W float32 [N, K] -> (cols int32 [C], lut float16 [N, 16], idx uint8 [N, (K-C)/2],
+    ocodes int8 [N, C], oscales float16 [N, C/32])."""
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    dev = W.device
+    cols = torch.empty(C, dtype=torch.int32, device=dev)
+    lut = torch.empty((N, 16), dtype=torch.float16, device=dev)
+    idx = torch.empty((N, (K - C) // 2), dtype=torch.uint8, device=dev)
+    oc = torch.empty((N, C), dtype=torch.int8, device=dev)
+    osc = torch.empty((N, C // 32), dtype=torch.float16, device=dev)
+    nb = int(lib().qmv_int4km_o8_encode_workspace_bytes(N, K, int(C)))
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+    _call("qmv_encode_int4km_o8", _ptr(W), N, K, int(C), int(iters), _ptr(cols), _ptr(lut), _ptr(idx), _ptr(oc),
+          _ptr(osc), _ptr(ws), ws.numel(), _stream(stream))
+    return cols, lut, idx, oc, osc
+
+
+def int4km_o8_workspace(B: int, K: int, C: int, device=None) -> torch.Tensor:
+    """A workspace for matvec_int4km_o8 (reusable; one call at a time)."""
+    nb = int(lib().qmv_int4km_o8_matvec_workspace_bytes(int(B), int(K), int(C)))
+    return torch.empty(max(nb, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def matvec_int4km_o8(cols, lut, idx, oc, osc, x, workspace=None, out=None, stream=None):
+    """y float32 [B, N] = x Wdq^T for the mixed format; x float16 [B, K] (or [K])."""
+    _need(idx, "idx", torch.uint8)
+    _need(lut, "lut", torch.float16)
+    _need(oc, "ocodes", torch.int8)
+    _need(osc, "oscales", torch.float16)
+    _need(cols, "cols", torch.int32)
+    N = idx.shape[0]
+    C = cols.numel()
+    K = 2 * idx.shape[1] + C
+    if tuple(lut.shape) != (N, 16) or tuple(oc.shape) != (N, C) or tuple(osc.shape) != (N, C // 32):
+        raise ValueError("lut / ocodes / oscales shapes do not match idx and cols")
+    squeeze = x.dim() == 1
+    xx = x.unsqueeze(0) if squeeze else x
+    _need(xx, "x", torch.float16)
+    B = xx.shape[0]
+    if xx.shape[1] != K:
+        raise ValueError(f"x has {xx.shape[1]} features, weights have {K}")
+    if workspace is None:
+        workspace = int4km_o8_workspace(B, K, C, idx.device)
+    _need(workspace, "workspace", torch.uint8)
+    if out is None:
+        out = torch.empty((B, N), dtype=torch.float32, device=idx.device)
+    _need(out, "out", torch.float32, (B, N))
+    _call("qmv_matvec_int4km_o8", _ptr(idx), _ptr(lut), _ptr(oc), _ptr(osc), _ptr(cols), _ptr(xx), B, N, K, C,
+          _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream))
+    return out[0] if squeeze else out
 
 
 def set_weight_prefetch(enable: bool) -> None:

@@ -133,7 +133,7 @@ struct ArgmaxOut {
 
 qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
                          int64_t K, float* y, void* stream, bool gather, int E, const int32_t* ids, int topk,
-                         int x_per_slot, const ArgmaxOut* am = nullptr) {
+                         int x_per_slot, const ArgmaxOut* am = nullptr, bool accum = false) {
   if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8KM) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
   QMV_TRY(check_ptr(codes, "codes"));
   if (!aux) return fail(QMV_ERR_ARG, "scales/lut is null");
@@ -177,6 +177,7 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
                 (long long)K);
   p.status = st;
   p.prefetch = (!gather && g_weight_prefetch.load(std::memory_order_relaxed)) ? 1 : 0;
+  p.accum = accum ? 1 : 0;
   if (am) {
     if (N >= (int64_t(1) << 31)) return fail(QMV_ERR_SHAPE, "argmax needs N < 2^31");
     if (!am->ws || (reinterpret_cast<uintptr_t>(am->ws) & 15u)) return fail(QMV_ERR_ARG, "workspace null or not 16-byte aligned");
@@ -281,6 +282,115 @@ qmv_status qmv_matvec_int4aff(const uint8_t* codes, const uint8_t* aux, const ui
 qmv_status qmv_matvec_int8km(const uint8_t* idx, const uint16_t* lut, const uint16_t* x, int B, int64_t N,
                              int64_t K, float* y, void* stream) {
   return matvec_common(QMV_FMT_INT8KM, idx, lut, x, B, N, K, y, stream, false, 0, nullptr, 0, 0);
+}
+
+// ---- mixed int4km + int8 outlier columns ----
+
+static int64_t round256(int64_t v) { return (v + 255) / 256 * 256; }
+
+static qmv_status check_mixed_shape(int64_t N, int64_t K, int64_t C) {
+  QMV_TRY(check_shape(N, K));
+  if (C < 0 || C % 32 != 0 || C >= K)
+    return fail(QMV_ERR_SHAPE, "C must be a multiple of 32 in [0, K) (got %lld)", (long long)C);
+  return QMV_OK;
+}
+
+int64_t qmv_int4km_o8_encode_workspace_bytes(int64_t N, int64_t K, int64_t C) {
+  return round256(4 * N * (K - C)) + round256(4 * N * C) + round256(8 * K);
+}
+
+int64_t qmv_int4km_o8_matvec_workspace_bytes(int B, int64_t K, int64_t C) {
+  return round256(2 * (int64_t)B * (K - C)) + round256(2 * (int64_t)B * C);
+}
+
+qmv_status qmv_outlier_columns(const float* W, int64_t N, int64_t K, int64_t C, int32_t* cols, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  QMV_TRY(check_ptr(W, "W"));
+  QMV_TRY(check_mixed_shape(N, K, C));
+  if (C > 0 && (!cols || (reinterpret_cast<uintptr_t>(cols) & 3u))) return fail(QMV_ERR_ARG, "cols null or misaligned");
+  QMV_TRY(check_ptr(workspace, "workspace"));
+  if (workspace_bytes < (size_t)(8 * K)) return fail(QMV_ERR_ARG, "workspace has %zu bytes, needs %lld",
+                                                     workspace_bytes, (long long)(8 * K));
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  if (C == 0) return QMV_OK;
+  cudaError_t e = qmv::launch_outlier_columns(W, N, K, C, cols, static_cast<int*>(workspace), sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "outlier_columns launch");
+  return QMV_OK;
+}
+
+qmv_status qmv_encode_int4km_o8(const float* W, int64_t N, int64_t K, int64_t C, int iters, int32_t* cols,
+                                uint16_t* lut, uint8_t* idx, int8_t* ocodes, uint16_t* oscales, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  QMV_TRY(check_ptr(W, "W"));
+  QMV_TRY(check_mixed_shape(N, K, C));
+  QMV_TRY(check_ptr(idx, "idx"));
+  if (!lut || (reinterpret_cast<uintptr_t>(lut) & 1u)) return fail(QMV_ERR_ARG, "lut null or misaligned");
+  if (C > 0) {
+    if (!cols || (reinterpret_cast<uintptr_t>(cols) & 3u)) return fail(QMV_ERR_ARG, "cols null or misaligned");
+    QMV_TRY(check_ptr(ocodes, "ocodes"));
+    if (!oscales || (reinterpret_cast<uintptr_t>(oscales) & 1u)) return fail(QMV_ERR_ARG, "oscales null or misaligned");
+  }
+  if (iters < 0 || iters > 1000) return fail(QMV_ERR_ARG, "iters must be in [0, 1000] (got %d)", iters);
+  if (K - C > 16384) return fail(QMV_ERR_UNSUPPORTED, "K - C must be <= 16384 for the palette fit");
+  QMV_TRY(check_ptr(workspace, "workspace"));
+  const int64_t need = qmv_int4km_o8_encode_workspace_bytes(N, K, C);
+  if ((int64_t)workspace_bytes < need)
+    return fail(QMV_ERR_ARG, "workspace has %zu bytes, needs %lld", workspace_bytes, (long long)need);
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* Wmain = reinterpret_cast<float*>(ws);
+  float* Wout = reinterpret_cast<float*>(ws + round256(4 * N * (K - C)));
+  int* keys = reinterpret_cast<int*>(ws + round256(4 * N * (K - C)) + round256(4 * N * C));
+  cudaError_t e = cudaSuccess;
+  if (C > 0) {
+    e = qmv::launch_outlier_columns(W, N, K, C, cols, keys, sms, s);
+    if (e == cudaSuccess) e = qmv::launch_split_f32(W, N, K, cols, C, Wmain, Wout, sms, s);
+  }
+  if (e == cudaSuccess) e = qmv::launch_encode_int4km(C > 0 ? Wmain : W, N, K - C, iters, lut, idx, st, sms, s);
+  if (e == cudaSuccess && C > 0) {
+    qmv::ClipList cl{};
+    cl.v[0] = 1.0f;
+    cl.n = 1;
+    e = qmv::launch_encode_int(127, Wout, N, C, cl, reinterpret_cast<uint8_t*>(ocodes), oscales, st, sms, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "encode_int4km_o8 launch");
+  return QMV_OK;
+}
+
+qmv_status qmv_matvec_int4km_o8(const uint8_t* idx, const uint16_t* lut, const int8_t* ocodes, const uint16_t* oscales,
+                                const int32_t* cols, const uint16_t* x, int B, int64_t N, int64_t K, int64_t C,
+                                void* workspace, size_t workspace_bytes, float* y, void* stream) {
+  QMV_TRY(check_mixed_shape(N, K, C));
+  QMV_TRY(check_ptr(x, "x"));
+  if (B < 1 || B > 16) return fail(QMV_ERR_UNSUPPORTED, "B must be in [1, 16] (got %d)", B);
+  if (C > 0 && (!cols || (reinterpret_cast<uintptr_t>(cols) & 3u))) return fail(QMV_ERR_ARG, "cols null or misaligned");
+  QMV_TRY(check_ptr(workspace, "workspace"));
+  const int64_t need = qmv_int4km_o8_matvec_workspace_bytes(B, K, C);
+  if ((int64_t)workspace_bytes < need)
+    return fail(QMV_ERR_ARG, "workspace has %zu bytes, needs %lld", workspace_bytes, (long long)need);
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* xmain = reinterpret_cast<uint16_t*>(ws);
+  uint16_t* xout = reinterpret_cast<uint16_t*>(ws + round256(2 * (int64_t)B * (K - C)));
+  const uint16_t* xm = x;
+  if (C > 0) {
+    cudaError_t e = qmv::launch_split_f16(x, B, K, cols, C, xmain, xout, sms, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "column split launch");
+    xm = xmain;
+  }
+  // the int4km part writes y; the int8 part adds its outlier columns
+  QMV_TRY(matvec_common(QMV_FMT_INT4KM, idx, lut, xm, B, N, K - C, y, stream, false, 0, nullptr, 0, 0));
+  if (C > 0)
+    QMV_TRY(matvec_common(QMV_FMT_INT8, ocodes, oscales, xout, B, N, C, y, stream, false, 0, nullptr, 0, 0, nullptr,
+                          true));
+  return QMV_OK;
 }
 
 qmv_status qmv_matvec_argmax(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,

@@ -637,7 +637,8 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
         }
       }
     } else {
-      p.y[(int64_t)pair * p.N + n] = v;
+      float* out = p.y + (int64_t)pair * p.N + n;
+      *out = p.accum ? *out + v : v;  // accumulate: add to what the preceding kernel wrote
     }
   };
   float acc[NTX][4];

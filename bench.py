@@ -46,11 +46,18 @@ FORMATS = ("fp4", "int4", "int4km", "int8")
 FALLBACK_HBM_GBS = 6650.0
 
 
+O8_COLS = 64  # outlier columns of the mixed int4km + int8 format in the extra measurement
+
+
 def algorithmic_bytes(fmt: str, N: int, K: int, B: int) -> int:
     """Bytes a matvec must move: packed codes + block scales (or palette) +
     activations (fp16) + outputs (fp32)."""
-    codes = N * K // 2 if fmt != "int8" else N * K
-    aux = {"fp4": N * (K // 32), "int4": N * (K // 32) * 2, "int8": N * (K // 32) * 2, "int4km": N * 16 * 2}[fmt]
+    if fmt == "int4km_o8":  # main int4km columns + int8 outlier columns with scales, the column list
+        C = O8_COLS
+        return N * (K - C) // 2 + N * 16 * 2 + N * C + N * (C // 32) * 2 + C * 4 + B * K * 2 + B * N * 4
+    codes = N * K if fmt in ("int8", "int8km") else N * K // 2
+    aux = {"fp4": N * (K // 32), "int4": N * (K // 32) * 2, "int8": N * (K // 32) * 2, "int4km": N * 16 * 2,
+           "int4aff": N * (2 * (K // 32) + (K // 32 + 1) // 2), "int8km": ((N + 31) // 32) * 256 * 2}[fmt]
     return codes + aux + B * K * 2 + B * N * 4
 
 
@@ -324,6 +331,7 @@ def run_ours(args, rank, world, local_rank):
     dstep = (measure_decode_step(q, ops["int4km"][0], ops["int4km"][1], dev, stream)
              if not args.no_extras and "int4km" in formats else None)
     amax = None if args.no_extras else measure_argmax(q, ops, fmt_id, x, dev, stream, formats)
+    nxt = None if args.no_extras else measure_next_formats(q, x, dev, stream, peak)
 
     # end to end through the C ABI with host buffers: H2D x, the matvecs, D2H y
     e2e = None if args.no_extras else measure_e2e(q, ops, fmt_id, x, dev, stream, formats,
@@ -333,8 +341,55 @@ def run_ours(args, rank, world, local_rank):
         "ms_per_step": ms_step, "value": value, "per_fmt": per_fmt, "roofline": roof, "clocks": clocks,
         "encode_ms": enc_ms, "batches": extra, "e2e": e2e, "bytes_step": bytes_step,
         "gpu_launches": len(formats) * args.steps, "step_us_without_graph": round(plain_us, 2),
-        "decode_step_int4km": dstep, "argmax_b1": amax,
+        "decode_step_int4km": dstep, "argmax_b1": amax, "next_formats": nxt,
     }
+
+
+def measure_next_formats(q, x, dev, stream, peak):
+    """The formats beyond the step's four, on the same head at batch 1 (graphs
+    of 10 launches): affine int4 and the mixed int4km + int8 outlier columns
+    (64), both encoded on the GPU from the same synthetic weights, and int8km
+    (stand-in tables: no GPU fit for 256-entry palettes)."""
+    import torch
+    from weight_only_quantized_qmv_b200 import synth
+    g = synth.generator(0, dev)
+    W, _ = synth.weights(N_HEAD, K_HEAD, g, n_outlier_cols=2)
+    res = {}
+    calls = {}
+    enc = {}
+
+    def timed(fn):
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        r = fn()
+        b.record()
+        torch.cuda.synchronize()
+        return r, a.elapsed_time(b)
+
+    (c4a, a4a), enc["int4aff"] = timed(lambda: q.encode_int4aff(W))
+    o8, enc["int4km_o8"] = timed(lambda: q.encode_int4km_o8(W, O8_COLS))
+    del W
+    torch.cuda.empty_cache()
+    lut8, idx8 = synth.palette_tables8(N_HEAD, K_HEAD, synth.generator(1, dev))
+    if q.status_fetch():
+        raise RuntimeError("encoder status flags")
+    out = torch.empty((1, N_HEAD), dtype=torch.float32, device=dev)
+    ws = q.int4km_o8_workspace(1, K_HEAD, O8_COLS, dev)
+    calls["int4aff"] = lambda: q.matvec_int4aff(c4a, a4a, x, out=out, stream=stream)
+    calls["int8km"] = lambda: q.matvec_int8km(idx8, lut8, x, out=out, stream=stream)
+    calls["int4km_o8"] = lambda: q.matvec_int4km_o8(*o8, x, workspace=ws, out=out, stream=stream)
+    for f, fn in calls.items():
+        gr = capture(fn, stream, 10)
+        us = graph_us(gr, stream, 10, 5)
+        del gr
+        nb = algorithmic_bytes(f, N_HEAD, K_HEAD, 1)
+        gbs = nb / (us * 1e-6) / 1e9
+        res[f] = {"us": round(us, 3), "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
+                  "bytes": nb, "encode_ms": round(enc[f], 2) if f in enc else None}
+    res["int4km_o8"]["launches_per_call"] = 3
+    res["int8km"]["weights"] = "stand-in tables (random indices, sorted N(0, 0.02) palettes)"
+    return res
 
 
 def measure_batches(q, ops, dev, stream):
@@ -578,6 +633,34 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- main
 
+def profile_case(name: str) -> int:
+    """A small case for a profiler: one kernel's matvec on 65536 x 2048
+    weights (larger than L2, a few hundred MB on the device), three launches,
+    batch 1.  Prints one line and exits."""
+    import torch
+    import weight_only_quantized_qmv_b200 as q
+    from weight_only_quantized_qmv_b200 import synth
+    N, K = 65536, K_HEAD
+    g = synth.generator(0, "cuda")
+    x = synth.activations(1, K, g)
+    if name == "int8km":
+        lut, idx = synth.palette_tables8(N, K, g)
+        run = lambda: q.matvec_int8km(idx, lut, x)
+    else:  # int4km_o8
+        W, _ = synth.weights(N, K, g, n_outlier_cols=2)
+        enc = q.encode_int4km_o8(W, O8_COLS)
+        del W
+        ws = q.int4km_o8_workspace(1, K, O8_COLS)
+        run = lambda: q.matvec_int4km_o8(*enc, x, workspace=ws)
+    for _ in range(3):
+        y = run()
+    torch.cuda.synchronize()
+    flags = q.status_fetch()
+    print(json.dumps({"profile_case": name, "N": N, "K": K, "launches": 3, "y_abs_sum": float(y.abs().sum()),
+                      "flags": flags}), flush=True)
+    return 1 if flags else 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -590,7 +673,11 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e and batch-4/16 measurements")
     ap.add_argument("--no-prefetch", action="store_true",
                     help="keep weight reads behind the preceding launch (qmv_set_weight_prefetch(0))")
+    ap.add_argument("--profile-case", choices=("int8km", "int4km_o8"),
+                    help="run one small case for a profiler (65536 x 2048, three launches) and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        return profile_case(args.profile_case)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
@@ -639,7 +726,7 @@ def main():
             "step_us_without_graph": r["step_us_without_graph"], "decode_step_int4km": r["decode_step_int4km"],
             "argmax_b1": r["argmax_b1"],
             "gpu_launches": r["gpu_launches"] * world, "clocks": r["clocks"], "encode_ms": r["encode_ms"],
-            "batch_verify": r["batches"],
+            "batch_verify": r["batches"], "next_formats": r["next_formats"],
         }
         print(json.dumps(out), flush=True)
     if world > 1:

@@ -16,10 +16,9 @@
 //    all 32 banks, so the lookup of lane l reads bank l: one conflict-free
 //    32-bit load per weight whatever the indices.  Two table buffers: the
 //    next unit's LUT is written while this one is read.
-//  * Index bytes go from global memory straight to registers (one 16-byte
-//    load per row and chunk, one chunk ahead); the next unit's index rows are
-//    prefetched into L2 (128-byte lines, spread over the CTA's threads)
-//    while this one is computed.
+//  * Index bytes go from global memory straight to registers (16-byte loads,
+//    one chunk ahead, across unit boundaries).  Explicit L2 prefetches of
+//    the next units' rows (line or bulk) measured slower and are not used.
 //  * The looked-up fp16 values form the m16n8k16 A fragments directly: lane
 //    (g, t) owns in-features 16t..16t+15 of a chunk, word s of its bytes is
 //    the A operand of MMA step s, so the activations stay in natural order.
@@ -39,8 +38,6 @@ __device__ __forceinline__ uint4 ldg_stream_128(const void* p) {
                : "l"(p));
   return v;
 }
-// L2 prefetch of the line holding p
-__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // The LUT table: 256 rows of 256 bytes at the start of the dynamic shared
 // memory; row c holds entry c of buffer 0 in words 0..31 and of buffer 1 in
@@ -95,36 +92,9 @@ __device__ __forceinline__ void km8_chunk(float (&acc)[NT][4], const uint4& cg, 
   }
 }
 
-// Batch 1 (dense): no tensor cores.  The table holds fp32 values and the
-// activations are staged as fp32, 16 per lane and chunk (chunk c of the
-// staged row: 256 bytes, the 16 bytes of lane quarter t and word i at
-// 64 i + 16 t, so the four quarters of a load are conflict-free).  Each
-// weight is one byte permute, one shared load and one fp32 fma; the even
-// and odd in-features of a row accumulate separately (shorter chains).
-template <bool PARTIAL>
-__device__ __forceinline__ void km8_chunk_b1(float (&ag)[2], float (&ah)[2], const uint4& cg, const uint4& ch,
-                                             uint32_t xa, int64_t c, uint32_t lb, uint32_t tb, int t) {
-  if (PARTIAL && t >= 2) return;
-  const uint32_t wg[4] = {cg.x, cg.y, cg.z, cg.w}, wh[4] = {ch.x, ch.y, ch.z, ch.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 xv = lds128(xa + 256u * (uint32_t)c + 64u * (uint32_t)i);
-    const float x0 = __uint_as_float(xv.x), x1 = __uint_as_float(xv.y);
-    const float x2 = __uint_as_float(xv.z), x3 = __uint_as_float(xv.w);
-    ag[0] = fmaf(__uint_as_float(km8_lookup<0>(wg[i], lb, tb)), x0, ag[0]);
-    ah[0] = fmaf(__uint_as_float(km8_lookup<0>(wh[i], lb, tb)), x0, ah[0]);
-    ag[1] = fmaf(__uint_as_float(km8_lookup<1>(wg[i], lb, tb)), x1, ag[1]);
-    ah[1] = fmaf(__uint_as_float(km8_lookup<1>(wh[i], lb, tb)), x1, ah[1]);
-    ag[0] = fmaf(__uint_as_float(km8_lookup<2>(wg[i], lb, tb)), x2, ag[0]);
-    ah[0] = fmaf(__uint_as_float(km8_lookup<2>(wh[i], lb, tb)), x2, ah[0]);
-    ag[1] = fmaf(__uint_as_float(km8_lookup<3>(wg[i], lb, tb)), x3, ag[1]);
-    ah[1] = fmaf(__uint_as_float(km8_lookup<3>(wh[i], lb, tb)), x3, ah[1]);
-  }
-}
-
-// NT: activation n-tiles of 8 columns (1 or 2), or 0: dense batch 1 on the
-// fp32 path above.  WARPS: 8 (two CTAs per SM) or 16 (one CTA per SM, when
-// the staged activations are large).
+// NT: activation n-tiles of 8 columns (1 or 2).  WARPS: 8 (two CTAs per SM)
+// or 16 (one CTA per SM, when the staged activations are large).  Dense
+// batch 1 runs km8b1_kernel below.
 //
 // Per unit, with one barrier: the next unit's LUT entries are requested at
 // the start (registers) and written to the other table buffer at the end;
@@ -136,10 +106,9 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
   constexpr int kT = 32 * WARPS;
   constexpr int KP = 8;                  // K parts per unit
   constexpr int PPW = KP / (WARPS / 2);  // parts per warp
-  constexpr bool kF = NT == 0;           // the batch-1 fp32 path
-  constexpr int NTX = kF ? 1 : NT;
+  constexpr int NTX = NT;
   constexpr int EPW = 256 / WARPS;       // LUT entries per warp in a table build
-  constexpr int kRedFloats = kF ? KP * 2 * 2 * 32 : KP * 2 * NTX * 4 * 32;  // one partial-sum buffer
+  constexpr int kRedFloats = KP * 2 * NTX * 4 * 32;  // one partial-sum buffer
   __shared__ GroupTable gt;
   __shared__ int s_ids[kMaxPairs];
   __shared__ int s_nvalid;
@@ -150,7 +119,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
   const int g = lane >> 2, t = lane & 3;
   const uint32_t sbase = smem_addr(km8_smem);  // the LUT table: [256][2 buffers][32] words
   const uint32_t xbase = sbase + p.off_x;
-  // partial sums, two buffers of [KP][2 tiles][NT][4][32] (batch-1 path: [KP][2 tiles][2 rows][32])
+  // partial sums, two buffers of [KP][2 tiles][NT][4][32]
   float* red0 = reinterpret_cast<float*>(km8_smem + p.off_red);
   const int64_t K = p.K;
   const int64_t G = p.tiles;  // row groups of 32
@@ -174,14 +143,6 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
     base = p.codes + (int64_t)gt.expert[grp] * p.expert_code_bytes + rg * 32 * K;
     nrows = (int)min((int64_t)32, p.N - rg * 32);
   };
-  auto prefetch_unit = [&](int64_t u) {  // whole CTA; at most 256 KB
-    int64_t rg;
-    int grp, nrows;
-    const uint8_t* base;
-    unit_codes(u, rg, grp, base, nrows);
-    const int64_t bytes = min((int64_t)nrows * K, (int64_t)1 << 18);
-    for (int64_t off = 128 * (int64_t)tid; off < bytes; off += 128 * kT) prefetch_l2(base + off);
-  };
   // this thread's LUT entry of unit u (lanes < EPW), in the table's word format
   auto lut_entry = [&](int64_t u) -> uint32_t {
     int64_t rg;
@@ -193,7 +154,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
     uint32_t v = 0u;
     if (lane < EPW) {
       const uint32_t h = lut[warp * EPW + lane];
-      v = kF ? __float_as_uint(__half2float(__ushort_as_half((unsigned short)h))) : (h | (h << 16));
+      v = h | (h << 16);
     }
     return v;
   };
@@ -208,61 +169,11 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
              make_uint4(w, w, w, w));
     }
   };
-  if ((int64_t)blockIdx.x < total) prefetch_unit(blockIdx.x);  // weights only
-  if ((int64_t)blockIdx.x + grid < total) prefetch_unit(blockIdx.x + grid);
-
-  if (p.prefetch) grid_wait_preceding();
-  if constexpr (kF) {
-    // one fp32 row: in-features 64c + 16t + 4i .. +3 at byte 256c + 64i + 16t,
-    // zero-padded to whole chunks
-    const int64_t n8 = p.XS / 32;  // 8-feature pieces of the padded row
-    for (int64_t j = tid; j < n8; j += kT) {
-      float f[8];
-      if (j < K / 8) {
-        const uint4 v = ldg_nc_128(p.x + 8 * j);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __half2 h = *reinterpret_cast<const __half2*>(&w4[e]);
-          f[2 * e] = __low2float(h);
-          f[2 * e + 1] = __high2float(h);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = 0.0f;
-      }
-      const int64_t k = 8 * j, c = k / 64, tq = (k % 64) / 16, i = (k % 16) / 4;  // i even
-      const uint32_t a = xbase + (uint32_t)(256 * c + 64 * i + 16 * tq);
-      sts128(a, make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3])));
-      sts128(a + 64u, make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]), __float_as_uint(f[6]), __float_as_uint(f[7])));
-    }
-  } else {
-    // activations in natural order, each row zero-padded to whole 64-wide chunks
-    const int64_t per_row = p.XS / 16;  // 16-byte pieces of a staged row
-    const int64_t k16 = K / 8;          // pieces holding activations
-    const int64_t n16 = (int64_t)p.n_xrows * per_row;
-    for (int64_t i = tid; i < n16; i += kT) {
-      const int64_t r = i / per_row, j = i - r * per_row;
-      const uint4 v = j < k16 ? ldg_nc_128(p.x + r * K + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
-      sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
-    }
-  }
-  if ((int64_t)blockIdx.x < total) write_table(lut_entry(blockIdx.x), 0);
-  __syncthreads();  // the first table and the activations
-
   const int tile = warp & 1;
   const int nch = (int)((K + 63) / 64);
   const int kp0 = (warp >> 1) * PPW;
   const int cA = kp0 * nch / KP, cB = (kp0 + PPW) * nch / KP;  // this warp's chunks, every unit
   const int rgi = tile * 16 + g;  // row g of this warp's tile within a unit
-
-  unsigned long long best[NTX];
-  int bcol[NTX];
-#pragma unroll
-  for (int i = 0; i < NTX; ++i) {
-    best[i] = 0ull;
-    bcol[i] = -1;
-  }
 
   // the first chunk of this warp in unit u (zero where past K)
   auto first_chunk = [&](int64_t u, uint4& cg, uint4& ch) {
@@ -277,8 +188,33 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
       ch = ldg_stream_128(base + (int64_t)min(rgi + 8, nrows - 1) * K + 64 * cA + 16 * t);
     }
   };
+  // weights only before the wait (early weight reads): the first index chunk and LUT entries
   uint4 cg, ch;
   first_chunk(blockIdx.x, cg, ch);
+  const uint32_t lut0 = (int64_t)blockIdx.x < total ? lut_entry(blockIdx.x) : 0u;
+
+  if (p.prefetch) grid_wait_preceding();
+  {
+    // activations in natural order, each row zero-padded to whole 64-wide chunks
+    const int64_t per_row = p.XS / 16;  // 16-byte pieces of a staged row
+    const int64_t k16 = K / 8;          // pieces holding activations
+    const int64_t n16 = (int64_t)p.n_xrows * per_row;
+    for (int64_t i = tid; i < n16; i += kT) {
+      const int64_t r = i / per_row, j = i - r * per_row;
+      const uint4 v = j < k16 ? ldg_nc_128(p.x + r * K + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
+      sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
+    }
+  }
+  if ((int64_t)blockIdx.x < total) write_table(lut0, 0);
+  __syncthreads();  // the first table and the activations
+
+  unsigned long long best[NTX];
+  int bcol[NTX];
+#pragma unroll
+  for (int i = 0; i < NTX; ++i) {
+    best[i] = 0ull;
+    bcol[i] = -1;
+  }
 
   int buf = 0;
   for (int64_t u = blockIdx.x; u < total; u += grid, buf ^= 1) {
@@ -293,7 +229,6 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
 
     // the next unit's LUT entries, written to the other buffer after this unit's lookups
     const uint32_t lutv = has_next ? lut_entry(u + grid) : 0u;
-    if (u + 2 * grid < total) prefetch_unit(u + 2 * grid);
 
     const uint8_t* row_g = ubase + (int64_t)min(rgi, nrows - 1) * K + 16 * t;
     const uint8_t* row_h = ubase + (int64_t)min(rgi + 8, nrows - 1) * K + 16 * t;
@@ -311,13 +246,12 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
       }
       xa[n] = xbase + (uint32_t)xrow * p.XS + 32u * (uint32_t)t;
     }
-    if constexpr (kF) xa[0] = xbase + 16u * (uint32_t)t;
 
 #pragma unroll 1
     for (int part = 0; part < PPW; ++part) {
       const int kp = kp0 + part;
       const int c0 = kp * nch / KP, c1 = (kp + 1) * nch / KP;
-      float acc[NTX][4];  // batch-1 path: acc[0][0..1] row g, acc[0][2..3] row g+8
+      float acc[NTX][4];
 #pragma unroll
       for (int n = 0; n < NTX; ++n)
 #pragma unroll
@@ -335,36 +269,17 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
         } else {
           first_chunk(u + grid, ng, nh);
         }
-        const bool full = 64 * (int64_t)c + 64 <= K;
-        if constexpr (kF) {
-          float ag[2] = {acc[0][0], acc[0][1]}, ah[2] = {acc[0][2], acc[0][3]};
-          if (full)
-            km8_chunk_b1<false>(ag, ah, cg, ch, xa[0], c, lb, sbase, t);
-          else
-            km8_chunk_b1<true>(ag, ah, cg, ch, xa[0], c, lb, sbase, t);
-          acc[0][0] = ag[0];
-          acc[0][1] = ag[1];
-          acc[0][2] = ah[0];
-          acc[0][3] = ah[1];
-        } else {
-          if (full)
-            km8_chunk<NTX, false>(acc, cg, ch, xa, xon, c, lb, sbase, t);
-          else
-            km8_chunk<NTX, true>(acc, cg, ch, xa, xon, c, lb, sbase, t);
-        }
+        if (64 * (int64_t)c + 64 <= K)
+          km8_chunk<NTX, false>(acc, cg, ch, xa, xon, c, lb, sbase, t);
+        else
+          km8_chunk<NTX, true>(acc, cg, ch, xa, xon, c, lb, sbase, t);
         cg = ng;
         ch = nh;
       }
-      if constexpr (kF) {
-        red[((kp * 2 + tile) * 2 + 0) * 32 + lane] = acc[0][0] + acc[0][1];
-        red[((kp * 2 + tile) * 2 + 1) * 32 + lane] = acc[0][2] + acc[0][3];
-      } else {
 #pragma unroll
-        for (int n = 0; n < NTX; ++n)
+      for (int n = 0; n < NTX; ++n)
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            red[(((kp * 2 + tile) * NTX + n) * 4 + q) * 32 + lane] = acc[n][q];
-      }
+        for (int q = 0; q < 4; ++q) red[(((kp * 2 + tile) * NTX + n) * 4 + q) * 32 + lane] = acc[n][q];
     }
     if (cA >= cB) first_chunk(u + grid, cg, ch);  // (no chunks: nothing was loaded ahead)
 
@@ -375,27 +290,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
     __syncthreads();
 
     // ---- the K parts meet, in order (read while the next unit runs) ----
-    if (kF) {
-      if (tid < 32) {
-        // row tid of the unit: tile tid / 16, lanes (g, 0..3) of rows g (rr 0) / g+8 (rr 1)
-        const int tl = tid >> 4, rw = tid & 15, gg = rw & 7, rr = rw >> 3;
-        float v = 0.0f;
-#pragma unroll
-        for (int k = 0; k < KP; ++k)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) v += red[((k * 2 + tl) * 2 + rr) * 32 + gg * 4 + q];  // part, lane order
-        if (tid < nrows) {
-          const int64_t nrow = rg * 32 + tid;
-          if constexpr (AM) {
-            const unsigned long long key = argmax_key(v, nrow);
-            best[0] = key > best[0] ? key : best[0];
-            bcol[0] = 0;
-          } else {
-            p.y[nrow] = v;
-          }
-        }
-      }
-    } else if (tid < 256) {
+    if (tid < 256) {
       // thread: tile tid / 128, accumulator q, lane ln; its column of n-tile n is 8n + 2(ln % 4) + q % 2
       const int tl = tid >> 7, q = (tid >> 5) & 3, ln = tid & 31;
       const int row = tl * 16 + (ln >> 2) + 8 * (q >> 1);
@@ -424,6 +319,212 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
 }
 
 // ---------------------------------------------------------------------------
+// Dense batch 1: its own kernel, without tensor cores.  128-wide chunks:
+// lane (g, t) owns in-features 128c + 32t .. +31 of rows g and g+8 (two
+// 16-byte index loads per row), the activations are staged as fp32 with
+// chunk c at byte 512c and the 16 bytes of (word i, quarter t) at
+// 64i + 16t (the quarters of a load are conflict-free), and each pair of
+// weights takes two permutes, two shared loads and one paired fp32 fma
+// (f32x2).  The four lanes of a row add their sums by shuffles before they
+// go to shared memory.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack_f32x2(uint64_t v) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+// per element: d = fma(a, b, c), round to nearest
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// one 128-wide chunk of rows g, g+8 (index words g0/g1, h0/h1 of this lane)
+__device__ __forceinline__ void km8b1_chunk(uint64_t (&acc)[4], const uint4& g0, const uint4& g1, const uint4& h0,
+                                            const uint4& h1, uint32_t xc, uint32_t lb, uint32_t tb) {
+  const uint32_t wg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+  const uint32_t wh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 xv = lds128(xc + 64u * (uint32_t)i);
+    const uint64_t x01 = pack_f32x2(xv.x, xv.y), x23 = pack_f32x2(xv.z, xv.w);
+    acc[0] = fma_f32x2(pack_f32x2(km8_lookup<0>(wg[i], lb, tb), km8_lookup<1>(wg[i], lb, tb)), x01, acc[0]);
+    acc[1] = fma_f32x2(pack_f32x2(km8_lookup<2>(wg[i], lb, tb), km8_lookup<3>(wg[i], lb, tb)), x23, acc[1]);
+    acc[2] = fma_f32x2(pack_f32x2(km8_lookup<0>(wh[i], lb, tb), km8_lookup<1>(wh[i], lb, tb)), x01, acc[2]);
+    acc[3] = fma_f32x2(pack_f32x2(km8_lookup<2>(wh[i], lb, tb), km8_lookup<3>(wh[i], lb, tb)), x23, acc[3]);
+  }
+}
+
+template <int WARPS, bool AM>
+__global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8b1_kernel(const __grid_constant__ MvParams p) {
+  constexpr int kT = 32 * WARPS;
+  constexpr int KP = 8;                  // K parts per unit
+  constexpr int PPW = KP / (WARPS / 2);  // parts per warp
+  constexpr int EPW = 256 / WARPS;       // LUT entries per warp in a table build
+  constexpr int kRedFloats = KP * 2 * 16;  // one partial-sum buffer: [part][tile][16 rows]
+  __shared__ unsigned long long s_best[kMaxCols];
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t sbase = smem_addr(km8_smem);  // the LUT table: [256][2 buffers][32] words (fp32 values)
+  const uint32_t xbase = sbase + p.off_x;
+  float* red0 = reinterpret_cast<float*>(km8_smem + p.off_red);
+  const int64_t K = p.K;
+  const int64_t total = p.tiles;  // row groups of 32
+  const int64_t grid = gridDim.x;
+
+  grid_launch_dependents();
+  if (!p.prefetch) grid_wait_preceding();
+  if (tid < kMaxCols) s_best[tid] = 0ull;
+
+  auto unit_base = [&](int64_t u) { return p.codes + u * 32 * K; };
+  auto unit_rows = [&](int64_t u) { return (int)min((int64_t)32, p.N - u * 32); };
+  auto lut_entry = [&](int64_t u) -> uint32_t {
+    const uint16_t* lut = reinterpret_cast<const uint16_t*>(p.aux) + u * 256;
+    return lane < EPW ? __float_as_uint(__half2float(__ushort_as_half(lut[warp * EPW + lane]))) : 0u;
+  };
+  auto write_table = [&](uint32_t v, int b) {
+#pragma unroll
+    for (int j = 0; j < EPW / 4; ++j) {
+      const int r = 4 * j + (lane >> 3);
+      const uint32_t w = __shfl_sync(0xffffffffu, v, r);
+      sts128(sbase + (uint32_t)(warp * EPW + r) * 256u + 128u * (uint32_t)b + 16u * (uint32_t)(lane & 7),
+             make_uint4(w, w, w, w));
+    }
+  };
+  const int tile = warp & 1;
+  const int nch = (int)((K + 127) / 128);
+  const int kp0 = (warp >> 1) * PPW;
+  const int cA = kp0 * nch / KP, cB = (kp0 + PPW) * nch / KP;  // this warp's chunks, every unit
+  const int rgi = tile * 16 + g;
+  const uint32_t xq = xbase + 16u * (uint32_t)t;
+
+  // index words of this lane for chunk c of unit u (zero where past K)
+  auto load_chunk = [&](int64_t u, int c, uint4& a0, uint4& a1, uint4& b0, uint4& b1) {
+    a0 = a1 = b0 = b1 = make_uint4(0u, 0u, 0u, 0u);
+    if (u < total && 128 * (int64_t)c + 32 * t < K) {
+      const int nr = unit_rows(u);
+      const uint8_t* base = unit_base(u) + 128 * (int64_t)c + 32 * t;
+      const uint8_t* rg_ = base + (int64_t)min(rgi, nr - 1) * K;
+      const uint8_t* rh_ = base + (int64_t)min(rgi + 8, nr - 1) * K;
+      a0 = ldg_stream_128(rg_);
+      a1 = ldg_stream_128(rg_ + 16);
+      b0 = ldg_stream_128(rh_);
+      b1 = ldg_stream_128(rh_ + 16);
+    }
+  };
+  // weights only before the wait (early weight reads): the first index chunk and LUT entries
+  uint4 cg0, cg1, ch0, ch1;
+  load_chunk(blockIdx.x, cA, cg0, cg1, ch0, ch1);
+  const uint32_t lut0 = (int64_t)blockIdx.x < total ? lut_entry(blockIdx.x) : 0u;
+
+  if (p.prefetch) grid_wait_preceding();
+  {
+    // fp32 activations: in-feature k = 128c + 32q + 4i + e at byte 512c + 64i + 16q + 4e,
+    // zero-padded to whole chunks
+    const int64_t n8 = p.XS / 32;  // 8-feature pieces of the padded row
+    for (int64_t j = tid; j < n8; j += kT) {
+      float f[8];
+      if (j < K / 8) {
+        const uint4 v = ldg_nc_128(p.x + 8 * j);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __half2 h = *reinterpret_cast<const __half2*>(&w4[e]);
+          f[2 * e] = __low2float(h);
+          f[2 * e + 1] = __high2float(h);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+      }
+      const int64_t k = 8 * j, c = k / 128, qq = (k % 128) / 32, i = (k % 32) / 4;  // i even
+      const uint32_t a = xbase + (uint32_t)(512 * c + 64 * i + 16 * qq);
+      sts128(a, make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3])));
+      sts128(a + 64u, make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]), __float_as_uint(f[6]), __float_as_uint(f[7])));
+    }
+  }
+  if ((int64_t)blockIdx.x < total) write_table(lut0, 0);
+  __syncthreads();  // the first table and the activations
+
+  unsigned long long best[1] = {0ull};
+  int bcol[1] = {-1};
+
+  int buf = 0;
+  for (int64_t u = blockIdx.x; u < total; u += grid, buf ^= 1) {
+    const int nrows = unit_rows(u);
+    const bool has_next = u + grid < total;
+    float* red = red0 + (p.red_bufs == 2 ? buf : 0) * kRedFloats;
+    if (p.red_bufs == 1) __syncthreads();  // one partial-sum buffer: the previous unit's sums have been read
+    const uint32_t lutv = has_next ? lut_entry(u + grid) : 0u;
+    const uint32_t lb = 128u * (uint32_t)buf + 4u * (uint32_t)lane;
+
+#pragma unroll 1
+    for (int part = 0; part < PPW; ++part) {
+      const int kp = kp0 + part;
+      const int c0 = kp * nch / KP, c1 = (kp + 1) * nch / KP;
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // row g: in-features (4i, 4i+1), (4i+2, 4i+3); row g+8 the same
+      for (int c = c0; c < c1; ++c) {
+        uint4 ng0, ng1, nh0, nh1;
+        if (c + 1 < cB)
+          load_chunk(u, c + 1, ng0, ng1, nh0, nh1);
+        else
+          load_chunk(u + grid, cA, ng0, ng1, nh0, nh1);
+        if (128 * (int64_t)c + 32 * t < K) km8b1_chunk(acc, cg0, cg1, ch0, ch1, xq + 512u * (uint32_t)c, lb, sbase);
+        cg0 = ng0;
+        cg1 = ng1;
+        ch0 = nh0;
+        ch1 = nh1;
+      }
+      // this part's sums of rows g, g+8: lane, then the row's four lanes (fixed order)
+      const float2 a = unpack_f32x2(acc[0]), b = unpack_f32x2(acc[1]);
+      const float2 d = unpack_f32x2(acc[2]), e = unpack_f32x2(acc[3]);
+      float sg = (a.x + a.y) + (b.x + b.y), sh = (d.x + d.y) + (e.x + e.y);
+      sg += __shfl_xor_sync(0xffffffffu, sg, 1);
+      sh += __shfl_xor_sync(0xffffffffu, sh, 1);
+      sg += __shfl_xor_sync(0xffffffffu, sg, 2);
+      sh += __shfl_xor_sync(0xffffffffu, sh, 2);
+      if (t == 0) {
+        red[(kp * 2 + tile) * 16 + g] = sg;
+        red[(kp * 2 + tile) * 16 + g + 8] = sh;
+      }
+    }
+    if (cA >= cB) load_chunk(u + grid, cA, cg0, cg1, ch0, ch1);  // (no chunks: nothing was loaded ahead)
+
+    if (has_next) write_table(lutv, buf ^ 1);
+    __syncthreads();
+
+    if (tid < 32) {  // row tid of the unit: parts in order
+      const int tl = tid >> 4, r16 = tid & 15;
+      float v = 0.0f;
+#pragma unroll
+      for (int k = 0; k < KP; ++k) v += red[(k * 2 + tl) * 16 + r16];
+      if (tid < nrows) {
+        const int64_t nrow = u * 32 + tid;
+        if constexpr (AM) {
+          const unsigned long long key = argmax_key(v, nrow);
+          best[0] = key > best[0] ? key : best[0];
+          bcol[0] = 0;
+        } else {
+          float* out = p.y + nrow;
+          *out = v;
+        }
+      }
+    }
+  }
+
+  if constexpr (AM) argmax_finish<1, kT>(best, bcol, s_best, s_last, p, tid, lane);
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 
@@ -443,8 +544,8 @@ bool plan_km8(MvParams& p, int num_sms) {
   const int nt = p.B > 8 ? 2 : 1;
   // dense batch 1: the fp32 path (one fp32 row, in its own chunk layout)
   p.one = (!p.gather && p.B == 1) ? 1 : 0;
-  if (p.one) p.XS = (int)(256 * ((p.K + 63) / 64));
-  const int64_t red_one = p.one ? (int64_t)8 * 2 * 2 * 32 * 4 : (int64_t)8 * 2 * nt * 4 * 32 * 4;  // one buffer
+  if (p.one) p.XS = (int)(512 * ((p.K + 127) / 128));
+  const int64_t red_one = p.one ? (int64_t)8 * 2 * 16 * 4 : (int64_t)8 * 2 * nt * 4 * 32 * 4;  // one buffer
   const int64_t units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
   // layouts in order of preference: two 8-warp CTAs per SM, one 16-warp CTA;
@@ -494,10 +595,35 @@ static cudaError_t launch_km8_t(const MvParams& p, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, km8_kernel<NT, WARPS, AM>, p);
 }
 
+template <int WARPS, bool AM>
+static cudaError_t launch_km8b1_t(const MvParams& p, cudaStream_t stream) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 64 && !attr_set[dev]) {
+    err = cudaFuncSetAttribute(km8b1_kernel<WARPS, AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSmemLimit - kStaticSmem);
+    if (err != cudaSuccess) return err;
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.grid);
+  cfg.blockDim = dim3(32 * WARPS);
+  cfg.dynamicSmemBytes = (size_t)p.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, km8b1_kernel<WARPS, AM>, p);
+}
+
 template <bool AM>
 static cudaError_t launch_km8_a(const MvParams& p, cudaStream_t stream) {
   const bool wide = p.warps == 16;
-  if (p.one) return wide ? launch_km8_t<0, 16, AM>(p, stream) : launch_km8_t<0, 8, AM>(p, stream);
+  if (p.one) return wide ? launch_km8b1_t<16, AM>(p, stream) : launch_km8b1_t<8, AM>(p, stream);
   if (p.B > 8) return wide ? launch_km8_t<2, 16, AM>(p, stream) : launch_km8_t<2, 8, AM>(p, stream);
   return wide ? launch_km8_t<1, 16, AM>(p, stream) : launch_km8_t<1, 8, AM>(p, stream);
 }

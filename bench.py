@@ -70,13 +70,19 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def csrc_digest() -> str:
+# the sources mv_kernel (the step's kernel) is built from: its counters in
+# profiles/ stay valid while these are unchanged
+MV_KERNEL_SOURCES = ("weight_only_quantized_qmv_b200/csrc/qmv_matvec.cu",
+                     "weight_only_quantized_qmv_b200/csrc/qmv_device.cuh",
+                     "weight_only_quantized_qmv_b200/csrc/qmv_kernel_common.cuh",
+                     "weight_only_quantized_qmv_b200/csrc/qmv_internal.h", "include/qmv.h")
+
+
+def csrc_digest(sources=MV_KERNEL_SOURCES) -> str:
     d = hashlib.sha256()
-    src = os.path.join(ROOT, "weight_only_quantized_qmv_b200", "csrc")
-    for name in sorted(os.listdir(src)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(src, name), "rb") as f:
-                d.update(name.encode() + f.read())
+    for rel in sources:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            d.update(os.path.basename(rel).encode() + f.read())
     return d.hexdigest()[:16]
 
 

@@ -207,13 +207,12 @@ qmv_status qmv_matvec_int8km(const uint8_t* idx, const uint16_t* lut, const uint
  *   (clip 1.0); the other K - C columns, ascending, are an int4km matrix.
  *   y[b, n] = sum_{k main} x[b, k] lut[n][idx] + sum_{k outlier} x[b, k] q s
  * Arrays: cols int32 [C] (ascending), lut fp16 [N, 16], idx uint8
- * [N, (K-C)/2], ocodes int8 [N, C], oscales fp16 [N, C/32].  Workspaces
- * are caller-owned device memory (16-byte aligned) of the sizes below.
+ * [N, (K-C)/2], ocodes int8 [N, C], oscales fp16 [N, C/32].  The encoder's
+ * workspace is caller-owned device memory (16-byte aligned).
  * --------------------------------------------------------------------- */
 
-/* Bytes of the workspace of qmv_encode_int4km_o8 / qmv_matvec_int4km_o8. */
+/* Bytes of the workspace of qmv_encode_int4km_o8. */
 int64_t qmv_int4km_o8_encode_workspace_bytes(int64_t N, int64_t K, int64_t C);
-int64_t qmv_int4km_o8_matvec_workspace_bytes(int B, int64_t K, int64_t C);
 
 /* The C outlier columns of W fp32 [N, K] into cols (ascending).
  * workspace: at least 8 * K bytes. */
@@ -228,13 +227,13 @@ qmv_status qmv_encode_int4km_o8(const float* W, int64_t N, int64_t K, int64_t C,
                                 uint16_t* oscales, void* workspace, size_t workspace_bytes,
                                 void* stream);
 
-/* y fp32 [B, N] for x fp16 [B, K]: the activations are split by column
- * (workspace), the int4km kernel writes y from the main columns and the
- * int8 kernel adds the outlier columns.  Three launches on `stream`. */
+/* y fp32 [B, N] for x fp16 [B, K]: the int4km kernel stages the main
+ * columns of x and writes y; a second kernel adds the outlier columns
+ * (two launches on `stream`, the second a dependent launch).  No
+ * workspace. */
 qmv_status qmv_matvec_int4km_o8(const uint8_t* idx, const uint16_t* lut, const int8_t* ocodes,
                                 const uint16_t* oscales, const int32_t* cols, const uint16_t* x,
-                                int B, int64_t N, int64_t K, int64_t C, void* workspace,
-                                size_t workspace_bytes, float* y, void* stream);
+                                int B, int64_t N, int64_t K, int64_t C, float* y, void* stream);
 
 /* ---------------------------------------------------------------------
  * Fused matvec + argmax (greedy next token from the lm_head; the pages'

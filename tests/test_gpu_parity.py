@@ -783,6 +783,20 @@ def test_matvec_int4km_o8_parity(q, N, K, C, B):
     assert q.status_fetch() == 0
 
 
+def test_matvec_int4km_o8_main_part_staging(q):
+    """With the outlier codes zeroed, the mixed matvec is the int4km kernel
+    on the main columns of x, bit for bit (the kernel's column map)."""
+    N, K, C, B = 300, 2048, 96, 3
+    W = _outlier_w(N, K, C, seed=61)
+    c_o, lut_o, idx_o, oc_o, osc_o, _ = orc.encode_int4km_o8(W, C)
+    x = synth.activations(B, K, synth.generator(62, "cpu")).numpy()
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    y = q.matvec_int4km_o8(t(c_o), t(lut_o), t(idx_o), t(np.zeros_like(oc_o)), t(osc_o), t(x))
+    main = np.setdiff1d(np.arange(K), c_o)
+    y_main = q.matvec_int4km(t(idx_o), t(lut_o), t(x[:, main]))
+    assert torch.equal(y, y_main)
+
+
 def test_matvec_int4km_o8_no_outliers_is_int4km(q):
     N, K, B = 300, 2048, 2
     W = _outlier_w(N, K, 32, seed=51)
@@ -826,8 +840,9 @@ def test_int4km_o8_argument_errors(q):
     assert ei.value.status == q.ERR_SHAPE
     cols, lut, idx, oc, osc = q.encode_int4km_o8(W, 32)
     x = torch.zeros(1, 256, dtype=torch.float16, device="cuda")
-    ws = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ValueError):
+        q.matvec_int4km_o8(cols, lut, idx, oc[:, :16].contiguous(), osc, x)  # outlier codes of the wrong width
     with pytest.raises(q.QmvError) as ei:
-        q.matvec_int4km_o8(cols, lut, idx, oc, osc, x, workspace=ws)
-    assert ei.value.status == q.ERR_ARG
+        q.matvec_int4km_o8(cols, lut, idx, oc, osc, torch.zeros(17, 256, dtype=torch.float16, device="cuda"))
+    assert ei.value.status == q.ERR_UNSUPPORTED  # B > 16
     assert q.status_fetch() == 0

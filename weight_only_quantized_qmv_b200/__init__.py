@@ -58,10 +58,9 @@ SIGNATURES = {
     "qmv_matvec_int4aff": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_matvec_int8km": [_P, _P, _P, _I32, _I64, _I64, _P, _P],
     "qmv_int4km_o8_encode_workspace_bytes": [_I64, _I64, _I64],
-    "qmv_int4km_o8_matvec_workspace_bytes": [_I32, _I64, _I64],
     "qmv_outlier_columns": [_P, _I64, _I64, _I64, _P, _P, ctypes.c_size_t, _P],
     "qmv_encode_int4km_o8": [_P, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
-    "qmv_matvec_int4km_o8": [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P],
+    "qmv_matvec_int4km_o8": [_P, _P, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P],
     "qmv_gather_matvec": [_I32, _P, _P, _I32, _I64, _I64, _P, _I32, _I32, _P, _I32, _P, _P],
     "qmv_matvec_argmax": [_I32, _P, _P, _P, _I32, _I64, _I64, _P, ctypes.c_size_t, _P, _P, _P],
     "qmv_argmax_workspace_bytes": [ctypes.POINTER(ctypes.c_size_t)],
@@ -396,13 +395,7 @@ def encode_int4km_o8(W: torch.Tensor, C: int, iters: int = KMEANS_ITERS, stream=
     return cols, lut, idx, oc, osc
 
 
-def int4km_o8_workspace(B: int, K: int, C: int, device=None) -> torch.Tensor:
-    """A workspace for matvec_int4km_o8 (reusable; one call at a time)."""
-    nb = int(lib().qmv_int4km_o8_matvec_workspace_bytes(int(B), int(K), int(C)))
-    return torch.empty(max(nb, 16), dtype=torch.uint8, device=device or "cuda")
-
-
-def matvec_int4km_o8(cols, lut, idx, oc, osc, x, workspace=None, out=None, stream=None):
+def matvec_int4km_o8(cols, lut, idx, oc, osc, x, out=None, stream=None):
     """y float32 [B, N] = x Wdq^T for the mixed format; x float16 [B, K] (or [K])."""
     _need(idx, "idx", torch.uint8)
     _need(lut, "lut", torch.float16)
@@ -420,14 +413,11 @@ def matvec_int4km_o8(cols, lut, idx, oc, osc, x, workspace=None, out=None, strea
     B = xx.shape[0]
     if xx.shape[1] != K:
         raise ValueError(f"x has {xx.shape[1]} features, weights have {K}")
-    if workspace is None:
-        workspace = int4km_o8_workspace(B, K, C, idx.device)
-    _need(workspace, "workspace", torch.uint8)
     if out is None:
         out = torch.empty((B, N), dtype=torch.float32, device=idx.device)
     _need(out, "out", torch.float32, (B, N))
     _call("qmv_matvec_int4km_o8", _ptr(idx), _ptr(lut), _ptr(oc), _ptr(osc), _ptr(cols), _ptr(xx), B, N, K, C,
-          _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream))
+          _ptr(out), _stream(stream))
     return out[0] if squeeze else out
 
 

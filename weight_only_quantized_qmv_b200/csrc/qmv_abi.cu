@@ -133,7 +133,8 @@ struct ArgmaxOut {
 
 qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint16_t* x, int B, int64_t N,
                          int64_t K, float* y, void* stream, bool gather, int E, const int32_t* ids, int topk,
-                         int x_per_slot, const ArgmaxOut* am = nullptr, bool accum = false) {
+                         int x_per_slot, const ArgmaxOut* am = nullptr, bool accum = false,
+                         const int32_t* xcols = nullptr, int64_t ncols = 0, int64_t xstride = 0) {
   if (fmt < QMV_FMT_FP4 || fmt > QMV_FMT_INT8KM) return fail(QMV_ERR_ARG, "unknown format %d", fmt);
   QMV_TRY(check_ptr(codes, "codes"));
   if (!aux) return fail(QMV_ERR_ARG, "scales/lut is null");
@@ -178,6 +179,9 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
   p.status = st;
   p.prefetch = (!gather && g_weight_prefetch.load(std::memory_order_relaxed)) ? 1 : 0;
   p.accum = accum ? 1 : 0;
+  p.xcols = xcols;
+  p.ncols = ncols;
+  p.xstride = xstride;
   if (am) {
     if (N >= (int64_t(1) << 31)) return fail(QMV_ERR_SHAPE, "argmax needs N < 2^31");
     if (!am->ws || (reinterpret_cast<uintptr_t>(am->ws) & 15u)) return fail(QMV_ERR_ARG, "workspace null or not 16-byte aligned");
@@ -299,10 +303,6 @@ int64_t qmv_int4km_o8_encode_workspace_bytes(int64_t N, int64_t K, int64_t C) {
   return round256(4 * N * (K - C)) + round256(4 * N * C) + round256(8 * K);
 }
 
-int64_t qmv_int4km_o8_matvec_workspace_bytes(int B, int64_t K, int64_t C) {
-  return round256(2 * (int64_t)B * (K - C)) + round256(2 * (int64_t)B * C);
-}
-
 qmv_status qmv_outlier_columns(const float* W, int64_t N, int64_t K, int64_t C, int32_t* cols, void* workspace,
                                size_t workspace_bytes, void* stream) {
   QMV_TRY(check_ptr(W, "W"));
@@ -364,32 +364,26 @@ qmv_status qmv_encode_int4km_o8(const float* W, int64_t N, int64_t K, int64_t C,
 
 qmv_status qmv_matvec_int4km_o8(const uint8_t* idx, const uint16_t* lut, const int8_t* ocodes, const uint16_t* oscales,
                                 const int32_t* cols, const uint16_t* x, int B, int64_t N, int64_t K, int64_t C,
-                                void* workspace, size_t workspace_bytes, float* y, void* stream) {
+                                float* y, void* stream) {
   QMV_TRY(check_mixed_shape(N, K, C));
   QMV_TRY(check_ptr(x, "x"));
   if (B < 1 || B > 16) return fail(QMV_ERR_UNSUPPORTED, "B must be in [1, 16] (got %d)", B);
-  if (C > 0 && (!cols || (reinterpret_cast<uintptr_t>(cols) & 3u))) return fail(QMV_ERR_ARG, "cols null or misaligned");
-  QMV_TRY(check_ptr(workspace, "workspace"));
-  const int64_t need = qmv_int4km_o8_matvec_workspace_bytes(B, K, C);
-  if ((int64_t)workspace_bytes < need)
-    return fail(QMV_ERR_ARG, "workspace has %zu bytes, needs %lld", workspace_bytes, (long long)need);
-  uint32_t* st;
-  int sms;
-  QMV_TRY(device_ctx(&st, &sms));
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint16_t* xmain = reinterpret_cast<uint16_t*>(ws);
-  uint16_t* xout = reinterpret_cast<uint16_t*>(ws + round256(2 * (int64_t)B * (K - C)));
-  const uint16_t* xm = x;
   if (C > 0) {
-    cudaError_t e = qmv::launch_split_f16(x, B, K, cols, C, xmain, xout, sms, (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "column split launch");
-    xm = xmain;
+    if (!cols || (reinterpret_cast<uintptr_t>(cols) & 3u)) return fail(QMV_ERR_ARG, "cols null or misaligned");
+    QMV_TRY(check_ptr(ocodes, "ocodes"));
+    if (!oscales || (reinterpret_cast<uintptr_t>(oscales) & 1u)) return fail(QMV_ERR_ARG, "oscales null or misaligned");
   }
-  // the int4km part writes y; the int8 part adds its outlier columns
-  QMV_TRY(matvec_common(QMV_FMT_INT4KM, idx, lut, xm, B, N, K - C, y, stream, false, 0, nullptr, 0, 0));
-  if (C > 0)
-    QMV_TRY(matvec_common(QMV_FMT_INT8, ocodes, oscales, xout, B, N, C, y, stream, false, 0, nullptr, 0, 0, nullptr,
-                          true));
+  // the int4km kernel stages the main columns of x and writes y; the outlier
+  // kernel adds the int8 columns
+  QMV_TRY(matvec_common(QMV_FMT_INT4KM, idx, lut, x, B, N, K - C, y, stream, false, 0, nullptr, 0, 0, nullptr, false,
+                        C > 0 ? cols : nullptr, C, K));
+  if (C > 0) {
+    uint32_t* st;
+    int sms;
+    QMV_TRY(device_ctx(&st, &sms));
+    cudaError_t e = qmv::launch_outlier_acc(ocodes, oscales, cols, x, B, N, K, C, y, sms, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "outlier columns launch");
+  }
   return QMV_OK;
 }
 

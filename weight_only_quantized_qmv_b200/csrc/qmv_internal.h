@@ -63,7 +63,10 @@ struct MvParams {
   int zoff;                // int4aff: byte offset of the slice's zero points in a staged aux row
   int off_tab;             // int8km: the replicated LUT table (64 KB, two buffers)
   int red_bufs;            // int8km: partial-sum buffers (2, or 1 where shared memory is short)
-  int accum;               // y += result (the int8 part of the mixed format) instead of y = result
+  int accum;               // y += result instead of y = result
+  const int32_t* xcols;    // mixed format: the outlier columns (ascending); x rows hold all columns and
+  int64_t ncols;           //   the kernel stages the K main ones (the others taken out)
+  int64_t xstride;         //   elements per activation row
   int prefetch;            // dense: weights may be read before the preceding grid completes
   int RS;                  // shared-memory bytes per staged code row
   int AS;                  // shared-memory bytes per staged scale row (kAuxRows)
@@ -116,13 +119,15 @@ cudaError_t launch_matvec(int fmt, const MvParams& p, cudaStream_t stream);
 // int8km (dense or gather; p.argmax for the fused argmax): geometry, launch.
 bool plan_km8(MvParams& p, int num_sms);
 // The mixed int4km + int8 outlier-column format: column choice (ws: 2K
-// ints), and the column splits of fp32 weights and fp16 activations.
+// ints) and the column split of fp32 weights.
 cudaError_t launch_outlier_columns(const float* W, int64_t N, int64_t K, int64_t C, int32_t* cols, int* ws,
                                    int num_sms, cudaStream_t stream);
 cudaError_t launch_split_f32(const float* W, int64_t N, int64_t K, const int32_t* cols, int64_t C, float* Wmain,
                              float* Wout, int num_sms, cudaStream_t stream);
-cudaError_t launch_split_f16(const uint16_t* x, int64_t B, int64_t K, const int32_t* cols, int64_t C,
-                             uint16_t* xmain, uint16_t* xout, int num_sms, cudaStream_t stream);
+// y[b, n] += sum over the C outlier columns of x[b, cols[c]] * q[n, c] * s[n, c / 32]
+// (dependent launch: weights read before the wait, y after it).
+cudaError_t launch_outlier_acc(const int8_t* q, const uint16_t* s, const int32_t* cols, const uint16_t* x, int B,
+                               int64_t N, int64_t K, int64_t C, float* y, int num_sms, cudaStream_t stream);
 cudaError_t launch_km8(const MvParams& p, cudaStream_t stream);
 
 // ---- encoders / dequant ------------------------------------------------------

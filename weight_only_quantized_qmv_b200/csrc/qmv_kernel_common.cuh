@@ -34,6 +34,28 @@ __device__ __forceinline__ uint8_t ldg_u8(const uint8_t* p) {
   return (uint8_t)v;
 }
 
+__device__ __forceinline__ uint32_t ldg_u16(const uint16_t* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+// The column of main in-feature j when the C columns in cols (ascending)
+// are taken out: j + m, m = #{i : cols[i] - i <= j} (cols[i] - i, the main
+// columns below outlier i, is non-decreasing).  The result is clamped to the
+// row (width) so a malformed column list cannot address outside it.
+__device__ __forceinline__ int64_t main_column(const int32_t* __restrict__ cols, int64_t C, int64_t j,
+                                               int64_t width) {
+  int64_t lo = 0, hi = C;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi) >> 1;
+    if ((int64_t)__ldg(cols + mid) - mid <= j) lo = mid + 1;
+    else hi = mid;
+  }
+  const int64_t k = j + lo;
+  return k < width ? k : width - 1;
+}
+
 // Programmatic dependent launch: let the next grid in the stream start, and
 // wait for the preceding one to complete (its writes visible).
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }

@@ -581,7 +581,18 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
     const int64_t n16 = (int64_t)p.n_xrows * per_row;
     for (int64_t i = tid; i < n16; i += kT) {
       const int64_t r = i / per_row, j = i - r * per_row;
-      uint4 v = ldg_nc_128(p.x + r * p.K + 8 * j);
+      uint4 v;
+      if (p.xcols) {
+        // the main columns of a wider activation row (the mixed format's
+        // int4km part): in-feature 8j + e is column main_column(8j + e)
+        uint32_t h[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          h[e] = ldg_u16(p.x + r * p.xstride + main_column(p.xcols, p.ncols, 8 * j + e, p.xstride));
+        v = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+      } else {
+        v = ldg_nc_128(p.x + r * p.K + 8 * j);
+      }
       if constexpr (F::kPermX && kOne) {  // (k0,k4), (k2,k6), (k1,k5), (k3,k7)
         v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.y, v.w, 0x5410u), prmt(v.x, v.z, 0x7632u),
                        prmt(v.y, v.w, 0x7632u));

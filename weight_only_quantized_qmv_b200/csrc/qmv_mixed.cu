@@ -1,7 +1,9 @@
 // qmv_mixed.cu -- the mixed int4km + int8 outlier-column format: the choice
-// of outlier columns, the column splits of weights and activations, and
-// the launchers that compose the int4km and int8 kernels ("Stream D", next
-// steps: a mixed int4 + int8-outlier matvec extending the int4km linear).
+// of outlier columns, the column split of the weights for encoding, and the
+// kernel that adds the outlier columns to the int4km kernel's output
+// ("Stream D", next steps: a mixed int4 + int8-outlier matvec extending the
+// int4km linear).  The int4km kernel itself stages the main columns of the
+// activations (MvParams::xcols).
 //
 // Format (the pages leave it open; the reading taken): the C input columns
 // (C % 32 == 0, C < K) with the largest max |w| (Inf/NaN the largest, ties
@@ -117,6 +119,121 @@ __global__ void split_kernel(const T* __restrict__ src, int64_t R, int64_t K, co
   }
 }
 
+// y[b, n] += sum_c x[b, cols[c]] * q[n, c] * s[n, c / 32].  A thread takes
+// one 32-column block of one row (GS threads per row, GS = the block count
+// rounded up to a power of two): the exact products add in fp32, take the
+// block's scale, and the row's threads combine their sums by a fixed
+// shuffle tree.  The outlier activations of the B rows are staged as fp32
+// in shared memory.  Dependent launch: it waits for the kernel that writes
+// y (the int4km part) before reading anything.
+constexpr int kAccThreads = 256;
+constexpr int kAccMaxC = 512;  // outlier columns per launch (<= 16 blocks, <= 33 KB of staged activations)
+
+// BT: a bound on the batch (1, 2, 4, 8 or 16), B <= BT; GS: threads per row
+template <int BT, int GS>
+__global__ void __launch_bounds__(kAccThreads) outlier_acc_kernel(const int8_t* __restrict__ q,
+                                                                  const uint16_t* __restrict__ sc,
+                                                                  const int32_t* __restrict__ cols,
+                                                                  const uint16_t* __restrict__ x, int B, int64_t N,
+                                                                  int64_t K, int64_t C, int64_t c0, int64_t cn,
+                                                                  float* __restrict__ y) {
+  // staged activations [B][cn / 32 blocks][33]: a block's 32 values plus one
+  // pad word, so the GS threads of a row (one block each) read distinct banks
+  extern __shared__ float xs[];
+  const int64_t cst = (cn / 32) * 33;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // y (and the step's inputs) complete
+  for (int64_t i = threadIdx.x; i < (int64_t)B * cn; i += kAccThreads) {
+    const int64_t b = i / cn, c = i - b * cn;
+    int64_t col = cols[c0 + c];
+    col = col < 0 ? 0 : (col >= K ? K - 1 : col);  // a malformed column list stays inside the row
+    xs[b * cst + (c >> 5) * 33 + (c & 31)] = __half2float(__ushort_as_half(x[b * K + col]));
+  }
+  __syncthreads();
+  const int blk = (int)(threadIdx.x % GS);
+  // a grid-stride loop over the rows: the staged activations serve them all
+  for (int64_t t0 = (int64_t)blockIdx.x * kAccThreads; t0 < N * GS; t0 += (int64_t)gridDim.x * kAccThreads) {
+  const int64_t n = (t0 + threadIdx.x) / GS;
+  float acc[BT];
+#pragma unroll
+  for (int b = 0; b < BT; ++b) acc[b] = 0.0f;
+  if (n < N && 32 * blk < cn) {
+    const int8_t* qr = q + n * C + c0 + 32 * blk;
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const uint4 w = *reinterpret_cast<const uint4*>(qr + 16 * v);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float qi = (float)(int8_t)(ws[i / 4] >> (8 * (i % 4)));
+        const int c = 33 * blk + 16 * v + i;
+#pragma unroll
+        for (int b = 0; b < BT; ++b)
+          if (b < B) acc[b] = fmaf(qi, xs[b * cst + c], acc[b]);
+      }
+    }
+    const float s = __half2float(__ushort_as_half(sc[n * (C / 32) + (c0 / 32) + blk]));
+#pragma unroll
+    for (int b = 0; b < BT; ++b) acc[b] *= s;
+  }
+  // the row's GS threads are consecutive lanes: a fixed tree
+#pragma unroll
+  for (int o = 1; o < GS; o *= 2)
+#pragma unroll
+    for (int b = 0; b < BT; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+  if (n < N && blk == 0) {
+#pragma unroll
+    for (int b = 0; b < BT; ++b)
+      if (b < B) y[(int64_t)b * N + n] += acc[b];
+  }
+  }
+}
+
+template <int BT, int GS>
+static cudaError_t launch_acc_t(const int8_t* q, const uint16_t* s, const int32_t* cols, const uint16_t* x, int B,
+                                int64_t N, int64_t K, int64_t C, int64_t c0, int64_t cn, float* y, int num_sms,
+                                cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  const int64_t want = (N * GS + kAccThreads - 1) / kAccThreads, cap = (int64_t)num_sms * 8;
+  cfg.gridDim = dim3((unsigned)(want < cap ? want : cap));
+  cfg.blockDim = dim3(kAccThreads);
+  cfg.dynamicSmemBytes = (size_t)(4 * B * (cn / 32) * 33);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, outlier_acc_kernel<BT, GS>, q, s, cols, x, B, N, K, C, c0, cn, y);
+}
+
+template <int BT>
+static cudaError_t launch_acc_b(const int8_t* q, const uint16_t* s, const int32_t* cols, const uint16_t* x, int B,
+                                int64_t N, int64_t K, int64_t C, int64_t c0, int64_t cn, float* y, int num_sms,
+                                cudaStream_t stream) {
+  const int64_t nb = cn / 32;  // 1..16 blocks
+  if (nb <= 1) return launch_acc_t<BT, 1>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream);
+  if (nb <= 2) return launch_acc_t<BT, 2>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream);
+  if (nb <= 4) return launch_acc_t<BT, 4>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream);
+  if (nb <= 8) return launch_acc_t<BT, 8>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream);
+  return launch_acc_t<BT, 16>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream);
+}
+
+cudaError_t launch_outlier_acc(const int8_t* q, const uint16_t* s, const int32_t* cols, const uint16_t* x, int B,
+                               int64_t N, int64_t K, int64_t C, float* y, int num_sms, cudaStream_t stream) {
+  for (int64_t c0 = 0; c0 < C; c0 += kAccMaxC) {
+    const int64_t cn = C - c0 < kAccMaxC ? C - c0 : kAccMaxC;
+    const cudaError_t e =
+        B <= 1 ? launch_acc_b<1>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream)
+        : B <= 2 ? launch_acc_b<2>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream)
+        : B <= 4 ? launch_acc_b<4>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream)
+        : B <= 8 ? launch_acc_b<8>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream)
+                 : launch_acc_b<16>(q, s, cols, x, B, N, K, C, c0, cn, y, num_sms, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 static int grid_for_n(int64_t n, int threads, int num_sms) {
   const int64_t b = (n + threads - 1) / threads;
   const int64_t cap = (int64_t)num_sms * 16;
@@ -142,10 +259,5 @@ cudaError_t launch_split_f32(const float* W, int64_t N, int64_t K, const int32_t
   return cudaGetLastError();
 }
 
-cudaError_t launch_split_f16(const uint16_t* x, int64_t B, int64_t K, const int32_t* cols, int64_t C,
-                             uint16_t* xmain, uint16_t* xout, int num_sms, cudaStream_t stream) {
-  split_kernel<uint16_t><<<grid_for_n(B * K, 256, num_sms), 256, 0, stream>>>(x, B, K, cols, C, xmain, xout);
-  return cudaGetLastError();
-}
 
 }  // namespace qmv

@@ -526,9 +526,18 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       if (ic == 0) cp_async16(da + (uint32_t)cr * 32u + 16u * ch, asrc);  // the palette rides with the first slice
     } else if (aux_fast) {
       const int sb = (kc / 32) * F::kSB;  // scale bytes per row, a multiple of 8
+      const uint8_t* seg = asrc - 8 * ch;  // row cr's scale segment of this slice
+      if ((reinterpret_cast<uintptr_t>(seg) & 15u) == 0 && sb % 16 == 0) {
+        // 16-byte pieces, the row's two lanes alternating (8-byte copies of
+        // scales cost several times the shared-memory wavefronts)
 #pragma unroll
-      for (int j = 0; j < kAuxSteps; ++j)
-        if (16 * j + 8 * ch < sb) cp_async8(da + (uint32_t)cr * p.AS + 16u * j + 8u * ch, asrc + 16 * j);
+        for (int j = 0; j < kAuxSteps; j += 2)
+          if (16 * (j + ch) < sb) cp_async16(da + (uint32_t)cr * p.AS + 16u * (j + ch), seg + 16 * (j + ch));
+      } else {
+#pragma unroll
+        for (int j = 0; j < kAuxSteps; ++j)
+          if (16 * j + 8 * ch < sb) cp_async8(da + (uint32_t)cr * p.AS + 16u * j + 8u * ch, asrc + 16 * j);
+      }
       asrc += sb;
       if constexpr (F::kZp) {
         const int zb = kc / 64;  // zero-point bytes per row, a multiple of 4

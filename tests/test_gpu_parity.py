@@ -281,15 +281,16 @@ def test_matvec_one_hot_columns_bit_exact(q, fmt):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("N,K", [(100, 512), (37, 2048)])
+@pytest.mark.parametrize("N,K", [(100, 512), (37, 2048), (40, 1056)])
 def test_matvec_batch1_one_hot_bit_exact(q, fmt, N, K):
     """Batch 1 with K a multiple of 256 takes the form whose MMA columns carry
     blocks: x = e_k, one launch per k, must return column k of Wdq exactly
-    (pins the block-to-column and in-block k mapping of that form)."""
+    (pins the block-to-column and in-block k mapping of that form; int8km's
+    batch-1 kernel: its 512-wide chunks, ragged at K = 1056)."""
     c_o, s_o, _ = _inputs(fmt, N, K, 1, seed=23 + K)
     c, s = torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda()
     D = orc.dequant(FID[fmt], c_o, s_o, N, K)
-    for k in [0, 1, 2, 3, 4, 7, 8, 9, 15, 16, 31, 32, 33, 63, 64, 100, 255, 256, 300, K - 1]:
+    for k in [0, 1, 2, 3, 4, 7, 8, 9, 15, 16, 31, 32, 33, 63, 64, 100, 255, 256, 300, K - 33, K - 1]:
         x = torch.zeros((1, K), dtype=torch.float16, device="cuda")
         x[0, k] = 1.0
         y = q.matvec(q.__dict__["FMT_" + fmt.upper()], c, s, x).cpu().numpy()

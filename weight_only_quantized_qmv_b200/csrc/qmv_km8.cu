@@ -319,14 +319,17 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
 }
 
 // ---------------------------------------------------------------------------
-// Dense batch 1: its own kernel, without tensor cores.  128-wide chunks:
-// lane (g, t) owns in-features 128c + 32t .. +31 of rows g and g+8 (two
-// 16-byte index loads per row), the activations are staged as fp32 with
-// chunk c at byte 512c and the 16 bytes of (word i, quarter t) at
-// 64i + 16t (the quarters of a load are conflict-free), and each pair of
-// weights takes two permutes, two shared loads and one paired fp32 fma
-// (f32x2).  The four lanes of a row add their sums by shuffles before they
-// go to shared memory.
+// Dense batch 1: its own kernel, without tensor cores, laid out so that one
+// staged activation load serves eight rows.  512-wide chunks: lane l owns
+// in-features 512c + 16l .. +15 of every row (one 16-byte index load per
+// row), warp w takes rows 8 (w % 4) .. +7 of the unit and K part w / 4 (two
+// parts of whole chunks), and the activations are staged as fp32 with piece
+// j (in-features 4j .. 4j+3 of a lane's 16) of lane l at byte
+// 2048c + 512j + 16l, so a warp's 16-byte activation loads are
+// conflict-free.  Each pair of weights takes two permutes, two shared loads
+// and one paired fp32 fma (f32x2); a part's eight row sums leave the warp
+// through a transposing shuffle reduction (nine shuffles), and the two
+// parts meet in shared memory in part order.
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
@@ -346,34 +349,56 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
   return d;
 }
 
-// one 128-wide chunk of rows g, g+8 (index words g0/g1, h0/h1 of this lane)
-__device__ __forceinline__ void km8b1_chunk(uint64_t (&acc)[4], const uint4& g0, const uint4& g1, const uint4& h0,
-                                            const uint4& h1, uint32_t xc, uint32_t lb, uint32_t tb) {
-  const uint32_t wg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-  const uint32_t wh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+// One row's 16 weights of a chunk (index word w of this lane) against the
+// lane's activation pairs xp (in-features (2i, 2i+1) of its 16).
+__device__ __forceinline__ void km8b1_row(uint64_t& acc, const uint4& w, const uint64_t (&xp)[8], uint32_t lb,
+                                          uint32_t tb) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint4 xv = lds128(xc + 64u * (uint32_t)i);
-    const uint64_t x01 = pack_f32x2(xv.x, xv.y), x23 = pack_f32x2(xv.z, xv.w);
-    acc[0] = fma_f32x2(pack_f32x2(km8_lookup<0>(wg[i], lb, tb), km8_lookup<1>(wg[i], lb, tb)), x01, acc[0]);
-    acc[1] = fma_f32x2(pack_f32x2(km8_lookup<2>(wg[i], lb, tb), km8_lookup<3>(wg[i], lb, tb)), x23, acc[1]);
-    acc[2] = fma_f32x2(pack_f32x2(km8_lookup<0>(wh[i], lb, tb), km8_lookup<1>(wh[i], lb, tb)), x01, acc[2]);
-    acc[3] = fma_f32x2(pack_f32x2(km8_lookup<2>(wh[i], lb, tb), km8_lookup<3>(wh[i], lb, tb)), x23, acc[3]);
+  for (int s = 0; s < 4; ++s) {
+    acc = fma_f32x2(pack_f32x2(km8_lookup<0>(ws[s], lb, tb), km8_lookup<1>(ws[s], lb, tb)), xp[2 * s], acc);
+    acc = fma_f32x2(pack_f32x2(km8_lookup<2>(ws[s], lb, tb), km8_lookup<3>(ws[s], lb, tb)), xp[2 * s + 1], acc);
   }
 }
 
-template <int WARPS, bool AM>
-__global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8b1_kernel(const __grid_constant__ MvParams p) {
-  constexpr int kT = 32 * WARPS;
-  constexpr int KP = 8;                  // K parts per unit
-  constexpr int PPW = KP / (WARPS / 2);  // parts per warp
-  constexpr int EPW = 256 / WARPS;       // LUT entries per warp in a table build
-  constexpr int kRedFloats = KP * 2 * 16;  // one partial-sum buffer: [part][tile][16 rows]
+// Each lane holds one sum of each of 8 rows; returns, in lane l, the sum over
+// the warp of row l / 4 (lanes exchange half of what they hold at each of
+// the first three steps, then add whole values).
+__device__ __forceinline__ float reduce_rows8(const float (&s)[8], int lane) {
+  const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0, h4 = (lane & 4) != 0;
+  float v4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // rows 4 h16 + i
+    const float give = h16 ? s[i] : s[i + 4];
+    const float keep = h16 ? s[i + 4] : s[i];
+    v4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
+  }
+  float v2[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {  // rows 4 h16 + 2 h8 + i
+    const float give = h8 ? v4[i] : v4[i + 2];
+    const float keep = h8 ? v4[i + 2] : v4[i];
+    v2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+  }
+  const float give = h4 ? v2[0] : v2[1];
+  const float keep = h4 ? v2[1] : v2[0];
+  float v = keep + __shfl_xor_sync(0xffffffffu, give, 4);  // row 4 h16 + 2 h8 + h4 = l / 4
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v;
+}
+
+template <bool AM>
+__global__ void __launch_bounds__(256, 2) km8b1_kernel(const __grid_constant__ MvParams p) {
+  constexpr int kT = 256;
+  constexpr int kR = 8;                  // rows per warp
+  constexpr int KP = 2;                  // K parts per unit
+  constexpr int EPW = 256 / 8;           // LUT entries per warp in a table build
+  constexpr int kRedFloats = KP * 32;    // one partial-sum buffer: [part][32 rows]
   __shared__ unsigned long long s_best[kMaxCols];
   __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
   const uint32_t sbase = smem_addr(km8_smem);  // the LUT table: [256][2 buffers][32] words (fp32 values)
   const uint32_t xbase = sbase + p.off_x;
   float* red0 = reinterpret_cast<float*>(km8_smem + p.off_red);
@@ -385,7 +410,6 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8b1_kernel(c
   if (!p.prefetch) grid_wait_preceding();
   if (tid < kMaxCols) s_best[tid] = 0ull;
 
-  auto unit_base = [&](int64_t u) { return p.codes + u * 32 * K; };
   auto unit_rows = [&](int64_t u) { return (int)min((int64_t)32, p.N - u * 32); };
   auto lut_entry = [&](int64_t u) -> uint32_t {
     const uint16_t* lut = reinterpret_cast<const uint16_t*>(p.aux) + u * 256;
@@ -400,35 +424,30 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8b1_kernel(c
              make_uint4(w, w, w, w));
     }
   };
-  const int tile = warp & 1;
-  const int nch = (int)((K + 127) / 128);
-  const int kp0 = (warp >> 1) * PPW;
-  const int cA = kp0 * nch / KP, cB = (kp0 + PPW) * nch / KP;  // this warp's chunks, every unit
-  const int rgi = tile * 16 + g;
-  const uint32_t xq = xbase + 16u * (uint32_t)t;
+  const int rg = warp & 3, part = warp >> 2;
+  const int nch = (int)((K + 511) / 512);
+  const int cA = part * nch / KP, cB = (part + 1) * nch / KP;  // this warp's chunks, every unit
+  const int64_t lk = 16 * (int64_t)lane;                       // this lane's first in-feature of a chunk
 
-  // index words of this lane for chunk c of unit u (zero where past K)
-  auto load_chunk = [&](int64_t u, int c, uint4& a0, uint4& a1, uint4& b0, uint4& b1) {
-    a0 = a1 = b0 = b1 = make_uint4(0u, 0u, 0u, 0u);
-    if (u < total && 128 * (int64_t)c + 32 * t < K) {
-      const int nr = unit_rows(u);
-      const uint8_t* base = unit_base(u) + 128 * (int64_t)c + 32 * t;
-      const uint8_t* rg_ = base + (int64_t)min(rgi, nr - 1) * K;
-      const uint8_t* rh_ = base + (int64_t)min(rgi + 8, nr - 1) * K;
-      a0 = ldg_stream_128(rg_);
-      a1 = ldg_stream_128(rg_ + 16);
-      b0 = ldg_stream_128(rh_);
-      b1 = ldg_stream_128(rh_ + 16);
+  // this lane's index word of row 8 rg + r of unit u, chunk c (zero where
+  // past K or past the units; rows past N repeat the unit's last row)
+  auto load_row = [&](int64_t u, int c, int r) -> uint4 {
+    if (u < total && 512 * (int64_t)c + lk < K) {
+      const int64_t row = u * 32 + min(kR * rg + r, unit_rows(u) - 1);
+      return ldg_stream_128(p.codes + row * K + 512 * (int64_t)c + lk);
     }
+    return make_uint4(0u, 0u, 0u, 0u);
   };
-  // weights only before the wait (early weight reads): the first index chunk and LUT entries
-  uint4 cg0, cg1, ch0, ch1;
-  load_chunk(blockIdx.x, cA, cg0, cg1, ch0, ch1);
+
+  // weights only before the wait (early weight reads): the first chunk's index words and LUT entries
+  uint4 cw[kR];
+#pragma unroll
+  for (int r = 0; r < kR; ++r) cw[r] = cA < cB ? load_row(blockIdx.x, cA, r) : make_uint4(0u, 0u, 0u, 0u);
   const uint32_t lut0 = (int64_t)blockIdx.x < total ? lut_entry(blockIdx.x) : 0u;
 
   if (p.prefetch) grid_wait_preceding();
   {
-    // fp32 activations: in-feature k = 128c + 32q + 4i + e at byte 512c + 64i + 16q + 4e,
+    // fp32 activations: in-feature k = 512c + 16l + 4j + e at byte 2048c + 512j + 16l + 4e,
     // zero-padded to whole chunks
     const int64_t n8 = p.XS / 32;  // 8-feature pieces of the padded row
     for (int64_t j = tid; j < n8; j += kT) {
@@ -446,10 +465,10 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8b1_kernel(c
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = 0.0f;
       }
-      const int64_t k = 8 * j, c = k / 128, qq = (k % 128) / 32, i = (k % 32) / 4;  // i even
-      const uint32_t a = xbase + (uint32_t)(512 * c + 64 * i + 16 * qq);
+      const int64_t k = 8 * j, c = k / 512, l = (k % 512) / 16, q = (k % 16) / 4;  // q even
+      const uint32_t a = xbase + (uint32_t)(2048 * c + 512 * q + 16 * l);
       sts128(a, make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3])));
-      sts128(a + 64u, make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]), __float_as_uint(f[6]), __float_as_uint(f[7])));
+      sts128(a + 512u, make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]), __float_as_uint(f[6]), __float_as_uint(f[7])));
     }
   }
   if ((int64_t)blockIdx.x < total) write_table(lut0, 0);
@@ -467,56 +486,62 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8b1_kernel(c
     const uint32_t lutv = has_next ? lut_entry(u + grid) : 0u;
     const uint32_t lb = 128u * (uint32_t)buf + 4u * (uint32_t)lane;
 
+    uint64_t acc[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) acc[r] = 0ull;
 #pragma unroll 1
-    for (int part = 0; part < PPW; ++part) {
-      const int kp = kp0 + part;
-      const int c0 = kp * nch / KP, c1 = (kp + 1) * nch / KP;
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // row g: in-features (4i, 4i+1), (4i+2, 4i+3); row g+8 the same
-      for (int c = c0; c < c1; ++c) {
-        uint4 ng0, ng1, nh0, nh1;
-        if (c + 1 < cB)
-          load_chunk(u, c + 1, ng0, ng1, nh0, nh1);
-        else
-          load_chunk(u + grid, cA, ng0, ng1, nh0, nh1);
-        if (128 * (int64_t)c + 32 * t < K) km8b1_chunk(acc, cg0, cg1, ch0, ch1, xq + 512u * (uint32_t)c, lb, sbase);
-        cg0 = ng0;
-        cg1 = ng1;
-        ch0 = nh0;
-        ch1 = nh1;
+    for (int c = cA; c < cB; ++c) {
+      const bool on = 512 * (int64_t)c + lk < K;  // the lane's in-features are inside K (else zero padding)
+      uint64_t xp[8];
+      const uint32_t xa = xbase + 2048u * (uint32_t)c + 16u * (uint32_t)lane;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = lds128(xa + 512u * (uint32_t)q);
+        xp[2 * q] = pack_f32x2(v.x, v.y);
+        xp[2 * q + 1] = pack_f32x2(v.z, v.w);
       }
-      // this part's sums of rows g, g+8: lane, then the row's four lanes (fixed order)
-      const float2 a = unpack_f32x2(acc[0]), b = unpack_f32x2(acc[1]);
-      const float2 d = unpack_f32x2(acc[2]), e = unpack_f32x2(acc[3]);
-      float sg = (a.x + a.y) + (b.x + b.y), sh = (d.x + d.y) + (e.x + e.y);
-      sg += __shfl_xor_sync(0xffffffffu, sg, 1);
-      sh += __shfl_xor_sync(0xffffffffu, sh, 1);
-      sg += __shfl_xor_sync(0xffffffffu, sg, 2);
-      sh += __shfl_xor_sync(0xffffffffu, sh, 2);
-      if (t == 0) {
-        red[(kp * 2 + tile) * 16 + g] = sg;
-        red[(kp * 2 + tile) * 16 + g + 8] = sh;
+      // the index words that follow: the next chunk of this part, else the next unit's first
+      const int64_t un = c + 1 < cB ? u : u + grid;
+      const int cn = c + 1 < cB ? c + 1 : cA;
+      const bool ld = un < total && 512 * (int64_t)cn + lk < K;
+      const uint8_t* nb = p.codes + (ld ? un * 32 * K + 512 * (int64_t)cn + lk : 0);
+      const int nlast = ld ? unit_rows(un) - 1 : 0;
+      if (512 * (int64_t)(c + 1) <= K) {  // (uniform) a whole chunk: no per-row branch
+#pragma unroll
+        for (int r = 0; r < kR; ++r) {
+          km8b1_row(acc[r], cw[r], xp, lb, sbase);
+          cw[r] = ld ? ldg_stream_128(nb + (int64_t)min(kR * rg + r, nlast) * K) : make_uint4(0u, 0u, 0u, 0u);
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < kR; ++r) {
+          if (on) km8b1_row(acc[r], cw[r], xp, lb, sbase);
+          cw[r] = ld ? ldg_stream_128(nb + (int64_t)min(kR * rg + r, nlast) * K) : make_uint4(0u, 0u, 0u, 0u);
+        }
       }
     }
-    if (cA >= cB) load_chunk(u + grid, cA, cg0, cg1, ch0, ch1);  // (no chunks: nothing was loaded ahead)
+    // this part's sums of the warp's 8 rows: lane pairs, then the warp (fixed order)
+    float s[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      const float2 a = unpack_f32x2(acc[r]);
+      s[r] = a.x + a.y;
+    }
+    const float v = reduce_rows8(s, lane);
+    if ((lane & 3) == 0) red[part * 32 + kR * rg + (lane >> 2)] = v;
 
     if (has_next) write_table(lutv, buf ^ 1);
     __syncthreads();
 
-    if (tid < 32) {  // row tid of the unit: parts in order
-      const int tl = tid >> 4, r16 = tid & 15;
-      float v = 0.0f;
-#pragma unroll
-      for (int k = 0; k < KP; ++k) v += red[(k * 2 + tl) * 16 + r16];
-      if (tid < nrows) {
-        const int64_t nrow = u * 32 + tid;
-        if constexpr (AM) {
-          const unsigned long long key = argmax_key(v, nrow);
-          best[0] = key > best[0] ? key : best[0];
-          bcol[0] = 0;
-        } else {
-          float* out = p.y + nrow;
-          *out = v;
-        }
+    if (tid < 32 && tid < nrows) {  // row tid of the unit: parts in order
+      const float y = red[tid] + red[32 + tid];
+      const int64_t nrow = u * 32 + tid;
+      if constexpr (AM) {
+        const unsigned long long key = argmax_key(y, nrow);
+        best[0] = key > best[0] ? key : best[0];
+        bcol[0] = 0;
+      } else {
+        p.y[nrow] = y;
       }
     }
   }
@@ -544,22 +569,23 @@ bool plan_km8(MvParams& p, int num_sms) {
   const int nt = p.B > 8 ? 2 : 1;
   // dense batch 1: the fp32 path (one fp32 row, in its own chunk layout)
   p.one = (!p.gather && p.B == 1) ? 1 : 0;
-  if (p.one) p.XS = (int)(512 * ((p.K + 127) / 128));
-  const int64_t red_one = p.one ? (int64_t)8 * 2 * 16 * 4 : (int64_t)8 * 2 * nt * 4 * 32 * 4;  // one buffer
+  if (p.one) p.XS = (int)(2048 * ((p.K + 511) / 512));
+  const int64_t red_one = p.one ? (int64_t)2 * 32 * 4 : (int64_t)8 * 2 * nt * 4 * 32 * 4;  // one buffer
   const int64_t units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
-  // layouts in order of preference: two 8-warp CTAs per SM, one 16-warp CTA;
-  // two partial-sum buffers, else one
+  // layouts in order of preference: two 8-warp CTAs per SM, one 16-warp CTA
+  // (batch 1: one 8-warp CTA); two partial-sum buffers, else one
   const int cand[4][3] = {{8, 2, 2}, {16, 1, 2}, {8, 2, 1}, {16, 1, 1}};
   for (int ci = 0; ci < 4; ++ci) {
-    const int warps = cand[ci][0], ctas = cand[ci][1];
+    const int warps = p.one ? 8 : cand[ci][0], ctas = cand[ci][1];
     p.warps = warps;
     p.red_bufs = cand[ci][2];
     p.off_tab = 0;  // 64 KB: 256 rows x 2 buffers x 128 bytes
     p.off_red = 256 * 256;
     p.off_x = (int)round_up8(p.off_red + p.red_bufs * red_one, 128);
     const int64_t bytes = p.off_x + (int64_t)p.n_xrows * p.XS;
-    if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
+    const int64_t stat = p.one ? 1024 : kStaticSmem;  // the batch-1 kernel's static shared memory is the argmax keys
+    if (bytes <= dyn_limit && ctas * (bytes + stat + 1024) <= kSmemPerSM) {
       p.smem_bytes = (int)bytes;
       p.ctas_per_sm = ctas;
       const int64_t slots = (int64_t)num_sms * ctas;
@@ -595,21 +621,21 @@ static cudaError_t launch_km8_t(const MvParams& p, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, km8_kernel<NT, WARPS, AM>, p);
 }
 
-template <int WARPS, bool AM>
+template <bool AM>
 static cudaError_t launch_km8b1_t(const MvParams& p, cudaStream_t stream) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 64 && !attr_set[dev]) {
-    err = cudaFuncSetAttribute(km8b1_kernel<WARPS, AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(km8b1_kernel<AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
     attr_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
-  cfg.blockDim = dim3(32 * WARPS);
+  cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = (size_t)p.smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -617,13 +643,13 @@ static cudaError_t launch_km8b1_t(const MvParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, km8b1_kernel<WARPS, AM>, p);
+  return cudaLaunchKernelEx(&cfg, km8b1_kernel<AM>, p);
 }
 
 template <bool AM>
 static cudaError_t launch_km8_a(const MvParams& p, cudaStream_t stream) {
   const bool wide = p.warps == 16;
-  if (p.one) return wide ? launch_km8b1_t<16, AM>(p, stream) : launch_km8b1_t<8, AM>(p, stream);
+  if (p.one) return launch_km8b1_t<AM>(p, stream);
   if (p.B > 8) return wide ? launch_km8_t<2, 16, AM>(p, stream) : launch_km8_t<2, 8, AM>(p, stream);
   return wide ? launch_km8_t<1, 16, AM>(p, stream) : launch_km8_t<1, 8, AM>(p, stream);
 }

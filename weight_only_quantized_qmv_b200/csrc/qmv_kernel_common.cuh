@@ -40,6 +40,31 @@ __device__ __forceinline__ uint32_t ldg_u16(const uint16_t* p) {
   return v;
 }
 
+// Paired fp32 arithmetic (two lanes of a 64-bit register, each element
+// rounded as its scalar operation would be).
+__device__ __forceinline__ uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack_f32x2(uint64_t v) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+// per element: d = fma(a, b, c), round to nearest
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// per element: d = a - b, round to nearest
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // The column of main in-feature j when the C columns in cols (ascending)
 // are taken out: j + m, m = #{i : cols[i] - i <= j} (cols[i] - i, the main
 // columns below outlier i, is non-decreasing).  The result is clamped to the

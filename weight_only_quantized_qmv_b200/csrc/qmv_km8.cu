@@ -332,23 +332,6 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? 2 : 1) km8_kernel(con
 // parts meet in shared memory in part order.
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 unpack_f32x2(uint64_t v) {
-  uint32_t lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
-  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
-}
-// per element: d = fma(a, b, c), round to nearest
-__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
 // One row's 16 weights of a chunk (index word w of this lane) against the
 // lane's activation pairs xp (in-features (2i, 2i+1) of its 16).
 __device__ __forceinline__ void km8b1_row(uint64_t& acc, const uint4& w, const uint64_t (&xp)[8], uint32_t lb,

@@ -345,20 +345,28 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
         d[2] = fmaf(fmaf(d[2], 16.0f, dh[2]), 1048576.0f, -8.0f * xs.x);
         d[3] = fmaf(fmaf(d[3], 16.0f, dh[3]), 1048576.0f, -8.0f * xs.y);
       } else if constexpr (kSub) {
-        // block partial = 2^20 * (16 * dlo + dhi) - z * sum(x): the scaling by
-        // 2^20 is exact, so one rounding for the sum and one for the fma
-        const float2 xs = *sptr<float2>(xs_t + (uint32_t)(4 * 8 * gi));
+        // block partial / 2^20 = (16 * dlo + dhi) - z * sum(x) / 2^20: one
+        // rounding for the sum and one for the fma, as for int4 (the exact
+        // power-of-two scale is restored once per row at the output); the
+        // two blocks of a row go as one paired operation
+        const float2 xs = *sptr<float2>(xs_t + (uint32_t)(4 * 8 * gi));  // block sums / 2^20
         const uint32_t zg = lds_u8(sa_g + zo + (uint32_t)(4 * gi + t));  // blocks 2t (low), 2t+1 (high)
         const uint32_t zh = lds_u8(sa_g8 + zo + (uint32_t)(4 * gi + t));
-        // z as a float: 2^23 + z spliced into the mantissa, minus 2^23 (exact)
-        const float z0 = __uint_as_float(0x4B000000u | (zg & 15u)) - 8388608.0f;
-        const float z1 = __uint_as_float(0x4B000000u | (zg >> 4)) - 8388608.0f;
-        const float z2 = __uint_as_float(0x4B000000u | (zh & 15u)) - 8388608.0f;
-        const float z3 = __uint_as_float(0x4B000000u | (zh >> 4)) - 8388608.0f;
-        d[0] = fmaf(-z0, xs.x, fmaf(d[0], 16.0f, dh[0]) * 1048576.0f);
-        d[1] = fmaf(-z1, xs.y, fmaf(d[1], 16.0f, dh[1]) * 1048576.0f);
-        d[2] = fmaf(-z2, xs.x, fmaf(d[2], 16.0f, dh[2]) * 1048576.0f);
-        d[3] = fmaf(-z3, xs.y, fmaf(d[3], 16.0f, dh[3]) * 1048576.0f);
+        // -z as floats: 2^23 minus (2^23 + z spliced into the mantissa), exact
+        const uint64_t e23 = pack_f32x2(0x4B000000u, 0x4B000000u);
+        const uint64_t nzg = sub_f32x2(e23, pack_f32x2(0x4B000000u | (zg & 15u), 0x4B000000u | (zg >> 4)));
+        const uint64_t nzh = sub_f32x2(e23, pack_f32x2(0x4B000000u | (zh & 15u), 0x4B000000u | (zh >> 4)));
+        const uint64_t x2 = pack_f32x2(__float_as_uint(xs.x), __float_as_uint(xs.y));
+        const uint64_t c16 = pack_f32x2(0x41800000u, 0x41800000u);  // 16.0f
+        const uint64_t tg = fma_f32x2(pack_f32x2(__float_as_uint(d[0]), __float_as_uint(d[1])), c16,
+                                      pack_f32x2(__float_as_uint(dh[0]), __float_as_uint(dh[1])));
+        const uint64_t th = fma_f32x2(pack_f32x2(__float_as_uint(d[2]), __float_as_uint(d[3])), c16,
+                                      pack_f32x2(__float_as_uint(dh[2]), __float_as_uint(dh[3])));
+        const float2 rg = unpack_f32x2(fma_f32x2(nzg, x2, tg)), rh = unpack_f32x2(fma_f32x2(nzh, x2, th));
+        d[0] = rg.x;
+        d[1] = rg.y;
+        d[2] = rh.x;
+        d[3] = rh.y;
       }
       acc[0] = fmaf(d[0], s0, acc[0]);
       acc[0] = fmaf(d[1], s1, acc[0]);
@@ -625,6 +633,8 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
             sum += (double)__low2float(hv) + (double)__high2float(hv);
           }
         }
+        // affine int4 keeps its block partials scaled by 2^-20 (exact): the sums too
+        if constexpr (FMT == QMV_FMT_INT4AFF) sum *= 0x1p-20;
         *reinterpret_cast<float*>(smem + p.off_xsum + 4 * b) = (float)sum;
       }
     }
@@ -774,6 +784,8 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
     // ---- outputs: lane (g, t) holds rows g, g+8, columns 2t, 2t+1 of each n-tile ----
     const float f = (FMT == QMV_FMT_FP4) ? 0.5f : 1.0f;  // the fp4 block scales carried a factor 2
     if constexpr (kOne) {
+      // (affine int4's batch-1 partials were kept scaled by 2^-20)
+      const float f1 = FMT == QMV_FMT_INT4AFF ? 1048576.0f : f;
       // rows g, g+8: the four lanes of a row hold disjoint blocks; add them
       float r0 = F::kLut ? dl[0] + dl[1] : acc1[0];
       float r1 = F::kLut ? dl[2] + dl[3] : acc1[1];
@@ -784,8 +796,8 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       const int pair = gt.sorted[gstart];
       if (!it.split) {
         if (t == 0) {
-          if (g < nrows) emit(0, pair, row0 + g, r0 * f);
-          if (g + 8 < nrows) emit(0, pair, row0 + g + 8, r1 * f);
+          if (g < nrows) emit(0, pair, row0 + g, r0 * f1);
+          if (g + 8 < nrows) emit(0, pair, row0 + g + 8, r1 * f1);
         }
       } else {
         if (t == 0) {
@@ -797,7 +809,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
           float v = 0.0f;
 #pragma unroll
           for (int w = 0; w < WARPS; ++w) v += red[w * 16 + tid];
-          if (tid < nrows) emit(0, pair, row0 + tid, v * f);
+          if (tid < nrows) emit(0, pair, row0 + tid, v * f1);
         }
         __syncthreads();
       }

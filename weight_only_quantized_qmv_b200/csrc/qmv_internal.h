@@ -125,7 +125,7 @@ cudaError_t launch_outlier_columns(const float* W, int64_t N, int64_t K, int64_t
 cudaError_t launch_split_f32(const float* W, int64_t N, int64_t K, const int32_t* cols, int64_t C, float* Wmain,
                              float* Wout, int num_sms, cudaStream_t stream);
 // y[b, n] += sum over the C outlier columns of x[b, cols[c]] * q[n, c] * s[n, c / 32]
-// (dependent launch: weights read before the wait, y after it).
+// (dependent launch: everything is read after the wait for the int4km part).
 cudaError_t launch_outlier_acc(const int8_t* q, const uint16_t* s, const int32_t* cols, const uint16_t* x, int B,
                                int64_t N, int64_t K, int64_t C, float* y, int num_sms, cudaStream_t stream);
 cudaError_t launch_km8(const MvParams& p, cudaStream_t stream);

@@ -179,6 +179,22 @@ def test_int4aff_unaligned_aux(q):
     assert q.status_fetch() == 0
 
 
+@pytest.mark.parametrize("K", [32768, 65536])
+def test_int8km_batch1_long_rows(q, K):
+    """Batch 1 with long rows: at K = 32768 the batch-1 kernel's fp32
+    activation row leaves room for one CTA per SM; at K = 65536 it does not
+    fit at all and the general kernel (fp16 rows) takes the call.  Both match
+    the oracle on stand-in tables."""
+    N = 40
+    c_o, s_o, xn = _inputs("int8km", N, K, 1, seed=K + 3)
+    y = q.matvec_int8km(torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(),
+                        torch.from_numpy(xn).cuda()).cpu().numpy()
+    r = orc.matvec(FID["int8km"], c_o, s_o, xn, N, K)
+    e = rel_err(y, r)
+    assert e < TOL, e
+    assert q.status_fetch() == 0
+
+
 def test_int8km_lut_checks_and_unaligned_lut(q):
     """The binding rejects a LUT of the wrong group count; a LUT plane that
     starts 2 bytes past a 16-byte boundary gives the same outputs."""

@@ -544,36 +544,39 @@ bool plan_km8(MvParams& p, int num_sms) {
   p.tiles = (p.N + 31) / 32;  // row groups
   p.expert_code_bytes = p.N * p.K;
   p.expert_aux_bytes = p.tiles * 512;
-  // staged activation rows: natural order, whole 64-wide chunks, the row
-  // stride at 16 mod 128 bytes so the 16-byte reads of 8 lanes (two rows,
-  // four in-feature quarters) fall in distinct banks
-  p.XS = (int)(round_up8(2 * round_up8(p.K, 64), 128) + 16);
   p.n_xrows = p.gather ? (p.x_per_slot ? p.B * p.topk : p.B) : p.B;
   const int nt = p.B > 8 ? 2 : 1;
-  // dense batch 1: the fp32 path (one fp32 row, in its own chunk layout)
-  p.one = (!p.gather && p.B == 1) ? 1 : 0;
-  if (p.one) p.XS = (int)(2048 * ((p.K + 511) / 512));
-  const int64_t red_one = p.one ? (int64_t)2 * 32 * 4 : (int64_t)8 * 2 * nt * 4 * 32 * 4;  // one buffer
   const int64_t units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
-  // layouts in order of preference: two 8-warp CTAs per SM, one 16-warp CTA
-  // (batch 1: one 8-warp CTA); two partial-sum buffers, else one
-  const int cand[4][3] = {{8, 2, 2}, {16, 1, 2}, {8, 2, 1}, {16, 1, 1}};
-  for (int ci = 0; ci < 4; ++ci) {
-    const int warps = p.one ? 8 : cand[ci][0], ctas = cand[ci][1];
-    p.warps = warps;
-    p.red_bufs = cand[ci][2];
-    p.off_tab = 0;  // 64 KB: 256 rows x 2 buffers x 128 bytes
-    p.off_red = 256 * 256;
-    p.off_x = (int)round_up8(p.off_red + p.red_bufs * red_one, 128);
-    const int64_t bytes = p.off_x + (int64_t)p.n_xrows * p.XS;
-    const int64_t stat = p.one ? 1024 : kStaticSmem;  // the batch-1 kernel's static shared memory is the argmax keys
-    if (bytes <= dyn_limit && ctas * (bytes + stat + 1024) <= kSmemPerSM) {
-      p.smem_bytes = (int)bytes;
-      p.ctas_per_sm = ctas;
-      const int64_t slots = (int64_t)num_sms * ctas;
-      p.grid = (int)(units < slots ? units : slots);
-      return true;
+  // dense batch 1 takes its own kernel (one fp32 activation row, in its own
+  // chunk layout); where that row does not fit, the general kernel (fp16
+  // rows, half the bytes)
+  for (int one = (!p.gather && p.B == 1) ? 1 : 0; one >= 0; --one) {
+    p.one = one;
+    // staged activation rows: natural order, whole 64-wide chunks, the row
+    // stride at 16 mod 128 bytes so the 16-byte reads of 8 lanes (two rows,
+    // four in-feature quarters) fall in distinct banks
+    p.XS = one ? (int)(2048 * ((p.K + 511) / 512)) : (int)(round_up8(2 * round_up8(p.K, 64), 128) + 16);
+    const int64_t red_one = one ? (int64_t)2 * 32 * 4 : (int64_t)8 * 2 * nt * 4 * 32 * 4;  // one buffer
+    // layouts in order of preference: two 8-warp CTAs per SM, one 16-warp CTA
+    // (batch 1: one 8-warp CTA); two partial-sum buffers, else one
+    const int cand[4][3] = {{8, 2, 2}, {16, 1, 2}, {8, 2, 1}, {16, 1, 1}};
+    for (int ci = 0; ci < 4; ++ci) {
+      const int warps = one ? 8 : cand[ci][0], ctas = cand[ci][1];
+      p.warps = warps;
+      p.red_bufs = cand[ci][2];
+      p.off_tab = 0;  // 64 KB: 256 rows x 2 buffers x 128 bytes
+      p.off_red = 256 * 256;
+      p.off_x = (int)round_up8(p.off_red + p.red_bufs * red_one, 128);
+      const int64_t bytes = p.off_x + (int64_t)p.n_xrows * p.XS;
+      const int64_t stat = one ? 1024 : kStaticSmem;  // the batch-1 kernel's static shared memory is the argmax keys
+      if (bytes <= dyn_limit && ctas * (bytes + stat + 1024) <= kSmemPerSM) {
+        p.smem_bytes = (int)bytes;
+        p.ctas_per_sm = ctas;
+        const int64_t slots = (int64_t)num_sms * ctas;
+        p.grid = (int)(units < slots ? units : slots);
+        return true;
+      }
     }
   }
   return false;

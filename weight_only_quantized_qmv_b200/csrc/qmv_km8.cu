@@ -94,7 +94,8 @@ __device__ __forceinline__ void km8_chunk(float (&acc)[NT][4], const uint4& cg, 
 
 // NT: activation n-tiles of 8 columns (1 or 2).  WARPS: 8 (two CTAs per SM)
 // or 16 (one CTA per SM, when the staged activations are large).  Dense
-// batch 1 runs km8b1_kernel below.
+// batch 1 runs km8b1_kernel below, unless its fp32 activation row does not
+// fit (then this kernel, with B = 1 as one column).
 //
 // Per unit, with one barrier: the next unit's LUT entries are requested at
 // the start (registers) and written to the other table buffer at the end;

@@ -39,6 +39,10 @@ MUTANTS = {
     "outlier columns by the smallest maximum": ("if (x->m != y->m) return (x->m > y->m) ? -1 : 1;",
                                                 "if (x->m != y->m) return (x->m > y->m) ? 1 : -1;"),
     "outlier dequant with the first scale only": ("oscales[n * (C / 32) + jo / 32]", "oscales[n * (C / 32)]"),
+    "int8km LUT shared by 16 rows in dequant": ("aux)[(n / ORC_KM8_GROUP) * 256 + j]", "aux)[(n / 16) * 256 + j]"),
+    "mixed main-part nibbles swapped in dequant": ("int e = (jm % 2) ? (byte >> 4) : (byte & 15);\n        Wdq",
+                                                   "int e = (jm % 2) ? (byte & 15) : (byte >> 4);\n        Wdq"),
+    "outlier membership off by one column": ("return lo < C && cols[lo] == k;", "return lo < C && cols[lo] == k + 1;"),
 }
 
 

@@ -180,6 +180,9 @@ class ClockSampler:
 # ----------------------------------------------------------------- workload
 
 def build_workload(device, formats=FORMATS):
+    """The head's weights encoded by the library in each format.  Each
+    encoder runs once on a small slice first (module load and first-launch
+    costs), then its time on the full head is taken with CUDA events."""
     import torch
     import weight_only_quantized_qmv_b200 as q
     from weight_only_quantized_qmv_b200 import synth
@@ -192,13 +195,14 @@ def build_workload(device, formats=FORMATS):
                     ("int4km", q.encode_int4km)):
         if fmt not in formats:
             continue
+        fn(W[:256].contiguous())  # warm-up launch
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         codes, aux = fn(W)
         b.record()
         torch.cuda.synchronize()
-        enc_ms[fmt] = a.elapsed_time(b)
+        enc_ms[fmt] = round(a.elapsed_time(b), 3)
         ops[fmt] = (codes, aux)  # int4km: (indices, palette)
     del W
     torch.cuda.empty_cache()
@@ -235,6 +239,76 @@ def graph_us(g, stream, reps_per_graph, replays):
         e1.record(stream)
     stream.synchronize()
     return e0.elapsed_time(e1) * 1e3 / (replays * reps_per_graph)
+
+
+def graph_us_samples(g, stream, reps_per_graph, replays):
+    """Device time per call (us) of each of `replays` replays of a captured
+    graph: every replay is bracketed by its own CUDA events on the graph's
+    stream (one warm-up replay first)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+    with torch.cuda.stream(stream):
+        g.replay()
+        for a, b in evs:
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+    stream.synchronize()
+    return [a.elapsed_time(b) * 1e3 / reps_per_graph for a, b in evs]
+
+
+def spread(samples):
+    """median / p10 / p90 / mean of a list of per-call times (us)."""
+    v = sorted(samples)
+    n = len(v)
+
+    def q(f):  # nearest-rank percentile
+        return v[min(n - 1, max(0, int(round(f * (n - 1)))))]
+    return {"median": round(statistics.median(v), 3), "p10": round(q(0.10), 3), "p90": round(q(0.90), 3),
+            "mean": round(statistics.mean(v), 3), "reps": n}
+
+
+STAT_REPLAYS = 25  # replays per figure: >= 20 samples for median / p10 / p90
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (lscpu, else /proc/cpuinfo)."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def read_ceiling_gbs(dev, stream, gib=2):
+    """A read-only streaming ceiling for this GPU: the best of a few full
+    reductions (torch amax, int32) over a buffer of `gib` GiB, larger than L2;
+    bytes read / device time.  A measurement aid, not part of the library."""
+    import torch
+    n = gib * (1 << 30) // 4
+    buf = torch.ones(n, dtype=torch.int32, device=dev)
+    best = 0.0
+    with torch.cuda.stream(stream):
+        torch.amax(buf)
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            torch.amax(buf)
+            b.record(stream)
+            stream.synchronize()
+            best = max(best, n * 4 / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del buf
+    torch.cuda.empty_cache()
+    return best
 
 
 def run_ours(args, rank, world, local_rank):
@@ -303,23 +377,28 @@ def run_ours(args, rank, world, local_rank):
     bytes_step = sum(algorithmic_bytes(f, N_HEAD, K_HEAD, 1) for f in formats)
     value = whole_job_gbs(bytes_step, world, ms_step)
 
-    # per-format kernel time: a graph of 10 back-to-back launches of one format
+    # per-format kernel time: graphs of 10 back-to-back launches of one
+    # format, each replay timed with its own events (median / p10 / p90)
     peak, peak_src = hbm_peak()
+    read_ceiling = None if args.no_extras else read_ceiling_gbs(dev, stream)
     per_fmt = {}
-    replays = max(3, min(30, args.steps // 100))
     for f in formats:
         g = capture(lambda f=f: launch(f), stream, 10)
-        us = graph_us(g, stream, 10, replays)
+        st = spread(graph_us_samples(g, stream, 10, STAT_REPLAYS))
         del g
-        gbs = algorithmic_bytes(f, N_HEAD, K_HEAD, 1) / (us * 1e-6) / 1e9
-        per_fmt[f] = {"us": round(us, 3), "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
-                      "frac_of_8tbs": round(gbs / 8000.0, 4), "bytes": algorithmic_bytes(f, N_HEAD, K_HEAD, 1)}
+        us = st["median"]
+        nb = algorithmic_bytes(f, N_HEAD, K_HEAD, 1)
+        gbs = nb / (us * 1e-6) / 1e9
+        per_fmt[f] = {"us": us, "us_p10": st["p10"], "us_p90": st["p90"], "reps": st["reps"], "gbs": round(gbs, 1),
+                      "frac_of_measured_hbm": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / 8000.0, 4),
+                      "frac_of_read_ceiling": round(gbs / read_ceiling, 4) if read_ceiling else None,
+                      "bytes": nb}
     dom = max(formats, key=lambda f: per_fmt[f]["us"])
     roof = {"bound": "hbm", "kernel": f"mv_kernel<{dom}> lm_head 248320x2048 B=1",
             "achieved": per_fmt[dom]["gbs"], "peak": peak, "unit": "GB/s",
             "frac": round(per_fmt[dom]["gbs"] / peak, 4), "peak_source": f"{peak_src} (hbm copy)",
             "traffic": profiled_traffic(dom), "algorithmic_bytes": per_fmt[dom]["bytes"],
-            "timing": "CUDA events around replays of a graph of 10 launches"}
+            "timing": f"median of {STAT_REPLAYS} replays of a graph of 10 launches, CUDA events per replay"}
 
     # the same step launched call by call (no graph), for context
     with torch.cuda.stream(stream):
@@ -339,16 +418,85 @@ def run_ours(args, rank, world, local_rank):
     amax = None if args.no_extras else measure_argmax(q, ops, fmt_id, x, dev, stream, formats)
     nxt = None if args.no_extras else measure_next_formats(q, x, dev, stream, peak)
 
-    # end to end through the C ABI with host buffers: H2D x, the matvecs, D2H y
-    e2e = None if args.no_extras else measure_e2e(q, ops, fmt_id, x, dev, stream, formats,
+    # the same-box fp16 lm_head matvec (the pages' per-op comparison) and the
+    # int8 head at its own shape
+    fp16 = None if args.no_extras else measure_fp16_head(dev, stream, per_fmt)
+    c2 = None if args.no_extras else measure_int8_head_c2(q, dev, stream, peak)
+
+    # end to end through the C ABI with host buffers: H2D x, the matvecs, D2H
+    # y, all on the step's stream; the step's outputs are the check
+    ref_outs = {}
+    with torch.cuda.stream(stream):
+        step_graph.replay()
+    stream.synchronize()
+    for f in formats:
+        ref_outs[f] = outs[f].cpu()
+    e2e = None if args.no_extras else measure_e2e(q, ops, fmt_id, x, dev, stream, formats, ref_outs,
                                                     steps=min(200, max(20, args.steps // 10)))
 
     return {
         "ms_per_step": ms_step, "value": value, "per_fmt": per_fmt, "roofline": roof, "clocks": clocks,
         "encode_ms": enc_ms, "batches": extra, "e2e": e2e, "bytes_step": bytes_step,
         "gpu_launches": len(formats) * args.steps, "step_us_without_graph": round(plain_us, 2),
-        "decode_step_int4km": dstep, "argmax_b1": amax, "next_formats": nxt,
+        "decode_step_int4km": dstep, "argmax_b1": amax, "next_formats": nxt, "fp16_head": fp16,
+        "int8_head_130560": c2, "read_ceiling_gbs": round(read_ceiling, 1) if read_ceiling else None,
     }
+
+
+def measure_fp16_head(dev, stream, per_fmt):
+    """The same head in fp16 on this GPU: torch (cuBLAS) y = x W^T with W
+    float16 [248320, 2048] (seeded N(0, 0.02)), batch 1, graphs of 10 calls.
+    Bytes: W + x + y (fp16), ~1018 MB.  The ratios are the B200 counterpart
+    of the pages' per-op 'int4km vs fp16' figure."""
+    import torch
+    from weight_only_quantized_qmv_b200 import synth
+    g = synth.generator(3, dev)
+    W16 = synth.weights(N_HEAD, K_HEAD, g)[0].to(torch.float16)
+    x16 = synth.activations(1, K_HEAD, g)
+    y16 = torch.empty((1, N_HEAD), dtype=torch.float16, device=dev)
+    gr = capture(lambda: torch.matmul(x16, W16.t(), out=y16), stream, 10)
+    st = spread(graph_us_samples(gr, stream, 10, STAT_REPLAYS))
+    del gr, W16
+    torch.cuda.empty_cache()
+    nb = N_HEAD * K_HEAD * 2 + K_HEAD * 2 + N_HEAD * 2
+    return {"us": st["median"], "us_p10": st["p10"], "us_p90": st["p90"], "bytes": nb,
+            "gbs": round(nb / (st["median"] * 1e-6) / 1e9, 1), "kernel": "torch.matmul (cuBLAS), fp16",
+            "speedup_vs_fp16": {f: round(st["median"] / v["us"], 3) for f, v in per_fmt.items()}}
+
+
+def measure_int8_head_c2(q, dev, stream, peak):
+    """The int8 head at its own shape (130560 x 2048, N(0, 0.02), clip 1.0):
+    encode (after a warm-up launch) and the batch-1 matvec, timed apart."""
+    import torch
+    from weight_only_quantized_qmv_b200 import synth
+    N = 130560
+    g = synth.generator(0, dev)
+    W, _ = synth.weights(N, K_HEAD, g)
+    x = synth.activations(1, K_HEAD, g)
+    q.encode_int8(W[:256].contiguous())
+    enc = []
+    for _ in range(3):
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        codes, scales = q.encode_int8(W)
+        b.record()
+        torch.cuda.synchronize()
+        enc.append(a.elapsed_time(b))
+    del W
+    torch.cuda.empty_cache()
+    out = torch.empty((1, N), dtype=torch.float32, device=dev)
+    gr = capture(lambda: q.matvec_int8(codes, scales, x, out=out, stream=stream), stream, 10)
+    st = spread(graph_us_samples(gr, stream, 10, STAT_REPLAYS))
+    del gr
+    if q.status_fetch(stream):
+        raise RuntimeError("int8 head status flags")
+    nb = algorithmic_bytes("int8", N, K_HEAD, 1)
+    gbs = nb / (st["median"] * 1e-6) / 1e9
+    return {"shape": [N, K_HEAD], "encode_ms": round(statistics.median(enc), 3),
+            "encode_read_gbs": round(N * K_HEAD * 4 / (statistics.median(enc) * 1e-3) / 1e9, 1),
+            "matvec_us": st["median"], "matvec_us_p10": st["p10"], "matvec_us_p90": st["p90"],
+            "bytes": nb, "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4)}
 
 
 def measure_next_formats(q, x, dev, stream, peak):
@@ -386,11 +534,13 @@ def measure_next_formats(q, x, dev, stream, peak):
     calls["int4km_o8"] = lambda: q.matvec_int4km_o8(*o8, x, out=out, stream=stream)
     for f, fn in calls.items():
         gr = capture(fn, stream, 10)
-        us = graph_us(gr, stream, 10, 5)
+        st = spread(graph_us_samples(gr, stream, 10, STAT_REPLAYS))
         del gr
+        us = st["median"]
         nb = algorithmic_bytes(f, N_HEAD, K_HEAD, 1)
         gbs = nb / (us * 1e-6) / 1e9
-        res[f] = {"us": round(us, 3), "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peak, 4),
+        res[f] = {"us": us, "us_p10": st["p10"], "us_p90": st["p90"], "gbs": round(gbs, 1),
+                  "frac_of_measured_hbm": round(gbs / peak, 4),
                   "bytes": nb, "encode_ms": round(enc[f], 2) if f in enc else None}
     res["int4km_o8"]["launches_per_call"] = 2
     res["int8km"]["weights"] = "stand-in tables (random indices, sorted N(0, 0.02) palettes)"
@@ -407,9 +557,10 @@ def measure_batches(q, ops, dev, stream):
         out = torch.empty((B, N_HEAD), dtype=torch.float32, device=dev)
         c, a = ops["fp4"]
         g = capture(lambda: q.matvec_fp4(c, a, x, out=out, stream=stream), stream, 10)
-        us = graph_us(g, stream, 10, 5)
+        st = spread(graph_us_samples(g, stream, 10, STAT_REPLAYS))
         del g
-        res[f"fp4_b{B}"] = {"us": round(us, 3),
+        us = st["median"]
+        res[f"fp4_b{B}"] = {"us": us, "us_p10": st["p10"], "us_p90": st["p90"],
                             "gbs": round(algorithmic_bytes("fp4", N_HEAD, K_HEAD, B) / (us * 1e-6) / 1e9, 1)}
     return res
 
@@ -499,7 +650,13 @@ def measure_decode_step(q, lm_idx, lm_lut, dev, stream, reps=20):
     return res
 
 
-def measure_e2e(q, ops, fmt_id, x, dev, stream, formats, steps):
+def measure_e2e(q, ops, fmt_id, x, dev, stream, formats, ref_outs, steps):
+    """The step end to end through the public API with host buffers: per step
+    the activations are copied in from pinned host memory, the four matvecs
+    run, and every output is copied back to pinned host memory, all in order
+    on one stream.  CUDA events on that stream bracket copy-in .. copy-out,
+    the wall clock runs until the stream has drained, and the host copies of
+    the last step are compared bit for bit with the graph step's outputs."""
     import torch
     x_host = x.cpu().pin_memory()
     y_host = {f: torch.empty((1, N_HEAD), dtype=torch.float32).pin_memory() for f in formats}
@@ -507,35 +664,41 @@ def measure_e2e(q, ops, fmt_id, x, dev, stream, formats, steps):
     outs = {f: torch.empty((1, N_HEAD), dtype=torch.float32, device=dev) for f in formats}
 
     def one():
-        x_dev.copy_(x_host, non_blocking=True)
-        for f in formats:
-            c, a = ops[f]
-            q.matvec(fmt_id[f], c, a, x_dev, out=outs[f], stream=stream)
-            y_host[f].copy_(outs[f], non_blocking=True)
-        stream.synchronize()
+        with torch.cuda.stream(stream):
+            x_dev.copy_(x_host, non_blocking=True)
+            for f in formats:
+                c, a = ops[f]
+                q.matvec(fmt_id[f], c, a, x_dev, out=outs[f], stream=stream)
+                y_host[f].copy_(outs[f], non_blocking=True)
 
     for _ in range(5):
         one()
+        stream.synchronize()
+    for f in formats:
+        y_host[f].zero_()
     times = []
     for _ in range(steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        one_start = time.perf_counter()
-        x_dev.copy_(x_host, non_blocking=True)
-        for f in formats:
-            c, a = ops[f]
-            q.matvec(fmt_id[f], c, a, x_dev, out=outs[f], stream=stream)
-            y_host[f].copy_(outs[f], non_blocking=True)
-        e1.record(stream)
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+        one()
+        with torch.cuda.stream(stream):
+            e1.record(stream)
         stream.synchronize()
-        times.append((e0.elapsed_time(e1), (time.perf_counter() - one_start) * 1e3))
-    ms_dev = statistics.mean(t[0] for t in times)
-    ms_wall = statistics.mean(t[1] for t in times)
+        times.append((e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3))
+    checked = all(torch.equal(y_host[f], ref_outs[f]) for f in formats)
+    if not checked:
+        raise RuntimeError("e2e outputs differ from the graph step's outputs")
+    ms_dev = statistics.median(t[0] for t in times)
+    ms_wall = statistics.median(t[1] for t in times)
     bytes_step = sum(algorithmic_bytes(f, N_HEAD, K_HEAD, 1) for f in formats)
     return {"value": round(bytes_step / (ms_wall * 1e-3) / 1e9, 1), "unit": "GB/s",
             "ms_per_step_wall": round(ms_wall, 4), "ms_per_step_device": round(ms_dev, 4),
             "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(len(formats) * N_HEAD * 4),
-            "steps": steps}
+            "steps": steps, "checked": checked,
+            "how": "median per step; H2D x, 4 matvecs, 4 D2H y on one stream; wall clock until the stream drains; "
+                   "outputs equal the graph step's bit for bit"}
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -576,7 +739,7 @@ def cpu_baseline(W, x, seconds=12.0, rows=8192):
     Wn = W[:rows].cpu().numpy()
     xn = x.cpu().numpy()
     gbs, R, thr, dt, passes = oracle_sample(Wn, xn, seconds)
-    return {"value": round(gbs, 3), "unit": "GB/s", "cores": thr, "kind": "oracle",
+    return {"value": round(gbs, 3), "unit": "GB/s", "cores": thr, "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"fp64 oracle matvec, {R} of 248320 rows x 2048, all four formats, {passes} passes in "
                       f"{dt:.1f} s (bytes scaled by the algorithmic-bytes definition)"}
 
@@ -638,30 +801,44 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- main
 
+PROFILE_CASES = ("fp4", "int4", "int4km", "int8", "int4aff", "int8km", "int4km_o8", "fp4_b16")
+
+
 def profile_case(name: str) -> int:
-    """A small case for a profiler: one kernel's matvec on 65536 x 2048
-    weights (larger than L2, a few hundred MB on the device), three launches,
-    batch 1.  Prints one line and exits."""
+    """A small case for a profiler: one format's matvec on 65536 x 2048
+    weights (larger than L2, a few hundred MB on the device), encoded by the
+    library (int8km: stand-in tables), three launches at batch 1 (fp4_b16:
+    batch 16).  Prints one line and exits."""
     import torch
     import weight_only_quantized_qmv_b200 as q
     from weight_only_quantized_qmv_b200 import synth
     N, K = 65536, K_HEAD
     g = synth.generator(0, "cuda")
-    x = synth.activations(1, K, g)
+    B = 16 if name == "fp4_b16" else 1
+    x = synth.activations(B, K, g)
     if name == "int8km":
         lut, idx = synth.palette_tables8(N, K, g)
         run = lambda: q.matvec_int8km(idx, lut, x)
-    else:  # int4km_o8
+    else:
         W, _ = synth.weights(N, K, g, n_outlier_cols=2)
-        enc = q.encode_int4km_o8(W, O8_COLS)
+        if name == "int4km_o8":
+            enc = q.encode_int4km_o8(W, O8_COLS)
+            run = lambda: q.matvec_int4km_o8(*enc, x)
+        else:
+            fmt = name.split("_")[0]
+            fid = {"fp4": q.FMT_FP4, "int4": q.FMT_INT4, "int4km": q.FMT_INT4KM, "int8": q.FMT_INT8,
+                   "int4aff": q.FMT_INT4AFF}[fmt]
+            encf = {"fp4": q.encode_fp4, "int4": q.encode_int4, "int4km": q.encode_int4km, "int8": q.encode_int8,
+                    "int4aff": q.encode_int4aff}[fmt]
+            c, a = encf(W)
+            run = lambda: q.matvec(fid, c, a, x)
         del W
-        run = lambda: q.matvec_int4km_o8(*enc, x)
     for _ in range(3):
         y = run()
     torch.cuda.synchronize()
     flags = q.status_fetch()
-    print(json.dumps({"profile_case": name, "N": N, "K": K, "launches": 3, "y_abs_sum": float(y.abs().sum()),
-                      "flags": flags}), flush=True)
+    print(json.dumps({"profile_case": name, "N": N, "K": K, "B": B, "launches": 3,
+                      "y_abs_sum": float(y.abs().sum()), "flags": flags}), flush=True)
     return 1 if flags else 0
 
 
@@ -677,7 +854,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e and batch-4/16 measurements")
     ap.add_argument("--no-prefetch", action="store_true",
                     help="keep weight reads behind the preceding launch (qmv_set_weight_prefetch(0))")
-    ap.add_argument("--profile-case", choices=("int8km", "int4km_o8"),
+    ap.add_argument("--profile-case", choices=PROFILE_CASES,
                     help="run one small case for a profiler (65536 x 2048, three launches) and exit")
     args = ap.parse_args()
     if args.profile_case:
@@ -730,7 +907,9 @@ def main():
             "step_us_without_graph": r["step_us_without_graph"], "decode_step_int4km": r["decode_step_int4km"],
             "argmax_b1": r["argmax_b1"],
             "gpu_launches": r["gpu_launches"] * world, "clocks": r["clocks"], "encode_ms": r["encode_ms"],
-            "batch_verify": r["batches"], "next_formats": r["next_formats"],
+            "batch_verify": r["batches"], "next_formats": r["next_formats"], "fp16_head": r["fp16_head"],
+            "int8_head_130560": r["int8_head_130560"], "read_ceiling_gbs": r["read_ceiling_gbs"],
+            "host_cpu": {"model": cpu_model(), "cores": os.cpu_count()},
         }
         print(json.dumps(out), flush=True)
     if world > 1:

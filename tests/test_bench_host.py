@@ -51,3 +51,10 @@ def test_algorithmic_bytes_are_the_encoded_bytes(fmt, B):
 def test_whole_job_rate_counts_every_rank():
     # 2 ranks x 1 GB in 0.5 ms (the slowest rank's time) = 4000 GB/s
     assert bench.whole_job_gbs(1_000_000_000, 2, 0.5) == pytest.approx(4000.0)
+
+
+def test_spread_percentiles():
+    # 1..25: median 13, nearest-rank p10 / p90 at positions 2.4 -> 2 and 21.6 -> 22 (0-based)
+    st = bench.spread([float(v) for v in range(25, 0, -1)])
+    assert st["median"] == 13.0 and st["p10"] == 3.0 and st["p90"] == 23.0
+    assert st["mean"] == 13.0 and st["reps"] == 25

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "qmv_internal.h"
 
@@ -30,8 +31,12 @@ qmv_status cuda_fail(cudaError_t e, const char* what) {
 __device__ uint32_t g_status_word;
 
 constexpr int kMaxDevices = 64;
-uint32_t* g_status_ptr[kMaxDevices] = {nullptr};
-int g_num_sms[kMaxDevices] = {0};
+// Filled on a device's first call; several host threads may make that first
+// call at once, so the values are published with release stores after the
+// set-up ran under g_setup_mutex, and read with acquire loads.
+std::atomic<uint32_t*> g_status_ptr[kMaxDevices];
+std::atomic<int> g_num_sms[kMaxDevices];
+std::mutex g_setup_mutex;
 
 // Per-device set-up (current device): the status word's device address and
 // the SM count.  Runs on a device's first call.
@@ -40,18 +45,24 @@ qmv_status device_ctx(uint32_t** status, int* num_sms) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(QMV_ERR_UNSUPPORTED, "device %d out of range", dev);
-  if (!g_status_ptr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_status_word);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
-    int sms = 0;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-    g_num_sms[dev] = sms;
-    g_status_ptr[dev] = static_cast<uint32_t*>(ptr);
+  uint32_t* sp = g_status_ptr[dev].load(std::memory_order_acquire);
+  if (!sp) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    sp = g_status_ptr[dev].load(std::memory_order_acquire);
+    if (!sp) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_status_word);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+      int sms = 0;
+      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+      g_num_sms[dev].store(sms, std::memory_order_relaxed);
+      sp = static_cast<uint32_t*>(ptr);
+      g_status_ptr[dev].store(sp, std::memory_order_release);
+    }
   }
-  *status = g_status_ptr[dev];
-  *num_sms = g_num_sms[dev];
+  *status = sp;
+  *num_sms = g_num_sms[dev].load(std::memory_order_relaxed);
   return QMV_OK;
 }
 
@@ -107,20 +118,24 @@ qmv_status encode_int(int qmax, const float* W, int64_t N, int64_t K, const floa
 // once per device.
 constexpr size_t kStaticArgmaxBytes = 16 + 512 * 2 * qmv::kMaxCols * sizeof(unsigned long long);
 __device__ __align__(256) unsigned char g_argmax_scratch[kStaticArgmaxBytes];
-void* g_argmax_scratch_ptr[kMaxDevices] = {};
+std::atomic<void*> g_argmax_scratch_ptr[kMaxDevices];
 
 qmv_status static_argmax_scratch(void** ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(QMV_ERR_UNSUPPORTED, "device %d out of range", dev);
-  if (!g_argmax_scratch_ptr[dev]) {
-    void* a = nullptr;
-    e = cudaGetSymbolAddress(&a, g_argmax_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(argmax scratch)");
-    g_argmax_scratch_ptr[dev] = a;
+  void* a = g_argmax_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!a) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    a = g_argmax_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!a) {
+      e = cudaGetSymbolAddress(&a, g_argmax_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(argmax scratch)");
+      g_argmax_scratch_ptr[dev].store(a, std::memory_order_release);
+    }
   }
-  *ptr = g_argmax_scratch_ptr[dev];
+  *ptr = a;
   return QMV_OK;
 }
 

@@ -22,6 +22,7 @@
 //  * The looked-up fp16 values form the m16n8k16 A fragments directly: lane
 //    (g, t) owns in-features 16t..16t+15 of a chunk, word s of its bytes is
 //    the A operand of MMA step s, so the activations stay in natural order.
+#include <atomic>
 #include <cstdint>
 #include <cuda_fp16.h>
 
@@ -585,15 +586,15 @@ bool plan_km8(MvParams& p, int num_sms) {
 
 template <int NT, int WARPS, bool AM>
 static cudaError_t launch_km8_t(const MvParams& p, cudaStream_t stream) {
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(km8_kernel<NT, WARPS, AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
@@ -610,15 +611,15 @@ static cudaError_t launch_km8_t(const MvParams& p, cudaStream_t stream) {
 
 template <bool AM>
 static cudaError_t launch_km8b1_t(const MvParams& p, cudaStream_t stream) {
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(km8b1_kernel<AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);

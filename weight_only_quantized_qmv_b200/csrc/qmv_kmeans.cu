@@ -29,6 +29,8 @@
 // equal the rule's assignment when no two centres tie in computed double
 // distance at a weight other than by equal values; for weights of one row
 // that needs a dynamic range beyond 2^50.)
+#include <atomic>
+
 #include "qmv_device.cuh"
 
 namespace qmv {
@@ -233,14 +235,14 @@ cudaError_t launch_encode_int4km(const float* W, int64_t N, int64_t K, int iters
   if (warps > 8) warps = 8;
   if (warps < 1) return cudaErrorInvalidValue;
   const size_t smem = (size_t)warps * per_warp;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(km_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 16 * 1024);
     if (err != cudaSuccess) return err;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const int64_t want = (N + warps - 1) / warps;
   const int64_t cap = (int64_t)num_sms * 8;

@@ -26,6 +26,8 @@
 // applied in fp32 to each 32-block's partial sum; the palette format carries
 // its scale in the table and accumulates straight through.  Each output is
 // accumulated by one lane in a fixed order and written once (deterministic).
+#include <atomic>
+
 #include "qmv_device.cuh"
 #include "qmv_kernel_common.cuh"
 
@@ -960,15 +962,15 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
 
 template <int FMT, int NT, int WARPS, bool AM>
 static cudaError_t launch_t(const MvParams& p, cudaStream_t stream) {
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(mv_kernel<FMT, NT, WARPS, AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);

@@ -594,59 +594,81 @@ def measure_argmax(q, ops, fmt_id, x, dev, stream, formats):
     return res
 
 
-def measure_decode_step(q, lm_idx, lm_lut, dev, stream, reps=20):
-    """The int4km decode step of the workload list, timed as one CUDA graph per
-    batch size: the 248320x2048 lm_head, 10 layers of q (4096x2048) and o
-    (2048x4096), and one routed-expert layer (256 experts; gate and up
-    512x2048, down 2048x512; top-8 uniform routing).  Random palettes and
-    indices of the fitted shapes; each launch reads fixed synthetic
-    activations (the step's data flow between layers is not modelled)."""
-    import torch
+DECODE_E, DECODE_TOPK, DECODE_H, DECODE_I, DECODE_LAYERS = 256, 8, 2048, 512, 10
+
+
+def decode_step_weights(dev):
+    """Stand-in int4km weights of the decode step (fitted shapes, random
+    palettes and indices): 10 layers of q (4096x2048) and o (2048x4096), one
+    routed-expert layer (gate and up [256, 512, 2048], down [256, 2048, 512])."""
     from weight_only_quantized_qmv_b200 import synth
     g = synth.generator(11, dev)
-    E, topk, H, I = 256, 8, 2048, 512
+    E, H, I = DECODE_E, DECODE_H, DECODE_I
     layers = []
-    for _ in range(10):
+    for _ in range(DECODE_LAYERS):
         ql, qi = synth.palette_tables(4096, H, g)
         ol, oi = synth.palette_tables(H, 4096, g)
         layers.append((qi, ql, oi, ol))
     gl, gi = synth.palette_tables(E * I, H, g)
     ul, ui = synth.palette_tables(E * I, H, g)
     dl, di = synth.palette_tables(E * H, I, g)
-    gi, gl = gi.view(E, I, H // 2), gl.view(E, I, 16)
-    ui, ul = ui.view(E, I, H // 2), ul.view(E, I, 16)
-    di, dl = di.view(E, H, I // 2), dl.view(E, H, 16)
+    experts = (gi.view(E, I, H // 2), gl.view(E, I, 16), ui.view(E, I, H // 2), ul.view(E, I, 16),
+               di.view(E, H, I // 2), dl.view(E, H, 16))
+    return layers, experts, g
+
+
+def decode_step_fn(q, layers, experts, lm_idx, lm_lut, B, dev, stream, g):
+    """The decode step's 24 launches for B tokens, as a closure on `stream`,
+    and the number of distinct experts its routing selects."""
+    import torch
+    from weight_only_quantized_qmv_b200 import synth
+    E, topk, H, I = DECODE_E, DECODE_TOPK, DECODE_H, DECODE_I
+    gi, gl, ui, ul, di, dl = experts
+    x_h = synth.activations(B, H, g)
+    x_o = synth.activations(B, 4096, g)
+    x_d = synth.activations(B, I, g, extra_shape=(topk,))
+    ids = synth.routing(B, topk, E, g).to(dev)
+    y_lm = torch.empty((B, lm_idx.shape[0]), dtype=torch.float32, device=dev)
+    y_q = torch.empty((B, 4096), dtype=torch.float32, device=dev)
+    y_o = torch.empty((B, H), dtype=torch.float32, device=dev)
+    y_g = torch.empty((B, topk, I), dtype=torch.float32, device=dev)
+    y_u = torch.empty((B, topk, I), dtype=torch.float32, device=dev)
+    y_d = torch.empty((B, topk, H), dtype=torch.float32, device=dev)
+
+    def step():
+        for qi, ql, oi, ol in layers:
+            q.matvec_int4km(qi, ql, x_h, out=y_q, stream=stream)
+            q.matvec_int4km(oi, ol, x_o, out=y_o, stream=stream)
+        q.gather_matvec(q.FMT_INT4KM, gi, gl, ids, x_h, out=y_g, stream=stream)
+        q.gather_matvec(q.FMT_INT4KM, ui, ul, ids, x_h, out=y_u, stream=stream)
+        q.gather_matvec(q.FMT_INT4KM, di, dl, ids, x_d, x_per_slot=True, out=y_d, stream=stream)
+        q.matvec_int4km(lm_idx, lm_lut, x_h, out=y_lm, stream=stream)
+
+    return step, len(set(ids.flatten().tolist()))
+
+
+def measure_decode_step(q, lm_idx, lm_lut, dev, stream, reps=STAT_REPLAYS):
+    """The int4km decode step of the workload list, timed as one CUDA graph per
+    batch size: the 248320x2048 lm_head, 10 layers of q (4096x2048) and o
+    (2048x4096), and one routed-expert layer (256 experts; gate and up
+    512x2048, down 2048x512; top-8 uniform routing).  Random palettes and
+    indices of the fitted shapes; each launch reads fixed synthetic
+    activations (the step's data flow between layers is not modelled)."""
+    layers, experts, g = decode_step_weights(dev)
+    E, topk, H, I = DECODE_E, DECODE_TOPK, DECODE_H, DECODE_I
     res = {}
     for B in (1, 8):
-        x_h = synth.activations(B, H, g)
-        x_o = synth.activations(B, 4096, g)
-        x_d = synth.activations(B, I, g, extra_shape=(topk,))
-        ids = synth.routing(B, topk, E, g).to(dev)
-        y_lm = torch.empty((B, N_HEAD), dtype=torch.float32, device=dev)
-        y_q = torch.empty((B, 4096), dtype=torch.float32, device=dev)
-        y_o = torch.empty((B, H), dtype=torch.float32, device=dev)
-        y_g = torch.empty((B, topk, I), dtype=torch.float32, device=dev)
-        y_u = torch.empty((B, topk, I), dtype=torch.float32, device=dev)
-        y_d = torch.empty((B, topk, H), dtype=torch.float32, device=dev)
-
-        def step():
-            for qi, ql, oi, ol in layers:
-                q.matvec_int4km(qi, ql, x_h, out=y_q, stream=stream)
-                q.matvec_int4km(oi, ol, x_o, out=y_o, stream=stream)
-            q.gather_matvec(q.FMT_INT4KM, gi, gl, ids, x_h, out=y_g, stream=stream)
-            q.gather_matvec(q.FMT_INT4KM, ui, ul, ids, x_h, out=y_u, stream=stream)
-            q.gather_matvec(q.FMT_INT4KM, di, dl, ids, x_d, x_per_slot=True, out=y_d, stream=stream)
-            q.matvec_int4km(lm_idx, lm_lut, x_h, out=y_lm, stream=stream)
-
+        step, n_exp = decode_step_fn(q, layers, experts, lm_idx, lm_lut, B, dev, stream, g)
         gph = capture(step, stream, 1)
-        us = graph_us(gph, stream, 1, reps)
+        st = spread(graph_us_samples(gph, stream, 1, reps))
         del gph
-        n_exp = len(set(ids.flatten().tolist()))
+        us = st["median"]
         dense = (algorithmic_bytes("int4km", N_HEAD, H, B)
                  + 10 * (algorithmic_bytes("int4km", 4096, H, B) + algorithmic_bytes("int4km", H, 4096, B)))
         expert = n_exp * (2 * (I * H // 2 + I * 32) + (H * I // 2 + H * 32))
-        res[f"b{B}"] = {"us": round(us, 2), "launches": 24, "distinct_experts": n_exp,
-                        "bytes": dense + expert, "gbs": round((dense + expert) / (us * 1e-6) / 1e9, 1)}
+        res[f"b{B}"] = {"us": us, "us_p10": st["p10"], "us_p90": st["p90"], "launches": 24,
+                        "distinct_experts": n_exp, "bytes": dense + expert,
+                        "gbs": round((dense + expert) / (us * 1e-6) / 1e9, 1)}
     return res
 
 
@@ -801,7 +823,8 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- main
 
-PROFILE_CASES = ("fp4", "int4", "int4km", "int8", "int4aff", "int8km", "int4km_o8", "fp4_b16")
+PROFILE_CASES = ("fp4", "int4", "int4km", "int8", "int4aff", "int8km", "int4km_o8", "fp4_b16",
+                 "decode_step_b1", "decode_step_b8")
 
 
 def profile_case(name: str) -> int:
@@ -813,6 +836,25 @@ def profile_case(name: str) -> int:
     import weight_only_quantized_qmv_b200 as q
     from weight_only_quantized_qmv_b200 import synth
     N, K = 65536, K_HEAD
+    if name.startswith("decode_step"):
+        # the full decode step (24 launches: lm_head, 10 x (q, o), gate, up,
+        # down), captured as a graph and replayed three times
+        B = int(name[-1])
+        dev = torch.device("cuda", 0)
+        stream = torch.cuda.Stream(device=dev)
+        layers, experts, g = decode_step_weights(dev)
+        lm_lut, lm_idx = synth.palette_tables(N_HEAD, K, g)
+        step, n_exp = decode_step_fn(q, layers, experts, lm_idx, lm_lut, B, dev, stream, g)
+        q.set_weight_prefetch(True)
+        gph = capture(step, stream, 1)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                gph.replay()
+        stream.synchronize()
+        flags = q.status_fetch()
+        print(json.dumps({"profile_case": name, "launches_per_step": 24, "steps": 5, "distinct_experts": n_exp,
+                          "flags": flags}), flush=True)
+        return 1 if flags else 0
     g = synth.generator(0, "cuda")
     B = 16 if name == "fp4_b16" else 1
     x = synth.activations(B, K, g)

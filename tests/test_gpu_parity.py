@@ -280,6 +280,35 @@ def test_matvec_parity(q, fmt, N, K, B):
     assert q.status_fetch() == 0
 
 
+@pytest.mark.parametrize("B", [7, 8])
+def test_int4km_palette_copy_fallback_parity(q, B):
+    """int4km at up to 8 columns looks rows g+8 up in lane palette copies in
+    shared memory where they fit beside the staged activations: at K = 8704
+    they just fit with 7 columns (one 8-warp CTA per SM), and with 8 columns
+    they do not, so the byte-permute lookups serve that launch (no refusal)."""
+    N, K = 300, 8704
+    c_o, s_o, xn = _inputs("int4km", N, K, B, seed=91 + B)
+    y = q.matvec_int4km(torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(), torch.from_numpy(xn).cuda())
+    r = orc.matvec(FID["int4km"], c_o, s_o, xn, N, K)
+    assert rel_err(y.cpu().numpy(), r) < TOL
+    assert q.status_fetch() == 0
+
+
+def test_int4km_palette_copy_equals_register_lookup(q):
+    """The shared-memory palette lookups (8 columns) and the byte-permute
+    lookups (9 columns) return the same fp16 weights: on a shape where every
+    output is one lane's sum over all of K, the first 8 outputs of the 9-column
+    launch equal the 8-column launch bit for bit."""
+    N, K = 37905, 2048
+    g = synth.generator(17, "cuda")
+    lut, idx = synth.palette_tables(N, K, g)
+    x9 = synth.activations(9, K, g)
+    y8 = q.matvec_int4km(idx, lut, x9[:8].contiguous())
+    y9 = q.matvec_int4km(idx, lut, x9)
+    assert torch.equal(y8, y9[:8])
+    assert q.status_fetch() == 0
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_matvec_one_hot_columns_bit_exact(q, fmt):
     """x = e_k picks column k of Wdq: the kernel must return it exactly

@@ -149,10 +149,12 @@ __device__ __forceinline__ uint32_t opaque(uint32_t c) {
 // Multipliers kept opaque so the decoders' shifts-by-multiply stay integer
 // multiply-adds on the FMA pipe.
 struct Mul {
-  uint32_t p4, e23;  // 2^4, 2^23
+  uint32_t p4, p8, p16, e23;  // 2^4, 2^8, 2^16, 2^23
   __device__ __forceinline__ static Mul make() {
     Mul m;
     m.p4 = opaque(1u << 4);
+    m.p8 = opaque(1u << 8);
+    m.p16 = opaque(1u << 16);
     m.e23 = opaque(1u << 23);
     return m;
   }
@@ -272,6 +274,39 @@ __device__ __forceinline__ void dec_int4km(const Palette& p, uint32_t w, uint32_
   s0hi = prmt(lo_a, hi_a, 0x7362u);
   s1lo = prmt(lo_b, hi_b, 0x5140u);
   s1hi = prmt(lo_b, hi_b, 0x7362u);
+}
+
+// INT4KM through a lane-private copy of one row's palette in shared memory,
+// a second lookup unit beside the byte permutes (which load the ALU pipe).
+// Entry j of the lane's copy is the 16-bit word at tb + 256 j, in the lane's
+// own bank, so the warp's 32 loads are one conflict-free wavefront; tb has
+// bits 8..11 clear, so a nibble standing at bits 8..11 of a word is its own
+// offset: one LOP3 ((v & 0xF00) | tb) forms each address.  Nibble 2 is in
+// place, nibbles 0 and 1 move up by a multiply (FMA pipe), nibble 3 and the
+// word's high half take one shift each, after which the high half's nibbles
+// 4..6 move like 0..2.  Per 8 weights: 3 shifts and 8 address LOP3s on the
+// ALU pipe (the byte-permute form takes 19), 8 16-bit loads, and 4
+// multiply-adds pack entry pairs into f16x2.  Emits (k0,k1) (k2,k3) (k4,k5)
+// (k6,k7) like dec_int4km.
+__device__ __forceinline__ uint32_t km_entry(uint32_t v, uint32_t tb) {
+  return *sptr<uint16_t>(lop3_and_or(v, 0xF00u, tb));
+}
+
+__device__ __forceinline__ void dec_int4km_smem(uint32_t tb, uint32_t w, uint32_t& s0lo, uint32_t& s0hi,
+                                                uint32_t& s1lo, uint32_t& s1hi, const Mul& m) {
+  const uint32_t hi = w >> 16;
+  const uint32_t e0 = km_entry(w * m.p8, tb);
+  const uint32_t e1 = km_entry(w * m.p4, tb);
+  const uint32_t e2 = km_entry(w, tb);
+  const uint32_t e3 = km_entry(w >> 4, tb);
+  const uint32_t e4 = km_entry(hi * m.p8, tb);
+  const uint32_t e5 = km_entry(hi * m.p4, tb);
+  const uint32_t e6 = km_entry(hi, tb);
+  const uint32_t e7 = km_entry(hi >> 4, tb);
+  s0lo = e1 * m.p16 + e0;
+  s0hi = e3 * m.p16 + e2;
+  s1lo = e5 * m.p16 + e4;
+  s1hi = e7 * m.p16 + e6;
 }
 
 }  // namespace qmv

@@ -62,6 +62,8 @@ struct MvParams {
   int64_t zplane;          // int4aff: byte offset of the zero points in an aux row
   int zoff;                // int4aff: byte offset of the slice's zero points in a staged aux row
   int off_tab;             // int8km: the replicated LUT table (64 KB, two buffers)
+  int off_kmtab;           // int4km: lane palette copies (4 KB per four warps, 4 KB aligned at run time)
+  int km_smem;             // int4km: rows g+8 look up their palette copy in shared memory
   int red_bufs;            // int8km: partial-sum buffers (2, or 1 where shared memory is short)
   int accum;               // y += result instead of y = result
   const int32_t* xcols;    // mixed format: the outlier columns (ascending); x rows hold all columns and

@@ -109,11 +109,12 @@ __device__ __forceinline__ float half_at(const uint4& v) {
 }
 
 // Decode one block's codes of rows g and g+8 into the two m16n8k16 A fragments
-// (zg / zh: the block's zero points of rows g / g+8, affine int4 only).
-template <int FMT>
+// (zg / zh: the block's zero points of rows g / g+8, affine int4 only; KMS:
+// int4km row g+8 through the lane's palette copy at ktb in shared memory).
+template <int FMT, bool KMS>
 __device__ __forceinline__ void decode_block(uint32_t crow_g, uint32_t crow_g8, int b, int t, const Palette& pg,
                                              const Palette& pg8, const Mul& m, uint32_t (&a0)[4], uint32_t (&a1)[4],
-                                             uint32_t zg = 0u, uint32_t zh = 0u) {
+                                             uint32_t zg, uint32_t zh, uint32_t ktb) {
   uint32_t g0lo, g0hi, g1lo, g1hi, h0lo, h0hi, h1lo, h1hi;  // row g / g+8, step 0 / 1
   if constexpr (FmtT<FMT>::kBits == 8) {
     const uint2 vg = lds64(crow_g + 32u * b + 8u * t);
@@ -136,7 +137,10 @@ __device__ __forceinline__ void decode_block(uint32_t crow_g, uint32_t crow_g8, 
       DecInt4::run_z(wh, h0lo, h0hi, h1lo, h1hi, int4_zp_sub(zh), int4_zp_neg(zh));
     } else {
       dec_int4km(pg, wg, g0lo, g0hi, g1lo, g1hi, m);
-      dec_int4km(pg8, wh, h0lo, h0hi, h1lo, h1hi, m);
+      if constexpr (KMS)
+        dec_int4km_smem(ktb, wh, h0lo, h0hi, h1lo, h1hi, m);
+      else
+        dec_int4km(pg8, wh, h0lo, h0hi, h1lo, h1hi, m);
     }
   }
   a0[0] = g0lo; a0[1] = h0lo; a0[2] = g0hi; a0[3] = h0hi;
@@ -168,10 +172,10 @@ __device__ __forceinline__ void mac_block(float (&acc)[NT][4], const uint32_t (&
 // A warp's NB blocks of a full K-slice, unrolled: every shared-memory address
 // is a base plus an immediate, and the slice's scales of a row are read with
 // one or two 128-bit loads (zo: offset of the zero points from the scales).
-template <int FMT, int NT, int NB>
+template <int FMT, int NT, int NB, bool KMS>
 __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g, uint32_t crow_g8, uint32_t sa_g,
                                            uint32_t sa_g8, uint32_t zo, const uint32_t (&xb)[NT], int t,
-                                           const Palette& pg, const Palette& pg8, const Mul& m) {
+                                           const Palette& pg, const Palette& pg8, const Mul& m, uint32_t ktb) {
   using F = FmtT<FMT>;
   uint4 sg0 = make_uint4(0u, 0u, 0u, 0u), sh0 = sg0, sg1 = sg0, sh1 = sg0;
   if constexpr (!F::kLut) {
@@ -204,7 +208,7 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g,
       zg = ((i < 8 ? zwg.x : zwg.y) >> (4 * (i & 7))) & 15u;
       zh = ((i < 8 ? zwh.x : zwh.y) >> (4 * (i & 7))) & 15u;
     }
-    decode_block<FMT>(crow_g, crow_g8, i, t, pg, pg8, m, a0, a1, zg, zh);
+    decode_block<FMT, KMS>(crow_g, crow_g8, i, t, pg, pg8, m, a0, a1, zg, zh, ktb);
     float sg = 0.0f, sh = 0.0f;
     if constexpr (FMT == QMV_FMT_FP4) {
       const uint32_t q = (uint32_t)i >> 2;
@@ -251,10 +255,11 @@ __device__ __forceinline__ void slice_full(float (&acc)[NT][4], uint32_t crow_g,
 // exact sum of n * x, and the offset (8, or the block's zero point z for
 // affine int4, staged zo bytes after the scales) is removed with the block's
 // sum of activations (xsum, exact in fp64, rounded once to fp32).
-template <int FMT, int NG>
+template <int FMT, int NG, bool KMS>
 __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint32_t crow_g, uint32_t crow_g8,
                                           uint32_t sa_g, uint32_t sa_g8, uint32_t zo, uint32_t xl0, uint32_t xl1,
-                                          uint32_t xs_t, int t, const Palette& pg, const Palette& pg8, const Mul& m) {
+                                          uint32_t xs_t, int t, const Palette& pg, const Palette& pg8, const Mul& m,
+                                          uint32_t ktb) {
   using F = FmtT<FMT>;
   constexpr int kBB = F::kBits * 4;  // code bytes per block and row
   constexpr bool kSub = FMT == QMV_FMT_INT4 || FMT == QMV_FMT_INT4AFF;  // the subnormal int4 decode
@@ -310,7 +315,10 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
           DecInt4::run(wh[i], h0lo, h0hi, h1lo, h1hi, m);
         } else {
           dec_int4km(pg, wg[i], g0lo, g0hi, g1lo, g1hi, m);
-          dec_int4km(pg8, wh[i], h0lo, h0hi, h1lo, h1hi, m);
+          if constexpr (KMS)  // row g+8 through the lane's palette copy in shared memory
+            dec_int4km_smem(ktb, wh[i], h0lo, h0hi, h1lo, h1hi, m);
+          else
+            dec_int4km(pg8, wh[i], h0lo, h0hi, h1lo, h1hi, m);
         }
         if constexpr (F::kLut) {
           mma16816(dl, g0lo, h0lo, g0hi, h0hi, xv.x, xv.y);
@@ -384,7 +392,9 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
 // WARPS: warps per CTA (8, two CTAs per SM; or 16, one CTA per SM, when the
 // staged activations leave room for only one 8-warp CTA).
 // AM: fused argmax (outputs folded into per-row maxima instead of stored).
-template <int FMT, int NT, int WARPS, bool AM>
+// KMS: int4km with lane palette copies in shared memory for rows g+8 (the
+// host sets it where they fit; batch <= 8).
+template <int FMT, int NT, int WARPS, bool AM, bool KMS>
 __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kernel(const __grid_constant__ MvParams p) {
   using F = FmtT<FMT>;
   constexpr bool kOne = NT == 0;
@@ -676,6 +686,11 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   float acc[NTX][4];
   float acc1[2], dl[4];  // batch-1 form: rows g, g+8 / the palette format's running MMA sums
   Palette pg, pg8;
+  // int4km (KMS): this lane's copy of row g+8's palette, entry j at ktb +
+  // 256 j.  Four warps share a 4 KB region (two 128-byte rows per entry, two
+  // 16-bit halves per 4-byte slot); every lane stays in its own bank.
+  const uint32_t ktb = ((sbase + (uint32_t)p.off_kmtab + 4095u) & ~4095u) + 4096u * (uint32_t)(warp >> 2) +
+                       128u * (uint32_t)((warp >> 1) & 1) + 2u * (uint32_t)(warp & 1) + 4u * (uint32_t)lane;
   uint32_t xa[NTX];
   int xa_grp = -1;
   uint32_t cons = ring;
@@ -728,7 +743,17 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
           e1[0] = b0.x; e1[1] = b0.y; e1[2] = b0.z; e1[3] = b0.w;
           e1[4] = b1.x; e1[5] = b1.y; e1[6] = b1.z; e1[7] = b1.w;
           pg = palette_from_words(e0);
-          pg8 = palette_from_words(e1);
+          if constexpr (KMS) {
+            // the lane's copy of row g+8's palette (read only by this lane,
+            // after this lane's earlier lookups in program order)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              sts_u16(ktb + 512u * j, e1[j] & 0xFFFFu);
+              sts_u16(ktb + 512u * j + 256u, e1[j] >> 16);
+            }
+          } else {
+            pg8 = palette_from_words(e1);
+          }
         }
       }
       const uint32_t crow_g = cons + (uint32_t)g * p.RS, crow_g8 = cons + (uint32_t)(g + 8) * p.RS;
@@ -743,10 +768,11 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
         const uint32_t tb = (uint32_t)(t * F::kBits * 4);
         const uint32_t xs_t = sbase + p.off_xsum + 4u * (uint32_t)(k0 / 32 + 2 * t);  // block sums of this lane
         if (kNB >= 16 && kc == kNB * 32)
-          slice_one<FMT, (kNB >= 16 ? kNB / 8 : 1)>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, zo, xl0, xl1,
-                                                    xs_t, t, pg, pg8, mul);
+          slice_one<FMT, (kNB >= 16 ? kNB / 8 : 1), KMS>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, zo, xl0,
+                                                         xl1, xs_t, t, pg, pg8, mul, ktb);
         else
-          slice_one<FMT, 1>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, zo, xl0, xl1, xs_t, t, pg, pg8, mul);
+          slice_one<FMT, 1, KMS>(acc1, dl, crow_g + tb, crow_g8 + tb, sa_g, sa_g8, zo, xl0, xl1, xs_t, t, pg, pg8,
+                                 mul, ktb);
         __syncwarp();
         cons = (cons + p.stage_bytes == ring_end) ? ring : cons + p.stage_bytes;
         continue;
@@ -755,9 +781,9 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
 #pragma unroll
       for (int n = 0; n < NTX; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
       if (kc == kNB * 32 && aux_fast) {
-        slice_full<FMT, NTX, kNB>(acc, crow_g, crow_g8, sa_g, sa_g8, zo, xb, t, pg, pg8, mul);
+        slice_full<FMT, NTX, kNB, KMS>(acc, crow_g, crow_g8, sa_g, sa_g8, zo, xb, t, pg, pg8, mul, ktb);
       } else if (kc == kNB * 16 && aux_fast) {
-        slice_full<FMT, NTX, kNB / 2>(acc, crow_g, crow_g8, sa_g, sa_g8, zo, xb, t, pg, pg8, mul);
+        slice_full<FMT, NTX, kNB / 2, KMS>(acc, crow_g, crow_g8, sa_g, sa_g8, zo, xb, t, pg, pg8, mul, ktb);
       } else {
         const int nbc = kc / 32;
         for (int b = 0; b < nbc; ++b) {
@@ -770,7 +796,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
             zg = (lds_u8(sa_g + zo + (uint32_t)(b >> 1)) >> (4 * (b & 1))) & 15u;
             zh = (lds_u8(sa_g8 + zo + (uint32_t)(b >> 1)) >> (4 * (b & 1))) & 15u;
           }
-          decode_block<FMT>(crow_g, crow_g8, b, t, pg, pg8, mul, a0, a1, zg, zh);
+          decode_block<FMT, KMS>(crow_g, crow_g8, b, t, pg, pg8, mul, a0, a1, zg, zh, ktb);
           float sg = 0.0f, sh = 0.0f;
           if constexpr (!F::kLut) {
             sg = stage_scale<FMT>(sa_g + (uint32_t)b * F::kSB, mul);
@@ -929,45 +955,59 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   const int cand[3][2] = {{kWarps, kMinCtas}, {2 * kWarps, 1}, {kWarps, 1}};
   // one CTA per (group, tile) unit up to the resident-CTA slots
   const int64_t upper_units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
+  // int4km up to 8 activation columns: lane palette copies in shared memory
+  // (4 KB per four warps + alignment) where they fit beside the staging,
+  // within each layout; without them otherwise.  (At 16 columns the copies
+  // cost ring depth that the byte-permute lookups do not need: measured
+  // slower.)
+  const bool km_ok = fi.lut && p.B <= 8;
   for (int ci = 0; ci < 3; ++ci) {
     const int warps = cand[ci][0], ctas = cand[ci][1];
     if (warps != kWarps && p.one) continue;  // the batch-1 form fits two 8-warp CTAs
-    p.warps = warps;
-    const int64_t slots = (int64_t)num_sms * ctas;
-    p.grid = (int)(upper_units < slots ? upper_units : slots);
-    // Units are split along K (partial sums meet in shared memory) only when
-    // there are fewer than the grid's warps; a (group, tile) count of at
-    // least p.tiles means that can happen only if p.tiles is below it.
-    const bool may_split = p.tiles < (int64_t)p.grid * warps;
-    p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
-    p.off_x = may_split ? (int)round_up((int64_t)warps * nt * 4 * 32 * 4, 128) : 0;
-    // the zero region starts 32 bytes past a 128-byte line: its reads and the
-    // activation reads of the same instruction fall in different banks
-    p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
-    p.off_xsum = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
-    const bool xsum = p.one && (fmt == QMV_FMT_INT4 || fmt == QMV_FMT_INT4AFF);
-    p.off_stage = (int)round_up(p.off_xsum + (xsum ? 4 * (p.K / 32) : 0), 128);
-    for (int st = kStages; st >= 2; --st) {
-      const int64_t bytes = p.off_stage + (int64_t)warps * st * p.stage_bytes;
-      if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
-        p.stages = st;
-        p.smem_bytes = (int)bytes;
-        p.ctas_per_sm = ctas;
-        return true;
+    for (int km = km_ok ? 1 : 0; km >= 0; --km) {
+      p.warps = warps;
+      p.km_smem = km;
+      const int64_t slots = (int64_t)num_sms * ctas;
+      p.grid = (int)(upper_units < slots ? upper_units : slots);
+      // Units are split along K (partial sums meet in shared memory) only when
+      // there are fewer than the grid's warps; a (group, tile) count of at
+      // least p.tiles means that can happen only if p.tiles is below it.
+      const bool may_split = p.tiles < (int64_t)p.grid * warps;
+      p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
+      p.off_x = may_split ? (int)round_up((int64_t)warps * nt * 4 * 32 * 4, 128) : 0;
+      // the zero region starts 32 bytes past a 128-byte line: its reads and the
+      // activation reads of the same instruction fall in different banks
+      p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
+      p.off_xsum = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
+      const bool xsum = p.one && (fmt == QMV_FMT_INT4 || fmt == QMV_FMT_INT4AFF);
+      // the copies' region is aligned to 4 KB at run time: with the dynamic
+      // shared memory 1 KB aligned and this offset a multiple of 1 KB, the
+      // alignment moves it by at most 3 KB
+      p.off_kmtab = (int)round_up(p.off_xsum + (xsum ? 4 * (p.K / 32) : 0), km ? 1024 : 128);
+      const int64_t kmtab = km ? 4096 * (int64_t)((warps + 3) / 4) + 3072 : 0;
+      p.off_stage = (int)round_up(p.off_kmtab + kmtab, 128);
+      for (int st = kStages; st >= 2; --st) {
+        const int64_t bytes = p.off_stage + (int64_t)warps * st * p.stage_bytes;
+        if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
+          p.stages = st;
+          p.smem_bytes = (int)bytes;
+          p.ctas_per_sm = ctas;
+          return true;
+        }
       }
     }
   }
   return false;
 }
 
-template <int FMT, int NT, int WARPS, bool AM>
+template <int FMT, int NT, int WARPS, bool AM, bool KMS = false>
 static cudaError_t launch_t(const MvParams& p, cudaStream_t stream) {
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
-    err = cudaFuncSetAttribute(mv_kernel<FMT, NT, WARPS, AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(mv_kernel<FMT, NT, WARPS, AM, KMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
     attr_set[dev].store(true, std::memory_order_release);
@@ -982,15 +1022,21 @@ static cudaError_t launch_t(const MvParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT, WARPS, AM>, p);
+  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT, WARPS, AM, KMS>, p);
 }
 
 template <int FMT, bool AM>
 static cudaError_t launch_fa(const MvParams& p, cudaStream_t stream) {
   // activation columns served per pass: dense B, gather at most B pairs per
   // expert when ids are distinct per token (groups are capped at 8 * NT)
-  if (p.one) return launch_t<FMT, 0, kWarps, AM>(p, stream);
   const bool wide = p.warps == 2 * kWarps;
+  if constexpr (FMT == QMV_FMT_INT4KM) {  // the palette-copy instances (batch <= 8)
+    if (p.km_smem) {
+      if (p.one) return launch_t<FMT, 0, kWarps, AM, true>(p, stream);
+      return wide ? launch_t<FMT, 1, 2 * kWarps, AM, true>(p, stream) : launch_t<FMT, 1, kWarps, AM, true>(p, stream);
+    }
+  }
+  if (p.one) return launch_t<FMT, 0, kWarps, AM>(p, stream);
   if (p.B > 8) return wide ? launch_t<FMT, 2, 2 * kWarps, AM>(p, stream) : launch_t<FMT, 2, kWarps, AM>(p, stream);
   return wide ? launch_t<FMT, 1, 2 * kWarps, AM>(p, stream) : launch_t<FMT, 1, kWarps, AM>(p, stream);
 }

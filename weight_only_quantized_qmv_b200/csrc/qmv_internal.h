@@ -56,6 +56,7 @@ struct MvParams {
   int topk, E, x_per_slot, gather;
   int KC, nchunks;         // in-features per warp slice, slices per tile
   int gk;                  // K granule of split units (in-features)
+  int min_part;            // split units: the least granules a warp's part of K keeps
   int one;                 // batch-1 block-column form (dense B == 1, K % 256 == 0)
   int off_zero;            // its zero activation region
   int off_xsum;            // its per-block activation sums (int4, int4aff)

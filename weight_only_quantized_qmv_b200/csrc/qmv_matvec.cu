@@ -421,40 +421,40 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   const uint32_t xbase = sbase + p.off_x;
 
   // ---- the warp's work items ------------------------------------------------
-  // Units are (column group, 16-row tile) pairs.  With at least as many
-  // units as warps (W), each warp takes whole units round robin (all of K,
-  // one warp, no reduction).  With fewer, units are dealt to CTAs and a CTA's
-  // 8 warps split each one along K, adding their partial sums in shared
-  // memory in warp order (deterministic).  Each warp streams its items
-  // through a private ring of S slices (kc in-features of 16 rows) filled by
-  // 16-byte asynchronous copies S-1 slices ahead of the math.
+  // Units are (column group, 16-row tile) pairs, each taken by a group of P
+  // warps of one CTA (P a power of two up to the CTA's warps): the group's
+  // warps split the unit's K in whole granules of p.gk and add their partial
+  // sums in shared memory in warp order (deterministic), behind the group's
+  // own named barrier.  P is the largest power of two with P * units <= the
+  // grid's warps whose parts keep at least p.min_part granules, so units are
+  // spread over every warp without cutting K finer than needed; with at
+  // least as many units as warps, P = 1 (whole units, no reduction).  Groups
+  // are numbered group-major across CTAs, so the units of a partial last
+  // round spread over the CTAs (and SMs) instead of filling whole CTAs
+  // first.  Each warp streams its items through a private ring of S slices
+  // (kc in-features of 16 rows) filled by 16-byte asynchronous copies S-1
+  // slices ahead of the math.
   const int ngroups = gt.ngroups;
   const int64_t total = (int64_t)ngroups * p.tiles;
   const int grid = (int)gridDim.x;
-  const int64_t W = (int64_t)grid * WARPS;
-  // Warps are numbered warp-major across CTAs, so the units of a partial last
-  // round land 4-5 per CTA instead of filling whole CTAs (and SMs) first.
-  const int64_t gwarp = (int64_t)warp * grid + blockIdx.x;
-  int64_t R, tail0;
-  int T;
-  if (total >= W) {  // whole units only: this warp's units gwarp, gwarp + W, ...
-    R = (total - gwarp + W - 1) / W;
-    tail0 = total;
-    T = 0;
-  } else {  // fewer units than warps: each CTA splits its units along K
-    R = 0;
-    tail0 = 0;
-    T = total > (int64_t)blockIdx.x ? (int)((total - blockIdx.x + grid - 1) / grid) : 0;
-  }
-  const int nitems = (int)R + T;
-  // this warp's share of K in the split units: whole granules of p.gk
   const int Kg = (int)((p.K + p.gk - 1) / p.gk);
-  const int kb_w = (int)min(p.K, (int64_t)(warp * Kg / WARPS) * p.gk);
-  const int ke_w = (int)min(p.K, (int64_t)((warp + 1) * Kg / WARPS) * p.gk);
+  int P = 1;
+  if (total < (int64_t)grid * WARPS) {  // (then every count below fits 32 bits)
+    const int units = (int)total, W = grid * WARPS;
+    while (2 * P <= WARPS && units * 2 * P <= W && Kg >= 2 * P * p.min_part) P *= 2;
+  }
+  const int gi = warp / P, wr = warp - gi * P;  // this warp's group in the CTA, its rank in the group
+  const int NG = grid * (WARPS / P);
+  const int ggrp = gi * grid + (int)blockIdx.x;
+  const int nitems = total > ggrp ? (int)((total - ggrp + NG - 1) / NG) : 0;
+  // this warp's part of K: whole granules of p.gk
+  const int kb_w = (int)min(p.K, (int64_t)(wr * Kg / P) * p.gk);
+  const int ke_w = (int)min(p.K, (int64_t)((wr + 1) * Kg / P) * p.gk);
   const int KC = p.KC;
-  const int nsl_main = p.nchunks;
-  const int nsl_tail = ke_w > kb_w ? (ke_w - kb_w + KC - 1) / KC : 0;
-  const int n_issue = nsl_tail > 0 ? nitems : (int)R;  // items that move any bytes
+  const int nsl_w = ke_w > kb_w ? (ke_w - kb_w + KC - 1) / KC : 0;
+  const int n_issue = nsl_w > 0 ? nitems : 0;  // items that move any bytes
+  // a group's barrier: id 1 + gi (0 is the CTA barrier), its P warps
+  auto group_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(32 * P) : "memory"); };
 
   struct Item {
     int64_t tile;
@@ -463,14 +463,8 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   };
   auto item_at = [&](int i) {
     Item it;
-    int64_t u;
-    if (i < R) {
-      u = gwarp + (int64_t)i * W;
-      it.kbeg = 0; it.kend = (int)p.K; it.nsl = nsl_main; it.split = false;
-    } else {
-      u = tail0 + blockIdx.x + (int64_t)(i - R) * grid;
-      it.kbeg = kb_w; it.kend = ke_w; it.nsl = nsl_tail; it.split = true;
-    }
+    const int64_t u = ggrp + (int64_t)i * NG;
+    it.kbeg = kb_w; it.kend = ke_w; it.nsl = nsl_w; it.split = P > 1;
     if (ngroups == 1) {
       it.grp = 0; it.tile = u;
     } else {
@@ -832,14 +826,15 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
           red[warp * 16 + g] = r0;
           red[warp * 16 + g + 8] = r1;
         }
-        __syncthreads();
-        if (tid < kTileRows) {
+        group_sync();
+        if (wr == 0 && lane < kTileRows) {  // the group's first warp adds its P partials in warp order
           float v = 0.0f;
 #pragma unroll
-          for (int w = 0; w < WARPS; ++w) v += red[w * 16 + tid];
-          if (tid < nrows) emit(0, pair, row0 + tid, v * f1);
+          for (int w = 0; w < WARPS; ++w)
+            if (w < P) v += red[(gi * P + w) * 16 + lane];
+          if (lane < nrows) emit(0, pair, row0 + lane, v * f1);
         }
-        __syncthreads();
+        group_sync();  // red is free again
       }
       continue;
     }
@@ -857,25 +852,32 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
         }
       }
     } else {
-      // split unit: partial sums of all 8 warps, added in warp order
+      // split unit: the group's P partial sums, added in warp order by the
+      // group's first warp (lane (g, t) keeps its own outputs)
 #pragma unroll
       for (int n = 0; n < NT; ++n)
 #pragma unroll
         for (int q = 0; q < 4; ++q) red[((warp * NT + n) * 4 + q) * 32 + lane] = acc[n][q];
-      __syncthreads();
-      if (tid < NT * 4 * 32) {
-        const int ln = tid & 31, q = (tid >> 5) & 3, n = tid >> 7;
-        float v = 0.0f;
+      group_sync();
+      if (wr == 0) {
 #pragma unroll
-        for (int w = 0; w < WARPS; ++w) v += red[((w * NT + n) * 4 + q) * 32 + ln];
-        const int col = 8 * n + 2 * (ln & 3) + (q & 1);
-        const int row = (ln >> 2) + 8 * (q >> 1);
-        if (col < ncols && row < nrows) {
-          const int pair = gt.sorted[gstart + col];
-          emit(0, pair, row0 + row, v * f);
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float v = 0.0f;
+#pragma unroll
+            for (int w = 0; w < WARPS; ++w)
+              if (w < P) v += red[(((gi * P + w) * NT + n) * 4 + q) * 32 + lane];
+            const int col = 8 * n + 2 * t + (q & 1);
+            const int row = g + 8 * (q >> 1);
+            if (col < ncols && row < nrows) {
+              const int pair = gt.sorted[gstart + col];
+              emit(2 * n + (q & 1), pair, row0 + row, v * f);
+            }
+          }
         }
       }
-      __syncthreads();
+      group_sync();  // red is free again
     }
   }
   cp_async_wait(0);
@@ -897,34 +899,13 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   p.expert_code_bytes = p.N * p.code_row_bytes;
   p.expert_aux_bytes = p.N * p.aux_row_bytes;
   p.tiles = (p.N + kTileRows - 1) / kTileRows;
-  // a warp's K-slice: kSliceBytes of codes per row
-  const int slice = kSliceBytes * 8 / fi.bits;
-  p.KC = (int)(p.K < slice ? p.K : slice);
-  p.nchunks = (int)((p.K + p.KC - 1) / p.KC);
-  const int64_t cb = (int64_t)p.KC * fi.bits / 8;
   // batch 1 (dense, 4-bit formats): the block-column form, for K in whole
   // groups of 8 blocks (int8 measured faster on the general form)
   p.one = (!p.gather && p.B == 1 && p.K % 256 == 0 && fi.bits == 4) ? 1 : 0;
-  // Row strides chosen so a warp's shared-memory reads are free of bank
-  // conflicts: 4-bit rows at 16 mod 128 bytes (32-bit loads), 8-bit rows at
-  // 32 mod 128 (64-bit loads); the batch-1 form's 128-bit loads want 4-bit
-  // rows at 64 mod 128 and 8-bit rows at 16 mod 128.
-  if (p.one)
-    p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 64 : 16));
-  else
-    p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 16 : 32));
-  int64_t aux_region;
-  // split units divide K in granules whose code and scale segments start on
-  // 16- and 8-byte boundaries
-  // (affine int4: 256, so a granule's zero points start on a 4-byte boundary)
-  p.gk = (p.one || fi.zp) ? 256 : (fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128));
   p.zoff = 0;
   if (fi.lut) {
     p.aux_mode = kAuxLut;
-    p.AS = 32;
-    aux_region = kTileRows * 32;
   } else {
-    const int64_t slice_sc = (int64_t)(p.KC / 32) * fi.scale_bytes;
     // asynchronous 8-byte scale copies when every row's scales start on an
     // 8-byte boundary and come in whole 8-byte pieces (affine int4: and the
     // zero points of every slice in whole 4-byte pieces)
@@ -932,27 +913,60 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
     const bool zp_ok = !fi.zp || (p.zplane % 4 == 0 && p.K % 256 == 0);
     p.aux_mode = (based && p.aux_row_bytes % 8 == 0 && zp_ok) ? kAuxRows : kAuxBlock;
     if (p.aux_mode == kAuxBlock) p.one = 0;
-    // a staged row: the slice's scales, then (affine int4) its zero points
-    p.zoff = fi.zp ? (int)round_up(slice_sc, 8) : 0;
-    const int64_t row_bytes = fi.zp ? p.zoff + (p.KC / 32 + 1) / 2 : slice_sc;
-    int64_t j = (row_bytes + 15) / 16;
-    // the batch-1 form reads 4 bytes of rows g = 0..7 per load: an odd
-    // multiple of 16 bytes puts them in distinct banks (elsewhere the scale
-    // loads are a few per slice and the tighter rows let more warps fit)
-    if (p.one && j % 2 == 0) ++j;
-    p.AS = (int)(16 * j);
-    aux_region = kTileRows * p.AS;
   }
-  p.aux_off = kTileRows * p.RS;
-  p.stage_bytes = (int)round_up(p.aux_off + aux_region, 128);
+  // split units divide K in granules whose code and scale segments start on
+  // 16- and 8-byte boundaries
+  // (affine int4: 256, so a granule's zero points start on a 4-byte boundary)
+  p.gk = (p.one || fi.zp) ? 256 : (fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128));
+  // a warp's part of a split unit keeps at least 256 in-features
+  p.min_part = 256 / p.gk > 1 ? 256 / p.gk : 1;
+  // A warp's K-slice: kSliceBytes of codes per row, or half of that where
+  // the full ring leaves no room for enough warps (large staged activations).
+  auto slice_geometry = [&](int slice_bytes) {
+    const int slice = slice_bytes * 8 / fi.bits;
+    p.KC = (int)(p.K < slice ? p.K : slice);
+    p.nchunks = (int)((p.K + p.KC - 1) / p.KC);
+    const int64_t cb = (int64_t)p.KC * fi.bits / 8;
+    // Row strides chosen so a warp's shared-memory reads are free of bank
+    // conflicts: 4-bit rows at 16 mod 128 bytes (32-bit loads), 8-bit rows at
+    // 32 mod 128 (64-bit loads); the batch-1 form's 128-bit loads want 4-bit
+    // rows at 64 mod 128 and 8-bit rows at 16 mod 128.
+    if (p.one)
+      p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 64 : 16));
+    else
+      p.RS = (int)(round_up(cb, 128) + (fi.bits == 4 ? 16 : 32));
+    int64_t aux_region;
+    if (fi.lut) {
+      p.AS = 32;
+      aux_region = kTileRows * 32;
+    } else {
+      const int64_t slice_sc = (int64_t)(p.KC / 32) * fi.scale_bytes;
+      // a staged row: the slice's scales, then (affine int4) its zero points
+      p.zoff = fi.zp ? (int)round_up(slice_sc, 8) : 0;
+      const int64_t row_bytes = fi.zp ? p.zoff + (p.KC / 32 + 1) / 2 : slice_sc;
+      int64_t j = (row_bytes + 15) / 16;
+      // the batch-1 form reads 4 bytes of rows g = 0..7 per load: an odd
+      // multiple of 16 bytes puts them in distinct banks (elsewhere the scale
+      // loads are a few per slice and the tighter rows let more warps fit)
+      if (p.one && j % 2 == 0) ++j;
+      p.AS = (int)(16 * j);
+      aux_region = kTileRows * p.AS;
+    }
+    p.aux_off = kTileRows * p.RS;
+    p.stage_bytes = (int)round_up(p.aux_off + aux_region, 128);
+  };
   p.XS = (int)(round_up(2 * p.K, 128) + 64);  // 64 mod 128: conflict-free 128-bit reads
   p.n_xrows = p.gather ? (p.x_per_slot ? p.B * p.topk : p.B) : p.B;
   const int nt = p.B > 8 ? 2 : 1;
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
-  // Layouts in order of preference: two 8-warp CTAs per SM, else one 16-warp
-  // CTA (the staged activations shared by 16 warps), else one 8-warp CTA;
-  // within each the deepest ring (<= kStages slices per warp) that fits.
-  const int cand[3][2] = {{kWarps, kMinCtas}, {2 * kWarps, 1}, {kWarps, 1}};
+  // Layouts in order of preference (warps, CTAs per SM, slice halved):
+  // two 8-warp CTAs per SM, else one 16-warp CTA (the staged activations
+  // shared by 16 warps), then the 16-warp CTA with half slices (more warps
+  // beat longer slices where the activations leave little room), else one
+  // 8-warp CTA; within each the deepest ring (<= kStages slices per warp)
+  // that fits.  (Half slices in two 8-warp CTAs measured slower than one
+  // 16-warp CTA with whole slices, so that layout is not tried.)
+  const int cand[5][3] = {{kWarps, kMinCtas, 0}, {2 * kWarps, 1, 0}, {2 * kWarps, 1, 1}, {kWarps, 1, 0}, {kWarps, 1, 1}};
   // one CTA per (group, tile) unit up to the resident-CTA slots
   const int64_t upper_units = (p.gather ? (int64_t)p.B * p.topk : 1) * p.tiles;
   // int4km up to 8 activation columns: lane palette copies in shared memory
@@ -961,9 +975,10 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   // cost ring depth that the byte-permute lookups do not need: measured
   // slower.)
   const bool km_ok = fi.lut && p.B <= 8;
-  for (int ci = 0; ci < 3; ++ci) {
+  for (int ci = 0; ci < 5; ++ci) {
     const int warps = cand[ci][0], ctas = cand[ci][1];
     if (warps != kWarps && p.one) continue;  // the batch-1 form fits two 8-warp CTAs
+    slice_geometry(cand[ci][2] ? kSliceBytes / 2 : kSliceBytes);
     for (int km = km_ok ? 1 : 0; km >= 0; --km) {
       p.warps = warps;
       p.km_smem = km;
@@ -1036,7 +1051,9 @@ static cudaError_t launch_fa(const MvParams& p, cudaStream_t stream) {
       return wide ? launch_t<FMT, 1, 2 * kWarps, AM, true>(p, stream) : launch_t<FMT, 1, kWarps, AM, true>(p, stream);
     }
   }
-  if (p.one) return launch_t<FMT, 0, kWarps, AM>(p, stream);
+  if constexpr (FMT != QMV_FMT_INT8) {  // the batch-1 form (4-bit formats)
+    if (p.one) return launch_t<FMT, 0, kWarps, AM>(p, stream);
+  }
   if (p.B > 8) return wide ? launch_t<FMT, 2, 2 * kWarps, AM>(p, stream) : launch_t<FMT, 2, kWarps, AM>(p, stream);
   return wide ? launch_t<FMT, 1, 2 * kWarps, AM>(p, stream) : launch_t<FMT, 1, kWarps, AM>(p, stream);
 }

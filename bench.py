@@ -600,7 +600,9 @@ DECODE_E, DECODE_TOPK, DECODE_H, DECODE_I, DECODE_LAYERS = 256, 8, 2048, 512, 10
 def decode_step_weights(dev):
     """Stand-in int4km weights of the decode step (fitted shapes, random
     palettes and indices): 10 layers of q (4096x2048) and o (2048x4096), one
-    routed-expert layer (gate and up [256, 512, 2048], down [256, 2048, 512])."""
+    routed-expert layer: gate and up [256, 512, 2048] stored as one stack
+    [256, 1024, 2048] (each expert's gate rows, then its up rows) so that one
+    gather launch serves both, and down [256, 2048, 512]."""
     from weight_only_quantized_qmv_b200 import synth
     g = synth.generator(11, dev)
     E, H, I = DECODE_E, DECODE_H, DECODE_I
@@ -609,21 +611,20 @@ def decode_step_weights(dev):
         ql, qi = synth.palette_tables(4096, H, g)
         ol, oi = synth.palette_tables(H, 4096, g)
         layers.append((qi, ql, oi, ol))
-    gl, gi = synth.palette_tables(E * I, H, g)
-    ul, ui = synth.palette_tables(E * I, H, g)
+    gl, gi = synth.palette_tables(E * 2 * I, H, g)
     dl, di = synth.palette_tables(E * H, I, g)
-    experts = (gi.view(E, I, H // 2), gl.view(E, I, 16), ui.view(E, I, H // 2), ul.view(E, I, 16),
-               di.view(E, H, I // 2), dl.view(E, H, 16))
+    experts = (gi.view(E, 2 * I, H // 2), gl.view(E, 2 * I, 16), di.view(E, H, I // 2), dl.view(E, H, 16))
     return layers, experts, g
 
 
 def decode_step_fn(q, layers, experts, lm_idx, lm_lut, B, dev, stream, g):
-    """The decode step's 24 launches for B tokens, as a closure on `stream`,
-    and the number of distinct experts its routing selects."""
+    """The decode step's 23 launches for B tokens (lm_head, 10 x (q, o),
+    gate+up, down), as a closure on `stream`, and the number of distinct
+    experts its routing selects."""
     import torch
     from weight_only_quantized_qmv_b200 import synth
     E, topk, H, I = DECODE_E, DECODE_TOPK, DECODE_H, DECODE_I
-    gi, gl, ui, ul, di, dl = experts
+    gui, gul, di, dl = experts
     x_h = synth.activations(B, H, g)
     x_o = synth.activations(B, 4096, g)
     x_d = synth.activations(B, I, g, extra_shape=(topk,))
@@ -631,16 +632,14 @@ def decode_step_fn(q, layers, experts, lm_idx, lm_lut, B, dev, stream, g):
     y_lm = torch.empty((B, lm_idx.shape[0]), dtype=torch.float32, device=dev)
     y_q = torch.empty((B, 4096), dtype=torch.float32, device=dev)
     y_o = torch.empty((B, H), dtype=torch.float32, device=dev)
-    y_g = torch.empty((B, topk, I), dtype=torch.float32, device=dev)
-    y_u = torch.empty((B, topk, I), dtype=torch.float32, device=dev)
+    y_gu = torch.empty((B, topk, 2 * I), dtype=torch.float32, device=dev)
     y_d = torch.empty((B, topk, H), dtype=torch.float32, device=dev)
 
     def step():
         for qi, ql, oi, ol in layers:
             q.matvec_int4km(qi, ql, x_h, out=y_q, stream=stream)
             q.matvec_int4km(oi, ol, x_o, out=y_o, stream=stream)
-        q.gather_matvec(q.FMT_INT4KM, gi, gl, ids, x_h, out=y_g, stream=stream)
-        q.gather_matvec(q.FMT_INT4KM, ui, ul, ids, x_h, out=y_u, stream=stream)
+        q.gather_matvec(q.FMT_INT4KM, gui, gul, ids, x_h, out=y_gu, stream=stream)
         q.gather_matvec(q.FMT_INT4KM, di, dl, ids, x_d, x_per_slot=True, out=y_d, stream=stream)
         q.matvec_int4km(lm_idx, lm_lut, x_h, out=y_lm, stream=stream)
 
@@ -651,7 +650,7 @@ def measure_decode_step(q, lm_idx, lm_lut, dev, stream, reps=STAT_REPLAYS):
     """The int4km decode step of the workload list, timed as one CUDA graph per
     batch size: the 248320x2048 lm_head, 10 layers of q (4096x2048) and o
     (2048x4096), and one routed-expert layer (256 experts; gate and up
-    512x2048, down 2048x512; top-8 uniform routing).  Random palettes and
+    512x2048 in one launch, down 2048x512; top-8 uniform routing).  Random palettes and
     indices of the fitted shapes; each launch reads fixed synthetic
     activations (the step's data flow between layers is not modelled)."""
     layers, experts, g = decode_step_weights(dev)
@@ -666,7 +665,7 @@ def measure_decode_step(q, lm_idx, lm_lut, dev, stream, reps=STAT_REPLAYS):
         dense = (algorithmic_bytes("int4km", N_HEAD, H, B)
                  + 10 * (algorithmic_bytes("int4km", 4096, H, B) + algorithmic_bytes("int4km", H, 4096, B)))
         expert = n_exp * (2 * (I * H // 2 + I * 32) + (H * I // 2 + H * 32))
-        res[f"b{B}"] = {"us": us, "us_p10": st["p10"], "us_p90": st["p90"], "launches": 24,
+        res[f"b{B}"] = {"us": us, "us_p10": st["p10"], "us_p90": st["p90"], "launches": 23,
                         "distinct_experts": n_exp, "bytes": dense + expert,
                         "gbs": round((dense + expert) / (us * 1e-6) / 1e9, 1)}
     return res
@@ -837,7 +836,7 @@ def profile_case(name: str) -> int:
     from weight_only_quantized_qmv_b200 import synth
     N, K = 65536, K_HEAD
     if name.startswith("decode_step"):
-        # the full decode step (24 launches: lm_head, 10 x (q, o), gate, up,
+        # the full decode step (23 launches: lm_head, 10 x (q, o), gate+up,
         # down), captured as a graph and replayed three times
         B = int(name[-1])
         dev = torch.device("cuda", 0)
@@ -852,7 +851,7 @@ def profile_case(name: str) -> int:
                 gph.replay()
         stream.synchronize()
         flags = q.status_fetch()
-        print(json.dumps({"profile_case": name, "launches_per_step": 24, "steps": 5, "distinct_experts": n_exp,
+        print(json.dumps({"profile_case": name, "launches_per_step": 23, "steps": 5, "distinct_experts": n_exp,
                           "flags": flags}), flush=True)
         return 1 if flags else 0
     g = synth.generator(0, "cuda")

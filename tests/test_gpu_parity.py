@@ -750,7 +750,8 @@ def test_full_int4km_head_248320x2048(q):
 @pytest.mark.parametrize("B", [1, 8])
 def test_full_decode_step_int4km(q, B):
     """lm_head + 10 x (q_proj 2048->4096, o_proj 4096->2048) + routed experts
-    256 x (gate/up 2048->512, down 512->2048), top-8 routing."""
+    256 x (gate/up 2048->512, down 512->2048), top-8 routing; gate and up as
+    one [256, 1024, 2048] stack (one gather launch serves both)."""
     g = synth.generator(1000 + B, "cuda")
     dense = [(248320, 2048)] + [(4096, 2048), (2048, 4096)] * 10
     for i, (N, K) in enumerate(dense):
@@ -762,7 +763,7 @@ def test_full_decode_step_int4km(q, B):
         assert rel_err(y.cpu().numpy()[:, rows], r) < TOL, (i, N, K)
     E, topk = 256, 8
     ids = synth.routing(B, topk, E, g)
-    for name, N, K, per_slot in (("gate", 512, 2048, 0), ("up", 512, 2048, 0), ("down", 2048, 512, 1)):
+    for name, N, K, per_slot in (("gate_up", 1024, 2048, 0), ("down", 2048, 512, 1)):
         lut, idx = synth.palette_tables(E * N, K, g)
         lut, idx = lut.view(E, N, 16), idx.view(E, N, K // 2)
         x = synth.activations(B, K, g, extra_shape=(topk,) if per_slot else ())

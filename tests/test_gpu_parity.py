@@ -267,8 +267,10 @@ def _inputs(fmt, N, K, B, seed):
 def test_matvec_parity(q, fmt, N, K, B):
     c_o, s_o, xn = _inputs(fmt, N, K, B, seed=N * 7 + K + B)
     c, s, x = torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(), torch.from_numpy(xn).cuda()
-    if B * K * 2 > 160 * 1024:
-        # activations beyond the on-chip staging are rejected on the host
+    if B * K * 2 > 160 * 1024 and fmt == "int8km":
+        # int8km's kernel stages all of K: activations beyond the on-chip
+        # staging are rejected on the host (the other formats stage them in
+        # K-phases)
         with pytest.raises(q.QmvError) as ei:
             q.matvec(q.__dict__["FMT_" + fmt.upper()], c, s, x)
         assert ei.value.status == q.ERR_UNSUPPORTED
@@ -306,6 +308,62 @@ def test_int4km_palette_copy_equals_register_lookup(q):
     y8 = q.matvec_int4km(idx, lut, x9[:8].contiguous())
     y9 = q.matvec_int4km(idx, lut, x9)
     assert torch.equal(y8, y9[:8])
+    assert q.status_fetch() == 0
+
+
+PHASED_FMTS = ("fp4", "int4", "int4km", "int8", "int4aff")
+
+
+@pytest.mark.parametrize("fmt", PHASED_FMTS)
+@pytest.mark.parametrize("N,K,B", [(100, 16384, 16), (40, 6144, 9), (300, 8192, 12), (33, 32768, 3)])
+def test_matvec_phased_staging_parity(q, fmt, N, K, B):
+    """Activations larger than the on-chip staging (B * K * 2 bytes beyond
+    ~160 KB) are staged one K-phase at a time: the result still matches the
+    oracle (several phases, ragged row tiles, 3..16 columns)."""
+    c_o, s_o, xn = _inputs(fmt, N, K, B, seed=N + K + B)
+    y = q.matvec(q.__dict__["FMT_" + fmt.upper()], torch.from_numpy(c_o).cuda(), torch.from_numpy(s_o).cuda(),
+                 torch.from_numpy(xn).cuda()).cpu().numpy()
+    r = orc.matvec(FID[fmt], c_o, s_o, xn, N, K)
+    assert rel_err(y, r) < TOL
+    assert q.status_fetch() == 0
+
+
+@pytest.mark.parametrize("fmt", ("fp4", "int4km"))
+def test_gather_phased_staging_parity(q, fmt):
+    """Per-slot activations of 64 (token, slot) pairs at K = 4096 (512 KB)
+    are staged in K-phases: every slot still equals the oracle's matvec with
+    its expert."""
+    E, N, K, B, topk = 16, 64, 4096, 8, 8
+    g = synth.generator(77, "cpu")
+    W, _ = synth.weights(E * N, K, g)
+    Wn = W.numpy()
+    c_o, s_o, _ = encode_orc(fmt, Wn)
+    ids = synth.routing(B, topk, E, g)
+    x = synth.activations(B, K, g, extra_shape=(topk,))
+    c = torch.from_numpy(c_o).cuda().view(E, N, -1)
+    a = torch.from_numpy(s_o).cuda().view(E, N, -1)
+    y = q.gather_matvec(q.__dict__["FMT_" + fmt.upper()], c, a, ids.cuda(), x.cuda(), x_per_slot=True).cpu().numpy()
+    xn, ids_n = x.numpy(), ids.numpy()
+    for b in range(B):
+        for j in range(topk):
+            e = ids_n[b, j]
+            r = orc.matvec(FID[fmt], c_o[e * N:(e + 1) * N], s_o[e * N:(e + 1) * N], xn[b, j][None], N, K)
+            assert rel_err(y[b, j][None], r) < TOL, (b, j)
+    assert q.status_fetch() == 0
+
+
+def test_argmax_phased_staging(q):
+    """The fused argmax over a launch with phased activation staging equals
+    torch.argmax of the unfused outputs (16 columns, K = 12288)."""
+    N, K, B = 3000, 12288, 16
+    g = synth.generator(78, "cuda")
+    W, _ = synth.weights(N, K, g)
+    codes, scales = q.encode_fp4(W)
+    x = synth.activations(B, K, g)
+    y = q.matvec_fp4(codes, scales, x)
+    idx, val = q.matvec_argmax(q.FMT_FP4, codes, scales, x, q.argmax_workspace())
+    assert torch.equal(idx.long(), torch.argmax(y, dim=1))
+    assert torch.equal(val, y.max(dim=1).values)
     assert q.status_fetch() == 0
 
 

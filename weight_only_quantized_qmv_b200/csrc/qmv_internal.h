@@ -76,6 +76,7 @@ struct MvParams {
   int aux_mode;
   int stages, stage_bytes, aux_off;  // ring geometry; aux_off: scale region inside a stage
   int XS;                  // shared-memory bytes per staged activation row
+  int64_t xphase;          // 0: all of K staged; else in-features staged per phase (a multiple of KC)
   int n_xrows;             // activation rows staged
   int off_red, off_x, off_stage;  // dynamic shared-memory offsets
   int smem_bytes;

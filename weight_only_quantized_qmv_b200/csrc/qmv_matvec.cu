@@ -394,7 +394,9 @@ __device__ __forceinline__ void slice_one(float (&acc)[2], float (&dl)[4], uint3
 // AM: fused argmax (outputs folded into per-row maxima instead of stored).
 // KMS: int4km with lane palette copies in shared memory for rows g+8 (the
 // host sets it where they fit; batch <= 8).
-template <int FMT, int NT, int WARPS, bool AM, bool KMS>
+// PH: activations staged one K-phase at a time (p.xphase in-features), for
+// activations beyond the on-chip staging (the general form, whole units).
+template <int FMT, int NT, int WARPS, bool AM, bool KMS, bool PH>
 __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kernel(const __grid_constant__ MvParams p) {
   using F = FmtT<FMT>;
   constexpr bool kOne = NT == 0;
@@ -439,7 +441,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   const int grid = (int)gridDim.x;
   const int Kg = (int)((p.K + p.gk - 1) / p.gk);
   int P = 1;
-  if (total < (int64_t)grid * WARPS) {  // (then every count below fits 32 bits)
+  if (total < (int64_t)grid * WARPS && !(PH && !kOne)) {  // (then every count below fits 32 bits)
     const int units = (int)total, W = grid * WARPS;
     while (2 * P <= WARPS && units * 2 * P <= W && Kg >= 2 * P * p.min_part) P *= 2;
   }
@@ -596,25 +598,26 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
 
   if (p.prefetch) grid_wait_preceding();  // weights only before this point
 
-  // The activations are staged while the first weight slices are in flight.
-  // Activations once per CTA: row r at xbase + r * XS, in the k order the
-  // format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7) per 8).
-  {
-    const int64_t per_row = p.K / 8;
+  // Activations are staged once per CTA: row r at xbase + r * XS, in the k
+  // order the format's decoder emits (int4: (k0,k4),(k1,k5),(k2,k6),(k3,k7)
+  // per 8).
+  auto stage_x = [&](int64_t k_lo, int64_t k_hi) {
+    const int64_t per_row = (k_hi - k_lo) / 8;
     const int64_t n16 = (int64_t)p.n_xrows * per_row;
     for (int64_t i = tid; i < n16; i += kT) {
       const int64_t r = i / per_row, j = i - r * per_row;
+      const int64_t k = k_lo + 8 * j;
       uint4 v;
       if (p.xcols) {
         // the main columns of a wider activation row (the mixed format's
-        // int4km part): in-feature 8j + e is column main_column(8j + e)
+        // int4km part): in-feature k + e is column main_column(k + e)
         uint32_t h[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          h[e] = ldg_u16(p.x + r * p.xstride + main_column(p.xcols, p.ncols, 8 * j + e, p.xstride));
+          h[e] = ldg_u16(p.x + r * p.xstride + main_column(p.xcols, p.ncols, k + e, p.xstride));
         v = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
       } else {
-        v = ldg_nc_128(p.x + r * p.K + 8 * j);
+        v = ldg_nc_128(p.x + r * p.K + k);
       }
       if constexpr (F::kPermX && kOne) {  // (k0,k4), (k2,k6), (k1,k5), (k3,k7)
         v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.y, v.w, 0x5410u), prmt(v.x, v.z, 0x7632u),
@@ -625,6 +628,13 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       }
       sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
     }
+  };
+  // The activations are staged while the first weight slices are in flight
+  // (all of K; or, where they do not fit on chip, one K-phase at a time in
+  // the consume loop below).
+  constexpr bool phased = PH && !kOne;
+  {
+    if (!phased) stage_x(0, p.K);
     if constexpr (kOne && (FMT == QMV_FMT_INT4 || FMT == QMV_FMT_INT4AFF)) {
       // per-block activation sums: exact in fp64 (32 fp16 terms), one rounding to fp32
       for (int64_t b = tid; b < p.K / 32; b += kT) {
@@ -688,13 +698,19 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
   uint32_t xa[NTX];
   int xa_grp = -1;
   uint32_t cons = ring;
-  for (int i = 0; i < nitems; ++i) {
-    const Item it = item_at(i);
-    const int grp = it.grp;
+  // Phased staging: every warp runs the same rounds of whole units (a warp
+  // without a unit in the last round only takes part in the staging), and
+  // the CTA stages phase f's activations at the slice where it begins.
+  const int rounds = phased ? (int)((total + NG - 1) / NG) : nitems;
+  int xk0 = 0;  // first in-feature of the staged activations
+  for (int i = 0; i < rounds; ++i) {
+    const bool has = !phased || i < nitems;
+    const Item it = item_at(has ? i : 0);
+    const int grp = has ? it.grp : 0;
     const int64_t row0 = it.tile * kTileRows;
     const int nrows = (int)min((int64_t)kTileRows, p.N - row0);
     const int ncols = gt.count[grp], gstart = gt.start[grp];
-    if (grp != xa_grp) {  // activation rows of this column group
+    if (has && grp != xa_grp) {  // activation rows of this column group
       xa_grp = grp;
 #pragma unroll
       for (int n = 0; n < NTX; ++n) {
@@ -716,7 +732,26 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
     acc1[0] = acc1[1] = 0.0f;
     dl[0] = dl[1] = dl[2] = dl[3] = 0.0f;
 
-    for (int c = 0; c < it.nsl; ++c) {
+    for (int c = 0; c < (has ? it.nsl : p.nchunks); ++c) {
+      if (phased && (c * KC) % (int)p.xphase == 0) {
+        // one K-phase of every activation row (the general form: natural
+        // order, or int4's (k0,k4),(k1,k5),... per 8); 32-bit indices, the
+        // staged phase fits in shared memory
+        __syncthreads();  // every warp is done with the previous phase
+        xk0 = c * KC;
+        const int per_row = min((int)p.xphase, (int)p.K - xk0) / 8;
+        const int n16 = p.n_xrows * per_row;
+        for (int e = tid; e < n16; e += kT) {
+          const int r = e / per_row, j = e - r * per_row;
+          uint4 v = ldg_nc_128(p.x + (int64_t)r * p.K + xk0 + 8 * j);
+          if constexpr (F::kPermX)
+            v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
+                           prmt(v.y, v.w, 0x7632u));
+          sts128(xbase + (uint32_t)(r * p.XS + 16 * j), v);
+        }
+        __syncthreads();
+      }
+      if (phased && !has) continue;
       // keep S-1 slices in flight: refill the stage freed by the previous slice
       if (ii < n_issue) issue_next(fill);
       cp_async_commit();
@@ -773,7 +808,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       }
       uint32_t xb[NTX];
 #pragma unroll
-      for (int n = 0; n < NTX; ++n) xb[n] = xa[n] + (uint32_t)k0 * 2u;
+      for (int n = 0; n < NTX; ++n) xb[n] = xa[n] + (uint32_t)(k0 - xk0) * 2u;
       if (kc == kNB * 32 && aux_fast) {
         slice_full<FMT, NTX, kNB, KMS>(acc, crow_g, crow_g8, sa_g, sa_g8, zo, xb, t, pg, pg8, mul, ktb);
       } else if (kc == kNB * 16 && aux_fast) {
@@ -802,6 +837,7 @@ __global__ void __launch_bounds__(32 * WARPS, WARPS == 8 ? kMinCtas : 1) mv_kern
       __syncwarp();  // all lanes are done with this stage before it is refilled
       cons = (cons + p.stage_bytes == ring_end) ? ring : cons + p.stage_bytes;
     }
+    if (phased && !has) continue;
 
     // ---- outputs: lane (g, t) holds rows g, g+8, columns 2t, 2t+1 of each n-tile ----
     const float f = (FMT == QMV_FMT_FP4) ? 0.5f : 1.0f;  // the fp4 block scales carried a factor 2
@@ -914,12 +950,6 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
     p.aux_mode = (based && p.aux_row_bytes % 8 == 0 && zp_ok) ? kAuxRows : kAuxBlock;
     if (p.aux_mode == kAuxBlock) p.one = 0;
   }
-  // split units divide K in granules whose code and scale segments start on
-  // 16- and 8-byte boundaries
-  // (affine int4: 256, so a granule's zero points start on a 4-byte boundary)
-  p.gk = (p.one || fi.zp) ? 256 : (fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128));
-  // a warp's part of a split unit keeps at least 256 in-features
-  p.min_part = 256 / p.gk > 1 ? 256 / p.gk : 1;
   // A warp's K-slice: kSliceBytes of codes per row, or half of that where
   // the full ring leaves no room for enough warps (large staged activations).
   auto slice_geometry = [&](int slice_bytes) {
@@ -955,7 +985,6 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
     p.aux_off = kTileRows * p.RS;
     p.stage_bytes = (int)round_up(p.aux_off + aux_region, 128);
   };
-  p.XS = (int)(round_up(2 * p.K, 128) + 64);  // 64 mod 128: conflict-free 128-bit reads
   p.n_xrows = p.gather ? (p.x_per_slot ? p.B * p.topk : p.B) : p.B;
   const int nt = p.B > 8 ? 2 : 1;
   const int64_t dyn_limit = (int64_t)kSmemLimit - kStaticSmem;
@@ -975,54 +1004,82 @@ bool plan_matvec(int fmt, MvParams& p, int num_sms) {
   // cost ring depth that the byte-permute lookups do not need: measured
   // slower.)
   const bool km_ok = fi.lut && p.B <= 8;
-  for (int ci = 0; ci < 5; ++ci) {
-    const int warps = cand[ci][0], ctas = cand[ci][1];
-    if (warps != kWarps && p.one) continue;  // the batch-1 form fits two 8-warp CTAs
-    slice_geometry(cand[ci][2] ? kSliceBytes / 2 : kSliceBytes);
-    for (int km = km_ok ? 1 : 0; km >= 0; --km) {
-      p.warps = warps;
-      p.km_smem = km;
-      const int64_t slots = (int64_t)num_sms * ctas;
-      p.grid = (int)(upper_units < slots ? upper_units : slots);
-      // Units are split along K (partial sums meet in shared memory) only when
-      // there are fewer than the grid's warps; a (group, tile) count of at
-      // least p.tiles means that can happen only if p.tiles is below it.
-      const bool may_split = p.tiles < (int64_t)p.grid * warps;
-      p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
-      p.off_x = may_split ? (int)round_up((int64_t)warps * nt * 4 * 32 * 4, 128) : 0;
-      // the zero region starts 32 bytes past a 128-byte line: its reads and the
-      // activation reads of the same instruction fall in different banks
-      p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
-      p.off_xsum = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
-      const bool xsum = p.one && (fmt == QMV_FMT_INT4 || fmt == QMV_FMT_INT4AFF);
-      // the copies' region is aligned to 4 KB at run time: with the dynamic
-      // shared memory 1 KB aligned and this offset a multiple of 1 KB, the
-      // alignment moves it by at most 3 KB
-      p.off_kmtab = (int)round_up(p.off_xsum + (xsum ? 4 * (p.K / 32) : 0), km ? 1024 : 128);
-      const int64_t kmtab = km ? 4096 * (int64_t)((warps + 3) / 4) + 3072 : 0;
-      p.off_stage = (int)round_up(p.off_kmtab + kmtab, 128);
-      for (int st = kStages; st >= 2; --st) {
-        const int64_t bytes = p.off_stage + (int64_t)warps * st * p.stage_bytes;
-        if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
-          p.stages = st;
-          p.smem_bytes = (int)bytes;
-          p.ctas_per_sm = ctas;
-          return true;
+  auto try_layouts = [&](bool phased) -> bool {
+    // split units divide K in granules whose code and scale segments start on
+    // 16- and 8-byte boundaries
+    // (affine int4: 256, so a granule's zero points start on a 4-byte boundary)
+    p.gk = (p.one || fi.zp) ? 256 : (fi.lut ? 32 : (fi.scale_bytes == 1 ? 256 : 128));
+    // a warp's part of a split unit keeps at least 256 in-features
+    p.min_part = 256 / p.gk > 1 ? 256 / p.gk : 1;
+    // staged activation rows: all of K, or one phase
+    p.XS = (int)(round_up(2 * (p.xphase ? p.xphase : p.K), 128) + 64);  // 64 mod 128: conflict-free 128-bit reads
+    for (int ci = 0; ci < 5; ++ci) {
+      const int warps = cand[ci][0], ctas = cand[ci][1];
+      if (warps != kWarps && p.one) continue;  // the batch-1 form fits two 8-warp CTAs
+      if (phased && warps != 2 * kWarps) continue;  // phased staging: the 16-warp instances
+      slice_geometry(cand[ci][2] ? kSliceBytes / 2 : kSliceBytes);
+      for (int km = (km_ok && !phased) ? 1 : 0; km >= 0; --km) {
+        p.warps = warps;
+        p.km_smem = km;
+        const int64_t slots = (int64_t)num_sms * ctas;
+        p.grid = (int)(upper_units < slots ? upper_units : slots);
+        // Units are split along K (partial sums meet in shared memory) only when
+        // there are fewer than the grid's warps; a (group, tile) count of at
+        // least p.tiles means that can happen only if p.tiles is below it.
+        const bool may_split = p.tiles < (int64_t)p.grid * warps && p.xphase == 0;
+        p.off_red = 0;  // split-unit partial sums: [warp][nt][4][32] floats
+        p.off_x = may_split ? (int)round_up((int64_t)warps * nt * 4 * 32 * 4, 128) : 0;
+        // the zero region starts 32 bytes past a 128-byte line: its reads and the
+        // activation reads of the same instruction fall in different banks
+        p.off_zero = (int)round_up(p.off_x + (int64_t)p.n_xrows * p.XS, 128) + 32;
+        p.off_xsum = (int)round_up(p.off_zero + (p.one ? kZeroBytes : 0), 128);
+        const bool xsum = p.one && (fmt == QMV_FMT_INT4 || fmt == QMV_FMT_INT4AFF);
+        // the copies' region is aligned to 4 KB at run time: with the dynamic
+        // shared memory 1 KB aligned and this offset a multiple of 1 KB, the
+        // alignment moves it by at most 3 KB
+        p.off_kmtab = (int)round_up(p.off_xsum + (xsum ? 4 * (p.K / 32) : 0), km ? 1024 : 128);
+        const int64_t kmtab = km ? 4096 * (int64_t)((warps + 3) / 4) + 3072 : 0;
+        p.off_stage = (int)round_up(p.off_kmtab + kmtab, 128);
+        for (int st = kStages; st >= 2; --st) {
+          const int64_t bytes = p.off_stage + (int64_t)warps * st * p.stage_bytes;
+          if (bytes <= dyn_limit && ctas * (bytes + kStaticSmem + 1024) <= kSmemPerSM) {
+            p.stages = st;
+            p.smem_bytes = (int)bytes;
+            p.ctas_per_sm = ctas;
+            return true;
+          }
         }
       }
     }
+    return false;
+  };
+  p.xphase = 0;
+  if (try_layouts(false)) return true;
+  // Activations beyond the on-chip staging: stage them one K-phase at a time
+  // (whole slices; the general form).  The fewest phases that fit.  (Not for
+  // the mixed format's main part, whose staged columns are remapped.)
+  if (p.xcols) return false;
+  p.one = 0;
+  const int64_t full_kc = kSliceBytes * 8 / fi.bits;
+  int64_t prev = p.K;
+  for (int64_t nph = 2; nph <= (p.K + full_kc - 1) / full_kc; ++nph) {
+    p.xphase = round_up((p.K + nph - 1) / nph, full_kc);
+    if (p.xphase >= prev) continue;  // the same phase as fewer phases gave
+    prev = p.xphase;
+    if (try_layouts(true)) return true;
   }
+  p.xphase = 0;
   return false;
 }
 
-template <int FMT, int NT, int WARPS, bool AM, bool KMS = false>
+template <int FMT, int NT, int WARPS, bool AM, bool KMS = false, bool PH = false>
 static cudaError_t launch_t(const MvParams& p, cudaStream_t stream) {
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
-    err = cudaFuncSetAttribute(mv_kernel<FMT, NT, WARPS, AM, KMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(mv_kernel<FMT, NT, WARPS, AM, KMS, PH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemLimit - kStaticSmem);
     if (err != cudaSuccess) return err;
     attr_set[dev].store(true, std::memory_order_release);
@@ -1037,7 +1094,7 @@ static cudaError_t launch_t(const MvParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT, WARPS, AM, KMS>, p);
+  return cudaLaunchKernelEx(&cfg, mv_kernel<FMT, NT, WARPS, AM, KMS, PH>, p);
 }
 
 template <int FMT, bool AM>
@@ -1045,6 +1102,9 @@ static cudaError_t launch_fa(const MvParams& p, cudaStream_t stream) {
   // activation columns served per pass: dense B, gather at most B pairs per
   // expert when ids are distinct per token (groups are capped at 8 * NT)
   const bool wide = p.warps == 2 * kWarps;
+  if (p.xphase)  // phased activation staging: 16-warp CTAs, register lookups
+    return p.B > 8 ? launch_t<FMT, 2, 2 * kWarps, AM, false, true>(p, stream)
+                   : launch_t<FMT, 1, 2 * kWarps, AM, false, true>(p, stream);
   if constexpr (FMT == QMV_FMT_INT4KM) {  // the palette-copy instances (batch <= 8)
     if (p.km_smem) {
       if (p.one) return launch_t<FMT, 0, kWarps, AM, true>(p, stream);

@@ -39,9 +39,11 @@
  *  - Errors: argument checks run on the host before anything is enqueued
  *    and return QMV_ERR_ARG (null or misaligned pointer, bad format or clip
  *    list), QMV_ERR_SHAPE (N < 1, K < 32, K % 32 != 0, E < 1) or
- *    QMV_ERR_UNSUPPORTED (B or topk outside [1, 16], or a shape whose
- *    activations do not fit the kernel's on-chip staging); a failed launch
- *    returns QMV_ERR_CUDA.  Bad DATA is found on the device: the kernel sets
+ *    QMV_ERR_UNSUPPORTED (B or topk outside [1, 16]; for int8km, and for the
+ *    int4km part of the mixed format, a shape whose activations do not fit
+ *    the kernel's on-chip staging -- the other formats stage such
+ *    activations one K-phase at a time); a failed launch returns
+ *    QMV_ERR_CUDA.  Bad DATA is found on the device: the kernel sets
  *    a bit of a library-owned device status word (QMV_FLAG_*) and carries
  *    on; qmv_status_fetch reads and clears it.  No kernel traps.
  *  - The library-owned status word is per device; calls that run on several

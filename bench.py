@@ -822,7 +822,7 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- main
 
-PROFILE_CASES = ("fp4", "int4", "int4km", "int8", "int4aff", "int8km", "int4km_o8", "fp4_b16",
+PROFILE_CASES = ("fp4", "int4", "int4km", "int8", "int4aff", "int8km", "int4km_o8", "fp4_b16", "fp4_b16_tc",
                  "decode_step_b1", "decode_step_b8")
 
 
@@ -830,7 +830,8 @@ def profile_case(name: str) -> int:
     """A small case for a profiler: one format's matvec on 65536 x 2048
     weights (larger than L2, a few hundred MB on the device), encoded by the
     library (int8km: stand-in tables), three launches at batch 1 (fp4_b16:
-    batch 16).  Prints one line and exits."""
+    batch 16 on the mma.sync kernel; fp4_b16_tc: on the tcgen05 kernel).
+    Prints one line and exits."""
     import torch
     import weight_only_quantized_qmv_b200 as q
     from weight_only_quantized_qmv_b200 import synth
@@ -855,7 +856,8 @@ def profile_case(name: str) -> int:
                           "flags": flags}), flush=True)
         return 1 if flags else 0
     g = synth.generator(0, "cuda")
-    B = 16 if name == "fp4_b16" else 1
+    B = 16 if name.startswith("fp4_b16") else 1
+    q.set_fp4_tensor_cores(name == "fp4_b16_tc")
     x = synth.activations(B, K, g)
     if name == "int8km":
         lut, idx = synth.palette_tables8(N, K, g)

@@ -82,6 +82,7 @@ enum {
 #define QMV_FLAG_NONFINITE 0x1u      /* encode: a block held Inf/NaN (block written as zeros) */
 #define QMV_FLAG_SCALE_OVERFLOW 0x2u /* encode: no clip gave a finite fp16 scale (block zeroed) */
 #define QMV_FLAG_BAD_EXPERT 0x4u     /* gather: expert id outside [0, E) (that output row zeroed) */
+#define QMV_FLAG_TIMEOUT 0x8u        /* a kernel's bounded wait on its own tensor-core work gave up (that launch's outputs are invalid) */
 
 /* ---------------------------------------------------------------------
  * Encoders (offline conversion; [P1] sec. 1-2).
@@ -317,6 +318,22 @@ qmv_status qmv_status_fetch(void* stream, uint32_t* flags);
  * encoder call on the same stream, synchronize or keep it off.  Default 0.
  * Returns QMV_ERR_ARG if enable is not 0 or 1. */
 qmv_status qmv_set_weight_prefetch(int enable);
+
+/* fp4 matvecs at 2..16 activation columns on the tcgen05 tensor cores.
+ * With mode = 1, dense fp4 matvec launches made afterwards (any stream, any
+ * thread) with 2 <= B <= 16, K a multiple of 512 no larger than 4608 (16
+ * activation columns and two 16 KB code stages in shared memory), 16-byte
+ * aligned codes, scales and x, and neither the fused argmax nor the
+ * mixed format's accumulation, run the tensor-memory kernel: 128-row tiles,
+ * codes streamed by TMA, each row's E2M1 weights times its block scales
+ * decoded exactly to fp16 relative to the row's largest block exponent, the
+ * MMA (M = 128, N = 16) accumulating in fp32 ("Dense-path int4km coverage",
+ * sec. 8).  Blocks more than 2^36 below the row's largest scale are dropped
+ * (their terms lie below fp32's resolution of the result).  Other launches
+ * keep the mma.sync kernel.  mode = 0 uses the mma.sync kernel everywhere.
+ * A bounded wait inside the kernel that gives up sets QMV_FLAG_TIMEOUT.
+ * Returns QMV_ERR_ARG if mode is not 0 or 1. */
+qmv_status qmv_set_fp4_tensor_cores(int mode);
 
 /* Text of the last error of this host thread ("" if none). */
 const char* qmv_last_error(void);

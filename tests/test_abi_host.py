@@ -109,6 +109,14 @@ def test_weight_prefetch_option(L):
     assert L.qmv_set_weight_prefetch(0) == q.OK
 
 
+def test_fp4_tensor_core_option(L):
+    import weight_only_quantized_qmv_b200 as q
+    assert L.qmv_set_fp4_tensor_cores(2) == q.ERR_ARG
+    assert L.qmv_set_fp4_tensor_cores(-1) == q.ERR_ARG
+    assert L.qmv_set_fp4_tensor_cores(1) == q.OK
+    assert L.qmv_set_fp4_tensor_cores(0) == q.OK
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     import weight_only_quantized_qmv_b200 as q

@@ -25,7 +25,7 @@ FMT_FP4, FMT_INT4, FMT_INT4KM, FMT_INT8, FMT_INT4AFF, FMT_INT8KM = 0, 1, 2, 3, 4
 FMT_NAMES = {FMT_FP4: "fp4", FMT_INT4: "int4", FMT_INT4KM: "int4km", FMT_INT8: "int8", FMT_INT4AFF: "int4aff",
              FMT_INT8KM: "int8km"}
 KM8_GROUP = 32  # int8km: output rows sharing one 256-entry LUT
-FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT = 1, 2, 4
+FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, FLAG_BAD_EXPERT, FLAG_TIMEOUT = 1, 2, 4, 8
 OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_DATA, ERR_CUDA = 0, -1, -2, -3, -4, -5
 
 # Clip lists of the workloads: int4 searches 1.00, 0.95, ..., 0.50 (float32
@@ -68,6 +68,7 @@ SIGNATURES = {
     "qmv_dequant": [_I32, _P, _P, _I64, _I64, _P, _P],
     "qmv_status_fetch": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "qmv_set_weight_prefetch": [_I32],
+    "qmv_set_fp4_tensor_cores": [_I32],
     "qmv_last_error": [],
     "qmv_version": [],
 }
@@ -426,6 +427,13 @@ def set_weight_prefetch(enable: bool) -> None:
     work in their stream completes (only while nothing in flight writes the
     weights; see qmv_set_weight_prefetch in include/qmv.h)."""
     _call("qmv_set_weight_prefetch", int(bool(enable)))
+
+
+def set_fp4_tensor_cores(enable: bool) -> None:
+    """Run dense fp4 matvecs at 2..16 activation columns on the tcgen05
+    tensor-memory kernel where their shape allows (see
+    qmv_set_fp4_tensor_cores in include/qmv.h); off: the mma.sync kernel."""
+    _call("qmv_set_fp4_tensor_cores", int(bool(enable)))
 
 
 def status_fetch(stream=None) -> int:

@@ -13,6 +13,7 @@ namespace {
 
 thread_local char g_err[512] = "";
 std::atomic<int> g_weight_prefetch{0};  // qmv_set_weight_prefetch
+std::atomic<int> g_fp4_tc{0};           // qmv_set_fp4_tensor_cores
 
 qmv_status fail(qmv_status code, const char* fmt, ...) {
   va_list ap;
@@ -188,7 +189,9 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
   int sms;
   QMV_TRY(device_ctx(&st, &sms));
   const bool km8 = fmt == QMV_FMT_INT8KM;
-  if (!(km8 ? qmv::plan_km8(p, sms) : qmv::plan_matvec(fmt, p, sms)))
+  const bool tc = fmt == QMV_FMT_FP4 && !gather && !am && !accum && !xcols && B >= 2 &&
+                  g_fp4_tc.load(std::memory_order_relaxed) && qmv::plan_fp4_tc(p, sms);
+  if (!tc && !(km8 ? qmv::plan_km8(p, sms) : qmv::plan_matvec(fmt, p, sms)))
     return fail(QMV_ERR_UNSUPPORTED, "activations (%d rows x %lld) do not fit the on-chip staging", p.n_xrows,
                 (long long)K);
   p.status = st;
@@ -210,7 +213,9 @@ qmv_status matvec_common(int fmt, const void* codes, const void* aux, const uint
     p.am_idx = am->idx;
     p.am_val = am->val;
   }
-  cudaError_t e = km8 ? qmv::launch_km8(p, (cudaStream_t)stream) : qmv::launch_matvec(fmt, p, (cudaStream_t)stream);
+  cudaError_t e = tc    ? qmv::launch_fp4_tc(p, (cudaStream_t)stream)
+                  : km8 ? qmv::launch_km8(p, (cudaStream_t)stream)
+                        : qmv::launch_matvec(fmt, p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "matvec launch");
   return QMV_OK;
 }
@@ -481,6 +486,12 @@ const char* qmv_last_error(void) { return g_err; }
 qmv_status qmv_set_weight_prefetch(int enable) {
   if (enable != 0 && enable != 1) return fail(QMV_ERR_ARG, "enable must be 0 or 1 (got %d)", enable);
   g_weight_prefetch.store(enable, std::memory_order_relaxed);
+  return QMV_OK;
+}
+
+qmv_status qmv_set_fp4_tensor_cores(int mode) {
+  if (mode != 0 && mode != 1) return fail(QMV_ERR_ARG, "mode must be 0 or 1 (got %d)", mode);
+  g_fp4_tc.store(mode, std::memory_order_relaxed);
   return QMV_OK;
 }
 

@@ -133,6 +133,10 @@ cudaError_t launch_split_f32(const float* W, int64_t N, int64_t K, const int32_t
 cudaError_t launch_outlier_acc(const int8_t* q, const uint16_t* s, const int32_t* cols, const uint16_t* x, int B,
                                int64_t N, int64_t K, int64_t C, float* y, int num_sms, cudaStream_t stream);
 cudaError_t launch_km8(const MvParams& p, cudaStream_t stream);
+// fp4 at 1..16 activation columns on the tcgen05 tensor cores (dense only;
+// the activations of all K staged per CTA): geometry, launch.
+bool plan_fp4_tc(MvParams& p, int num_sms);
+cudaError_t launch_fp4_tc(const MvParams& p, cudaStream_t stream);
 
 // ---- encoders / dequant ------------------------------------------------------
 struct ClipList {

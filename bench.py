@@ -87,9 +87,10 @@ def csrc_digest(sources=MV_KERNEL_SOURCES) -> str:
 
 
 def profiled_traffic(kernel_fmt: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", "qmv_matvec_lm_head_248320x2048_b1.md")
+    """DRAM bytes of one full-head launch from the committed ncu summary (the
+    65536-row capture scaled by rows: the kernel streams each weight byte
+    once), if it was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "qmv_matvec_formats_65536x2048_b1.md")
     if not os.path.exists(p):
         return None
     txt = open(p).read()

@@ -502,9 +502,10 @@ def measure_int8_head_c2(q, dev, stream, peak):
 
 def measure_next_formats(q, x, dev, stream, peak):
     """The formats beyond the step's four, on the same head at batch 1 (graphs
-    of 10 launches): affine int4 and the mixed int4km + int8 outlier columns
-    (64), both encoded on the GPU from the same synthetic weights, and int8km
-    (stand-in tables: no GPU fit for 256-entry palettes)."""
+    of 10 launches): affine int4, the mixed int4km + int8 outlier columns
+    (64) and int8km (256-entry palettes per 32 rows, 20 Lloyd steps), all
+    encoded on the GPU from the same synthetic weights (each encoder warmed
+    up on a 64-row slice first)."""
     import torch
     from weight_only_quantized_qmv_b200 import synth
     g = synth.generator(0, dev)
@@ -522,11 +523,14 @@ def measure_next_formats(q, x, dev, stream, peak):
         torch.cuda.synchronize()
         return r, a.elapsed_time(b)
 
+    q.encode_int4aff(W[:64].contiguous())
+    q.encode_int4km_o8(W[:64].contiguous(), O8_COLS)
+    q.encode_int8km(W[:64].contiguous())
     (c4a, a4a), enc["int4aff"] = timed(lambda: q.encode_int4aff(W))
     o8, enc["int4km_o8"] = timed(lambda: q.encode_int4km_o8(W, O8_COLS))
+    (idx8, lut8), enc["int8km"] = timed(lambda: q.encode_int8km(W))
     del W
     torch.cuda.empty_cache()
-    lut8, idx8 = synth.palette_tables8(N_HEAD, K_HEAD, synth.generator(1, dev))
     if q.status_fetch():
         raise RuntimeError("encoder status flags")
     out = torch.empty((1, N_HEAD), dtype=torch.float32, device=dev)
@@ -544,7 +548,7 @@ def measure_next_formats(q, x, dev, stream, peak):
                   "frac_of_measured_hbm": round(gbs / peak, 4),
                   "bytes": nb, "encode_ms": round(enc[f], 2) if f in enc else None}
     res["int4km_o8"]["launches_per_call"] = 2
-    res["int8km"]["weights"] = "stand-in tables (random indices, sorted N(0, 0.02) palettes)"
+    res["int8km"]["weights"] = "GPU k-means fit (qmv_encode_int8km, 20 Lloyd steps)"
     return res
 
 
@@ -830,7 +834,7 @@ PROFILE_CASES = ("fp4", "int4", "int4km", "int8", "int4aff", "int8km", "int4km_o
 def profile_case(name: str) -> int:
     """A small case for a profiler: one format's matvec on 65536 x 2048
     weights (larger than L2, a few hundred MB on the device), encoded by the
-    library (int8km: stand-in tables), three launches at batch 1 (fp4_b16:
+    library, three launches at batch 1 (fp4_b16:
     batch 16 on the mma.sync kernel; fp4_b16_tc: on the tcgen05 kernel).
     Prints one line and exits."""
     import torch
@@ -860,11 +864,11 @@ def profile_case(name: str) -> int:
     B = 16 if name.startswith("fp4_b16") else 1
     q.set_fp4_tensor_cores(name == "fp4_b16_tc")
     x = synth.activations(B, K, g)
+    W, _ = synth.weights(N, K, g, n_outlier_cols=2)
     if name == "int8km":
-        lut, idx = synth.palette_tables8(N, K, g)
+        idx, lut = q.encode_int8km(W)
         run = lambda: q.matvec_int8km(idx, lut, x)
     else:
-        W, _ = synth.weights(N, K, g, n_outlier_cols=2)
         if name == "int4km_o8":
             enc = q.encode_int4km_o8(W, O8_COLS)
             run = lambda: q.matvec_int4km_o8(*enc, x)
@@ -876,7 +880,7 @@ def profile_case(name: str) -> int:
                     "int4aff": q.encode_int4aff}[fmt]
             c, a = encf(W)
             run = lambda: q.matvec(fid, c, a, x)
-        del W
+    del W
     for _ in range(3):
         y = run()
     torch.cuda.synchronize()

@@ -157,6 +157,34 @@ int64_t qmv_int4aff_aux_row_bytes(int64_t K);
 qmv_status qmv_encode_int4km(const float* W, int64_t N, int64_t K, int iters, uint16_t* lut, uint8_t* idx,
                              void* stream);
 
+/* int8km encode: per group of 32 consecutive output rows a 256-entry fp16
+ * palette by scalar 1-D k-means and one 8-bit index per weight ([P3]
+ * "Palettization": per-grouped-channel LUTs, 2^n_bits centroids; [P5]
+ * "int8 k-means > whole-model int4": 8-bit k-means, group size 32).  Per
+ * group of n = rows * K weights (a last group of N % 32 rows is fitted on
+ * the rows it has) the steps of qmv_encode_int4km with 256 centres: sort
+ * ascending (-0 before +0); centre k starts at sorted[floor((2k+1) n / 512)];
+ * `iters` Lloyd steps (nearest centre by double distance, ties to the lower
+ * index; a non-empty centre becomes float(double sum of its members in
+ * ascending order / count), an empty one keeps its value); palette = fp16
+ * RNE of the centres; index = nearest palette entry (double distance, ties
+ * to the lower index).  A group with Inf/NaN is written as zeros and sets
+ * QMV_FLAG_NONFINITE.
+ *   W          [N, K] float32 (device)
+ *   K          multiple of 32, at most 16384
+ *   iters      0 .. 1000 (the workloads use 20)
+ *   lut        [ceil(N/32), 256] fp16 (out);  idx [N, K] uint8 (out)
+ *   workspace  device buffer of at least qmv_int8km_encode_workspace_bytes
+ *              (N, K) bytes, 16-byte aligned (sort scratch, overwritten)
+ * Errors: QMV_ERR_ARG (pointers, iters, short workspace), QMV_ERR_SHAPE
+ * (N, K % 32), QMV_ERR_UNSUPPORTED (K > 16384). */
+qmv_status qmv_encode_int8km(const float* W, int64_t N, int64_t K, int iters, uint16_t* lut, uint8_t* idx,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of the workspace of qmv_encode_int8km: at most 160 groups in
+ * flight, next_pow2(min(N, 32) * K) 4-byte keys each. */
+int64_t qmv_int8km_encode_workspace_bytes(int64_t N, int64_t K);
+
 /* ---------------------------------------------------------------------
  * Fused dequantize + matvec, y = x Wdq^T with fp32 accumulation
  * ([P2] sec. 1-3, 8).  x: [B, K] fp16; y: [B, N] float32 (overwritten).

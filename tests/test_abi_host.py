@@ -109,6 +109,29 @@ def test_weight_prefetch_option(L):
     assert L.qmv_set_weight_prefetch(0) == q.OK
 
 
+def test_encode_int8km_argument_checks(L):
+    import weight_only_quantized_qmv_b200 as q
+    nb = L.qmv_int8km_encode_workspace_bytes(100, 2048)
+    # 4 groups in flight, next_pow2(32 * 2048) keys of 4 bytes each
+    assert nb == 4 * 65536 * 4
+    assert L.qmv_int8km_encode_workspace_bytes(1000000, 96) == 160 * 4096 * 4
+    assert L.qmv_int8km_encode_workspace_bytes(5, 96) == 1 * 512 * 4
+    assert L.qmv_int8km_encode_workspace_bytes(0, 96) == 0
+    fn = L.qmv_encode_int8km
+    assert fn(None, 100, 2048, 20, FAKE, FAKE, FAKE, nb, None) == q.ERR_ARG
+    assert fn(FAKE, 100, 2048, 20, None, FAKE, FAKE, nb, None) == q.ERR_ARG
+    assert fn(FAKE, 100, 2048, 20, ctypes.c_void_p(0x10001), FAKE, FAKE, nb, None) == q.ERR_ARG
+    assert fn(FAKE, 100, 2048, 20, FAKE, None, FAKE, nb, None) == q.ERR_ARG
+    assert fn(FAKE, 100, 2048, -1, FAKE, FAKE, FAKE, nb, None) == q.ERR_ARG
+    assert fn(FAKE, 100, 2048, 1001, FAKE, FAKE, FAKE, nb, None) == q.ERR_ARG
+    assert fn(FAKE, 100, 2048, 20, FAKE, FAKE, None, nb, None) == q.ERR_ARG
+    assert fn(FAKE, 100, 2048, 20, FAKE, FAKE, FAKE, nb - 1, None) == q.ERR_ARG
+    assert "workspace" in _err(L)
+    assert fn(FAKE, 100, 2040, 20, FAKE, FAKE, FAKE, nb, None) == q.ERR_SHAPE
+    assert fn(FAKE, 0, 2048, 20, FAKE, FAKE, FAKE, nb, None) == q.ERR_SHAPE
+    assert fn(FAKE, 10, 16416, 20, FAKE, FAKE, FAKE, 1 << 30, None) == q.ERR_UNSUPPORTED
+
+
 def test_fp4_tensor_core_option(L):
     import weight_only_quantized_qmv_b200 as q
     assert L.qmv_set_fp4_tensor_cores(2) == q.ERR_ARG

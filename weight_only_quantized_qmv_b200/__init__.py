@@ -69,6 +69,8 @@ SIGNATURES = {
     "qmv_status_fetch": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "qmv_set_weight_prefetch": [_I32],
     "qmv_set_fp4_tensor_cores": [_I32],
+    "qmv_encode_int8km": [_P, _I64, _I64, _I32, _P, _P, _P, ctypes.c_size_t, _P],
+    "qmv_int8km_encode_workspace_bytes": [_I64, _I64],
     "qmv_last_error": [],
     "qmv_version": [],
 }
@@ -193,6 +195,20 @@ _CODES = {FMT_FP4: torch.uint8, FMT_INT4: torch.uint8, FMT_INT4KM: torch.uint8, 
           FMT_INT4AFF: torch.uint8, FMT_INT8KM: torch.uint8}
 _ENTRY = {FMT_FP4: "qmv_matvec_fp4", FMT_INT4: "qmv_matvec_int4", FMT_INT4KM: "qmv_matvec_int4km",
           FMT_INT8: "qmv_matvec_int8", FMT_INT4AFF: "qmv_matvec_int4aff", FMT_INT8KM: "qmv_matvec_int8km"}
+
+
+def encode_int8km(W: torch.Tensor, iters: int = KMEANS_ITERS, stream=None):
+    """W float32 [N, K] -> (idx uint8 [N, K], lut float16 [ceil(N/32), 256]):
+    a 256-entry k-means palette per 32 rows and one index per weight."""
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    idx = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    lut = torch.empty((int8km_groups(N), 256), dtype=torch.float16, device=W.device)
+    nb = int(lib().qmv_int8km_encode_workspace_bytes(N, K))
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=W.device)
+    _call("qmv_encode_int8km", _ptr(W), N, K, int(iters), _ptr(lut), _ptr(idx), _ptr(ws), ws.numel(),
+          _stream(stream))
+    return idx, lut
 
 
 def int8km_groups(N: int) -> int:

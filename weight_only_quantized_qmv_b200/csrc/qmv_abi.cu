@@ -340,6 +340,31 @@ qmv_status qmv_outlier_columns(const float* W, int64_t N, int64_t K, int64_t C, 
   return QMV_OK;
 }
 
+int64_t qmv_int8km_encode_workspace_bytes(int64_t N, int64_t K) {
+  if (N < 1 || K < 32 || K > 16384) return 0;
+  return qmv::km8fit_workspace_bytes(N, K);
+}
+
+qmv_status qmv_encode_int8km(const float* W, int64_t N, int64_t K, int iters, uint16_t* lut, uint8_t* idx,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  QMV_TRY(check_ptr(W, "W"));
+  QMV_TRY(check_ptr(idx, "idx"));
+  if (!lut || (reinterpret_cast<uintptr_t>(lut) & 1u)) return fail(QMV_ERR_ARG, "lut null or misaligned");
+  QMV_TRY(check_shape(N, K));
+  if (iters < 0 || iters > 1000) return fail(QMV_ERR_ARG, "iters must be in [0, 1000] (got %d)", iters);
+  if (K > 16384) return fail(QMV_ERR_UNSUPPORTED, "K must be <= 16384 for the int8km palette fit");
+  QMV_TRY(check_ptr(workspace, "workspace"));
+  const int64_t need = qmv::km8fit_workspace_bytes(N, K);
+  if ((int64_t)workspace_bytes < need)
+    return fail(QMV_ERR_ARG, "workspace has %zu bytes, needs %lld", workspace_bytes, (long long)need);
+  uint32_t* st;
+  int sms;
+  QMV_TRY(device_ctx(&st, &sms));
+  cudaError_t e = qmv::launch_encode_int8km(W, N, K, iters, lut, idx, workspace, st, sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "encode_int8km launch");
+  return QMV_OK;
+}
+
 qmv_status qmv_encode_int4km_o8(const float* W, int64_t N, int64_t K, int64_t C, int iters, int32_t* cols,
                                 uint16_t* lut, uint8_t* idx, int8_t* ocodes, uint16_t* oscales, void* workspace,
                                 size_t workspace_bytes, void* stream) {

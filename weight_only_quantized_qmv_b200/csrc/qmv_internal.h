@@ -133,6 +133,11 @@ cudaError_t launch_split_f32(const float* W, int64_t N, int64_t K, const int32_t
 cudaError_t launch_outlier_acc(const int8_t* q, const uint16_t* s, const int32_t* cols, const uint16_t* x, int B,
                                int64_t N, int64_t K, int64_t C, float* y, int num_sms, cudaStream_t stream);
 cudaError_t launch_km8(const MvParams& p, cudaStream_t stream);
+// int8km palette fit (256 entries per 32 rows) and its workspace: one slot
+// of next_pow2(min(N, 32) * K) keys per CTA.
+int64_t km8fit_workspace_bytes(int64_t N, int64_t K);
+cudaError_t launch_encode_int8km(const float* W, int64_t N, int64_t K, int iters, uint16_t* lut, uint8_t* idx,
+                                 void* workspace, uint32_t* status, int num_sms, cudaStream_t stream);
 // fp4 at 1..16 activation columns on the tcgen05 tensor cores (dense only;
 // the activations of all K staged per CTA): geometry, launch.
 bool plan_fp4_tc(MvParams& p, int num_sms);

@@ -1,7 +1,8 @@
 """bench.py's end-to-end leg on the GPU at a small size: the activations go
-in from pinned host memory, the matvecs run and the outputs come back to
-pinned host memory in stream order, and the host copies equal the device
-results of the same step bit for bit (the leg raises otherwise)."""
+in from pinned host memory, the matvecs run, each output comes back to
+pinned host memory on a copy stream ordered after its matvec by an event,
+and the host copies equal the device results of the same step bit for bit
+(the leg raises otherwise)."""
 import os
 import sys
 

@@ -741,21 +741,31 @@ def measure_e2e(q, ops, fmt_id, x, dev, stream, formats, ref_outs, steps):
 
 # ----------------------------------------------------------------- CPU oracle
 
-def oracle_sample(W_rows, x_np, seconds_target):
-    """Time the oracle's fp64 matvec on a row sample of the head for each
-    format; returns (GB/s on the algorithmic-bytes definition, rows, threads)."""
+def oracle_encodings(W_rows):
+    """The oracle's encodings of a row sample for the four formats (int4km:
+    stand-in tables of the fitted shapes; the CPU fit of 16 centres per row
+    is not part of the per-token path), with the encode times (s)."""
     import numpy as np
     import oracle
-    enc = {}
-    c, s, _ = oracle.encode_fp4(W_rows)
-    enc["fp4"] = (oracle.FMT_FP4, c, s)
-    c, s, _ = oracle.encode_int4(W_rows)
-    enc["int4"] = (oracle.FMT_INT4, c, s)
+    enc, secs = {}, {}
+    for f, fn in (("fp4", oracle.encode_fp4), ("int4", oracle.encode_int4), ("int8", oracle.encode_int8)):
+        t0 = time.perf_counter()
+        c, s, _ = fn(W_rows)
+        secs[f] = time.perf_counter() - t0
+        enc[f] = ({"fp4": oracle.FMT_FP4, "int4": oracle.FMT_INT4, "int8": oracle.FMT_INT8}[f], c, s)
     lut = np.sort(np.random.default_rng(0).standard_normal((W_rows.shape[0], 16)) * 0.02, axis=1).astype(np.float16)
     idx = np.random.default_rng(1).integers(0, 256, (W_rows.shape[0], K_HEAD // 2), dtype=np.uint8)
     enc["int4km"] = (oracle.FMT_INT4KM, idx, lut)
-    c, s, _ = oracle.encode_int8(W_rows)
-    enc["int8"] = (oracle.FMT_INT8, c, s)
+    return enc, secs
+
+
+def oracle_sample(W_rows, x_np, seconds_target, enc=None):
+    """Time the oracle's fp64 matvec on a row sample of the head for each
+    format; returns (GB/s on the algorithmic-bytes definition, rows, threads,
+    seconds, passes)."""
+    import oracle
+    if enc is None:
+        enc, _ = oracle_encodings(W_rows)
     R = W_rows.shape[0]
     t0 = time.perf_counter()
     done = 0
@@ -773,13 +783,27 @@ def oracle_sample(W_rows, x_np, seconds_target):
 
 
 def cpu_baseline(W, x, seconds=12.0, rows=8192):
-    import numpy as np
+    """The oracle on the host cores: encode (fp4, int4 with 11 clips, int8) and
+    the fp64 matvec of all four formats on a row sample, the matvec on all
+    cores (the reported value) and on one thread."""
+    import oracle
     Wn = W[:rows].cpu().numpy()
     xn = x.cpu().numpy()
-    gbs, R, thr, dt, passes = oracle_sample(Wn, xn, seconds)
+    enc, enc_s = oracle_encodings(Wn)
+    gbs, R, thr, dt, passes = oracle_sample(Wn, xn, seconds, enc)
+    n0 = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        gbs1, _, _, dt1, passes1 = oracle_sample(Wn, xn, 3.0, enc)
+    finally:
+        oracle.set_num_threads(n0)
     return {"value": round(gbs, 3), "unit": "GB/s", "cores": thr, "kind": "oracle", "cpu_model": cpu_model(),
+            "single_thread_gbs": round(gbs1, 4),
+            "encode_ms": {f: round(1e3 * v, 1) for f, v in enc_s.items()},
+            "encode_read_gbs": {f: round(4.0 * R * K_HEAD / v / 1e9, 3) for f, v in enc_s.items()},
             "sample": f"fp64 oracle matvec, {R} of 248320 rows x 2048, all four formats, {passes} passes in "
-                      f"{dt:.1f} s (bytes scaled by the algorithmic-bytes definition)"}
+                      f"{dt:.1f} s on {thr} threads and {passes1} in {dt1:.1f} s on one (bytes scaled by the "
+                      f"algorithmic-bytes definition); encoders timed once on the same rows ({thr} threads)"}
 
 
 def run_reference(args):

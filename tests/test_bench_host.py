@@ -58,3 +58,20 @@ def test_spread_percentiles():
     st = bench.spread([float(v) for v in range(25, 0, -1)])
     assert st["median"] == 13.0 and st["p10"] == 3.0 and st["p90"] == 23.0
     assert st["mean"] == 13.0 and st["reps"] == 25
+
+
+def test_cpu_baseline_reports_oracle_encode_and_thread_counts():
+    """The CPU leg times the oracle's encoders and its matvec on all cores
+    and on one thread, on a bounded row sample, and says so."""
+    import torch
+    from weight_only_quantized_qmv_b200 import synth
+    g = synth.generator(0, "cpu")
+    W, _ = synth.weights(64, bench.K_HEAD, g)
+    x = synth.activations(1, bench.K_HEAD, g)
+    r = bench.cpu_baseline(W, x, seconds=0.2, rows=64)
+    assert r["kind"] == "oracle" and r["unit"] == "GB/s"
+    assert r["value"] > 0 and r["single_thread_gbs"] > 0
+    assert r["cores"] == oracle.num_threads() >= 1
+    assert set(r["encode_ms"]) == {"fp4", "int4", "int8"} and all(v > 0 for v in r["encode_ms"].values())
+    assert "64 of 248320 rows" in r["sample"] and "on one" in r["sample"]
+    assert isinstance(W, torch.Tensor)

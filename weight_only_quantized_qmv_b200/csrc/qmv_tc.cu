@@ -10,15 +10,15 @@
 //
 // One persistent CTA per SM owns 128-row tiles (the MMA's M) round robin,
 // its warps split by role:
-//  * warp 16 (one thread) streams the tile's codes by TMA, 128 rows x 256
+//  * warp 8 (one thread) streams the tile's codes by TMA, 128 rows x 256
 //    in-features (16 KB, 128-byte swizzle) per stage of a ring, and the
 //    tile's scale rows (one padded 2D box) into one of two scale buffers;
-//  * warps 0-15 decode: warp w owns tensor-memory lanes 32 (w % 4) .. + 31
-//    (one row each) and quarter w / 4 of each chunk's in-features; a thread
-//    turns its 64 codes into fp16 pairs by the hardware E2M1 conversion,
-//    times the block scale as an exact fp16 power of two, and writes the 32
+//  * warps 0-7 decode: warp w owns tensor-memory lanes 32 (w % 4) .. + 31
+//    (one row each) and half w / 4 of each chunk's in-features; a thread
+//    turns its 128 codes into fp16 pairs by the hardware E2M1 conversion,
+//    times the block scale as an exact fp16 power of two, and writes the 64
 //    words into tensor memory as the MMA's A operand (two buffers);
-//  * warps 17-20 (one thread each) issue the MMAs, MMA s of a chunk by
+//  * warps 9-12 (one thread each) issue the MMAs, MMA s of a chunk by
 //    issuer s % 4 (an issuing thread waits ~60 cycles per MMA at N = 16;
 //    four of them keep the tensor core fed): M = 128, N = 16, K = 16 each,
 //    A from tensor memory, B = the activations staged once per CTA in
@@ -26,7 +26,7 @@
 //    accumulators in tensor memory: eight per tile (MMA s of a chunk adds
 //    into accumulator s % 8, so consecutive MMAs do not wait on each
 //    other's result), two tiles in flight;
-//  * warps 21-24 read each finished tile's accumulators back (tcgen05.ld),
+//  * warps 13-16 read each finished tile's accumulators back (tcgen05.ld),
 //    sum the eight and store y.
 // Scaled E2M1 values are fp16-exact for exponents 2^-23 .. 2^13.  Each row
 // is decoded relative to its largest block exponent (that block at 2^13) and
@@ -52,10 +52,10 @@ constexpr int kTcCols = 16;                                 // MMA N: activation
 constexpr int kTcChunk = 256;                               // in-features per staged code chunk
 constexpr int kTcChunkBytes = kTcRows * kTcChunk / 2;       // 16 KB
 constexpr int kTcMaxStages = 8;
-constexpr int kTcDecWarps = 16;                             // decoders: lanes 32 (w % 4).., in-feature quarter w / 4
-constexpr int kTcProdWarp = 16;                             // TMA producer
-constexpr int kTcMmaWarp0 = 17, kTcMmaWarps = 4;            // MMA issuers: MMA s of a chunk by issuer s % 4
-constexpr int kTcEpiWarp0 = 21, kTcWarps = 25;              // epilogue: warps 21..24
+constexpr int kTcDecWarps = 8;                              // decoders: lanes 32 (w % 4).., in-feature half w / 4
+constexpr int kTcProdWarp = 8;                              // TMA producer
+constexpr int kTcMmaWarp0 = 9, kTcMmaWarps = 4;             // MMA issuers: MMA s of a chunk by issuer s % 4
+constexpr int kTcEpiWarp0 = 13, kTcWarps = 17;              // epilogue: warps 13..16
 constexpr int kTcThreads = kTcWarps * 32;
 constexpr int kTcStageThreads = (kTcWarps - 1) * 32;        // every warp but the producer stages x
 constexpr int kTcAcc = 8;                                   // independent accumulators per tile (MMA s -> s % 8)
@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp < kTcDecWarps) {
     // ---- decoders ----
-    const int h = warp >> 2;                 // in-feature quarter of each chunk (two blocks)
+    const int h = warp >> 2;                 // in-feature half of each chunk (four blocks)
     const int r = (warp & 3) * 32 + lane;    // row within the tile
     const Mul mul = Mul::make();
     uint32_t gc = 0;
@@ -403,10 +403,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         const uint32_t crow = s_stage + (uint32_t)(st * kTcChunkBytes + r * 128);
-        uint4 cv[2];
+        uint4 cv[4];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) cv[j] = lds128(crow + ((uint32_t)((2 * h + j) ^ (r & 7)) << 4));
-        const uint32_t sc = *sptr<uint16_t>(srow + 8u * c + 2u * h);
+        for (int j = 0; j < 4; ++j) cv[j] = lds128(crow + ((uint32_t)((4 * h + j) ^ (r & 7)) << 4));
+        const uint32_t sc = lds32(srow + 8u * c + 4u * h);
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(smem_u32(&sh.empty[st]));
@@ -419,11 +419,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t t_a = tmem + lane_base + 128u * ab + 32u * h;
+        const uint32_t t_a = tmem + lane_base + 128u * ab + 64u * h;
         uint32_t a[32];
         decode_block16(cv[0], block_scale_h2((int)(sc & 0xFFu), emax), a, mul);
-        decode_block16(cv[1], block_scale_h2((int)(sc >> 8), emax), a + 16, mul);
+        decode_block16(cv[1], block_scale_h2((int)((sc >> 8) & 0xFFu), emax), a + 16, mul);
         tmem_st32(t_a, a);
+        decode_block16(cv[2], block_scale_h2((int)((sc >> 16) & 0xFFu), emax), a, mul);
+        decode_block16(cv[3], block_scale_h2((int)(sc >> 24), emax), a + 16, mul);
+        tmem_st32(t_a + 32u, a);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

@@ -30,8 +30,11 @@ def fit_both(q, Wn, iters):
 
 
 @pytest.mark.parametrize("N,K,iters", [(64, 512, 0), (64, 512, 1), (64, 512, 3), (70, 96, 3), (33, 544, 2),
-                                       (32, 2048, 2), (5, 2080, 3)])
+                                       (32, 2048, 2), (5, 2080, 3), (1, 96, 3), (33, 32, 2), (32, 16384, 1)])
 def test_encode_int8km_bit_exact(q, N, K, iters):
+    """Shapes: groups whose keys fit one shared-memory sort chunk and ones that
+    take the global strides (up to 32 x 16384 = 2^19 keys, the largest
+    group), a single row, K = 32 with a one-row last group."""
     g = synth.generator(N * 13 + K + iters, "cpu")
     W, _ = synth.weights(N, K, g, n_outlier_cols=2)
     (lut, idx, fl), (lut_o, idx_o, fl_o) = fit_both(q, W.numpy(), iters)
